@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Selective-scan (S6) layer-core throughput on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl axon|reference]
+                    [--workload NAME]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+the prefill (conv1d + SiLU + dt + selective recurrence + C/D epilogue + SiLU(z)
+gate, returning the (conv_cache, ssm_state) pair) of the Bit-Axon layer shape
+(B1 L2048 E7680 N16 K4, bf16 io, fp32 state), followed by one cached decode step
+on the returned caches.  Throughput is counted in token x channel units:
+B*(L+1)*E per step.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own independent
+sequences (different seeds); the path has no data exchange, so there is no
+collective on the data path; the elapsed time is the max over ranks and the
+value counts the units of all ranks (weak scaling).
+
+Rank 0 prints ONE JSON line.  `--impl reference` times the fp64 CPU oracle on a
+bounded sample of the same workload instead (rank 0 only; other ranks exit 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from selective_state_space_52_b200 import workloads as W  # noqa: E402
+
+METRIC = "selective-scan throughput (G token·channel/s) and % of HBM roofline, 1 B200"
+UNIT = "G token·channel/s"
+# Transcendental (MUFU) evaluations per token x channel: 16 decays exp(dt*A_n),
+# SiLU(xc) (exp + reciprocal), softplus (exp + log), SiLU(z) (exp + reciprocal).
+MUFU_PER_TOKEN_CH = 16 + 6
+MUFU_LANES_PER_SM_CLK = 16
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# --------------------------------------------------------------- distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend=backend,
+                                             timeout=datetime.timedelta(seconds=120))
+
+
+def reduce_max(value: float, device) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        if device is not None and device.type == "cuda":
+            torch.distributed.barrier(device_ids=[device.index])
+        else:
+            torch.distributed.barrier()
+
+
+def rank_seed(base: int, rank: int, k: int = 0) -> int:
+    """Seeds of the independent per-rank problems (rank 0 == the single-GPU run)."""
+    return base + 7919 * rank + 104729 * k
+
+
+def rank_units(units_per_rank: int, world: int) -> int:
+    return units_per_rank * world
+
+
+# --------------------------------------------------------------- peaks / model
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def scan_model(wl) -> dict:
+    """Algorithmic bytes and MUFU operations of one prefill launch."""
+    s = 2 if wl.io == "bf16" else 4
+    T = wl.B * wl.L * wl.E
+    bytes_ = (4 * T * s                       # x, z, dt_raw read; y written
+              + 2 * wl.B * wl.L * wl.N * s    # B, C read
+              + wl.E * (wl.K + 3 + wl.N) * 4  # conv_w, conv_b, dt_bias, D, A_log
+              + wl.B * wl.E * wl.N * 4        # ssm_state written
+              + wl.B * (wl.K - 1) * wl.E * s)  # conv_cache written
+    return {"bytes": bytes_, "mufu": MUFU_PER_TOKEN_CH * T, "token_ch": T}
+
+
+def step_model(wl) -> dict:
+    """Algorithmic bytes of one cached decode step (state and cache read + written)."""
+    s = 2 if wl.io == "bf16" else 4
+    BE = wl.B * wl.E
+    bytes_ = (BE * (4 * s + 2 * (wl.K - 1) * s + 2 * wl.N * 4)
+              + 2 * wl.B * wl.N * s + wl.E * (wl.K + 3 + wl.N) * 4)
+    return {"bytes": bytes_, "mufu": MUFU_PER_TOKEN_CH * BE, "token_ch": BE}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_state_space_52_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode())
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key: str, workload: str, units: int):
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu summary,
+    or None when no capture exists for the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    ent = d.get(kernel_key, {}).get(workload)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    per_unit = ent["dram_bytes"] / ent["units"]
+    return per_unit * units
+
+
+# --------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons of one GPU during the timed region (NVML)."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.error = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    self.h = h
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as ex:  # no NVML: report no samples rather than guess
+            self.nv = None
+            self.error = repr(ex)
+
+    def _run(self):
+        nv = self.nv
+        while True:
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception as ex:
+                self.error = repr(ex)
+            if self._stop.wait(self.period):
+                break
+
+    def start(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+
+    def stop(self) -> dict:
+        if self._thr is not None:
+            self._stop.set()
+            self._thr.join()
+        med = statistics.median(self.samples) if self.samples else None
+        out = {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+               "samples": len(self.samples), "source": "nvml"}
+        if self.error and not self.samples:
+            out["error"] = self.error
+        return out
+
+
+# --------------------------------------------------------------- CPU oracle
+def time_oracle(wl, inp, budget_s: float, block: int = 256):
+    """Time the fp64 oracle on the first channels of the workload until the
+    budget is spent; returns (token_ch/s, token_ch done, seconds, channels)."""
+    import oracle
+    oracle.build()
+    done_ch, t_total = 0, 0.0
+    E = wl.E
+    while done_ch < E and t_total < budget_s:
+        e0, e1 = done_ch, min(E, done_ch + block)
+        sl = slice(e0, e1)
+        args = [inp["x"][:, :, sl].contiguous(), inp["z"][:, :, sl].contiguous(),
+                inp["dt_raw"][:, :, sl].contiguous(), inp["B"], inp["C"],
+                inp["conv_w"][sl], inp["conv_b"][sl], inp["dt_bias"][sl], inp["A_log"][sl],
+                inp["D"][sl]]
+        t0 = time.perf_counter()
+        oracle.scan_fwd(*args)
+        t_total += time.perf_counter() - t0
+        done_ch = e1
+    units = done_ch * wl.B * wl.L
+    return units / t_total, units, t_total, done_ch
+
+
+def run_reference(args, wl):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    inp = W.make_inputs(wl)
+    per_step_budget = max(0.5, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
+    channels = None
+    rates = []
+    for i in range(args.warmup + args.steps):
+        rate, units, secs, ch = time_oracle(wl, inp, per_step_budget, block=64)
+        channels = ch
+        if i >= args.warmup:
+            rates.append((units, secs))
+    units = sum(u for u, _ in rates)
+    secs = sum(s for _, s in rates)
+    value = units / secs / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * secs / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(wl), "sample": f"first {channels} channels x {wl.L} tokens per step"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{channels} of {wl.E} channels x {wl.L} tokens per step, "
+                                   "fp64 C oracle, single thread"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_desc(wl) -> str:
+    return (f"{wl.name}: B{wl.B} L{wl.L} E{wl.E} N{wl.N} K{wl.K}, {wl.io} io, fp32 state; "
+            "step = prefill + 1 cached decode token")
+
+
+# --------------------------------------------------------------- GPU arm
+def run_axon(args, wl):
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU for --impl axon")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl")
+    from selective_state_space_52_b200 import axon_ssm
+
+    io = wl.torch_io
+    io_code = axon_ssm.AXON_BF16 if wl.io == "bf16" else axon_ssm.AXON_F32
+    B, L, E, N, K = wl.B, wl.L, wl.E, wl.N, wl.K
+
+    # inputs: several independent sets so that consecutive steps do not hit in L2
+    params_cpu = W.make_params(wl, g=torch.Generator().manual_seed(rank_seed(wl.seed, rank)))
+    params = {k: v.to(dev) for k, v in params_cpu.items()}
+    set_bytes = 3 * B * L * E * io.itemsize
+    n_sets = max(2, math.ceil(2 * L2_BYTES / max(1, set_bytes)) + 1)
+    n_sets = min(n_sets, 8)
+    sets = []
+    for k in range(n_sets):
+        g = torch.Generator().manual_seed(rank_seed(wl.seed + 1000, rank, k))
+        sets.append({kk: v.to(dev) for kk, v in W.make_sequence(wl, g=g).items()})
+    tok = {kk: v[0].to(dev) for kk, v in W.make_decode_inputs(
+        wl, 1, g=torch.Generator().manual_seed(rank_seed(wl.seed + 3000, rank))).items()}
+
+    y = torch.empty(B, L, E, dtype=io, device=dev)
+    cc = torch.empty(B, K - 1, E, dtype=io, device=dev)
+    ss = torch.empty(B, E, N, dtype=torch.float32, device=dev)
+    y_tok = torch.empty(B, E, dtype=io, device=dev)
+    ws_bytes = axon_ssm.axon_ssm_scan_workspace_bytes(B, L, E, N, K, io_code)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    scan_launches = axon_ssm.axon_ssm_scan_launch_count(B, L, E, N, K, io_code)
+    stream = torch.cuda.current_stream(dev)
+
+    def one_step(s):
+        axon_ssm.scan_fwd(s["x"], s["z"], s["dt_raw"], s["B"], s["C"], params, None,
+                          out=(y, cc, ss), workspace=ws)
+        axon_ssm.step(tok["x"], tok["z"], tok["dt_raw"], tok["B"], tok["C"], params, (cc, ss), y=y_tok)
+
+    for i in range(args.warmup):
+        one_step(sets[i % n_sets])
+    torch.cuda.synchronize(dev)
+
+    # ---- device-resident timed region: exactly K steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t_start.record(stream)
+    for i in range(args.steps):
+        s = sets[i % n_sets]
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        axon_ssm.scan_fwd(s["x"], s["z"], s["dt_raw"], s["B"], s["C"], params, None,
+                          out=(y, cc, ss), workspace=ws)
+        e1.record(stream)
+        axon_ssm.step(tok["x"], tok["z"], tok["dt_raw"], tok["B"], tok["C"], params, (cc, ss), y=y_tok)
+        e2.record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier(dev)
+    ms_local = t_start.elapsed_time(t_end)
+    ms = reduce_max(ms_local, dev)
+    scan_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    step_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+
+    units_step = B * (L + 1) * E
+    value = rank_units(units_step, world) * args.steps / (ms / 1e3) / 1e9
+
+    # ---- end to end through the public API with host buffers (pinned)
+    host = {k: v.cpu().pin_memory() for k, v in sets[0].items()}
+    host_tok = {k: v.cpu().pin_memory() for k, v in tok.items()}
+    dev_in = {k: torch.empty_like(v) for k, v in sets[0].items()}
+    dev_tok = {k: torch.empty_like(v) for k, v in tok.items()}
+    y_host = torch.empty(y.shape, dtype=io).pin_memory()
+    ytok_host = torch.empty(y_tok.shape, dtype=io).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values()) + \
+        sum(v.numel() * v.element_size() for v in host_tok.values())
+    d2h = y_host.numel() * y_host.element_size() + ytok_host.numel() * ytok_host.element_size()
+
+    def e2e_step():
+        for k in host:
+            dev_in[k].copy_(host[k], non_blocking=True)
+        for k in host_tok:
+            dev_tok[k].copy_(host_tok[k], non_blocking=True)
+        axon_ssm.scan_fwd(dev_in["x"], dev_in["z"], dev_in["dt_raw"], dev_in["B"], dev_in["C"],
+                          params, None, out=(y, cc, ss), workspace=ws)
+        axon_ssm.step(dev_tok["x"], dev_tok["z"], dev_tok["dt_raw"], dev_tok["B"], dev_tok["C"],
+                      params, (cc, ss), y=y_tok)
+        y_host.copy_(y, non_blocking=True)
+        ytok_host.copy_(y_tok, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = reduce_max(a.elapsed_time(b), dev)
+    e2e_value = rank_units(units_step, world) * e2e_steps / (e2e_ms / 1e3) / 1e9
+
+    # ---- roofline of the dominant kernel (the prefill scan)
+    peaks = measured_peaks()
+    sm = scan_model(wl)
+    props = torch.cuda.get_device_properties(dev)
+    sms = props.multi_processor_count
+    mufu_peak = sms * MUFU_LANES_PER_SM_CLK * peaks["sm_max_mhz"] * 1e6 / 1e9   # Gop/s
+    mufu_ach = sm["mufu"] / (scan_ms / 1e3) / 1e9
+    hbm_ach = sm["bytes"] / (scan_ms / 1e3) / 1e9
+    traffic = ncu_traffic("scan", wl.name, sm["token_ch"])
+    stm = step_model(wl)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": workload_desc(wl), "io_dtype": wl.io,
+                   "l2": f"{n_sets} rotating input sets of {set_bytes / 1e6:.0f} MB "
+                         f"({n_sets * set_bytes / 1e6:.0f} MB > 126 MB L2)",
+                   "parallelism": f"dp{world} (independent sequences per GPU, no collective)"},
+        "roofline": {"bound": "alu", "achieved": mufu_ach, "peak": mufu_peak, "unit": "Gop/s",
+                     "frac": mufu_ach / mufu_peak, "traffic": traffic,
+                     "kernel": "prefill scan (MUFU transcendentals: 22 per token x channel)",
+                     "peak_source": f"{sms} SMs x {MUFU_LANES_PER_SM_CLK} MUFU/clk x "
+                                    f"{peaks['sm_max_mhz']:.0f} MHz",
+                     "kernel_ms": scan_ms, "algorithmic_bytes": sm["bytes"],
+                     "hbm": {"achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": hbm_ach / peaks["hbm_gbs"],
+                             "peak_source": peaks["source"]}},
+        "decode_step": {"us": step_ms * 1e3, "algorithmic_bytes": stm["bytes"],
+                        "hbm_gbs": stm["bytes"] / (step_ms / 1e3) / 1e9},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "clocks": clk,
+        "gpu_launches": args.steps * (scan_launches + 1),
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp_cpu = {**params_cpu, **{k: v.cpu() for k, v in sets[0].items()}}
+        rate, units, secs, ch = time_oracle(wl, inp_cpu, args.cpu_budget)
+        line["cpu_baseline"] = {"value": rate / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": f"{ch} of {E} channels x {L} tokens (prefill), "
+                                          f"{secs:.1f} s, fp64 C oracle, single thread"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    barrier(dev)
+    if torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["axon", "reference"], default="axon")
+    ap.add_argument("--workload", default="bit_axon_layer", choices=[w.name for w in W.WORKLOADS])
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
+    wl = W.WORKLOAD_BY_NAME[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_axon(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,205 @@
+/*
+ * axon_ssm.h -- C ABI of the B200 (sm_100a) selective-scan (S6) layer core.
+ *
+ * The operation is the Axon-SSM layer core of the page "Axon-SSM: Selective
+ * State Space Model for Apple Silicon" (bit-axon docs), between its input and
+ * output projections (which are not part of this library):
+ *
+ *   xc_t  = conv_b + sum_{k<K} conv_w[k] * xpad[t+k]     causal depthwise conv1d,
+ *           xpad = conv_cache ++ x, tap K-1 meets x_t    (section "Implementation
+ *                                                         in Bit-Axon", code map
+ *                                                         `_causal_conv1d`)
+ *   u_t   = SiLU(xc_t)
+ *   dt_t  = clip(softplus(dt_raw_t + dt_bias), 1e-4, 100) (section "Selective
+ *                                                         mechanism")
+ *   A     = -exp(A_log), diagonal                         (section "Diagonal state
+ *                                                         matrix")
+ *   h_t   = exp(dt_t*A) (.) h_{t-1} + dt_t*B_t*u_t        (section "ZOH
+ *                                                         discretisation": the
+ *                                                         first-order form used by
+ *                                                         Axon-SSM, and the
+ *                                                         recurrence equation)
+ *   y_t   = (C_t . h_t + D*u_t) * SiLU(z_t)               (recurrence output and
+ *                                                         section "Gating")
+ *
+ * and the cached decode of section "Autoregressive decoding": the cache pair
+ * [conv_cache (B,K-1,E), ssm_state (B,E,N)] carries the conv padding and the
+ * hidden state from one call to the next.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Sizes: B batch rows, L tokens, E channels (d_inner), N states, K conv taps.
+ *    This build supports N == 16 and K == 4 only (the layer configuration table
+ *    of the Axon-SSM page); other values return AXON_ERR_UNSUPPORTED.
+ *  - Layouts are dense row-major, last index fastest:
+ *      x, z, dt_raw, y        (B, L, E)   io dtype
+ *      Bm, Cm                 (B, L, N)   io dtype, shared by all channels
+ *      conv_w                 (E, K)      float32
+ *      conv_b, dt_bias, D     (E)         float32
+ *      A_log                  (E, N)      float32
+ *      conv_cache             (B, K-1, E) io dtype; index 0 is the oldest input
+ *      ssm_state              (B, E, N)   float32
+ *    For axon_ssm_step the L axis is absent: x, z, dt_raw, y are (B, E) and
+ *    Bm, Cm are (B, N).
+ *  - io dtype: AXON_F32 (float) or AXON_BF16 (bfloat16 bits, round-to-nearest-
+ *    even on output).  Arithmetic is float32 throughout; the state is float32.
+ *  - Pointers are DEVICE pointers owned by the caller.  The library never
+ *    allocates, frees or retains them; scratch memory comes from the caller
+ *    through `workspace`.  Every pointer must be 16-byte aligned, and E must be
+ *    a multiple of 8 (bf16) or 4 (f32), else AXON_ERR_ALIGNMENT.  There is no
+ *    fallback path.
+ *  - Work is enqueued on `stream` and runs asynchronously.  Arguments are
+ *    checked on the host before anything is enqueued: an error return means
+ *    nothing was launched and no output was touched.  AXON_ERR_CUDA reports a
+ *    failed launch; faults that occur later surface at the caller's next
+ *    synchronisation, as for any CUDA kernel.
+ *  - The library holds no mutable global state; concurrent calls on different
+ *    streams with disjoint outputs are safe.
+ *  - `axon_stream_t` is the CUDA runtime's cudaStream_t (a CUstream_st
+ *    pointer); NULL means the legacy default stream.
+ */
+#ifndef AXON_SSM_H
+#define AXON_SSM_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define AXON_API __attribute__((visibility("default")))
+#else
+#define AXON_API
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *axon_stream_t;
+
+typedef enum {
+    AXON_F32 = 0,
+    AXON_BF16 = 1
+} axon_dtype;
+
+typedef enum {
+    AXON_OK = 0,
+    AXON_ERR_INVALID_ARG = 1,   /* negative size, NULL required pointer, bad aliasing */
+    AXON_ERR_UNSUPPORTED = 2,   /* N != 16, K != 4, unknown dtype, size beyond limits */
+    AXON_ERR_ALIGNMENT = 3,     /* pointer not 16-byte aligned, E not a multiple of 8/4 */
+    AXON_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+    AXON_ERR_CUDA = 5,          /* a kernel launch (or device query) failed */
+    AXON_ERR_TIMEOUT = 6        /* reserved: no entry point waits on the device */
+} axon_status;
+
+/* Version of this ABI (bumped on any incompatible change). */
+AXON_API int axon_ssm_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+AXON_API const char *axon_status_string(axon_status status);
+
+/*
+ * Bytes of device scratch memory `axon_ssm_scan_fwd` may need for a problem of
+ * this size: an upper bound over every launch plan the library can choose for
+ * it, independent of the device.  Returns 0 when no plan needs scratch, and 0
+ * for arguments axon_ssm_scan_fwd would reject.
+ *
+ * The scratch holds, per sequence segment after the first and per (b, e)
+ * channel, the segment's local end state (N floats) and its summed dt (one
+ * float): the chunk-carry summaries of a time-split scan (the chunked
+ * associative scan of the SSD article, intra-block pass plus inter-block
+ * carry).
+ */
+AXON_API size_t axon_ssm_scan_workspace_bytes(int B, int L, int E, int N, int K, axon_dtype io);
+
+/*
+ * Number of kernel launches axon_ssm_scan_fwd enqueues for a problem of this
+ * size on the current device (its launch plan), or -1 for arguments it would
+ * reject or when the device cannot be queried.  Lets a caller count the work
+ * it put on a stream; it launches nothing.
+ */
+AXON_API int axon_ssm_scan_launch_count(int B, int L, int E, int N, int K, axon_dtype io);
+
+/*
+ * Prefill: run the layer core over L tokens of B sequences.
+ *
+ *   x, z, dt_raw        (B,L,E) io   inputs (post-projection x branch, gate branch,
+ *                                    raw step size); required when L > 0
+ *   Bm, Cm              (B,L,N) io   input-dependent B_t and C_t; required when L > 0
+ *   conv_w, conv_b, dt_bias, A_log, D  float32 parameters; required
+ *   conv_cache_in       (B,K-1,E) io or NULL (NULL: zero padding)
+ *   ssm_state_in        (B,E,N) f32  or NULL (NULL: zero initial state)
+ *   y                   (B,L,E) io   output; required when L > 0; must not
+ *                                    overlap any input
+ *   conv_cache_out      (B,K-1,E) io the last K-1 entries of conv_cache_in ++ x
+ *                                    (raw inputs, bit-exact copies); required;
+ *                                    either the same pointer as conv_cache_in
+ *                                    (updated in place) or disjoint from it
+ *   ssm_state_out       (B,E,N) f32  h after the last token; required; same
+ *                                    pointer as ssm_state_in or disjoint
+ *   workspace, workspace_bytes       caller-owned device scratch of at least
+ *                                    axon_ssm_scan_workspace_bytes(...) bytes;
+ *                                    may be NULL when that query returns 0
+ *   stream                           stream to enqueue on
+ *
+ * L == 0 copies the initial caches (or zeros) to the outputs.  B == 0 or
+ * E == 0 is a no-op.  Passing the returned caches to the next call continues
+ * the sequence exactly (the streaming `model.step(chunk, state)` pattern of
+ * the wiki page "Selective State Space Models (Mamba)").
+ */
+AXON_API axon_status axon_ssm_scan_fwd(
+    int B, int L, int E, int N, int K, axon_dtype io,
+    const void *x, const void *z, const void *dt_raw,
+    const void *Bm, const void *Cm,
+    const float *conv_w, const float *conv_b,
+    const float *dt_bias, const float *A_log, const float *D,
+    const void *conv_cache_in, const float *ssm_state_in,
+    void *y, void *conv_cache_out, float *ssm_state_out,
+    void *workspace, size_t workspace_bytes, axon_stream_t stream);
+
+/*
+ * The prefill with an explicit time split: `num_segments` > 0 forces the
+ * sequence to be cut into that many segments processed in parallel, with the
+ * chunk carry passed through `workspace` (which must then hold at least
+ * (num_segments-1) * B * E * (N+1) floats; num_segments <= 64 and never more
+ * than L).  num_segments == 0 lets the library choose, exactly as
+ * axon_ssm_scan_fwd does.  Same arguments and errors as axon_ssm_scan_fwd
+ * otherwise.  Intended for tests and tuning; results agree with the unsplit
+ * scan to float32 rounding.
+ */
+AXON_API axon_status axon_ssm_scan_fwd_segments(
+    int B, int L, int E, int N, int K, axon_dtype io,
+    const void *x, const void *z, const void *dt_raw,
+    const void *Bm, const void *Cm,
+    const float *conv_w, const float *conv_b,
+    const float *dt_bias, const float *A_log, const float *D,
+    const void *conv_cache_in, const float *ssm_state_in,
+    void *y, void *conv_cache_out, float *ssm_state_out,
+    void *workspace, size_t workspace_bytes, int num_segments, axon_stream_t stream);
+
+/*
+ * Cached single-token decode (section "Autoregressive decoding"): one step of
+ * the layer core for B sequences, caches updated in place.
+ *
+ *   x, z, dt_raw        (B,E) io     this token's inputs
+ *   Bm, Cm              (B,N) io     this token's B_t, C_t
+ *   conv_w ... D                     float32 parameters, as for the prefill
+ *   conv_cache          (B,K-1,E) io read, then shifted by one with x appended
+ *   ssm_state           (B,E,N) f32  read-modify-written
+ *   y                   (B,E) io     output; must not overlap the other buffers
+ *
+ * Equivalent to axon_ssm_scan_fwd with L == 1 and in-place caches; its cost
+ * does not depend on how many tokens came before (O(1) state per token).
+ */
+AXON_API axon_status axon_ssm_step(
+    int B, int E, int N, int K, axon_dtype io,
+    const void *x, const void *z, const void *dt_raw,
+    const void *Bm, const void *Cm,
+    const float *conv_w, const float *conv_b,
+    const float *dt_bias, const float *A_log, const float *D,
+    void *conv_cache, float *ssm_state, void *y, axon_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AXON_SSM_H */

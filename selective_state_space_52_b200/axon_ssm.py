@@ -1,0 +1,203 @@
+"""Python binding of the C ABI in include/axon_ssm.h (ctypes, argument marshalling only).
+
+Every step of the layer core runs in the CUDA library ``libaxon_ssm.so`` built
+in-tree by ``selective_state_space_52_b200.build``.  There is no CPU or PyTorch
+fallback: importing this module raises if the library is missing, and every
+call raises ``AxonError`` on a non-OK status.  PyTorch provides device memory
+and the current stream.
+
+Functions named like the C entry points take torch tensors (device, contiguous)
+and pass their pointers through; ``scan_fwd`` and ``step`` additionally allocate
+outputs / workspace with torch for convenience.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libaxon_ssm.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"CUDA library not built: {LIB_PATH} is missing. "
+        "Run `python -m selective_state_space_52_b200.build` (nvcc, sm_100a).")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+AXON_F32 = 0
+AXON_BF16 = 1
+STATUS = {0: "AXON_OK", 1: "AXON_ERR_INVALID_ARG", 2: "AXON_ERR_UNSUPPORTED",
+          3: "AXON_ERR_ALIGNMENT", 4: "AXON_ERR_WORKSPACE", 5: "AXON_ERR_CUDA",
+          6: "AXON_ERR_TIMEOUT"}
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+_lib.axon_ssm_abi_version.restype = _i
+_lib.axon_ssm_abi_version.argtypes = []
+_lib.axon_status_string.restype = ctypes.c_char_p
+_lib.axon_status_string.argtypes = [_i]
+_lib.axon_ssm_scan_workspace_bytes.restype = _sz
+_lib.axon_ssm_scan_workspace_bytes.argtypes = [_i] * 6
+_lib.axon_ssm_scan_launch_count.restype = _i
+_lib.axon_ssm_scan_launch_count.argtypes = [_i] * 6
+_SCAN_ARGS = [_i] * 6 + [_vp] * 15 + [_vp, _sz]
+_lib.axon_ssm_scan_fwd.restype = _i
+_lib.axon_ssm_scan_fwd.argtypes = _SCAN_ARGS + [_vp]
+_lib.axon_ssm_scan_fwd_segments.restype = _i
+_lib.axon_ssm_scan_fwd_segments.argtypes = _SCAN_ARGS + [_i, _vp]
+_lib.axon_ssm_step.restype = _i
+_lib.axon_ssm_step.argtypes = [_i] * 5 + [_vp] * 13 + [_vp]
+
+
+class AxonError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return AXON_F32
+    if t == torch.bfloat16:
+        return AXON_BF16
+    raise TypeError(f"unsupported io dtype {t}; use float32 or bfloat16")
+
+
+def _p(t):
+    """Device pointer of a tensor (None -> NULL).  Tensors must be contiguous."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the C ABI must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise AxonError(rc, where)
+
+
+# ------------------------------------------------------------ C entry points
+def axon_ssm_abi_version() -> int:
+    return _lib.axon_ssm_abi_version()
+
+
+def axon_status_string(status: int) -> str:
+    return _lib.axon_status_string(int(status)).decode()
+
+
+def axon_ssm_scan_workspace_bytes(B, L, E, N=16, K=4, io=AXON_BF16) -> int:
+    return int(_lib.axon_ssm_scan_workspace_bytes(B, L, E, N, K, io))
+
+
+def axon_ssm_scan_launch_count(B, L, E, N=16, K=4, io=AXON_BF16) -> int:
+    return int(_lib.axon_ssm_scan_launch_count(B, L, E, N, K, io))
+
+
+def axon_ssm_scan_fwd(B, L, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias,
+                      A_log, D, conv_cache_in, ssm_state_in, y, conv_cache_out,
+                      ssm_state_out, workspace, workspace_bytes, stream=None, *,
+                      raise_on_error=True) -> int:
+    rc = _lib.axon_ssm_scan_fwd(B, L, E, N, K, io, _p(x), _p(z), _p(dt_raw), _p(Bm), _p(Cm),
+                                _p(conv_w), _p(conv_b), _p(dt_bias), _p(A_log), _p(D),
+                                _p(conv_cache_in), _p(ssm_state_in), _p(y),
+                                _p(conv_cache_out), _p(ssm_state_out), _p(workspace),
+                                int(workspace_bytes), _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_ssm_scan_fwd")
+    return rc
+
+
+def axon_ssm_scan_fwd_segments(B, L, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b,
+                               dt_bias, A_log, D, conv_cache_in, ssm_state_in, y,
+                               conv_cache_out, ssm_state_out, workspace, workspace_bytes,
+                               num_segments, stream=None, *, raise_on_error=True) -> int:
+    rc = _lib.axon_ssm_scan_fwd_segments(B, L, E, N, K, io, _p(x), _p(z), _p(dt_raw), _p(Bm),
+                                         _p(Cm), _p(conv_w), _p(conv_b), _p(dt_bias),
+                                         _p(A_log), _p(D), _p(conv_cache_in),
+                                         _p(ssm_state_in), _p(y), _p(conv_cache_out),
+                                         _p(ssm_state_out), _p(workspace),
+                                         int(workspace_bytes), int(num_segments),
+                                         _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_ssm_scan_fwd_segments")
+    return rc
+
+
+def axon_ssm_step(B, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
+                  conv_cache, ssm_state, y, stream=None, *, raise_on_error=True) -> int:
+    rc = _lib.axon_ssm_step(B, E, N, K, io, _p(x), _p(z), _p(dt_raw), _p(Bm), _p(Cm),
+                            _p(conv_w), _p(conv_b), _p(dt_bias), _p(A_log), _p(D),
+                            _p(conv_cache), _p(ssm_state), _p(y), _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_ssm_step")
+    return rc
+
+
+# ------------------------------------------------------------ conveniences
+PARAM_KEYS = ("conv_w", "conv_b", "dt_bias", "A_log", "D")
+
+
+def scan_fwd(x, z, dt_raw, Bm, Cm, params: dict, cache=None, *, num_segments=None,
+             out=None, workspace=None, stream=None):
+    """Prefill over (B, L, E) inputs on the GPU.
+
+    ``params`` holds conv_w, conv_b, dt_bias, A_log, D (float32, on the device);
+    ``cache`` is None or (conv_cache, ssm_state).  Returns
+    ``(y, (conv_cache, ssm_state))`` -- the cache pair of the Axon-SSM page's
+    "Autoregressive decoding" section, ready for the next call or for ``step``.
+    """
+    Bsz, L, E = x.shape
+    K = params["conv_w"].shape[1]
+    N = params["A_log"].shape[1]
+    io = _dtype_code(x.dtype)
+    dev = x.device
+    cc_in, ss_in = (None, None) if cache is None else cache
+    if out is None:
+        y = torch.empty_like(x)
+        cc_out = torch.empty(Bsz, K - 1, E, dtype=x.dtype, device=dev)
+        ss_out = torch.empty(Bsz, E, N, dtype=torch.float32, device=dev)
+    else:
+        y, cc_out, ss_out = out
+    if num_segments is None:
+        nbytes = axon_ssm_scan_workspace_bytes(Bsz, L, E, N, K, io)
+    else:
+        nbytes = max(num_segments - 1, 0) * Bsz * E * (N + 1) * 4
+    if workspace is None and nbytes > 0:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    args = (Bsz, L, E, N, K, io, x, z, dt_raw, Bm, Cm, *(params[k] for k in PARAM_KEYS),
+            cc_in, ss_in, y, cc_out, ss_out, workspace, wsz)
+    if num_segments is None:
+        axon_ssm_scan_fwd(*args, stream=stream)
+    else:
+        axon_ssm_scan_fwd_segments(*args, num_segments, stream=stream)
+    return y, (cc_out, ss_out)
+
+
+def step(x, z, dt_raw, Bm, Cm, params: dict, cache, *, y=None, stream=None):
+    """One cached decode step; ``cache = (conv_cache, ssm_state)`` is updated in place."""
+    Bsz, E = x.shape
+    K = params["conv_w"].shape[1]
+    N = params["A_log"].shape[1]
+    conv_cache, ssm_state = cache
+    if y is None:
+        y = torch.empty_like(x)
+    axon_ssm_step(Bsz, E, N, K, _dtype_code(x.dtype), x, z, dt_raw, Bm, Cm,
+                  *(params[k] for k in PARAM_KEYS), conv_cache, ssm_state, y, stream=stream)
+    return y

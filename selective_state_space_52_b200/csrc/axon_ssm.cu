@@ -1,0 +1,279 @@
+// axon_ssm.cu -- host side of the C ABI declared in include/axon_ssm.h:
+// argument checks (nothing is launched on any error), the launch plan, and the
+// kernel launches on the caller's stream.  The library allocates nothing.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "axon_ssm.h"
+#include "device_math.cuh"
+#include "scan_seq.cuh"
+#include "step.cuh"
+
+namespace axon {
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr int kMaxSegments = 64;      // time segments of a split scan
+constexpr int kMinSegLen = 128;       // shortest segment the planner picks
+constexpr int kScanThreads = 128;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+size_t io_bytes(axon_dtype io) { return io == AXON_BF16 ? 2 : 4; }
+
+// Common size/dtype checks shared by prefill and decode.
+axon_status check_shape(int B, int L, int E, int N, int K, axon_dtype io) {
+    if (B < 0 || L < 0 || E < 0) return AXON_ERR_INVALID_ARG;
+    if (N != kN || K != kK) return AXON_ERR_UNSUPPORTED;
+    if (io != AXON_F32 && io != AXON_BF16) return AXON_ERR_UNSUPPORTED;
+    // element counts must stay well inside 64-bit offsets and grid limits
+    if ((long long)B * (long long)E > (1LL << 31)) return AXON_ERR_UNSUPPORTED;
+    if (B > 65535) return AXON_ERR_UNSUPPORTED;
+    if ((E % (io == AXON_BF16 ? 8 : 4)) != 0) return AXON_ERR_ALIGNMENT;
+    return AXON_OK;
+}
+
+// Longest split the planner may use for a sequence of L tokens.
+int max_segments_for(int L) {
+    int p = L / kMinSegLen;
+    if (p > kMaxSegments) p = kMaxSegments;
+    return p < 1 ? 1 : p;
+}
+
+size_t ws_bytes_for(int B, int E, int P) {
+    if (P <= 1) return 0;
+    return (size_t)(P - 1) * (size_t)B * (size_t)E * (kN + 1) * sizeof(float);
+}
+
+int device_sm_count() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    return sms;
+}
+
+// Channel-parallel scan: one thread per (b, e).  Split the sequence only when
+// the channels alone cannot give every SM a few warps.
+int plan_segments(int B, int L, int E, int sms) {
+    const long long channels = (long long)B * E;
+    const long long want = (long long)sms * 1024;   // resident threads to aim for
+    if (channels >= want / 2) return 1;
+    long long p = (want + channels - 1) / channels;
+    const int pmax = max_segments_for(L);
+    if (p > pmax) p = pmax;
+    return (int)(p < 1 ? 1 : p);
+}
+
+template <class Io>
+axon_status launch_scan(ScanParams& prm, cudaStream_t st) {
+    const dim3 block(kScanThreads);
+    const unsigned gx = (unsigned)((prm.E + kScanThreads - 1) / kScanThreads);
+    if (prm.L == 0) {
+        copy_state_kernel<Io><<<dim3(gx, prm.B), block, 0, st>>>(prm);
+    } else {
+        const unsigned gz = (unsigned)(prm.num_seg > 1 ? prm.num_seg - 1 : 1);
+        scan_seq_phase1<Io><<<dim3(gx, prm.B, gz), block, 0, st>>>(prm);
+        if (prm.num_seg > 1)
+            scan_seq_phase2<Io><<<dim3(gx, prm.B, prm.num_seg - 1), block, 0, st>>>(prm);
+    }
+    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+}
+
+axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
+                      const void* x, const void* z, const void* dt_raw,
+                      const void* Bm, const void* Cm,
+                      const float* conv_w, const float* conv_b,
+                      const float* dt_bias, const float* A_log, const float* D,
+                      const void* conv_cache_in, const float* ssm_state_in,
+                      void* y, void* conv_cache_out, float* ssm_state_out,
+                      void* workspace, size_t workspace_bytes, int num_segments,
+                      cudaStream_t stream) {
+    axon_status st = check_shape(B, L, E, N, K, io);
+    if (st != AXON_OK) return st;
+    if (num_segments < 0) return AXON_ERR_INVALID_ARG;
+    if (B == 0 || E == 0) return AXON_OK;
+    if (!conv_w || !conv_b || !dt_bias || !A_log || !D || !conv_cache_out || !ssm_state_out)
+        return AXON_ERR_INVALID_ARG;
+    if (L > 0 && (!x || !z || !dt_raw || !Bm || !Cm || !y)) return AXON_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
+                          conv_cache_in, ssm_state_in, y, conv_cache_out, ssm_state_out};
+    for (const void* q : ptrs)
+        if (q && !aligned16(q)) return AXON_ERR_ALIGNMENT;
+
+    const size_t sio = io_bytes(io);
+    const size_t n_seq = (size_t)B * L * E * sio;
+    const size_t n_bc = (size_t)B * L * kN * sio;
+    const size_t n_cc = (size_t)B * (kK - 1) * E * sio;
+    const size_t n_ss = (size_t)B * E * kN * sizeof(float);
+    // outputs: caches either exactly in place or disjoint; y disjoint from all
+    if (conv_cache_in != conv_cache_out && overlaps(conv_cache_in, n_cc, conv_cache_out, n_cc))
+        return AXON_ERR_INVALID_ARG;
+    if ((const void*)ssm_state_in != (const void*)ssm_state_out &&
+        overlaps(ssm_state_in, n_ss, ssm_state_out, n_ss))
+        return AXON_ERR_INVALID_ARG;
+    if (L > 0) {
+        const void* ins[] = {x, z, dt_raw};
+        for (const void* q : ins) if (overlaps(q, n_seq, y, n_seq)) return AXON_ERR_INVALID_ARG;
+        if (overlaps(Bm, n_bc, y, n_seq) || overlaps(Cm, n_bc, y, n_seq)) return AXON_ERR_INVALID_ARG;
+        if (overlaps(conv_cache_in, n_cc, y, n_seq) || overlaps(conv_cache_out, n_cc, y, n_seq) ||
+            overlaps(ssm_state_in, n_ss, y, n_seq) || overlaps(ssm_state_out, n_ss, y, n_seq))
+            return AXON_ERR_INVALID_ARG;
+    }
+    if (overlaps(conv_cache_out, n_cc, ssm_state_out, n_ss)) return AXON_ERR_INVALID_ARG;
+
+    int P = 1;
+    int seg = L > 0 ? L : 1;
+    if (L > 0) {
+        if (num_segments > 0) {
+            if (num_segments > kMaxSegments) return AXON_ERR_INVALID_ARG;
+            P = num_segments;
+        } else {
+            const int sms = device_sm_count();
+            if (sms <= 0) return AXON_ERR_CUDA;
+            P = plan_segments(B, L, E, sms);
+        }
+        if (P > 1) {
+            seg = (L + P - 1) / P;
+            if (seg < kK) return AXON_ERR_INVALID_ARG;   // each segment must cover the conv window
+            P = (L + seg - 1) / seg;                       // drop empty trailing segments
+        }
+    }
+    const size_t need = ws_bytes_for(B, E, P);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return AXON_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return AXON_ERR_ALIGNMENT;
+        if (overlaps(workspace, need, y, n_seq) || overlaps(workspace, need, ssm_state_out, n_ss) ||
+            overlaps(workspace, need, conv_cache_out, n_cc))
+            return AXON_ERR_INVALID_ARG;
+    }
+
+    ScanParams prm;
+    prm.B = B; prm.L = L; prm.E = E;
+    prm.x = x; prm.z = z; prm.dt_raw = dt_raw; prm.Bm = Bm; prm.Cm = Cm;
+    prm.conv_w = conv_w; prm.conv_b = conv_b; prm.dt_bias = dt_bias; prm.A_log = A_log; prm.D = D;
+    prm.conv_cache_in = conv_cache_in; prm.ssm_state_in = ssm_state_in;
+    prm.y = y; prm.conv_cache_out = conv_cache_out; prm.ssm_state_out = ssm_state_out;
+    prm.num_seg = P;
+    prm.seg_len = seg;   // segments [s*seg, min(L, (s+1)*seg)), s < P, all non-empty
+    prm.ws_h = P > 1 ? static_cast<float*>(workspace) : nullptr;
+    prm.ws_sdt = P > 1 ? static_cast<float*>(workspace) + (size_t)(P - 1) * B * E * kN : nullptr;
+
+    return io == AXON_BF16 ? launch_scan<IoBF16>(prm, stream) : launch_scan<IoF32>(prm, stream);
+}
+
+}  // namespace
+}  // namespace axon
+
+using namespace axon;
+
+extern "C" {
+
+int axon_ssm_abi_version(void) { return kAbiVersion; }
+
+const char* axon_status_string(axon_status s) {
+    switch (s) {
+        case AXON_OK: return "AXON_OK";
+        case AXON_ERR_INVALID_ARG: return "AXON_ERR_INVALID_ARG";
+        case AXON_ERR_UNSUPPORTED: return "AXON_ERR_UNSUPPORTED";
+        case AXON_ERR_ALIGNMENT: return "AXON_ERR_ALIGNMENT";
+        case AXON_ERR_WORKSPACE: return "AXON_ERR_WORKSPACE";
+        case AXON_ERR_CUDA: return "AXON_ERR_CUDA";
+        case AXON_ERR_TIMEOUT: return "AXON_ERR_TIMEOUT";
+    }
+    return "AXON_ERR_UNKNOWN";
+}
+
+size_t axon_ssm_scan_workspace_bytes(int B, int L, int E, int N, int K, axon_dtype io) {
+    if (check_shape(B, L, E, N, K, io) != AXON_OK) return 0;
+    return ws_bytes_for(B, E, max_segments_for(L));
+}
+
+int axon_ssm_scan_launch_count(int B, int L, int E, int N, int K, axon_dtype io) {
+    if (check_shape(B, L, E, N, K, io) != AXON_OK) return -1;
+    if (B == 0 || E == 0) return 0;
+    if (L == 0) return 1;
+    const int sms = device_sm_count();
+    if (sms <= 0) return -1;
+    return plan_segments(B, L, E, sms) > 1 ? 2 : 1;
+}
+
+axon_status axon_ssm_scan_fwd(int B, int L, int E, int N, int K, axon_dtype io,
+                              const void* x, const void* z, const void* dt_raw,
+                              const void* Bm, const void* Cm,
+                              const float* conv_w, const float* conv_b,
+                              const float* dt_bias, const float* A_log, const float* D,
+                              const void* conv_cache_in, const float* ssm_state_in,
+                              void* y, void* conv_cache_out, float* ssm_state_out,
+                              void* workspace, size_t workspace_bytes, axon_stream_t stream) {
+    return scan_impl(B, L, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
+                     conv_cache_in, ssm_state_in, y, conv_cache_out, ssm_state_out,
+                     workspace, workspace_bytes, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+axon_status axon_ssm_scan_fwd_segments(int B, int L, int E, int N, int K, axon_dtype io,
+                                       const void* x, const void* z, const void* dt_raw,
+                                       const void* Bm, const void* Cm,
+                                       const float* conv_w, const float* conv_b,
+                                       const float* dt_bias, const float* A_log, const float* D,
+                                       const void* conv_cache_in, const float* ssm_state_in,
+                                       void* y, void* conv_cache_out, float* ssm_state_out,
+                                       void* workspace, size_t workspace_bytes, int num_segments,
+                                       axon_stream_t stream) {
+    return scan_impl(B, L, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
+                     conv_cache_in, ssm_state_in, y, conv_cache_out, ssm_state_out,
+                     workspace, workspace_bytes, num_segments,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+axon_status axon_ssm_step(int B, int E, int N, int K, axon_dtype io,
+                          const void* x, const void* z, const void* dt_raw,
+                          const void* Bm, const void* Cm,
+                          const float* conv_w, const float* conv_b,
+                          const float* dt_bias, const float* A_log, const float* D,
+                          void* conv_cache, float* ssm_state, void* y, axon_stream_t stream) {
+    axon_status st = check_shape(B, 1, E, N, K, io);
+    if (st != AXON_OK) return st;
+    if (B == 0 || E == 0) return AXON_OK;
+    if (!x || !z || !dt_raw || !Bm || !Cm || !conv_w || !conv_b || !dt_bias || !A_log || !D ||
+        !conv_cache || !ssm_state || !y)
+        return AXON_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
+                          conv_cache, ssm_state, y};
+    for (const void* q : ptrs)
+        if (!aligned16(q)) return AXON_ERR_ALIGNMENT;
+    const size_t sio = io_bytes(io);
+    const size_t n_y = (size_t)B * E * sio;
+    const size_t n_cc = (size_t)B * (kK - 1) * E * sio;
+    const size_t n_ss = (size_t)B * E * kN * sizeof(float);
+    const size_t n_bc = (size_t)B * kN * sio;
+    if (overlaps(y, n_y, conv_cache, n_cc) || overlaps(y, n_y, ssm_state, n_ss) ||
+        overlaps(conv_cache, n_cc, ssm_state, n_ss))
+        return AXON_ERR_INVALID_ARG;
+    const void* ins[] = {x, z, dt_raw};
+    for (const void* q : ins)
+        if (overlaps(q, n_y, y, n_y) || overlaps(q, n_y, conv_cache, n_cc) || overlaps(q, n_y, ssm_state, n_ss))
+            return AXON_ERR_INVALID_ARG;
+    if (overlaps(Bm, n_bc, y, n_y) || overlaps(Cm, n_bc, y, n_y)) return AXON_ERR_INVALID_ARG;
+
+    StepParams prm;
+    prm.B = B; prm.E = E;
+    prm.x = x; prm.z = z; prm.dt_raw = dt_raw; prm.Bm = Bm; prm.Cm = Cm;
+    prm.conv_w = conv_w; prm.conv_b = conv_b; prm.dt_bias = dt_bias; prm.A_log = A_log; prm.D = D;
+    prm.conv_cache = conv_cache; prm.ssm_state = ssm_state; prm.y = y;
+    const long long threads = (long long)B * E * 4;
+    const unsigned grid = (unsigned)((threads + 255) / 256);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (io == AXON_BF16) step_kernel<IoBF16><<<grid, 256, 0, s>>>(prm);
+    else step_kernel<IoF32><<<grid, 256, 0, s>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,114 @@
+// device_math.cuh -- float32 building blocks of the selective-scan layer core
+// for sm_100a: the MUFU exp2/log2/reciprocal instructions, SiLU, the clipped
+// softplus step size, and io-dtype loads/stores.
+//
+// Math follows the page "Axon-SSM: Selective State Space Model for Apple
+// Silicon": SiLU gating (section "Gating"), dt = clip(softplus(dt_raw + b_dt),
+// 1e-4, 100) (section "Selective mechanism"), abar = exp(dt*A) with
+// A = -exp(A_log) (sections "ZOH discretisation", "Diagonal state matrix").
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace axon {
+
+constexpr float kLog2e = 1.4426950408889634f;   // log2(e)
+constexpr float kLn2 = 0.6931471805599453f;     // ln(2)
+constexpr float kDtMin = 1e-4f;                 // epsilon of the dt clip
+constexpr float kDtMax = 100.0f;                // dt_max of the dt clip
+constexpr int kN = 16;                          // state size N
+constexpr int kK = 4;                           // conv taps K
+
+// Hardware (MUFU) approximations, issued directly as PTX instructions.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2_approx(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// SiLU(v) = v * sigmoid(v) = v / (1 + 2^(-v log2 e)).  For v -> -inf the
+// exponential overflows to +inf and the reciprocal to 0, giving -0.
+__device__ __forceinline__ float silu(float v) {
+    return v * rcp_approx(1.0f + ex2_approx(-v * kLog2e));
+}
+
+// log(1 + e) for e in [0, 1].  Below 2^-6 the first four terms of the Taylor
+// series e - e^2/2 + e^3/3 - e^4/4 are used (truncation below e^5/5, i.e. under
+// 2^-26 relative); above it, log2(1 + e) * ln 2, where rounding 1 + e costs at
+// most 2^-24 / log(1 + 2^-6) ~ 4e-6 relative.
+__device__ __forceinline__ float log1p_unit(float e) {
+    const float series = e * (1.0f - e * (0.5f - e * (0.33333334f - e * 0.25f)));
+    const float viaLog = lg2_approx(1.0f + e) * kLn2;
+    return e < 0.015625f ? series : viaLog;
+}
+
+// softplus(v) = max(v, 0) + log(1 + exp(-|v|)), overflow-free.
+__device__ __forceinline__ float softplus(float v) {
+    const float e = ex2_approx(-fabsf(v) * kLog2e);
+    return fmaxf(v, 0.0f) + log1p_unit(e);
+}
+
+// dt = clip(softplus(v), 1e-4, 100), bounds inclusive.
+__device__ __forceinline__ float dt_from_raw(float v) {
+    return fminf(fmaxf(softplus(v), kDtMin), kDtMax);
+}
+
+// ---------------------------------------------------------------- io dtypes
+struct IoF32 {
+    using T = float;
+    static constexpr int kBytes = 4;
+    __device__ __forceinline__ static float load(const T* p) { return __ldg(p); }
+    __device__ __forceinline__ static float load_rw(const T* p) { return *p; }
+    __device__ __forceinline__ static void store(T* p, float v) { *p = v; }
+    // 16 consecutive values of a B/C row (64 bytes, 16-byte aligned).
+    __device__ __forceinline__ static void load_row16(const T* p, float (&r)[kN]) {
+        const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float4 v = __ldg(q + i);
+            r[4 * i + 0] = v.x; r[4 * i + 1] = v.y; r[4 * i + 2] = v.z; r[4 * i + 3] = v.w;
+        }
+    }
+};
+
+struct IoBF16 {
+    using T = __nv_bfloat16;
+    static constexpr int kBytes = 2;
+    __device__ __forceinline__ static float bits_to_f(uint32_t b16) {
+        return __uint_as_float(b16 << 16);
+    }
+    __device__ __forceinline__ static float load(const T* p) {
+        return bits_to_f(__ldg(reinterpret_cast<const unsigned short*>(p)));
+    }
+    __device__ __forceinline__ static float load_rw(const T* p) {
+        return bits_to_f(*reinterpret_cast<const unsigned short*>(p));
+    }
+    __device__ __forceinline__ static void store(T* p, float v) { *p = __float2bfloat16_rn(v); }
+    // 16 consecutive bf16 values of a B/C row (32 bytes, 16-byte aligned).
+    __device__ __forceinline__ static void load_row16(const T* p, float (&r)[kN]) {
+        const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            uint4 v = __ldg(q + i);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                r[8 * i + 2 * j + 0] = __uint_as_float(w[j] << 16);
+                r[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+            }
+        }
+    }
+};
+
+}  // namespace axon

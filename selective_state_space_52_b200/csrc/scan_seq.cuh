@@ -1,0 +1,244 @@
+// scan_seq.cuh -- channel-parallel selective scan: one thread owns one (b, e)
+// channel and keeps its N = 16 states in registers while it walks a run of
+// tokens in order.  The conv1d + SiLU + dt prologue and the D-skip, C-contraction
+// and SiLU(z) epilogue are fused into the same loop.
+//
+// Used (a) for the whole sequence when there are enough channels to fill the
+// GPU (many sequences, e.g. decode prefill), and (b) as the two phases of a
+// time-split scan when there are not: the sequence is cut into P segments,
+// phase 1 walks segment 0 from the true initial state (writing y) and every
+// middle segment from a zero state (writing only its end state and summed dt
+// to the workspace), and phase 2 folds the summaries of the segments before it
+// into its carry-in (h_in(s) = exp(A * sum dt) (.) h_in(s-1) + h_loc) and walks
+// its segment again, writing y.  This is the intra-block pass + inter-block
+// carry structure of the chunked associative scan described in the SSD article;
+// it costs a second walk of the middle segments.
+//
+// Recurrence (Axon-SSM page, recurrence equation, first-order discretisation):
+//   h_n <- exp(dt * A_n) h_n + dt * u * B_n,   y = (sum_n C_n h_n + D u) * SiLU(z)
+#pragma once
+
+#include "device_math.cuh"
+
+namespace axon {
+
+struct ScanParams {
+    int B, L, E;
+    const void* x;
+    const void* z;
+    const void* dt_raw;
+    const void* Bm;
+    const void* Cm;
+    const float* conv_w;
+    const float* conv_b;
+    const float* dt_bias;
+    const float* A_log;
+    const float* D;
+    const void* conv_cache_in;    // may be null
+    const float* ssm_state_in;    // may be null
+    void* y;
+    void* conv_cache_out;
+    float* ssm_state_out;
+    float* ws_h;                  // (P-1, B, E, N): segment end states
+    float* ws_sdt;                // (P-1, B, E): summed dt of segments 1..P-2
+    int seg_len;                  // tokens per segment
+    int num_seg;                  // P
+};
+
+// Value of the padded input stream xpad at absolute time t (t < 0 reads the
+// incoming conv cache, whose row K-1+t holds time t; null cache means zeros).
+template <class Io>
+__device__ __forceinline__ float xpad_at(const ScanParams& p, int b, int e, int t) {
+    using T = typename Io::T;
+    if (t >= 0) return Io::load(static_cast<const T*>(p.x) + ((size_t)b * p.L + t) * p.E + e);
+    if (p.conv_cache_in == nullptr) return 0.0f;
+    return Io::load_rw(static_cast<const T*>(p.conv_cache_in) + ((size_t)b * (kK - 1) + (kK - 1 + t)) * p.E + e);
+}
+
+// Walk tokens [t0, t1) of channel (b, e) starting from state h.
+//   kWriteY: produce y (else only the state and the dt sum are tracked).
+template <class Io, bool kWriteY>
+__device__ __forceinline__ void walk(const ScanParams& p, int b, int e, int t0, int t1,
+                                     const float (&A2)[kN], float (&h)[kN], float& sdt,
+                                     float (&win)[kK - 1]) {
+    using T = typename Io::T;
+    const float w0 = __ldg(p.conv_w + (size_t)e * kK + 0);
+    const float w1 = __ldg(p.conv_w + (size_t)e * kK + 1);
+    const float w2 = __ldg(p.conv_w + (size_t)e * kK + 2);
+    const float w3 = __ldg(p.conv_w + (size_t)e * kK + 3);
+    const float cb = __ldg(p.conv_b + e);
+    const float db = __ldg(p.dt_bias + e);
+    const float Dv = __ldg(p.D + e);
+    const T* xs = static_cast<const T*>(p.x) + (size_t)b * p.L * p.E + e;
+    const T* zs = static_cast<const T*>(p.z) + (size_t)b * p.L * p.E + e;
+    const T* ds = static_cast<const T*>(p.dt_raw) + (size_t)b * p.L * p.E + e;
+    const T* Bs = static_cast<const T*>(p.Bm) + (size_t)b * p.L * kN;
+    const T* Cs = static_cast<const T*>(p.Cm) + (size_t)b * p.L * kN;
+    T* ys = static_cast<T*>(p.y) + (size_t)b * p.L * p.E + e;
+
+#pragma unroll 2
+    for (int t = t0; t < t1; ++t) {
+        const size_t o = (size_t)t * p.E;
+        const float xt = Io::load(xs + o);
+        const float dr = Io::load(ds + o);
+        float Bv[kN];
+        Io::load_row16(Bs + (size_t)t * kN, Bv);
+        // causal depthwise conv (cross-correlation: tap 3 meets x_t) + SiLU
+        float xc = fmaf(w0, win[0], cb);
+        xc = fmaf(w1, win[1], xc);
+        xc = fmaf(w2, win[2], xc);
+        xc = fmaf(w3, xt, xc);
+        win[0] = win[1]; win[1] = win[2]; win[2] = xt;
+        const float u = silu(xc);
+        const float dt = dt_from_raw(dr + db);
+        const float dtu = dt * u;
+        sdt += dt;
+        if constexpr (kWriteY) {
+            const float zt = Io::load(zs + o);
+            float Cv[kN];
+            Io::load_row16(Cs + (size_t)t * kN, Cv);
+            float acc[4] = {Dv * u, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int n = 0; n < kN; ++n) {
+                const float a = ex2_approx(dt * A2[n]);
+                h[n] = fmaf(a, h[n], dtu * Bv[n]);
+                acc[n & 3] = fmaf(Cv[n], h[n], acc[n & 3]);
+            }
+            const float yv = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * silu(zt);
+            Io::store(ys + o, yv);
+        } else {
+#pragma unroll
+            for (int n = 0; n < kN; ++n) {
+                const float a = ex2_approx(dt * A2[n]);
+                h[n] = fmaf(a, h[n], dtu * Bv[n]);
+            }
+        }
+    }
+}
+
+template <class Io>
+__device__ __forceinline__ void load_A2(const ScanParams& p, int e, float (&A2)[kN]) {
+    // A = -exp(A_log), pre-scaled by log2(e) so that exp(dt*A) = 2^(dt*A2).
+#pragma unroll
+    for (int n = 0; n < kN; ++n) A2[n] = -expf(__ldg(p.A_log + (size_t)e * kN + n)) * kLog2e;
+}
+
+template <class Io>
+__device__ __forceinline__ void write_final(const ScanParams& p, int b, int e,
+                                            const float (&h)[kN], const float (&win)[kK - 1]) {
+    using T = typename Io::T;
+    float4* so = reinterpret_cast<float4*>(p.ssm_state_out + ((size_t)b * p.E + e) * kN);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) so[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+    T* co = static_cast<T*>(p.conv_cache_out) + (size_t)b * (kK - 1) * p.E + e;
+#pragma unroll
+    for (int j = 0; j < kK - 1; ++j) Io::store(co + (size_t)j * p.E, win[j]);  // exact: values came from io
+}
+
+// Phase 1 (or the whole scan when num_seg == 1).  grid = (ceil(E/128), B, max(P-1, 1)).
+template <class Io>
+__global__ void __launch_bounds__(128) scan_seq_phase1(ScanParams p) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    const int b = blockIdx.y;
+    const int s = blockIdx.z;
+    if (e >= p.E) return;
+    const int t0 = s * p.seg_len;
+    const int t1 = min(p.L, t0 + p.seg_len);
+    float A2[kN];
+    load_A2<Io>(p, e, A2);
+    float win[kK - 1];
+#pragma unroll
+    for (int j = 0; j < kK - 1; ++j) win[j] = xpad_at<Io>(p, b, e, t0 - (kK - 1) + j);
+    float h[kN];
+    float sdt = 0.0f;
+    if (s == 0) {
+        if (p.ssm_state_in) {
+            const float4* si = reinterpret_cast<const float4*>(p.ssm_state_in + ((size_t)b * p.E + e) * kN);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float4 v = si[i];
+                h[4 * i] = v.x; h[4 * i + 1] = v.y; h[4 * i + 2] = v.z; h[4 * i + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int n = 0; n < kN; ++n) h[n] = 0.0f;
+        }
+        walk<Io, true>(p, b, e, t0, t1, A2, h, sdt, win);
+        if (p.num_seg == 1) {
+            write_final<Io>(p, b, e, h, win);
+        } else {
+            float4* wo = reinterpret_cast<float4*>(p.ws_h + ((size_t)b * p.E + e) * kN);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) wo[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+        }
+    } else {
+#pragma unroll
+        for (int n = 0; n < kN; ++n) h[n] = 0.0f;
+        walk<Io, false>(p, b, e, t0, t1, A2, h, sdt, win);
+        const size_t slot = ((size_t)s * p.B + b) * p.E + e;
+        float4* wo = reinterpret_cast<float4*>(p.ws_h + slot * kN);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) wo[i] = make_float4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+        p.ws_sdt[slot] = sdt;
+    }
+}
+
+// Phase 2: segments 1..P-1 fold the carry and walk again.  grid = (ceil(E/128), B, P-1).
+template <class Io>
+__global__ void __launch_bounds__(128) scan_seq_phase2(ScanParams p) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    const int b = blockIdx.y;
+    const int s = blockIdx.z + 1;
+    if (e >= p.E) return;
+    const int t0 = s * p.seg_len;
+    const int t1 = min(p.L, t0 + p.seg_len);
+    float A2[kN];
+    load_A2<Io>(p, e, A2);
+    float h[kN];
+    {
+        const float4* w0 = reinterpret_cast<const float4*>(p.ws_h + ((size_t)b * p.E + e) * kN);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float4 v = w0[i];
+            h[4 * i] = v.x; h[4 * i + 1] = v.y; h[4 * i + 2] = v.z; h[4 * i + 3] = v.w;
+        }
+    }
+    for (int r = 1; r < s; ++r) {
+        const size_t slot = ((size_t)r * p.B + b) * p.E + e;
+        const float sd = p.ws_sdt[slot];
+        const float4* wr = reinterpret_cast<const float4*>(p.ws_h + slot * kN);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float4 v = wr[i];
+            const float hl[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int n = 4 * i + j;
+                h[n] = fmaf(ex2_approx(sd * A2[n]), h[n], hl[j]);
+            }
+        }
+    }
+    float win[kK - 1];
+#pragma unroll
+    for (int j = 0; j < kK - 1; ++j) win[j] = xpad_at<Io>(p, b, e, t0 - (kK - 1) + j);
+    float sdt = 0.0f;
+    walk<Io, true>(p, b, e, t0, t1, A2, h, sdt, win);
+    if (s == p.num_seg - 1) write_final<Io>(p, b, e, h, win);
+}
+
+// L == 0: the outputs are the incoming caches (or zeros).  grid = (ceil(E/128), B).
+template <class Io>
+__global__ void __launch_bounds__(128) copy_state_kernel(ScanParams p) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    const int b = blockIdx.y;
+    if (e >= p.E) return;
+    float h[kN];
+#pragma unroll
+    for (int n = 0; n < kN; ++n) h[n] = p.ssm_state_in ? p.ssm_state_in[((size_t)b * p.E + e) * kN + n] : 0.0f;
+    float win[kK - 1];
+#pragma unroll
+    for (int j = 0; j < kK - 1; ++j) win[j] = xpad_at<Io>(p, b, e, j - (kK - 1));
+    write_final<Io>(p, b, e, h, win);
+}
+
+}  // namespace axon

@@ -1,0 +1,182 @@
+"""Host-only checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments with the documented status before
+launching anything.
+
+Every call below fails argument validation, so no kernel is ever launched
+with the fake (never dereferenced) pointers used here; these tests are safe
+with or without a GPU.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from selective_state_space_52_b200 import build
+    build.build()
+    return ctypes.CDLL(build.LIB)
+
+
+def declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if fn.endswith(".h"):
+            src = open(os.path.join(HEADER_DIR, fn)).read()
+            names += re.findall(r"AXON_API\s+[\w\s\*]+?\b(axon_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for required in ("axon_ssm_scan_fwd", "axon_ssm_step", "axon_ssm_scan_workspace_bytes",
+                     "axon_status_string", "axon_ssm_abi_version", "axon_ssm_scan_fwd_segments"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from selective_state_space_52_b200 import build
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s+(\w+)", out))
+    for name in declared_symbols():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_status_strings_and_version(lib):
+    lib.axon_status_string.restype = ctypes.c_char_p
+    assert lib.axon_status_string(0) == b"AXON_OK"
+    assert lib.axon_status_string(4) == b"AXON_ERR_WORKSPACE"
+    assert lib.axon_status_string(99) == b"AXON_ERR_UNKNOWN"
+    assert lib.axon_ssm_abi_version() == 1
+
+
+def test_workspace_query(lib):
+    q = lib.axon_ssm_scan_workspace_bytes
+    q.restype = ctypes.c_size_t
+    # (P_max - 1) * B * E * (N + 1) * 4 with P_max = min(64, L // 128)
+    assert q(1, 2048, 7680, 16, 4, 1) == 15 * 7680 * 17 * 4
+    assert q(1, 65536, 2048, 16, 4, 1) == 63 * 2048 * 17 * 4
+    assert q(64, 128, 7680, 16, 4, 1) == 0          # short sequences never split
+    assert q(1, 64, 32, 16, 4, 0) == 0
+    assert q(1, 4096, 64, 8, 4, 0) == 0             # unsupported N -> 0
+    assert q(1, 4096, 60, 16, 4, 1) == 0            # E % 8 != 0 for bf16 -> rejected -> 0
+
+
+# A fake, 16-byte aligned, never-dereferenced device address.
+FAKE = 1 << 40
+
+
+def _scan(lib, **over):
+    a = dict(B=1, L=64, E=32, N=16, K=4, io=0,
+             x=FAKE, z=FAKE + 0x10000, dt_raw=FAKE + 0x20000, Bm=FAKE + 0x30000, Cm=FAKE + 0x40000,
+             conv_w=FAKE + 0x50000, conv_b=FAKE + 0x60000, dt_bias=FAKE + 0x70000,
+             A_log=FAKE + 0x80000, D=FAKE + 0x90000, cc_in=None, ss_in=None,
+             y=FAKE + 0xA0000, cc_out=FAKE + 0xB0000, ss_out=FAKE + 0xC0000,
+             ws=None, ws_bytes=0, segs=0)
+    a.update(over)
+    f = lib.axon_ssm_scan_fwd_segments
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 15 + [ctypes.c_void_p, ctypes.c_size_t,
+                                                               ctypes.c_int, ctypes.c_void_p]
+    return f(a["B"], a["L"], a["E"], a["N"], a["K"], a["io"], a["x"], a["z"], a["dt_raw"],
+             a["Bm"], a["Cm"], a["conv_w"], a["conv_b"], a["dt_bias"], a["A_log"], a["D"],
+             a["cc_in"], a["ss_in"], a["y"], a["cc_out"], a["ss_out"], a["ws"], a["ws_bytes"],
+             a["segs"], None)
+
+
+OK, INVALID, UNSUPPORTED, ALIGNMENT, WORKSPACE = 0, 1, 2, 3, 4
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(B=-1), INVALID),
+    (dict(L=-5), INVALID),
+    (dict(E=-8), INVALID),
+    (dict(N=8), UNSUPPORTED),
+    (dict(N=32), UNSUPPORTED),
+    (dict(K=3), UNSUPPORTED),
+    (dict(io=7), UNSUPPORTED),
+    (dict(B=70000), UNSUPPORTED),
+    (dict(E=30), ALIGNMENT),                      # fp32 needs E % 4 == 0
+    (dict(E=36, io=1), ALIGNMENT),                # bf16 needs E % 8 == 0
+    (dict(x=None), INVALID),
+    (dict(Bm=None), INVALID),
+    (dict(y=None), INVALID),
+    (dict(conv_w=None), INVALID),
+    (dict(D=None), INVALID),
+    (dict(cc_out=None), INVALID),
+    (dict(ss_out=None), INVALID),
+    (dict(x=FAKE + 4), ALIGNMENT),
+    (dict(y=FAKE + 0xA0008), ALIGNMENT),
+    (dict(cc_in=FAKE + 0xD0002), ALIGNMENT),
+    (dict(y=FAKE), INVALID),                      # y overlaps x
+    (dict(y=FAKE + 0x40000), INVALID),            # y overlaps Cm
+    (dict(cc_in=FAKE + 0xB0010), INVALID),        # partial overlap of the cache in/out
+    (dict(ss_in=FAKE + 0xC0040), INVALID),        # partial overlap of the state in/out
+    (dict(ss_out=FAKE + 0xB0000 + 64), INVALID),  # state overlaps conv cache
+    (dict(segs=-1), INVALID),
+    (dict(segs=65, L=100000), INVALID),           # more than 64 segments
+    (dict(segs=32, L=64), INVALID),               # segments shorter than the conv window
+    (dict(segs=2, L=256), WORKSPACE),             # split needs workspace, none given
+    (dict(segs=2, L=256, ws=FAKE + 0x100000, ws_bytes=100), WORKSPACE),
+    (dict(segs=2, L=256, ws=FAKE + 0x100004, ws_bytes=1 << 20), ALIGNMENT),
+])
+def test_scan_rejects_bad_arguments(lib, over, status):
+    assert _scan(lib, **over) == status
+
+
+def test_scan_noop_sizes_launch_nothing(lib):
+    # B == 0 or E == 0: nothing to do, OK without touching the device
+    assert _scan(lib, B=0) == OK
+    assert _scan(lib, E=0) == OK
+
+
+def _step(lib, **over):
+    a = dict(B=2, E=16, N=16, K=4, io=1,
+             x=FAKE, z=FAKE + 0x10000, dt_raw=FAKE + 0x20000, Bm=FAKE + 0x30000, Cm=FAKE + 0x40000,
+             conv_w=FAKE + 0x50000, conv_b=FAKE + 0x60000, dt_bias=FAKE + 0x70000,
+             A_log=FAKE + 0x80000, D=FAKE + 0x90000, cc=FAKE + 0xA0000, ss=FAKE + 0xB0000,
+             y=FAKE + 0xC0000)
+    a.update(over)
+    f = lib.axon_ssm_step
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 14
+    return f(a["B"], a["E"], a["N"], a["K"], a["io"], a["x"], a["z"], a["dt_raw"], a["Bm"],
+             a["Cm"], a["conv_w"], a["conv_b"], a["dt_bias"], a["A_log"], a["D"], a["cc"],
+             a["ss"], a["y"], None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(B=-2), INVALID),
+    (dict(N=4), UNSUPPORTED),
+    (dict(K=2), UNSUPPORTED),
+    (dict(E=12), ALIGNMENT),
+    (dict(x=None), INVALID),
+    (dict(cc=None), INVALID),
+    (dict(ss=None), INVALID),
+    (dict(y=None), INVALID),
+    (dict(ss=FAKE + 0xB0004), ALIGNMENT),
+    (dict(y=FAKE + 0xA0000), INVALID),             # y overlaps the conv cache
+    (dict(ss=FAKE + 0xA0000 + 32), INVALID),       # state overlaps the conv cache
+    (dict(x=FAKE + 0xC0000), INVALID),             # x overlaps y
+])
+def test_step_rejects_bad_arguments(lib, over, status):
+    assert _step(lib, **over) == status
+
+
+def test_step_noop_sizes(lib):
+    assert _step(lib, B=0) == OK
+    assert _step(lib, E=0) == OK
+
+
+def test_binding_module_exposes_c_names():
+    from selective_state_space_52_b200 import axon_ssm
+    for name in declared_symbols():
+        assert callable(getattr(axon_ssm, name)), name

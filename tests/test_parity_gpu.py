@@ -1,0 +1,183 @@
+"""GPU parity: the CUDA prefill and decode step (through the C ABI) against the
+fp64 oracle, element by element, on seeded inputs.
+
+Small cases span several CUDA blocks and ragged tails; full-size workloads are
+checked on sampled channels (channels are independent, so the oracle can
+compute any one of them alone).  Tolerances are in tests/gpu_util.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from selective_state_space_52_b200 import workloads as W
+
+from gpu_util import (Guarded, check_close, compare_scan, oracle_scan, run_gpu_scan, state_tol,
+                      to_dev, tol_for)
+
+pytestmark = pytest.mark.gpu
+
+SWEEP_L = [1, 2, 3, 4, 5, 63, 64, 65, 127, 257, 1000]
+SWEEP_BE = [(1, 8), (3, 40), (2, 264)]
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("B,E", SWEEP_BE)
+@pytest.mark.parametrize("L", SWEEP_L)
+def test_sweep_small_shapes(cuda_lib, io, B, E, L):
+    wl = W.custom(B, L, E, io=io, seed=1000 + 7 * L + E + B)
+    with_state = (L + E) % 2 == 0
+    inp = W.make_inputs(wl, with_state=True)
+    compare_scan(inp, io, with_state=with_state, what=f"B{B} L{L} E{E} {io}")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("L,P", [(64, 2), (257, 3), (1000, 7), (2048, 16), (300, 60), (4096, 64)])
+def test_forced_time_split(cuda_lib, io, L, P):
+    """The segment-carry path (phase 1 summaries + carry fold + second walk)."""
+    if (L + P - 1) // P < 4:
+        pytest.skip("segment shorter than the conv window")
+    wl = W.custom(2, L, 24 if io == "f32" else 48, io=io, seed=77 + L + P)
+    inp = W.make_inputs(wl, with_state=True)
+    compare_scan(inp, io, num_segments=P, what=f"split P={P} L={L} {io}")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_split_equals_unsplit_closely(cuda_lib, io):
+    wl = W.custom(1, 1024, 64, io=io, seed=5)
+    inp = W.make_inputs(wl, with_state=True)
+    y1, cc1, ss1 = run_gpu_scan(inp, num_segments=1)
+    y8, cc8, ss8 = run_gpu_scan(inp, num_segments=8)
+    assert torch.equal(cc1, cc8)
+    check_close(y8, y1, tol_for(io, y1), "split vs unsplit")
+    check_close(ss8, ss1, state_tol(ss1), "split vs unsplit state")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("shift", [-200.0, 200.0, -9.21, 0.0, 4.0, 20.0, 21.0])
+def test_dt_clip_edges(cuda_lib, io, shift):
+    wl = W.custom(1, 96, 32, io=io, seed=int(abs(shift) * 10) + 3)
+    inp = W.make_inputs(wl, with_state=True)
+    inp["dt_raw"] = (inp["dt_raw"].float() * 0.01 + shift).to(inp["dt_raw"].dtype)
+    compare_scan(inp, io, what=f"dt shift {shift}")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_bimodal_dt_long_and_fast_memory(cuda_lib, io):
+    wl = W.Workload("bimodal_small", 2, 777, 40, io, 9, dt_mode="bimodal")
+    inp = W.make_inputs(wl, with_state=True)
+    compare_scan(inp, io, what="bimodal")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_empty_sequence_copies_caches(cuda_lib, io):
+    wl = W.custom(2, 0, 16, io=io, seed=3)
+    inp = W.make_inputs(wl, with_state=True)
+    y, cc, ss = run_gpu_scan(inp)
+    assert y.shape == (2, 0, 16)
+    assert torch.equal(cc, inp["conv_cache"])
+    np.testing.assert_array_equal(ss, inp["ssm_state"].numpy())
+    y, cc, ss = run_gpu_scan(inp, with_state=False)
+    assert torch.all(cc.float() == 0) and np.all(ss == 0)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("P", [1, 4])
+def test_in_place_caches(cuda_lib, io, P):
+    """conv_cache_out / ssm_state_out may be the input buffers themselves."""
+    from selective_state_space_52_b200 import axon_ssm
+    wl = W.custom(2, 512, 40, io=io, seed=41 + P)
+    inp = W.make_inputs(wl, with_state=True)
+    d = to_dev(inp)
+    params = {k: d[k] for k in axon_ssm.PARAM_KEYS}
+    cc, ss = d["conv_cache"].clone(), d["ssm_state"].clone()
+    y = torch.empty_like(d["x"])
+    axon_ssm.scan_fwd(d["x"], d["z"], d["dt_raw"], d["B"], d["C"], params, (cc, ss),
+                      num_segments=P, out=(y, cc, ss))
+    torch.cuda.synchronize()
+    y_ref, cc_ref, ss_ref = oracle_scan(inp)
+    check_close(y.float().cpu().numpy(), y_ref, tol_for(io, y_ref), "in-place y")
+    check_close(ss.cpu().numpy(), ss_ref, state_tol(ss_ref), "in-place state")
+    assert torch.equal(cc.cpu(), torch.from_numpy(cc_ref).to(cc.dtype))
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_chunked_prefill_continues_exactly(cuda_lib, io):
+    """scan(L1) then scan(L - L1) with the returned caches == one scan over L
+    (the streaming pattern of the wiki page "Selective State Space Models")."""
+    from selective_state_space_52_b200 import axon_ssm
+    wl = W.custom(2, 700, 32, io=io, seed=61)
+    inp = W.make_inputs(wl, with_state=True)
+    d = to_dev(inp)
+    params = {k: d[k] for k in axon_ssm.PARAM_KEYS}
+    cache = (d["conv_cache"], d["ssm_state"])
+    ys = []
+    for lo, hi in [(0, 1), (1, 3), (3, 300), (300, 700)]:
+        sl = {k: d[k][:, lo:hi].contiguous() for k in ("x", "z", "dt_raw", "B", "C")}
+        y, cache = axon_ssm.scan_fwd(sl["x"], sl["z"], sl["dt_raw"], sl["B"], sl["C"], params, cache)
+        ys.append(y)
+    torch.cuda.synchronize()
+    y = torch.cat(ys, dim=1).float().cpu().numpy()
+    y_ref, cc_ref, ss_ref = oracle_scan(inp)
+    check_close(y, y_ref, tol_for(io, y_ref), "chunked y")
+    check_close(cache[1].cpu().numpy(), ss_ref, state_tol(ss_ref), "chunked state")
+    assert torch.equal(cache[0].cpu(), torch.from_numpy(cc_ref).to(cache[0].dtype))
+
+
+def _run_steps(d, params, cache, steps_inp, guarded_y=True):
+    from selective_state_space_52_b200 import axon_ssm
+    ys = []
+    S = steps_inp["x"].shape[0]
+    for s in range(S):
+        xs = {k: steps_inp[k][s] for k in ("x", "z", "dt_raw", "B", "C")}
+        if guarded_y:
+            g = Guarded(tuple(xs["x"].shape), xs["x"].dtype)
+            y = axon_ssm.step(xs["x"], xs["z"], xs["dt_raw"], xs["B"], xs["C"], params, cache, y=g.t)
+            torch.cuda.synchronize()
+            assert g.canaries_intact()
+        else:
+            y = axon_ssm.step(xs["x"], xs["z"], xs["dt_raw"], xs["B"], xs["C"], params, cache)
+        ys.append(y.float().cpu().numpy())
+    return np.stack(ys)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("B,E", [(1, 8), (3, 40), (5, 264)])
+def test_decode_steps_equal_full_prefill(cuda_lib, io, B, E):
+    """prefill(L0) + (L - L0) cached steps on the GPU == oracle prefill over L."""
+    from selective_state_space_52_b200 import axon_ssm
+    L0, L = 13, 29
+    wl = W.custom(B, L, E, io=io, seed=500 + E)
+    inp = W.make_inputs(wl, with_state=True)
+    d = to_dev(inp)
+    params = {k: d[k] for k in axon_ssm.PARAM_KEYS}
+    y0, cache = axon_ssm.scan_fwd(*(d[k][:, :L0].contiguous() for k in ("x", "z", "dt_raw", "B", "C")),
+                                  params, (d["conv_cache"], d["ssm_state"]))
+    steps = {k: d[k][:, L0:].transpose(0, 1).contiguous() for k in ("x", "z", "dt_raw", "B", "C")}
+    ys = _run_steps(d, params, cache, steps)
+    y_gpu = np.concatenate([y0.float().cpu().numpy(), ys.transpose(1, 0, 2)], axis=1)
+    y_ref, cc_ref, ss_ref = oracle_scan(inp)
+    check_close(y_gpu, y_ref, tol_for(io, y_ref), "decode y")
+    check_close(cache[1].cpu().numpy(), ss_ref, state_tol(ss_ref), "decode state")
+    assert torch.equal(cache[0].cpu(), torch.from_numpy(cc_ref).to(cache[0].dtype))
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_step_matches_oracle_step(cuda_lib, io):
+    from selective_state_space_52_b200 import axon_ssm
+    wl = W.custom(7, 1, 136, io=io, seed=88)
+    inp = W.make_inputs(wl, with_state=True)
+    d = to_dev(inp)
+    params = {k: d[k] for k in axon_ssm.PARAM_KEYS}
+    cc, ss = d["conv_cache"].clone(), d["ssm_state"].clone()
+    y = axon_ssm.step(d["x"][:, 0].contiguous(), d["z"][:, 0].contiguous(),
+                      d["dt_raw"][:, 0].contiguous(), d["B"][:, 0].contiguous(),
+                      d["C"][:, 0].contiguous(), params, (cc, ss))
+    torch.cuda.synchronize()
+    y_ref, cc_ref, ss_ref = oracle.step(inp["x"][:, 0], inp["z"][:, 0], inp["dt_raw"][:, 0],
+                                        inp["B"][:, 0], inp["C"][:, 0], inp["conv_w"],
+                                        inp["conv_b"], inp["dt_bias"], inp["A_log"], inp["D"],
+                                        inp["conv_cache"], inp["ssm_state"])
+    check_close(y.float().cpu().numpy(), y_ref, tol_for(io, y_ref), "step y")
+    check_close(ss.cpu().numpy(), ss_ref, state_tol(ss_ref), "step state")
+    assert torch.equal(cc.cpu(), torch.from_numpy(cc_ref).to(cc.dtype))
