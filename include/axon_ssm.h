@@ -53,8 +53,9 @@
  *    nothing was launched and no output was touched.  AXON_ERR_CUDA reports a
  *    failed launch; faults that occur later surface at the caller's next
  *    synchronisation, as for any CUDA kernel.
- *  - The library holds no mutable global state; concurrent calls on different
- *    streams with disjoint outputs are safe.
+ *  - Apart from axon_ssm_scan_fwd_noalloc (below), the library holds no
+ *    mutable global state; concurrent calls on different streams with
+ *    disjoint outputs are safe.
  *  - `axon_stream_t` is the CUDA runtime's cudaStream_t (a CUstream_st
  *    pointer); NULL means the legacy default stream.
  */
@@ -175,6 +176,49 @@ AXON_API axon_status axon_ssm_scan_fwd_segments(
     const void *conv_cache_in, const float *ssm_state_in,
     void *y, void *conv_cache_out, float *ssm_state_out,
     void *workspace, size_t workspace_bytes, int num_segments, axon_stream_t stream);
+
+/*
+ * The prefill (axon_ssm_scan_fwd_segments semantics) for callers that cannot
+ * provide scratch memory.  The pages have no counterpart; this is a
+ * convenience of the library.
+ *
+ * Who needs it: a serving process whose memory pool reserved nearly all of
+ * HBM up front has no room for a cudaMalloc of its own, and a host program
+ * that must not call cudaMalloc/cudaFree inside its token loop (those calls
+ * can synchronise the device) has no workspace to hand over.  Both still own
+ * and pass every input and output buffer; only the time-split scratch moves
+ * into the library.
+ *
+ *  - The scratch is one library-owned 16 MiB device array
+ *    (AXON_NOALLOC_SCRATCH_BYTES).  Every GPU that loads the library holds it
+ *    until the process exits.  The entry point itself calls no cudaMalloc,
+ *    cudaFree or other allocating routine.
+ *  - Limit: a call is rejected with AXON_ERR_UNSUPPORTED, before anything is
+ *    launched, when its worst-case scratch exceeds that size, i.e. when
+ *    (P - 1) * B * E * (N + 1) * 4 bytes > 16 MiB, with P = num_segments if it
+ *    is > 0, else min(64, max(1, L / 128)) (the largest split the library plans
+ *    for L tokens; axon_ssm_scan_workspace_bytes gives the same bound).
+ *  - num_segments as for axon_ssm_scan_fwd_segments (0 = library's plan).
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any
+ *    stream capture on that device.
+ *  - All calls share the one array and it keeps the last call's contents;
+ *    every scratch word a call reads was written earlier in the same call, so
+ *    nothing needs clearing.  Calls whose executions overlap on the GPU (on
+ *    different streams, or from different threads) race on the array: order
+ *    them, e.g. keep them on one stream.
+ * Other arguments, layouts and errors are those of axon_ssm_scan_fwd.
+ */
+#define AXON_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+AXON_API axon_status axon_ssm_scan_fwd_noalloc(
+    int B, int L, int E, int N, int K, axon_dtype io,
+    const void *x, const void *z, const void *dt_raw,
+    const void *Bm, const void *Cm,
+    const float *conv_w, const float *conv_b,
+    const float *dt_bias, const float *A_log, const float *D,
+    const void *conv_cache_in, const float *ssm_state_in,
+    void *y, void *conv_cache_out, float *ssm_state_out,
+    int num_segments, axon_stream_t stream);
 
 /*
  * Cached single-token decode (section "Autoregressive decoding"): one step of

@@ -50,6 +50,9 @@ _lib.axon_ssm_scan_fwd.restype = _i
 _lib.axon_ssm_scan_fwd.argtypes = _SCAN_ARGS + [_vp]
 _lib.axon_ssm_scan_fwd_segments.restype = _i
 _lib.axon_ssm_scan_fwd_segments.argtypes = _SCAN_ARGS + [_i, _vp]
+_lib.axon_ssm_scan_fwd_noalloc.restype = _i
+_lib.axon_ssm_scan_fwd_noalloc.argtypes = [_i] * 6 + [_vp] * 15 + [_i, _vp]
+NOALLOC_SCRATCH_BYTES = 16 << 20
 _lib.axon_ssm_step.restype = _i
 _lib.axon_ssm_step.argtypes = [_i] * 5 + [_vp] * 13 + [_vp]
 
@@ -136,6 +139,22 @@ def axon_ssm_scan_fwd_segments(B, L, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, 
                                          _stream(stream))
     if raise_on_error:
         _check(rc, "axon_ssm_scan_fwd_segments")
+    return rc
+
+
+def axon_ssm_scan_fwd_noalloc(B, L, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b,
+                              dt_bias, A_log, D, conv_cache_in, ssm_state_in, y,
+                              conv_cache_out, ssm_state_out, num_segments=0, stream=None, *,
+                              raise_on_error=True) -> int:
+    """The prefill with its time-split scratch in the library's own 16 MiB device
+    array, for callers that cannot provide a workspace (see include/axon_ssm.h)."""
+    rc = _lib.axon_ssm_scan_fwd_noalloc(B, L, E, N, K, io, _p(x), _p(z), _p(dt_raw), _p(Bm),
+                                        _p(Cm), _p(conv_w), _p(conv_b), _p(dt_bias),
+                                        _p(A_log), _p(D), _p(conv_cache_in),
+                                        _p(ssm_state_in), _p(y), _p(conv_cache_out),
+                                        _p(ssm_state_out), int(num_segments), _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_ssm_scan_fwd_noalloc")
     return rc
 
 

@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "axon_ssm.h"
 #include "device_math.cuh"
@@ -169,6 +170,35 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
     return io == AXON_BF16 ? launch_scan<IoBF16>(prm, stream) : launch_scan<IoF32>(prm, stream);
 }
 
+// ---- scratch for axon_ssm_scan_fwd_noalloc --------------------------------
+// Library-owned device scratch for callers that cannot pass a workspace.  It
+// is a file-scope __device__ array, so every GPU that loads this library holds
+// it until the process exits.  In host code `g_static_scratch` is only a
+// host-side stand-in for the symbol: its device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;   // 16 MiB
+constexpr int kMaxScratchDevices = 64;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxScratchDevices] = {};
+
+// Device address of g_static_scratch on the current device (set up on first use).
+axon_status static_scratch_address(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return AXON_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxScratchDevices) return AXON_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
+            return AXON_ERR_CUDA;
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return AXON_OK;
+}
+
 }  // namespace
 }  // namespace axon
 
@@ -274,6 +304,36 @@ axon_status axon_ssm_step(int B, int E, int N, int K, axon_dtype io,
     if (io == AXON_BF16) step_kernel<IoBF16><<<grid, 256, 0, s>>>(prm);
     else step_kernel<IoF32><<<grid, 256, 0, s>>>(prm);
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+}
+
+axon_status axon_ssm_scan_fwd_noalloc(int B, int L, int E, int N, int K, axon_dtype io,
+                                      const void* x, const void* z, const void* dt_raw,
+                                      const void* Bm, const void* Cm,
+                                      const float* conv_w, const float* conv_b,
+                                      const float* dt_bias, const float* A_log, const float* D,
+                                      const void* conv_cache_in, const float* ssm_state_in,
+                                      void* y, void* conv_cache_out, float* ssm_state_out,
+                                      int num_segments, axon_stream_t stream) {
+    // Size checks first, on the host: nothing touches the device on rejection.
+    const axon_status shape = check_shape(B, L, E, N, K, io);
+    if (shape != AXON_OK) return shape;
+    if (num_segments < 0 || num_segments > kMaxSegments) return AXON_ERR_INVALID_ARG;
+    // Worst-case scratch of any plan for this call: the caller's forced split,
+    // or the library's largest split for a sequence of L tokens.
+    const int worst = num_segments > 0 ? num_segments : max_segments_for(L);
+    if (ws_bytes_for(B, E, worst) > kStaticScratchBytes) return AXON_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    if (B > 0 && E > 0 && L > 0) {
+        const axon_status st = static_scratch_address(&scratch);
+        if (st != AXON_OK) return st;
+    }
+    // Every scratch word the split reads is written earlier in the same call
+    // (segment end states and dt sums by the first phase), so stale contents
+    // left by a previous call need no clearing.
+    return scan_impl(B, L, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
+                     conv_cache_in, ssm_state_in, y, conv_cache_out, ssm_state_out,
+                     scratch, scratch ? kStaticScratchBytes : 0, num_segments,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
