@@ -158,14 +158,16 @@ AXON_API axon_status axon_ssm_scan_fwd(
     void *workspace, size_t workspace_bytes, axon_stream_t stream);
 
 /*
- * The prefill with an explicit time split: `num_segments` > 0 forces the
+ * The prefill with an explicit time split: `num_segments` >= 2 forces the
  * sequence to be cut into that many segments processed in parallel, with the
  * chunk carry passed through `workspace` (which must then hold at least
- * (num_segments-1) * B * E * (N+1) floats; num_segments <= 64 and never more
- * than L).  num_segments == 0 lets the library choose, exactly as
+ * (num_segments-1) * B * E * (N+1) floats; num_segments <= 64 and every
+ * segment at least K tokens long, else AXON_ERR_INVALID_ARG).
+ * num_segments == 1 runs the sequence unsplit (the chunked kernel, no
+ * workspace); num_segments == 0 lets the library choose, exactly as
  * axon_ssm_scan_fwd does.  Same arguments and errors as axon_ssm_scan_fwd
- * otherwise.  Intended for tests and tuning; results agree with the unsplit
- * scan to float32 rounding.
+ * otherwise.  Intended for tests and tuning; results agree with the library's
+ * own plan to float32 rounding.
  */
 AXON_API axon_status axon_ssm_scan_fwd_segments(
     int B, int L, int E, int N, int K, axon_dtype io,

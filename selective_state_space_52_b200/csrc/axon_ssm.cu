@@ -9,6 +9,7 @@
 
 #include "axon_ssm.h"
 #include "device_math.cuh"
+#include "scan_chunked.cuh"
 #include "scan_seq.cuh"
 #include "step.cuh"
 
@@ -73,6 +74,91 @@ int plan_segments(int B, int L, int E, int sms) {
     return (int)(p < 1 ? 1 : p);
 }
 
+// Few channels and a long sequence: the channel tiles alone cannot occupy the
+// GPU, so split the sequence into segments and carry between them.
+bool use_time_split(int B, int L, int E, int sms) {
+    return (long long)B * E < (long long)sms * 4 && L >= 2 * kMinSegLen;
+}
+
+int device_max_smem_optin() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return -1;
+    return v;
+}
+
+struct ChunkPlan {
+    int W, R, ET, tiles_per_b, pitch, smem;
+};
+
+// Chunked scan plan: channel tiles of ET channels (about one CTA per SM when
+// channels are scarce, 128-channel tiles when they are plentiful) and W runs of
+// R tokens per chunk, the largest that fits the shared memory.
+bool plan_chunked(int B, int E, int io_bytes, int sms, int max_smem, ChunkPlan* out) {
+    const long long channels = (long long)B * E;
+    ChunkPlan c{};
+    if (channels >= (long long)sms * 256) {
+        c.W = 1; c.R = 16;
+        c.ET = E < 128 ? E : 128;
+    } else {
+        // about one tile per SM; all W runs of a channel share a warp, so ET
+        // is a multiple of the 32/W channels a warp holds
+        int tpb = sms / (B > 0 ? B : 1);
+        if (tpb < 1) tpb = 1;
+        const int et_ideal = (E + tpb - 1) / tpb;
+        static const int opts[][2] = {{2, 16}, {4, 16}, {8, 16}, {16, 16}, {8, 8}, {16, 8}, {32, 8}};
+        int best_score = -1;
+        for (const auto& o : opts) {
+            const int W = o[0], R = o[1];
+            const int cpw = 32 / W;
+            const int ET = (et_ideal + cpw - 1) / cpw * cpw;
+            const int threads = ET * W;
+            if (threads > 512) continue;
+            const int pitch = ((ET * io_bytes + 15) & ~15) + 16;
+            if (ChunkSmem(W, R, ET, pitch, io_bytes).total > max_smem) continue;
+            // enough warps to hide latency first, then the fewest runs per channel
+            const int score = (threads < 256 ? threads : 256) * 64 - W;
+            if (score > best_score) { best_score = score; c.W = W; c.R = R; c.ET = ET; }
+        }
+        if (best_score < 0) {
+            c.W = 1; c.R = 16;
+            c.ET = et_ideal < 512 ? et_ideal : 512;
+        }
+    }
+    if (c.ET * c.W > 512) return false;   // the kernel's launch bound
+    c.tiles_per_b = (E + c.ET - 1) / c.ET;
+    c.pitch = ((c.ET * io_bytes + 15) & ~15) + 16;
+    c.smem = ChunkSmem(c.W, c.R, c.ET, c.pitch, io_bytes).total;
+    if (c.smem > max_smem) return false;
+    *out = c;
+    return true;
+}
+
+template <class Io, int W, int R>
+axon_status launch_chunked_t(const ChunkParams& prm, int smem, cudaStream_t st) {
+    auto kern = scan_chunked_kernel<Io, W, R>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return AXON_ERR_CUDA;
+    const unsigned grid = (unsigned)((long long)prm.B * prm.tiles_per_b);
+    kern<<<grid, prm.ET * W, smem, st>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+}
+
+template <class Io>
+axon_status launch_chunked(const ChunkParams& prm, const ChunkPlan& c, cudaStream_t st) {
+    switch (c.W * 100 + c.R) {
+        case 116: return launch_chunked_t<Io, 1, 16>(prm, c.smem, st);
+        case 216: return launch_chunked_t<Io, 2, 16>(prm, c.smem, st);
+        case 416: return launch_chunked_t<Io, 4, 16>(prm, c.smem, st);
+        case 808: return launch_chunked_t<Io, 8, 8>(prm, c.smem, st);
+        case 816: return launch_chunked_t<Io, 8, 16>(prm, c.smem, st);
+        case 1608: return launch_chunked_t<Io, 16, 8>(prm, c.smem, st);
+        case 1616: return launch_chunked_t<Io, 16, 16>(prm, c.smem, st);
+        case 3208: return launch_chunked_t<Io, 32, 8>(prm, c.smem, st);
+    }
+    return AXON_ERR_UNSUPPORTED;
+}
+
 template <class Io>
 axon_status launch_scan(ScanParams& prm, cudaStream_t st) {
     const dim3 block(kScanThreads);
@@ -132,14 +218,23 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
 
     int P = 1;
     int seg = L > 0 ? L : 1;
+    bool chunked = false;
+    ChunkPlan cplan{};
     if (L > 0) {
-        if (num_segments > 0) {
-            if (num_segments > kMaxSegments) return AXON_ERR_INVALID_ARG;
-            P = num_segments;
+        if (num_segments > kMaxSegments) return AXON_ERR_INVALID_ARG;
+        if (num_segments > 1) {
+            P = num_segments;                  // forced time split (segment carry)
         } else {
             const int sms = device_sm_count();
             if (sms <= 0) return AXON_ERR_CUDA;
-            P = plan_segments(B, L, E, sms);
+            if (num_segments == 0 && use_time_split(B, L, E, sms)) {
+                P = plan_segments(B, L, E, sms);
+            } else {
+                // unsplit: the chunked kernel (the channel walk is the fallback)
+                const int max_smem = device_max_smem_optin();
+                if (max_smem <= 0) return AXON_ERR_CUDA;
+                chunked = plan_chunked(B, E, (int)io_bytes(io), sms, max_smem, &cplan);
+            }
         }
         if (P > 1) {
             seg = (L + P - 1) / P;
@@ -154,6 +249,18 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
         if (overlaps(workspace, need, y, n_seq) || overlaps(workspace, need, ssm_state_out, n_ss) ||
             overlaps(workspace, need, conv_cache_out, n_cc))
             return AXON_ERR_INVALID_ARG;
+    }
+
+    if (chunked) {
+        ChunkParams cp;
+        cp.B = B; cp.L = L; cp.E = E;
+        cp.ET = cplan.ET; cp.tiles_per_b = cplan.tiles_per_b; cp.pitch = cplan.pitch;
+        cp.x = x; cp.z = z; cp.dt_raw = dt_raw; cp.Bm = Bm; cp.Cm = Cm;
+        cp.conv_w = conv_w; cp.conv_b = conv_b; cp.dt_bias = dt_bias; cp.A_log = A_log; cp.D = D;
+        cp.conv_cache_in = conv_cache_in; cp.ssm_state_in = ssm_state_in;
+        cp.y = y; cp.conv_cache_out = conv_cache_out; cp.ssm_state_out = ssm_state_out;
+        return io == AXON_BF16 ? launch_chunked<IoBF16>(cp, cplan, stream)
+                               : launch_chunked<IoF32>(cp, cplan, stream);
     }
 
     ScanParams prm;
@@ -232,7 +339,8 @@ int axon_ssm_scan_launch_count(int B, int L, int E, int N, int K, axon_dtype io)
     if (L == 0) return 1;
     const int sms = device_sm_count();
     if (sms <= 0) return -1;
-    return plan_segments(B, L, E, sms) > 1 ? 2 : 1;
+    if (use_time_split(B, L, E, sms)) return plan_segments(B, L, E, sms) > 1 ? 2 : 1;
+    return 1;
 }
 
 axon_status axon_ssm_scan_fwd(int B, int L, int E, int N, int K, axon_dtype io,

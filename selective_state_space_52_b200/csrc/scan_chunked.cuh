@@ -1,0 +1,489 @@
+// scan_chunked.cuh -- chunked, shared-memory-staged selective scan.
+//
+// One CTA owns a tile of ET consecutive channels of one batch row for the
+// whole sequence (ET need not be a power of two: the host picks it so that
+// the tiles cover B*E channels with about one CTA per SM).  The sequence is
+// walked in chunks of kT = W*R tokens; the ET*W threads of the CTA split each
+// chunk into W runs of R consecutive tokens.  All W runs of a channel sit in
+// one warp (lane = channel-in-warp * W + run; a warp holds 32/W channels), so
+// runs exchange their partial results with warp shuffles, never with a CTA
+// barrier.  Per chunk:
+//
+//   1. x (with a 3-token halo), z, dt_raw rows of the tile's byte window and
+//      the B, C rows are copied into shared memory with 16-byte cp.async, one
+//      chunk ahead (double buffered).  Rows past L are zero-filled.  B and C
+//      are then converted once per chunk to float32 (transposed to [n][t]
+//      when W > 1), shared by all channels of the tile.
+//   2. Prologue per item: causal conv (tap 3 meets x_t) + SiLU, dt =
+//      clip(softplus(dt_raw + dt_bias), 1e-4, 100), dt*u; y starts at D*u.
+//   3. W > 1: states are processed one at a time.  Each run walks its R items
+//      from a zero state with the decays a_i = 2^(dt_i * A_n log2 e) and forms
+//      its aggregate (prod a_i, local end state).  An
+//      inclusive warp-shuffle scan over the W runs combines the (decay, input)
+//      pairs, (A, H) o (A', H') = (A A', A H' + H); the exclusive prefix applied
+//      to the chunk's carry-in h_in gives each run its starting state; the
+//      first pass kept each item's cumulative decay A_i and zero-start state
+//      H_i, so h_i = A_i h_in + H_i for all items at once (no second
+//      exponential, no dependency chain) and y_i += C_i,n h_i.  The last run's
+//      end state is the next chunk's carry.  This is the intra-block pass + inter-block carry of the
+//      chunked associative scan in the SSD article, applied to the diagonal
+//      (S6) recurrence, where every state's chain is a scalar linear
+//      recurrence.
+//      W == 1 (enough channels to fill the GPU): each thread walks its
+//      channel straight through, 16 states in registers, item by item.
+//   4. Epilogue: y *= SiLU(z); the tile of y is staged in shared memory and
+//      written back in 16-byte stores (narrow stores only at the tile edges).
+//
+// Float32 pairs use the sm_100 packed FMA/FMUL (__ffma2_rn/__fmul2_rn): over
+// items (consecutive tokens) when W > 1, over states when W == 1.
+//
+// Recurrence and gating: Axon-SSM page, recurrence equation (first-order
+// discretisation), "Selective mechanism", "Diagonal state matrix", "Gating".
+#pragma once
+
+#include "device_math.cuh"
+
+namespace axon {
+
+struct ChunkParams {
+    int B, L, E;
+    int ET;           // channels per tile (threads per run)
+    int tiles_per_b;  // ceil(E / ET)
+    int pitch;        // bytes per shared-memory row of the x/z/dt/y tiles (multiple of 16)
+    const void* x;
+    const void* z;
+    const void* dt_raw;
+    const void* Bm;
+    const void* Cm;
+    const float* conv_w;
+    const float* conv_b;
+    const float* dt_bias;
+    const float* A_log;
+    const float* D;
+    const void* conv_cache_in;   // may be null
+    const float* ssm_state_in;   // may be null
+    void* y;
+    void* conv_cache_out;
+    float* ssm_state_out;
+};
+
+constexpr int kSkew = 16;   // bytes added per run of rows (breaks bank aliasing between runs)
+
+__host__ __device__ constexpr int ilog2c(int v) { return v <= 1 ? 0 : 1 + ilog2c(v >> 1); }
+
+// Byte layout of a CTA's dynamic shared memory; identical on host and device.
+struct ChunkSmem {
+    int xs, zs, ds, bs, cs, stage, bf, cf, ys, carry, a2, total, tpad;
+    __host__ __device__ static int rows_bytes(int rows, int pitch, int R) {
+        return rows * pitch + ((rows + R - 1) / R) * kSkew;
+    }
+    __host__ __device__ ChunkSmem(int W, int R, int ET, int pitch, int io_bytes) {
+        const int kT = W * R;
+        tpad = kT + 4 * W;                      // float stride of a transposed B/C row (4 pad floats per run)
+        int off = 0;
+        xs = off; off += rows_bytes(kT + kK - 1, pitch, R);
+        zs = off; off += rows_bytes(kT, pitch, R);
+        ds = off; off += rows_bytes(kT, pitch, R);
+        bs = off; off += kT * kN * io_bytes;
+        cs = off; off += kT * kN * io_bytes;
+        stage = (off + 15) & ~15;
+        off = 2 * stage;
+        bf = off; off += (W > 1 ? kN * tpad : kT * kN) * 4;
+        cf = off; off += (W > 1 ? kN * tpad : kT * kN) * 4;
+        ys = off; off += rows_bytes(kT, pitch, R);
+        off = (off + 15) & ~15;
+        carry = off; off += (W > 1) ? 2 * kN * ET * 4 : 0;
+        a2 = off; off += (W > 1) ? kN * ET * 4 : 0;
+        total = off;
+    }
+};
+
+// Byte offset of row j of a staged tile (rows of R tokens are skewed by 16 B).
+template <int R>
+__device__ __forceinline__ int row_off(int j, int pitch) {
+    return j * pitch + (j >> ilog2c(R)) * kSkew;
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src, bool valid) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    const int n = valid ? 16 : 0;   // 0 source bytes: the 16 destination bytes are zero-filled
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem_src), "r"(n)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
+
+// io-typed shared-memory access by byte address
+template <class Io> struct SmemIo;
+template <> struct SmemIo<IoF32> {
+    __device__ __forceinline__ static float ld(const unsigned char* p) { return *reinterpret_cast<const float*>(p); }
+    __device__ __forceinline__ static void st(unsigned char* p, float v) { *reinterpret_cast<float*>(p) = v; }
+    // 8 consecutive values (32 bytes)
+    __device__ __forceinline__ static void ld8(const unsigned char* p, float (&v)[8]) {
+        const float4 a = *reinterpret_cast<const float4*>(p);
+        const float4 b = *reinterpret_cast<const float4*>(p + 16);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+};
+template <> struct SmemIo<IoBF16> {
+    __device__ __forceinline__ static float ld(const unsigned char* p) {
+        return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const unsigned short*>(p)) << 16);
+    }
+    __device__ __forceinline__ static void st(unsigned char* p, float v) {
+        *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(v);
+    }
+    // 8 consecutive values (16 bytes)
+    __device__ __forceinline__ static void ld8(const unsigned char* p, float (&v)[8]) {
+        const uint4 a = *reinterpret_cast<const uint4*>(p);
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            v[2 * q] = __uint_as_float(w[q] << 16);
+            v[2 * q + 1] = __uint_as_float(w[q] & 0xffff0000u);
+        }
+    }
+};
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+
+template <class Io, int W, int R, int kMinBlocks = 1>
+__global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkParams p) {
+    static_assert(R % 4 == 0 && (R & (R - 1)) == 0, "R: power of two, multiple of 4");
+    using T = typename Io::T;
+    using SI = SmemIo<Io>;
+    constexpr int S = Io::kBytes;
+    constexpr int kT = W * R;
+    extern __shared__ __align__(16) unsigned char smem[];
+
+    const int NT = blockDim.x;
+    const int tid = threadIdx.x;
+    const int ET = p.ET;
+    constexpr int CPW = 32 / W;                 // channels per warp (W > 1)
+    const int c = (W == 1) ? tid : (tid >> 5) * CPW + (tid & 31) / W;
+    const int r = (W == 1) ? 0 : (tid & (W - 1));
+    const int b = blockIdx.x / p.tiles_per_b;
+    const int e0 = (blockIdx.x - b * p.tiles_per_b) * ET;
+    const int ne = min(ET, p.E - e0);
+    const bool active = c < ne;
+    const int e = e0 + (active ? c : 0);
+    const int pitch = p.pitch;
+    // 16-byte aligned byte window [wb0, wb1) of the tile inside an (E)-row
+    const int wb0 = (e0 * S) & ~15;
+    const int wb1 = ((e0 + ne) * S + 15) & ~15;
+    const int nch = (wb1 - wb0) >> 4;
+    const int coff = e0 * S - wb0 + c * S;
+    const ChunkSmem lay(W, R, ET, pitch, S);
+    const int tpad = lay.tpad;
+
+    const unsigned char* xg = static_cast<const unsigned char*>(p.x);
+    const unsigned char* zg = static_cast<const unsigned char*>(p.z);
+    const unsigned char* dg = static_cast<const unsigned char*>(p.dt_raw);
+    const unsigned char* bg = static_cast<const unsigned char*>(p.Bm);
+    const unsigned char* cg = static_cast<const unsigned char*>(p.Cm);
+    const unsigned char* ccg = static_cast<const unsigned char*>(p.conv_cache_in);
+    const size_t row_bytes = (size_t)p.E * S;
+
+    // ---- copy chunk k into stage st (every thread issues its share)
+    auto prefetch = [&](int k, int st) {
+        const int t0 = k * kT;
+        unsigned char* sb = smem + st * lay.stage;
+        const int nx = (kT + kK - 1) * nch;
+        for (int w = tid; w < nx; w += NT) {
+            const int row = w / nch;
+            const int ch = w - row * nch;
+            const int t = t0 - (kK - 1) + row;
+            const void* src = xg;
+            bool ok = false;
+            if (t >= 0 && t < p.L) {
+                src = xg + ((size_t)b * p.L + t) * row_bytes + wb0 + ch * 16;
+                ok = true;
+            } else if (t < 0 && ccg != nullptr) {
+                src = ccg + ((size_t)b * (kK - 1) + (kK - 1 + t)) * row_bytes + wb0 + ch * 16;
+                ok = true;
+            }
+            cp_async16(sb + lay.xs + row_off<R>(row, pitch) + ch * 16, src, ok);
+        }
+        const int nz = kT * nch;
+        for (int w = tid; w < nz; w += NT) {
+            const int row = w / nch;
+            const int ch = w - row * nch;
+            const int t = t0 + row;
+            const bool ok = t < p.L;
+            const size_t go = ok ? ((size_t)b * p.L + t) * row_bytes + wb0 + ch * 16 : 0;
+            const int so = row_off<R>(row, pitch) + ch * 16;
+            cp_async16(sb + lay.zs + so, zg + go, ok);
+            cp_async16(sb + lay.ds + so, dg + go, ok);
+        }
+        constexpr int nbc = kN * S / 16;     // 16-byte pieces per B/C row
+        for (int w = tid; w < kT * nbc; w += NT) {
+            const int row = w / nbc;
+            const int ch = w - row * nbc;
+            const int t = t0 + row;
+            const bool ok = t < p.L;
+            const size_t go = ok ? ((size_t)b * p.L + t) * (kN * S) + ch * 16 : 0;
+            cp_async16(sb + lay.bs + row * (kN * S) + ch * 16, bg + go, ok);
+            cp_async16(sb + lay.cs + row * (kN * S) + ch * 16, cg + go, ok);
+        }
+    };
+
+    // ---- per-channel constants
+    const float w0 = __ldg(p.conv_w + (size_t)e * kK + 0);
+    const float w1 = __ldg(p.conv_w + (size_t)e * kK + 1);
+    const float w2 = __ldg(p.conv_w + (size_t)e * kK + 2);
+    const float w3 = __ldg(p.conv_w + (size_t)e * kK + 3);
+    const float cb = __ldg(p.conv_b + e);
+    const float db = __ldg(p.dt_bias + e);
+    const float Dv = __ldg(p.D + e);
+
+    float* bf = reinterpret_cast<float*>(smem + lay.bf);
+    float* cf = reinterpret_cast<float*>(smem + lay.cf);
+    float* carry = reinterpret_cast<float*>(smem + lay.carry);     // [2][kN][ET]
+    float* a2s = reinterpret_cast<float*>(smem + lay.a2);           // [kN][ET]
+
+    // A = -exp(A_log) scaled by log2(e), so that exp(dt*A) = 2^(dt*A2): in
+    // registers (state pairs) for the direct walk, in shared memory otherwise.
+    float2 s2[W == 1 ? kN / 2 : 1];
+    float2 h2[W == 1 ? kN / 2 : 1];
+    if constexpr (W == 1) {
+#pragma unroll
+        for (int q = 0; q < kN / 2; ++q) {
+            s2[q] = f2(-expf(__ldg(p.A_log + (size_t)e * kN + 2 * q)) * kLog2e,
+                       -expf(__ldg(p.A_log + (size_t)e * kN + 2 * q + 1)) * kLog2e);
+            h2[q] = (p.ssm_state_in && active)
+                        ? f2(p.ssm_state_in[((size_t)b * p.E + e) * kN + 2 * q],
+                             p.ssm_state_in[((size_t)b * p.E + e) * kN + 2 * q + 1])
+                        : f2(0.0f, 0.0f);
+        }
+    } else if (r == 0) {
+#pragma unroll
+        for (int n = 0; n < kN; ++n) {
+            a2s[n * ET + c] = -expf(__ldg(p.A_log + (size_t)e * kN + n)) * kLog2e;
+            carry[n * ET + c] = (p.ssm_state_in && active) ? p.ssm_state_in[((size_t)b * p.E + e) * kN + n] : 0.0f;
+        }
+    }
+
+    const int nck = (p.L + kT - 1) / kT;
+    const int i0 = r * R;                 // first item of this run within a chunk
+    prefetch(0, 0);
+    cp_async_commit();
+
+    for (int k = 0; k < nck; ++k) {
+        const int st = k & 1;
+        if (k + 1 < nck) prefetch(k + 1, st ^ 1);
+        cp_async_commit();
+        cp_async_wait_1();
+        __syncthreads();
+        const unsigned char* sb = smem + st * lay.stage;
+        const int t0 = k * kT;
+
+        // ---- B, C to float32, once per chunk for the whole tile
+        for (int w = tid; w < 4 * kT; w += NT) {
+            const int t = w % kT;
+            const int q = w / kT;                          // 0,1: B halves; 2,3: C halves
+            const unsigned char* src = sb + (q < 2 ? lay.bs : lay.cs) + t * (kN * S) + (q & 1) * 8 * S;
+            float v[8];
+            SI::ld8(src, v);
+            float* dst = q < 2 ? bf : cf;
+            if constexpr (W == 1) {
+                float4* d4 = reinterpret_cast<float4*>(dst + t * kN + (q & 1) * 8);
+                d4[0] = make_float4(v[0], v[1], v[2], v[3]);
+                d4[1] = make_float4(v[4], v[5], v[6], v[7]);
+            } else {
+#pragma unroll
+                for (int m = 0; m < 8; ++m) dst[((q & 1) * 8 + m) * tpad + t + (t / R) * 4] = v[m];
+            }
+        }
+        __syncthreads();
+
+        unsigned char* yb = smem + lay.ys;
+        if constexpr (W == 1) {
+            // ---- direct walk: item by item, all 16 states in registers
+            const unsigned char* xc0 = sb + lay.xs + coff;
+            float xm3 = SI::ld(xc0 + row_off<R>(0, pitch));
+            float xm2 = SI::ld(xc0 + row_off<R>(1, pitch));
+            float xm1 = SI::ld(xc0 + row_off<R>(2, pitch));
+#pragma unroll 2
+            for (int i = 0; i < R; ++i) {
+                const float xt = SI::ld(xc0 + row_off<R>(i + 3, pitch));
+                float xc = fmaf(w0, xm3, cb);
+                xc = fmaf(w1, xm2, xc);
+                xc = fmaf(w2, xm1, xc);
+                xc = fmaf(w3, xt, xc);
+                xm3 = xm2; xm2 = xm1; xm1 = xt;
+                const float u = silu(xc);
+                const float dr = SI::ld(sb + lay.ds + row_off<R>(i, pitch) + coff);
+                const float dt = dt_from_raw(dr + db);
+                const bool live = (t0 + i) < p.L;
+                const float dtl = live ? dt : 0.0f;     // dt = 0: decay 1, no input
+                const float2 dt2 = f2(dtl, dtl);
+                const float dtu = live ? dt * u : 0.0f;
+                const float2 dtu2 = f2(dtu, dtu);
+                float2 yacc = f2(Dv * u, 0.0f);
+                const float4* bq = reinterpret_cast<const float4*>(bf + i * kN);
+                const float4* cq = reinterpret_cast<const float4*>(cf + i * kN);
+#pragma unroll
+                for (int q = 0; q < kN / 4; ++q) {
+                    const float4 bv = bq[q];
+                    const float4 cv = cq[q];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int pq = 2 * q + hh;
+                        const float2 arg = __fmul2_rn(dt2, s2[pq]);
+                        const float2 a = f2(ex2_approx(arg.x), ex2_approx(arg.y));
+                        const float2 bb = hh ? f2(bv.z, bv.w) : f2(bv.x, bv.y);
+                        const float2 cc = hh ? f2(cv.z, cv.w) : f2(cv.x, cv.y);
+                        h2[pq] = __ffma2_rn(a, h2[pq], __fmul2_rn(dtu2, bb));
+                        yacc = __ffma2_rn(cc, h2[pq], yacc);
+                    }
+                }
+                const float zt = SI::ld(sb + lay.zs + row_off<R>(i, pitch) + coff);
+                SI::st(yb + row_off<R>(i, pitch) + coff, (yacc.x + yacc.y) * silu(zt));
+            }
+        } else {
+            // ---- prologue for this run's R items (pairs of consecutive items)
+            float2 dtv[R / 2], dtu[R / 2], yv[R / 2];
+            {
+                const unsigned char* xc0 = sb + lay.xs + coff;
+                float xm3 = SI::ld(xc0 + row_off<R>(i0 + 0, pitch));
+                float xm2 = SI::ld(xc0 + row_off<R>(i0 + 1, pitch));
+                float xm1 = SI::ld(xc0 + row_off<R>(i0 + 2, pitch));
+#pragma unroll
+                for (int i = 0; i < R; ++i) {
+                    const float xt = SI::ld(xc0 + row_off<R>(i0 + i + 3, pitch));
+                    float xc = fmaf(w0, xm3, cb);
+                    xc = fmaf(w1, xm2, xc);
+                    xc = fmaf(w2, xm1, xc);
+                    xc = fmaf(w3, xt, xc);
+                    xm3 = xm2; xm2 = xm1; xm1 = xt;
+                    const float u = silu(xc);
+                    const float dr = SI::ld(sb + lay.ds + row_off<R>(i0 + i, pitch) + coff);
+                    const float dt = dt_from_raw(dr + db);
+                    const bool live = (t0 + i0 + i) < p.L;
+                    const float dtl = live ? dt : 0.0f;
+                    const float dtul = live ? dt * u : 0.0f;
+                    if (i & 1) { dtv[i / 2].y = dtl; dtu[i / 2].y = dtul; yv[i / 2].y = Dv * u; }
+                    else       { dtv[i / 2].x = dtl; dtu[i / 2].x = dtul; yv[i / 2].x = Dv * u; }
+                }
+            }
+            const float* cin = carry + (k & 1) * kN * ET;
+            float* cout = carry + ((k + 1) & 1) * kN * ET;
+#pragma unroll 1
+            for (int n = 0; n < kN; ++n) {
+                const float s = a2s[n * ET + c];
+                const float2 ss = f2(s, s);
+                const float4* brow = reinterpret_cast<const float4*>(bf + n * tpad + r * (R + 4));
+                const float4* crow = reinterpret_cast<const float4*>(cf + n * tpad + r * (R + 4));
+                // first pass from a zero state: cumulative decay Acum_i and local
+                // state Hloc_i of every item, kept as (item, item+1) pairs
+                float2 Ac[R / 2], Hl[R / 2];
+                float A = 1.0f, H = 0.0f;
+#pragma unroll
+                for (int i4 = 0; i4 < R / 4; ++i4) {
+                    const float4 bv = brow[i4];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int ip = 2 * i4 + hh;
+                        const float2 arg = __fmul2_rn(dtv[ip], ss);
+                        const float a0 = ex2_approx(arg.x), a1 = ex2_approx(arg.y);
+                        const float2 bu = __fmul2_rn(dtu[ip], hh ? f2(bv.z, bv.w) : f2(bv.x, bv.y));
+                        const float A0 = A * a0, H0 = fmaf(a0, H, bu.x);
+                        A = A0 * a1;
+                        H = fmaf(a1, H0, bu.y);
+                        Ac[ip] = f2(A0, A);
+                        Hl[ip] = f2(H0, H);
+                    }
+                }
+                // inclusive scan of the run aggregates (A, H) over the W runs of this
+                // channel (W consecutive lanes); later o earlier = (A A', A H' + H)
+                float As = A, Hs = H;
+#pragma unroll
+                for (int d = 1; d < W; d <<= 1) {
+                    const float Ap = __shfl_up_sync(0xffffffffu, As, d, W);
+                    const float Hp = __shfl_up_sync(0xffffffffu, Hs, d, W);
+                    if (r >= d) { Hs = fmaf(As, Hp, Hs); As *= Ap; }
+                }
+                // exclusive prefix (the runs before this one) applied to the carry-in
+                float Ae = __shfl_up_sync(0xffffffffu, As, 1, W);
+                float He = __shfl_up_sync(0xffffffffu, Hs, 1, W);
+                if (r == 0) { Ae = 1.0f; He = 0.0f; }
+                const float hc = cin[n * ET + c];
+                const float hin = fmaf(Ae, hc, He);
+                const float2 hin2 = f2(hin, hin);
+                // second pass, no dependency chain: h_i = Acum_i h_in + Hloc_i
+#pragma unroll
+                for (int i4 = 0; i4 < R / 4; ++i4) {
+                    const float4 cv = crow[i4];
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int ip = 2 * i4 + hh;
+                        const float2 h = __ffma2_rn(Ac[ip], hin2, Hl[ip]);
+                        yv[ip] = __ffma2_rn(hh ? f2(cv.z, cv.w) : f2(cv.x, cv.y), h, yv[ip]);
+                    }
+                }
+                if (r == W - 1) {
+                    const float hend = fmaf(As, hc, Hs);           // the chunk's end state
+                    cout[n * ET + c] = hend;
+                    if (k == nck - 1 && active) p.ssm_state_out[((size_t)b * p.E + e) * kN + n] = hend;
+                }
+            }
+            // ---- epilogue: gate, stage the y tile
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                const float zt = SI::ld(sb + lay.zs + row_off<R>(i0 + i, pitch) + coff);
+                const float yy = (i & 1) ? yv[i / 2].y : yv[i / 2].x;
+                SI::st(yb + row_off<R>(i0 + i, pitch) + coff, yy * silu(zt));
+            }
+        }
+        __syncthreads();
+        // ---- write the y tile: 16-byte stores inside the tile, narrow ones at its edges
+        {
+            const int lo = e0 * S, hi = (e0 + ne) * S;
+            unsigned char* yg = static_cast<unsigned char*>(p.y);
+            const int nyw = kT * nch;
+            for (int w = tid; w < nyw; w += NT) {
+                const int row = w / nch;
+                const int ch = w - row * nch;
+                const int t = t0 + row;
+                if (t >= p.L) continue;
+                const int gb = wb0 + ch * 16;
+                unsigned char* gp = yg + ((size_t)b * p.L + t) * row_bytes + gb;
+                const unsigned char* sp = yb + row_off<R>(row, pitch) + ch * 16;
+                if (gb >= lo && gb + 16 <= hi) {
+                    *reinterpret_cast<uint4*>(gp) = *reinterpret_cast<const uint4*>(sp);
+                } else {
+                    const int q0 = max(lo, gb) - gb, q1 = min(hi, gb + 16) - gb;
+                    for (int q = q0; q < q1; q += S)
+                        *reinterpret_cast<T*>(gp + q) = *reinterpret_cast<const T*>(sp + q);
+                }
+            }
+        }
+    }
+
+    // ---- final caches
+    if constexpr (W == 1) {
+        if (active) {
+            float4* so = reinterpret_cast<float4*>(p.ssm_state_out + ((size_t)b * p.E + e) * kN);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                so[q] = make_float4(h2[2 * q].x, h2[2 * q].y, h2[2 * q + 1].x, h2[2 * q + 1].y);
+        }
+    }
+    if (r == 0 && active) {
+        // the last K-1 raw inputs of conv_cache_in ++ x (read all before writing: may alias)
+        const T* xs = static_cast<const T*>(p.x);
+        const T* cc = static_cast<const T*>(p.conv_cache_in);
+        T v[kK - 1];
+#pragma unroll
+        for (int j = 0; j < kK - 1; ++j) {
+            const int t = p.L - (kK - 1) + j;
+            if (t >= 0) v[j] = xs[((size_t)b * p.L + t) * p.E + e];
+            else if (cc) v[j] = cc[((size_t)b * (kK - 1) + (kK - 1 + t)) * p.E + e];
+            else v[j] = T(0.0f);
+        }
+        T* co = static_cast<T*>(p.conv_cache_out);
+#pragma unroll
+        for (int j = 0; j < kK - 1; ++j) co[((size_t)b * (kK - 1) + j) * p.E + e] = v[j];
+    }
+}
+
+}  // namespace axon

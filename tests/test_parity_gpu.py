@@ -32,6 +32,38 @@ def test_sweep_small_shapes(cuda_lib, io, B, E, L):
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("B,E", SWEEP_BE)
+@pytest.mark.parametrize("L", [1, 5, 63, 257, 1000, 3001])
+def test_chunked_kernel_small_shapes(cuda_lib, io, B, E, L):
+    """The unsplit chunked kernel (num_segments=1) on tiny channel tiles with
+    16-byte windows that start mid-chunk, several chunks and ragged tails."""
+    wl = W.custom(B, L, E, io=io, seed=3000 + L + E + B)
+    inp = W.make_inputs(wl, with_state=True)
+    compare_scan(inp, io, num_segments=1, with_state=(L % 2 == 1), what=f"chunked B{B} L{L} E{E} {io}")
+
+
+# Shapes that steer the planner to each run count W (channels per tile ET =
+# ceil(E / (148 / B)); W is the largest of 16/8/4/2/1 with ET*W <= 512 whose
+# shared memory fits), including partial last tiles (E % ET != 0).
+PLANNER_SHAPES = [
+    (1, 1000, 300),     # ET 7, partial last tile, W 16
+    (1, 7680, 200),     # ET 52 (the Bit-Axon tiling), W 8
+    (2, 2048, 300),     # ET 28, two batch rows, W 16 (bf16) / 8 (fp32)
+    (1, 14800, 100),    # ET 100, W 4 (bf16)
+    (1, 29600, 40),     # ET 200, W 2 (bf16) / 1 (fp32)
+    (8, 4800, 40),      # 38400 channels: direct walk, W 1
+]
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("B,E,L", PLANNER_SHAPES)
+def test_chunked_kernel_planner_shapes(cuda_lib, io, B, E, L):
+    wl = W.custom(B, L, E, io=io, seed=4000 + E + L)
+    inp = W.make_inputs(wl, with_state=True)
+    compare_scan(inp, io, num_segments=1, with_state=True, what=f"planner B{B} E{E} L{L} {io}")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
 @pytest.mark.parametrize("L,P", [(64, 2), (257, 3), (1000, 7), (2048, 16), (300, 60), (4096, 64)])
 def test_forced_time_split(cuda_lib, io, L, P):
     """The segment-carry path (phase 1 summaries + carry fold + second walk)."""
