@@ -276,6 +276,64 @@ def run_reference(args, wl):
     return 0
 
 
+def bench_decode(dev, steps: int = 512, distinct: int = 8) -> dict:
+    """Cached decode on the decode workload's shapes (64 sequences, E=7680, bf16):
+    per-step time cold (L2 flushed before every step, events around each step)
+    and warm (all steps back to back in one CUDA graph; the 34 MB of state and
+    cache may then stay in the 126 MB L2)."""
+    from selective_state_space_52_b200 import axon_ssm
+    wl = W.WORKLOAD_BY_NAME["decode"]
+    params = {k: v.to(dev) for k, v in W.make_params(wl).items()}
+    st = {k: v.to(dev) for k, v in W.make_state(wl).items()}
+    toks = {k: v.to(dev) for k, v in W.make_decode_inputs(wl, distinct).items()}
+    cache = (st["conv_cache"], st["ssm_state"])
+    y = torch.empty(wl.B, wl.E, dtype=wl.torch_io, device=dev)
+    model = step_model(wl)
+    stream = torch.cuda.current_stream(dev)
+
+    def one(i):
+        axon_ssm.step(*(toks[k][i % distinct] for k in ("x", "z", "dt_raw", "B", "C")), params, cache, y=y)
+
+    for i in range(8):
+        one(i)
+    # read (not write) a buffer twice the L2 size before every step: the L2 then
+    # holds clean lines only, so the step does not pay for another buffer's write-back
+    flush = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    cold = []
+    for i in range(32):
+        flush.sum()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream); one(i); b.record(stream)
+        torch.cuda.synchronize(dev)
+        cold.append(a.elapsed_time(b))
+    cold_ms = statistics.median(cold[4:])
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        one(0)
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            one(i)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream); g.replay(); b.record(stream)
+    torch.cuda.synchronize(dev)
+    warm_ms = a.elapsed_time(b) / steps
+    del g
+    peaks = measured_peaks()
+    return {"workload": "decode: B64 E7680 N16 K4, bf16 io, fp32 state",
+            "algorithmic_bytes": model["bytes"],
+            "cold_us": cold_ms * 1e3, "cold_gbs": model["bytes"] / (cold_ms / 1e3) / 1e9,
+            "cold_frac_hbm": model["bytes"] / (cold_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "warm_us": warm_ms * 1e3, "warm_gbs": model["bytes"] / (warm_ms / 1e3) / 1e9,
+            "warm_note": f"{steps} steps in one CUDA graph; state + cache (34 MB) can stay in L2",
+            "token_ch_per_s_warm": wl.B * wl.E / (warm_ms / 1e3) / 1e9}
+
+
 def workload_desc(wl) -> str:
     return (f"{wl.name}: B{wl.B} L{wl.L} E{wl.E} N{wl.N} K{wl.K}, {wl.io} io, fp32 state; "
             "step = prefill + 1 cached decode token")
@@ -429,6 +487,8 @@ def run_axon(args, wl):
         "gpu_launches": args.steps * (scan_launches + 1),
     }
 
+    if not args.no_decode_bench:
+        line["decode"] = bench_decode(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inp_cpu = {**params_cpu, **{k: v.cpu() for k, v in sets[0].items()}}
         rate, units, secs, ch = time_oracle(wl, inp_cpu, args.cpu_budget)
@@ -452,6 +512,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="bit_axon_layer", choices=[w.name for w in W.WORKLOADS])
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode-bench", action="store_true",
+                    help="skip the separate cached-decode measurement (decode workload shapes)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     wl = W.WORKLOAD_BY_NAME[args.workload]

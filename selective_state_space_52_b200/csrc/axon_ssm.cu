@@ -406,11 +406,18 @@ axon_status axon_ssm_step(int B, int E, int N, int K, axon_dtype io,
     prm.x = x; prm.z = z; prm.dt_raw = dt_raw; prm.Bm = Bm; prm.Cm = Cm;
     prm.conv_w = conv_w; prm.conv_b = conv_b; prm.dt_bias = dt_bias; prm.A_log = A_log; prm.D = D;
     prm.conv_cache = conv_cache; prm.ssm_state = ssm_state; prm.y = y;
-    const long long threads = (long long)B * E * 4;
-    const unsigned grid = (unsigned)((threads + 255) / 256);
+    // batch rows per block: the fewest that keep the grid within ~8 resident
+    // blocks of 128 threads per SM (one wave), so each block's copy ring runs
+    // over several rows
+    const int sms = device_sm_count();
+    if (sms <= 0) return AXON_ERR_CUDA;
+    const long long bx = (E + kStepChan - 1) / kStepChan;
+    int rows = 1;
+    while (rows < kStepMaxRows && rows < B && bx * ((B + rows - 1) / rows) > 8LL * sms) rows *= 2;
+    const dim3 grid((unsigned)bx, (unsigned)((B + rows - 1) / rows));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (io == AXON_BF16) step_kernel<IoBF16><<<grid, 256, 0, s>>>(prm);
-    else step_kernel<IoF32><<<grid, 256, 0, s>>>(prm);
+    if (io == AXON_BF16) step_kernel<IoBF16><<<grid, kStepThreads, 0, s>>>(prm, rows);
+    else step_kernel<IoF32><<<grid, kStepThreads, 0, s>>>(prm, rows);
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
 

@@ -71,6 +71,12 @@ struct IoF32 {
     __device__ __forceinline__ static float load(const T* p) { return __ldg(p); }
     __device__ __forceinline__ static float load_rw(const T* p) { return *p; }
     __device__ __forceinline__ static void store(T* p, float v) { *p = v; }
+    // one value / four consecutive values (16-byte aligned) from shared memory
+    __device__ __forceinline__ static float sload(const void* p) { return *reinterpret_cast<const float*>(p); }
+    __device__ __forceinline__ static void sload4(const void* p, float (&r)[4]) {
+        const float4 v = *reinterpret_cast<const float4*>(p);
+        r[0] = v.x; r[1] = v.y; r[2] = v.z; r[3] = v.w;
+    }
     // 16 consecutive values of a B/C row (64 bytes, 16-byte aligned).
     __device__ __forceinline__ static void load_row16(const T* p, float (&r)[kN]) {
         const float4* q = reinterpret_cast<const float4*>(p);
@@ -95,6 +101,15 @@ struct IoBF16 {
         return bits_to_f(*reinterpret_cast<const unsigned short*>(p));
     }
     __device__ __forceinline__ static void store(T* p, float v) { *p = __float2bfloat16_rn(v); }
+    // one value / four consecutive values (8-byte aligned) from shared memory
+    __device__ __forceinline__ static float sload(const void* p) {
+        return bits_to_f(*reinterpret_cast<const unsigned short*>(p));
+    }
+    __device__ __forceinline__ static void sload4(const void* p, float (&r)[4]) {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        r[0] = __uint_as_float(v.x << 16); r[1] = __uint_as_float(v.x & 0xffff0000u);
+        r[2] = __uint_as_float(v.y << 16); r[3] = __uint_as_float(v.y & 0xffff0000u);
+    }
     // 16 consecutive bf16 values of a B/C row (32 bytes, 16-byte aligned).
     __device__ __forceinline__ static void load_row16(const T* p, float (&r)[kN]) {
         const uint4* q = reinterpret_cast<const uint4*>(p);

@@ -4,11 +4,10 @@
 // y, the shifted conv cache and the updated state in place.
 //
 // The step is bound by HBM traffic on the state read-modify-write (2 x 64 bytes
-// per channel of the 148 bytes it moves at bf16).  Four lanes share a channel:
-// each owns four consecutive states (one 16-byte vector), so a warp's state
-// load/store is one contiguous 512-byte run, and the C contraction is finished
-// with two butterfly shuffles.  The cheap per-channel prologue is recomputed
-// by the four lanes instead of being broadcast.
+// of the 148 bytes per channel it moves at bf16).  The state moves as 16-byte
+// pieces, four lanes per channel, through per-lane asynchronous-copy rings, and
+// every other input arrives through shared memory in one copy per block, so the
+// HBM traffic of later rows overlaps the arithmetic of the current one.
 #pragma once
 
 #include "device_math.cuh"
@@ -32,71 +31,142 @@ struct StepParams {
     void* y;
 };
 
-// grid = ceil(B*E*4 / 256) blocks of 256 threads; thread -> (channel, quarter).
+__device__ __forceinline__ void step_cp_async16(void* smem_dst, const void* gmem_src, bool valid) {
+    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    const int n = valid ? 16 : 0;   // 0 source bytes: zero-fill
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem_src), "r"(n) : "memory");
+}
+
+constexpr int kStepThreads = 128;  // 32 channels x 4 lanes
+constexpr int kStepChan = kStepThreads / 4;
+constexpr int kStepStages = 4;     // state rows in flight per lane (shared-memory ring)
+constexpr int kStepMaxRows = 32;   // batch rows per block
+
+// grid = (ceil(E / 32), ceil(B / rows)) blocks of 128 threads, rows <= 32.
+// Four lanes share a channel, each owning four consecutive states (one 16-byte
+// vector), so a warp's state traffic is one contiguous 512-byte run.  A block
+// owns 32 channels and walks `rows` batch rows:
+//  - at the start it copies, for all its rows, the channels' x, z, dt_raw and
+//    K-1 cache entries and the B_t, C_t rows into shared memory (one
+//    cooperative cp.async group, one barrier);
+//  - every lane streams its state pieces through a private kStepStages-deep
+//    shared-memory ring with cp.async (a lane reads back only its own copies);
+//  - A = -exp(A_log) is formed once per lane.
+// The conv/SiLU/dt prologue is recomputed by the four lanes of a channel
+// (cheaper than broadcasting it); C . h is finished with two shuffles.
 template <class Io>
-__global__ void __launch_bounds__(256) step_kernel(StepParams p) {
+__global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int rows) {
     using T = typename Io::T;
-    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    const long long nch = (long long)p.B * p.E;
-    // Every lane stays to the end so that the full-warp shuffles below are
-    // defined; lanes past the last channel compute channel 0 and store nothing.
-    const bool valid = (gid >> 2) < nch;
-    const long long ch = valid ? (gid >> 2) : 0;   // flattened (b, e)
-    const int q = (int)(gid & 3);                  // states 4q .. 4q+3
-    const int b = (int)(ch / p.E);
-    const int e = (int)(ch - (long long)b * p.E);
+    constexpr int S = Io::kBytes;
+    constexpr int kSmall = 3 + (kK - 1);              // x, z, dt_raw, cache rows 0..K-2
+    constexpr int kWin = kStepChan * S;               // bytes of a 32-channel window
+    const int tid = threadIdx.x;
+    const int q = tid & 3;                            // states 4q .. 4q+3
+    const int c = tid >> 2;
+    const int e0 = blockIdx.x * kStepChan;
+    const int e = e0 + c;
+    const int b0 = blockIdx.y * rows;
+    const int nb = min(rows, p.B - b0);
+    // Every lane stays to the end (the shuffles below need full warps); lanes
+    // past E compute channel E-1 and store nothing.
+    const bool live = e < p.E;
+    const int ec = live ? e : p.E - 1;
 
-    // conv window: oldest first, then this token
-    T* cc = static_cast<T*>(p.conv_cache) + (size_t)b * (kK - 1) * p.E + e;
-    const float c0 = Io::load_rw(cc);
-    const float c1 = Io::load_rw(cc + p.E);
-    const float c2 = Io::load_rw(cc + 2 * (size_t)p.E);
-    const size_t io_off = (size_t)b * p.E + e;
-    const float xt = Io::load(static_cast<const T*>(p.x) + io_off);
-    const float zt = Io::load(static_cast<const T*>(p.z) + io_off);
-    const float dr = Io::load(static_cast<const T*>(p.dt_raw) + io_off);
+    __shared__ __align__(16) unsigned char small[kStepMaxRows][kSmall][kWin];
+    __shared__ __align__(16) unsigned char bcs[kStepMaxRows][2][kN * S];
+    __shared__ float4 ring[kStepStages][kStepThreads];
 
-    const float4 w = __ldg(reinterpret_cast<const float4*>(p.conv_w) + e);
-    float xc = fmaf(w.x, c0, __ldg(p.conv_b + e));
-    xc = fmaf(w.y, c1, xc);
-    xc = fmaf(w.z, c2, xc);
-    xc = fmaf(w.w, xt, xc);
-    const float u = silu(xc);
-    const float dt = dt_from_raw(dr + __ldg(p.dt_bias + e));
-    const float dtu = dt * u;
-
-    // this lane's four states and their B, C, A entries
-    float Bv[4], Cv[4], A2[4];
+    {   // (1) every row's small inputs and B/C rows, 16-byte pieces
+        constexpr int kPw = kWin / 16, kPb = kN * S / 16;
+        constexpr int kPer = kSmall * kPw + 2 * kPb;   // pieces per row
+        const size_t row_bytes = (size_t)p.E * S;
+        for (int i = tid; i < nb * kPer; i += kStepThreads) {
+            const int j = i / kPer, t = i - j * kPer, b = b0 + j;
+            if (t < kSmall * kPw) {
+                const int k = t / kPw, pc = t - k * kPw;
+                const size_t col = (size_t)e0 * S + (size_t)pc * 16;
+                const bool ok = col + 16 <= row_bytes;           // E*S is a multiple of 16
+                const unsigned char* base;
+                if (k < 3) base = static_cast<const unsigned char*>(k == 0 ? p.x : (k == 1 ? p.z : p.dt_raw)) + (size_t)b * row_bytes;
+                else base = static_cast<const unsigned char*>(p.conv_cache) + ((size_t)b * (kK - 1) + (k - 3)) * row_bytes;
+                step_cp_async16(&small[j][k][pc * 16], ok ? base + col : static_cast<const void*>(p.x), ok);
+            } else {
+                const int u = t - kSmall * kPw, w2 = u / kPb, pc = u - w2 * kPb;
+                const unsigned char* base = static_cast<const unsigned char*>(w2 ? p.Cm : p.Bm) + (size_t)b * kN * S;
+                step_cp_async16(&bcs[j][w2][pc * 16], base + pc * 16, true);
+            }
+        }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    }
+    auto issue = [&](int j) {   // (2) row j's state piece -> this lane's ring slot
+        step_cp_async16(&ring[j % kStepStages][tid],
+                        reinterpret_cast<const float4*>(p.ssm_state + ((size_t)(b0 + j) * p.E + ec) * kN) + q, true);
+    };
+#pragma unroll
+    for (int j = 0; j < kStepStages - 1; ++j) {
+        if (j < nb) issue(j);
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    }
+    const float4 w = __ldg(reinterpret_cast<const float4*>(p.conv_w) + ec);
+    const float cb = __ldg(p.conv_b + ec);
+    const float db = __ldg(p.dt_bias + ec);
+    const float Dv = __ldg(p.D + ec);
+    float A2[4];
     {
-        const float4 al = __ldg(reinterpret_cast<const float4*>(p.A_log + (size_t)e * kN) + q);
-        A2[0] = -expf(al.x) * kLog2e; A2[1] = -expf(al.y) * kLog2e;
-        A2[2] = -expf(al.z) * kLog2e; A2[3] = -expf(al.w) * kLog2e;
-        const T* Bs = static_cast<const T*>(p.Bm) + (size_t)b * kN + 4 * q;
-        const T* Cs = static_cast<const T*>(p.Cm) + (size_t)b * kN + 4 * q;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) { Bv[j] = Io::load(Bs + j); Cv[j] = Io::load(Cs + j); }
+        // exp(dt*A) = 2^(dt * A2) with A2 = A log2 e, A = -exp(A_log) = -2^(A_log log2 e)
+        const float4 a4 = __ldg(reinterpret_cast<const float4*>(p.A_log + (size_t)ec * kN) + q);
+        A2[0] = -ex2_approx(a4.x * kLog2e) * kLog2e;
+        A2[1] = -ex2_approx(a4.y * kLog2e) * kLog2e;
+        A2[2] = -ex2_approx(a4.z * kLog2e) * kLog2e;
+        A2[3] = -ex2_approx(a4.w * kLog2e) * kLog2e;
     }
-    float4* sp = reinterpret_cast<float4*>(p.ssm_state + ((size_t)b * p.E + e) * kN) + q;
-    float4 hv = *sp;
-    float h[4] = {hv.x, hv.y, hv.z, hv.w};
-    float acc = 0.0f;
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(kStepStages - 1) : "memory");   // (1) landed
+    __syncthreads();
+
+    const int co = (ec - e0) * S;                     // this channel's byte offset in a window
+#pragma unroll 1
+    for (int j = 0; j < nb; ++j) {
+        const int b = b0 + j;
+        if (j + kStepStages - 1 < nb) issue(j + kStepStages - 1);
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+        asm volatile("cp.async.wait_group %0;\n" ::"n"(kStepStages - 1) : "memory");   // row j landed
+
+        const float x_t = Io::sload(&small[j][0][co]);
+        const float c0 = Io::sload(&small[j][3][co]);
+        const float c1 = Io::sload(&small[j][4][co]);
+        const float c2 = Io::sload(&small[j][5][co]);
+        float xc = fmaf(w.x, c0, cb);
+        xc = fmaf(w.y, c1, xc);
+        xc = fmaf(w.z, c2, xc);
+        xc = fmaf(w.w, x_t, xc);
+        const float u = silu(xc);
+        const float dt = dt_from_raw(Io::sload(&small[j][2][co]) + db);
+        const float dtu = dt * u;
+        float Bq[4], Cq[4];
+        Io::sload4(&bcs[j][0][4 * q * S], Bq);
+        Io::sload4(&bcs[j][1][4 * q * S], Cq);
+        const float4 hq = ring[j % kStepStages][tid];
+        float h[4] = {hq.x, hq.y, hq.z, hq.w};
+        float acc = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float a = ex2_approx(dt * A2[j]);
-        h[j] = fmaf(a, h[j], dtu * Bv[j]);
-        acc = fmaf(Cv[j], h[j], acc);
-    }
-    if (valid) *sp = make_float4(h[0], h[1], h[2], h[3]);
-    // sum over the four lanes of this channel (lanes 4c .. 4c+3 of the warp)
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (valid && q == 0) {
-        const float yv = fmaf(__ldg(p.D + e), u, acc) * silu(zt);
-        Io::store(static_cast<T*>(p.y) + io_off, yv);
-        // shift the cache: drop the oldest input, append x_t (exact copies)
-        Io::store(cc, c1);
-        Io::store(cc + p.E, c2);
-        Io::store(cc + 2 * (size_t)p.E, xt);
+        for (int i = 0; i < 4; ++i) {
+            h[i] = fmaf(ex2_approx(dt * A2[i]), h[i], dtu * Bq[i]);
+            acc = fmaf(Cq[i], h[i], acc);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        if (live) {
+            const size_t ch = (size_t)b * p.E + e;
+            reinterpret_cast<float4*>(p.ssm_state + ch * kN)[q] = make_float4(h[0], h[1], h[2], h[3]);
+            if (q == 0) {
+                Io::store(static_cast<T*>(p.y) + ch, fmaf(Dv, u, acc) * silu(Io::sload(&small[j][1][co])));
+                // shift the cache: drop the oldest input, append x_t (exact copies of the raw bits)
+                T* cc = static_cast<T*>(p.conv_cache) + (size_t)b * (kK - 1) * p.E + e;
+                cc[0] = *reinterpret_cast<const T*>(&small[j][4][co]);
+                cc[p.E] = *reinterpret_cast<const T*>(&small[j][5][co]);
+                cc[2 * (size_t)p.E] = *reinterpret_cast<const T*>(&small[j][0][co]);
+            }
+        }
     }
 }
 
