@@ -146,6 +146,20 @@ template <> struct SmemIo<IoBF16> {
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
+// Walks the flat indices w = tid, tid + NT, ... of a (rows x per_row) grid of
+// copy pieces as (row, piece) pairs without a division per step: the stride NT
+// is split once into whole rows (drow) and a remainder (dpc).
+struct PieceWalk {
+    int row, pc, drow, dpc, per_row;
+    __device__ __forceinline__ PieceWalk(int tid, int NT, int per_row_)
+        : row(tid / per_row_), pc(tid % per_row_), drow(NT / per_row_), dpc(NT % per_row_), per_row(per_row_) {}
+    __device__ __forceinline__ void next() {
+        row += drow;
+        pc += dpc;
+        if (pc >= per_row) { pc -= per_row; ++row; }
+    }
+};
+
 template <class Io, int W, int R, int kMinBlocks = 1>
 __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkParams p) {
     static_assert(R % 4 == 0 && (R & (R - 1)) == 0, "R: power of two, multiple of 4");
@@ -187,10 +201,8 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
     auto prefetch = [&](int k, int st) {
         const int t0 = k * kT;
         unsigned char* sb = smem + st * lay.stage;
-        const int nx = (kT + kK - 1) * nch;
-        for (int w = tid; w < nx; w += NT) {
-            const int row = w / nch;
-            const int ch = w - row * nch;
+        for (PieceWalk it(tid, NT, nch); it.row < kT + kK - 1; it.next()) {
+            const int row = it.row, ch = it.pc;
             const int t = t0 - (kK - 1) + row;
             const void* src = xg;
             bool ok = false;
@@ -203,10 +215,8 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
             }
             cp_async16(sb + lay.xs + row_off<R>(row, pitch) + ch * 16, src, ok);
         }
-        const int nz = kT * nch;
-        for (int w = tid; w < nz; w += NT) {
-            const int row = w / nch;
-            const int ch = w - row * nch;
+        for (PieceWalk it(tid, NT, nch); it.row < kT; it.next()) {
+            const int row = it.row, ch = it.pc;
             const int t = t0 + row;
             const bool ok = t < p.L;
             const size_t go = ok ? ((size_t)b * p.L + t) * row_bytes + wb0 + ch * 16 : 0;
@@ -439,12 +449,10 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
         {
             const int lo = e0 * S, hi = (e0 + ne) * S;
             unsigned char* yg = static_cast<unsigned char*>(p.y);
-            const int nyw = kT * nch;
-            for (int w = tid; w < nyw; w += NT) {
-                const int row = w / nch;
-                const int ch = w - row * nch;
+            for (PieceWalk it(tid, NT, nch); it.row < kT; it.next()) {
+                const int row = it.row, ch = it.pc;
                 const int t = t0 + row;
-                if (t >= p.L) continue;
+                if (t >= p.L) break;          // rows only grow along the walk
                 const int gb = wb0 + ch * 16;
                 unsigned char* gp = yg + ((size_t)b * p.L + t) * row_bytes + gb;
                 const unsigned char* sp = yb + row_off<R>(row, pitch) + ch * 16;
