@@ -52,8 +52,8 @@ constexpr int kStepMaxRows = 32;   // batch rows per block
 //  - every lane streams its state pieces through a private kStepStages-deep
 //    shared-memory ring with cp.async (a lane reads back only its own copies);
 //  - A = -exp(A_log) is formed once per lane.
-// The conv/SiLU/dt prologue is recomputed by the four lanes of a channel
-// (cheaper than broadcasting it); C . h is finished with two shuffles.
+// The conv/SiLU/dt prologue of four consecutive rows is spread over the four
+// lanes of a channel; C . h is finished with two shuffles.
 template <class Io>
 __global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int rows) {
     using T = typename Io::T;
@@ -124,47 +124,59 @@ __global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int ro
     __syncthreads();
 
     const int co = (ec - e0) * S;                     // this channel's byte offset in a window
+    // Rows go in rounds of four: lane q computes the conv / SiLU / dt prologue
+    // and SiLU(z) of row j0+q only; each row's dt and dt*u reach the other
+    // three lanes of the channel by shuffles, and the row's owner lane writes
+    // y and the shifted cache.
 #pragma unroll 1
-    for (int j = 0; j < nb; ++j) {
-        const int b = b0 + j;
-        if (j + kStepStages - 1 < nb) issue(j + kStepStages - 1);
-        asm volatile("cp.async.commit_group;\n" ::: "memory");
-        asm volatile("cp.async.wait_group %0;\n" ::"n"(kStepStages - 1) : "memory");   // row j landed
-
-        const float x_t = Io::sload(&small[j][0][co]);
-        const float c0 = Io::sload(&small[j][3][co]);
-        const float c1 = Io::sload(&small[j][4][co]);
-        const float c2 = Io::sload(&small[j][5][co]);
-        float xc = fmaf(w.x, c0, cb);
-        xc = fmaf(w.y, c1, xc);
-        xc = fmaf(w.z, c2, xc);
-        xc = fmaf(w.w, x_t, xc);
-        const float u = silu(xc);
-        const float dt = dt_from_raw(Io::sload(&small[j][2][co]) + db);
-        const float dtu = dt * u;
-        float Bq[4], Cq[4];
-        Io::sload4(&bcs[j][0][4 * q * S], Bq);
-        Io::sload4(&bcs[j][1][4 * q * S], Cq);
-        const float4 hq = ring[j % kStepStages][tid];
-        float h[4] = {hq.x, hq.y, hq.z, hq.w};
-        float acc = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            h[i] = fmaf(ex2_approx(dt * A2[i]), h[i], dtu * Bq[i]);
-            acc = fmaf(Cq[i], h[i], acc);
+    for (int j0 = 0; j0 < nb; j0 += 4) {
+        const int jq = min(j0 + q, nb - 1);
+        float uq, dtq, dtuq, gzq;
+        {
+            const float x_t = Io::sload(&small[jq][0][co]);
+            float xc = fmaf(w.x, Io::sload(&small[jq][3][co]), cb);
+            xc = fmaf(w.y, Io::sload(&small[jq][4][co]), xc);
+            xc = fmaf(w.z, Io::sload(&small[jq][5][co]), xc);
+            xc = fmaf(w.w, x_t, xc);
+            uq = silu(xc);
+            dtq = dt_from_raw(Io::sload(&small[jq][2][co]) + db);
+            dtuq = dtq * uq;
+            gzq = silu(Io::sload(&small[jq][1][co]));
         }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        if (live) {
-            const size_t ch = (size_t)b * p.E + e;
-            reinterpret_cast<float4*>(p.ssm_state + ch * kN)[q] = make_float4(h[0], h[1], h[2], h[3]);
-            if (q == 0) {
-                Io::store(static_cast<T*>(p.y) + ch, fmaf(Dv, u, acc) * silu(Io::sload(&small[j][1][co])));
-                // shift the cache: drop the oldest input, append x_t (exact copies of the raw bits)
-                T* cc = static_cast<T*>(p.conv_cache) + (size_t)b * (kK - 1) * p.E + e;
-                cc[0] = *reinterpret_cast<const T*>(&small[j][4][co]);
-                cc[p.E] = *reinterpret_cast<const T*>(&small[j][5][co]);
-                cc[2 * (size_t)p.E] = *reinterpret_cast<const T*>(&small[j][0][co]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int j = j0 + k;
+            if (j >= nb) break;                           // block-uniform
+            const int b = b0 + j;
+            if (j + kStepStages - 1 < nb) issue(j + kStepStages - 1);
+            asm volatile("cp.async.commit_group;\n" ::: "memory");
+            asm volatile("cp.async.wait_group %0;\n" ::"n"(kStepStages - 1) : "memory");   // row j landed
+            const float dt = __shfl_sync(0xffffffffu, dtq, k, 4);
+            const float dtu = __shfl_sync(0xffffffffu, dtuq, k, 4);
+            float Bq[4], Cq[4];
+            Io::sload4(&bcs[j][0][4 * q * S], Bq);
+            Io::sload4(&bcs[j][1][4 * q * S], Cq);
+            const float4 hq = ring[j % kStepStages][tid];
+            float h[4] = {hq.x, hq.y, hq.z, hq.w};
+            float acc = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                h[i] = fmaf(ex2_approx(dt * A2[i]), h[i], dtu * Bq[i]);
+                acc = fmaf(Cq[i], h[i], acc);
+            }
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (live) {
+                const size_t ch = (size_t)b * p.E + e;
+                reinterpret_cast<float4*>(p.ssm_state + ch * kN)[q] = make_float4(h[0], h[1], h[2], h[3]);
+                if (q == k) {
+                    Io::store(static_cast<T*>(p.y) + ch, fmaf(Dv, uq, acc) * gzq);
+                    // shift the cache: drop the oldest input, append x_t (exact copies of the raw bits)
+                    T* cc = static_cast<T*>(p.conv_cache) + (size_t)b * (kK - 1) * p.E + e;
+                    cc[0] = *reinterpret_cast<const T*>(&small[j][4][co]);
+                    cc[p.E] = *reinterpret_cast<const T*>(&small[j][5][co]);
+                    cc[2 * (size_t)p.E] = *reinterpret_cast<const T*>(&small[j][0][co]);
+                }
             }
         }
     }
