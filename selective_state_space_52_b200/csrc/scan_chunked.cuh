@@ -112,6 +112,7 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src,
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
 // io-typed shared-memory access by byte address
 template <class Io> struct SmemIo;
@@ -274,23 +275,13 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
 
     const int nck = (p.L + kT - 1) / kT;
     const int i0 = r * R;                 // first item of this run within a chunk
-    prefetch(0, 0);
-    cp_async_commit();
 
-    for (int k = 0; k < nck; ++k) {
-        const int st = k & 1;
-        if (k + 1 < nck) prefetch(k + 1, st ^ 1);
-        cp_async_commit();
-        cp_async_wait_1();
-        __syncthreads();
-        const unsigned char* sb = smem + st * lay.stage;
-        const int t0 = k * kT;
-
-        // ---- B, C to float32, once per chunk for the whole tile
+    // ---- B, C of a staged chunk to float32, once per chunk for the whole tile
+    auto convert_bc = [&](const unsigned char* sbc) {
         for (int w = tid; w < 4 * kT; w += NT) {
             const int t = w % kT;
             const int q = w / kT;                          // 0,1: B halves; 2,3: C halves
-            const unsigned char* src = sb + (q < 2 ? lay.bs : lay.cs) + t * (kN * S) + (q & 1) * 8 * S;
+            const unsigned char* src = sbc + (q < 2 ? lay.bs : lay.cs) + t * (kN * S) + (q & 1) * 8 * S;
             float v[8];
             SI::ld8(src, v);
             float* dst = q < 2 ? bf : cf;
@@ -303,7 +294,25 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
                 for (int m = 0; m < 8; ++m) dst[((q & 1) * 8 + m) * tpad + t + (t / R) * 4] = v[m];
             }
         }
-        __syncthreads();
+    };
+
+    prefetch(0, 0);
+    cp_async_commit();
+    cp_async_wait_0();
+    __syncthreads();
+    convert_bc(smem);
+
+    // Two barriers per chunk: (a) at the top, publishing the float B/C of this
+    // chunk; (b) at the end, after which every thread is done reading this
+    // chunk's stage and float B/C and the next chunk's copies have landed, so
+    // the y tile can be stored and the next chunk's B/C converted.
+    for (int k = 0; k < nck; ++k) {
+        const int st = k & 1;
+        if (k + 1 < nck) prefetch(k + 1, st ^ 1);
+        cp_async_commit();
+        __syncthreads();                                   // (a)
+        const unsigned char* sb = smem + st * lay.stage;
+        const int t0 = k * kT;
 
         unsigned char* yb = smem + lay.ys;
         if constexpr (W == 1) {
@@ -444,7 +453,8 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
                 SI::st(yb + row_off<R>(i0 + i, pitch) + coff, yy * silu(zt));
             }
         }
-        __syncthreads();
+        cp_async_wait_0();                                 // this thread's copies of chunk k+1
+        __syncthreads();                                   // (b)
         // ---- write the y tile: 16-byte stores inside the tile, narrow ones at its edges
         {
             const int lo = e0 * S, hi = (e0 + ne) * S;
@@ -465,6 +475,7 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
                 }
             }
         }
+        if (k + 1 < nck) convert_bc(smem + (st ^ 1) * lay.stage);
     }
 
     // ---- final caches
