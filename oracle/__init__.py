@@ -53,7 +53,10 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
+            # AXON_ORACLE_LIB points the pins at another build of this source
+            # (the mutation tests plant mistakes in copies of it).
+            path = os.environ.get("AXON_ORACLE_LIB") or build()
+            lib = ctypes.CDLL(path)
             lib.oracle_silu.restype = ctypes.c_double
             lib.oracle_silu.argtypes = [ctypes.c_double]
             lib.oracle_dt.restype = ctypes.c_double

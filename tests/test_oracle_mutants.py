@@ -1,0 +1,65 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a copy of oracle/axon_ssm_oracle.c (a dropped
+term, a wrong sign, a swapped operand, an index off by one, a reversed
+order), builds it, and runs tests/test_oracle_pins.py against that build: at
+least one pin must fail.  The real source is never modified.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "axon_ssm_oracle.c")
+
+MUTANTS = {
+    "dropped_D_skip": ("double y_ssm = acc + D[e] * u;", "double y_ssm = acc;"),
+    "A_sign": ("A[n] = -exp(A_log[(size_t)e * N + n]);", "A[n] = exp(A_log[(size_t)e * N + n]);"),
+    "C_replaced_by_B": ("acc += Cm[bn] * h[n];", "acc += Bm[bn] * h[n];"),
+    "conv_taps_reversed": ("xc += conv_w[(size_t)e * K + k] * xpad[t + k];",
+                           "xc += conv_w[(size_t)e * K + (K - 1 - k)] * xpad[t + k];"),
+    "dt_lower_clip": ("#define ORACLE_DT_MIN 1e-4", "#define ORACLE_DT_MIN 1e-3"),
+    "dt_upper_clip": ("#define ORACLE_DT_MAX 100.0", "#define ORACLE_DT_MAX 10.0"),
+    "B_time_index_shift": ("size_t bn = ((size_t)b * L + t) * N + n;",
+                           "size_t bn = ((size_t)b * L + (t > 0 ? t - 1 : 0)) * N + n;"),
+    "gate_without_silu": ("y[idx] = y_ssm * oracle_silu(z[idx]);", "y[idx] = y_ssm * z[idx];"),
+    "softplus_without_log1p": ("return log1p(exp(v));", "return exp(v);"),
+    "cache_order_reversed": ("conv_cache_out[((size_t)b * KM1 + j) * E + e] = xpad[L + j];",
+                             "conv_cache_out[((size_t)b * KM1 + j) * E + e] = xpad[L + KM1 - 1 - j];"),
+    "input_before_decay": ("h[n] = abar * h[n] + bbar * u;", "h[n] = abar * (h[n] + bbar * u);"),
+    "silu_as_sigmoid": ("double oracle_silu(double v) { return v / (1.0 + exp(-v)); }",
+                        "double oracle_silu(double v) { return 1.0 / (1.0 + exp(-v)); }"),
+    "zoh_missing_A_division": ("double bbar = zoh ? expm1(dt * A[n]) / A[n] * Bm[bn] : dt * Bm[bn];",
+                               "double bbar = zoh ? expm1(dt * A[n]) * Bm[bn] : dt * Bm[bn];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor for {name} not found in the oracle source"
+    mutated = tmp_path / "oracle_mutant.c"
+    mutated.write_text(src.replace(old, new))
+    lib = tmp_path / "liboracle_mutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fno-fast-math",
+                    "-ffp-contract=off", "-o", str(lib), str(mutated), "-lm"], check=True)
+    env = dict(os.environ, AXON_ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"no pin failed for the planted mistake {name}:\n{r.stdout[-2000:]}"
+    assert "failed" in r.stdout
+
+
+def test_unmutated_oracle_passes_the_pins(tmp_path):
+    lib = tmp_path / "liboracle_copy.so"
+    subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fno-fast-math",
+                    "-ffp-contract=off", "-o", str(lib), SRC, "-lm"], check=True)
+    env = dict(os.environ, AXON_ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:]
