@@ -334,6 +334,30 @@ def bench_decode(dev, steps: int = 512, distinct: int = 8) -> dict:
             "token_ch_per_s_warm": wl.B * wl.E / (warm_ms / 1e3) / 1e9}
 
 
+def bench_zoh_prefill(wl, sets, params, out, ws, dev, launches: int = 20) -> dict:
+    """The same prefill with the exact zero-order-hold discretisation (the
+    Axon-SSM page's ZOH form): mean event time of `launches` prefill calls."""
+    from selective_state_space_52_b200 import axon_ssm
+    stream = torch.cuda.current_stream(dev)
+    n_sets = len(sets)
+
+    def run(i):
+        s = sets[i % n_sets]
+        axon_ssm.scan_fwd(s["x"], s["z"], s["dt_raw"], s["B"], s["C"], params, None, out=out,
+                          workspace=ws, discretization="zoh")
+
+    for i in range(3):
+        run(i)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(launches)]
+    torch.cuda.synchronize(dev)
+    for i, (a, b) in enumerate(ev):
+        a.record(stream); run(i); b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    T = wl.B * wl.L * wl.E
+    return {"kernel_ms": ms, "value": T / (ms / 1e3) / 1e9, "unit": UNIT, "launches": launches}
+
+
 def workload_desc(wl) -> str:
     return (f"{wl.name}: B{wl.B} L{wl.L} E{wl.E} N{wl.N} K{wl.K}, {wl.io} io, fp32 state; "
             "step = prefill + 1 cached decode token")
@@ -489,6 +513,7 @@ def run_axon(args, wl):
 
     if not args.no_decode_bench:
         line["decode"] = bench_decode(dev)
+        line["prefill_zoh"] = bench_zoh_prefill(wl, sets, params, (y, cc, ss), ws, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inp_cpu = {**params_cpu, **{k: v.cpu() for k, v in sets[0].items()}}
         rate, units, secs, ch = time_oracle(wl, inp_cpu, args.cpu_budget)

@@ -82,6 +82,12 @@ typedef enum {
     AXON_BF16 = 1
 } axon_dtype;
 
+/* Discretisation of B (Axon-SSM page, section "ZOH discretisation"). */
+typedef enum {
+    AXON_DISC_FIRST_ORDER = 0,  /* Bbar = dt * B: the form Axon-SSM uses (default) */
+    AXON_DISC_ZOH = 1           /* Bbar = (exp(dt*A) - 1) / A * B: exact zero-order hold */
+} axon_discretization;
+
 typedef enum {
     AXON_OK = 0,
     AXON_ERR_INVALID_ARG = 1,   /* negative size, NULL required pointer, bad aliasing */
@@ -223,6 +229,25 @@ AXON_API axon_status axon_ssm_scan_fwd_noalloc(
     int num_segments, axon_stream_t stream);
 
 /*
+ * axon_ssm_scan_fwd_segments with a choice of discretisation: `disc` selects
+ * the first-order Bbar = dt*B (AXON_DISC_FIRST_ORDER, what every other entry
+ * point uses) or the exact zero-order hold Bbar = (exp(dt*A) - 1)/A * B
+ * (AXON_DISC_ZOH) of the Axon-SSM page's "ZOH discretisation" section.  The
+ * decay exp(dt*A) is the same in both.  An unknown `disc` returns
+ * AXON_ERR_UNSUPPORTED; all other arguments and errors are those of
+ * axon_ssm_scan_fwd_segments (num_segments == 0: the library's plan).
+ */
+AXON_API axon_status axon_ssm_scan_fwd_ex(
+    int B, int L, int E, int N, int K, axon_dtype io, axon_discretization disc,
+    const void *x, const void *z, const void *dt_raw,
+    const void *Bm, const void *Cm,
+    const float *conv_w, const float *conv_b,
+    const float *dt_bias, const float *A_log, const float *D,
+    const void *conv_cache_in, const float *ssm_state_in,
+    void *y, void *conv_cache_out, float *ssm_state_out,
+    void *workspace, size_t workspace_bytes, int num_segments, axon_stream_t stream);
+
+/*
  * Cached single-token decode (section "Autoregressive decoding"): one step of
  * the layer core for B sequences, caches updated in place.
  *
@@ -238,6 +263,18 @@ AXON_API axon_status axon_ssm_scan_fwd_noalloc(
  */
 AXON_API axon_status axon_ssm_step(
     int B, int E, int N, int K, axon_dtype io,
+    const void *x, const void *z, const void *dt_raw,
+    const void *Bm, const void *Cm,
+    const float *conv_w, const float *conv_b,
+    const float *dt_bias, const float *A_log, const float *D,
+    void *conv_cache, float *ssm_state, void *y, axon_stream_t stream);
+
+/*
+ * axon_ssm_step with a choice of discretisation (see axon_ssm_scan_fwd_ex).
+ * A decode that continues a prefill must use the same `disc` as the prefill.
+ */
+AXON_API axon_status axon_ssm_step_ex(
+    int B, int E, int N, int K, axon_dtype io, axon_discretization disc,
     const void *x, const void *z, const void *dt_raw,
     const void *Bm, const void *Cm,
     const float *conv_w, const float *conv_b,

@@ -53,6 +53,13 @@ _lib.axon_ssm_scan_fwd_segments.argtypes = _SCAN_ARGS + [_i, _vp]
 _lib.axon_ssm_scan_fwd_noalloc.restype = _i
 _lib.axon_ssm_scan_fwd_noalloc.argtypes = [_i] * 6 + [_vp] * 15 + [_i, _vp]
 NOALLOC_SCRATCH_BYTES = 16 << 20
+_lib.axon_ssm_scan_fwd_ex.restype = _i
+_lib.axon_ssm_scan_fwd_ex.argtypes = [_i] * 7 + [_vp] * 15 + [_vp, _sz, _i, _vp]
+_lib.axon_ssm_step_ex.restype = _i
+_lib.axon_ssm_step_ex.argtypes = [_i] * 6 + [_vp] * 13 + [_vp]
+AXON_DISC_FIRST_ORDER = 0
+AXON_DISC_ZOH = 1
+_DISC = {"first_order": AXON_DISC_FIRST_ORDER, "zoh": AXON_DISC_ZOH}
 _lib.axon_ssm_step.restype = _i
 _lib.axon_ssm_step.argtypes = [_i] * 5 + [_vp] * 13 + [_vp]
 
@@ -158,6 +165,30 @@ def axon_ssm_scan_fwd_noalloc(B, L, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, c
     return rc
 
 
+def axon_ssm_scan_fwd_ex(B, L, E, N, K, io, disc, x, z, dt_raw, Bm, Cm, conv_w, conv_b,
+                         dt_bias, A_log, D, conv_cache_in, ssm_state_in, y, conv_cache_out,
+                         ssm_state_out, workspace, workspace_bytes, num_segments=0, stream=None, *,
+                         raise_on_error=True) -> int:
+    rc = _lib.axon_ssm_scan_fwd_ex(B, L, E, N, K, io, int(disc), _p(x), _p(z), _p(dt_raw),
+                                   _p(Bm), _p(Cm), _p(conv_w), _p(conv_b), _p(dt_bias),
+                                   _p(A_log), _p(D), _p(conv_cache_in), _p(ssm_state_in), _p(y),
+                                   _p(conv_cache_out), _p(ssm_state_out), _p(workspace),
+                                   int(workspace_bytes), int(num_segments), _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_ssm_scan_fwd_ex")
+    return rc
+
+
+def axon_ssm_step_ex(B, E, N, K, io, disc, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias,
+                     A_log, D, conv_cache, ssm_state, y, stream=None, *, raise_on_error=True) -> int:
+    rc = _lib.axon_ssm_step_ex(B, E, N, K, io, int(disc), _p(x), _p(z), _p(dt_raw), _p(Bm),
+                               _p(Cm), _p(conv_w), _p(conv_b), _p(dt_bias), _p(A_log), _p(D),
+                               _p(conv_cache), _p(ssm_state), _p(y), _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_ssm_step_ex")
+    return rc
+
+
 def axon_ssm_step(B, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
                   conv_cache, ssm_state, y, stream=None, *, raise_on_error=True) -> int:
     rc = _lib.axon_ssm_step(B, E, N, K, io, _p(x), _p(z), _p(dt_raw), _p(Bm), _p(Cm),
@@ -173,7 +204,7 @@ PARAM_KEYS = ("conv_w", "conv_b", "dt_bias", "A_log", "D")
 
 
 def scan_fwd(x, z, dt_raw, Bm, Cm, params: dict, cache=None, *, num_segments=None,
-             out=None, workspace=None, stream=None):
+             out=None, workspace=None, stream=None, discretization="first_order"):
     """Prefill over (B, L, E) inputs on the GPU.
 
     ``params`` holds conv_w, conv_b, dt_bias, A_log, D (float32, on the device);
@@ -202,14 +233,18 @@ def scan_fwd(x, z, dt_raw, Bm, Cm, params: dict, cache=None, *, num_segments=Non
     wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
     args = (Bsz, L, E, N, K, io, x, z, dt_raw, Bm, Cm, *(params[k] for k in PARAM_KEYS),
             cc_in, ss_in, y, cc_out, ss_out, workspace, wsz)
-    if num_segments is None:
+    if discretization != "first_order":
+        axon_ssm_scan_fwd_ex(Bsz, L, E, N, K, io, _DISC[discretization], *args[6:],
+                             num_segments or 0, stream=stream)
+    elif num_segments is None:
         axon_ssm_scan_fwd(*args, stream=stream)
     else:
         axon_ssm_scan_fwd_segments(*args, num_segments, stream=stream)
     return y, (cc_out, ss_out)
 
 
-def step(x, z, dt_raw, Bm, Cm, params: dict, cache, *, y=None, stream=None):
+def step(x, z, dt_raw, Bm, Cm, params: dict, cache, *, y=None, stream=None,
+         discretization="first_order"):
     """One cached decode step; ``cache = (conv_cache, ssm_state)`` is updated in place."""
     Bsz, E = x.shape
     K = params["conv_w"].shape[1]
@@ -217,6 +252,10 @@ def step(x, z, dt_raw, Bm, Cm, params: dict, cache, *, y=None, stream=None):
     conv_cache, ssm_state = cache
     if y is None:
         y = torch.empty_like(x)
-    axon_ssm_step(Bsz, E, N, K, _dtype_code(x.dtype), x, z, dt_raw, Bm, Cm,
-                  *(params[k] for k in PARAM_KEYS), conv_cache, ssm_state, y, stream=stream)
+    args = (x, z, dt_raw, Bm, Cm, *(params[k] for k in PARAM_KEYS), conv_cache, ssm_state, y)
+    if discretization != "first_order":
+        axon_ssm_step_ex(Bsz, E, N, K, _dtype_code(x.dtype), _DISC[discretization], *args,
+                         stream=stream)
+    else:
+        axon_ssm_step(Bsz, E, N, K, _dtype_code(x.dtype), *args, stream=stream)
     return y

@@ -134,9 +134,9 @@ bool plan_chunked(int B, int E, int io_bytes, int sms, int max_smem, ChunkPlan* 
     return true;
 }
 
-template <class Io, int W, int R>
+template <class Io, int W, int R, bool Z>
 axon_status launch_chunked_t(const ChunkParams& prm, int smem, cudaStream_t st) {
-    auto kern = scan_chunked_kernel<Io, W, R>;
+    auto kern = scan_chunked_kernel<Io, W, R, Z>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return AXON_ERR_CUDA;
     const unsigned grid = (unsigned)((long long)prm.B * prm.tiles_per_b);
@@ -144,22 +144,22 @@ axon_status launch_chunked_t(const ChunkParams& prm, int smem, cudaStream_t st) 
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
 
-template <class Io>
+template <class Io, bool Z>
 axon_status launch_chunked(const ChunkParams& prm, const ChunkPlan& c, cudaStream_t st) {
     switch (c.W * 100 + c.R) {
-        case 116: return launch_chunked_t<Io, 1, 16>(prm, c.smem, st);
-        case 216: return launch_chunked_t<Io, 2, 16>(prm, c.smem, st);
-        case 416: return launch_chunked_t<Io, 4, 16>(prm, c.smem, st);
-        case 808: return launch_chunked_t<Io, 8, 8>(prm, c.smem, st);
-        case 816: return launch_chunked_t<Io, 8, 16>(prm, c.smem, st);
-        case 1608: return launch_chunked_t<Io, 16, 8>(prm, c.smem, st);
-        case 1616: return launch_chunked_t<Io, 16, 16>(prm, c.smem, st);
-        case 3208: return launch_chunked_t<Io, 32, 8>(prm, c.smem, st);
+        case 116: return launch_chunked_t<Io, 1, 16, Z>(prm, c.smem, st);
+        case 216: return launch_chunked_t<Io, 2, 16, Z>(prm, c.smem, st);
+        case 416: return launch_chunked_t<Io, 4, 16, Z>(prm, c.smem, st);
+        case 808: return launch_chunked_t<Io, 8, 8, Z>(prm, c.smem, st);
+        case 816: return launch_chunked_t<Io, 8, 16, Z>(prm, c.smem, st);
+        case 1608: return launch_chunked_t<Io, 16, 8, Z>(prm, c.smem, st);
+        case 1616: return launch_chunked_t<Io, 16, 16, Z>(prm, c.smem, st);
+        case 3208: return launch_chunked_t<Io, 32, 8, Z>(prm, c.smem, st);
     }
     return AXON_ERR_UNSUPPORTED;
 }
 
-template <class Io>
+template <class Io, bool Z>
 axon_status launch_scan(ScanParams& prm, cudaStream_t st) {
     const dim3 block(kScanThreads);
     const unsigned gx = (unsigned)((prm.E + kScanThreads - 1) / kScanThreads);
@@ -167,9 +167,9 @@ axon_status launch_scan(ScanParams& prm, cudaStream_t st) {
         copy_state_kernel<Io><<<dim3(gx, prm.B), block, 0, st>>>(prm);
     } else {
         const unsigned gz = (unsigned)(prm.num_seg > 1 ? prm.num_seg - 1 : 1);
-        scan_seq_phase1<Io><<<dim3(gx, prm.B, gz), block, 0, st>>>(prm);
+        scan_seq_phase1<Io, Z><<<dim3(gx, prm.B, gz), block, 0, st>>>(prm);
         if (prm.num_seg > 1)
-            scan_seq_phase2<Io><<<dim3(gx, prm.B, prm.num_seg - 1), block, 0, st>>>(prm);
+            scan_seq_phase2<Io, Z><<<dim3(gx, prm.B, prm.num_seg - 1), block, 0, st>>>(prm);
     }
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
@@ -182,7 +182,7 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
                       const void* conv_cache_in, const float* ssm_state_in,
                       void* y, void* conv_cache_out, float* ssm_state_out,
                       void* workspace, size_t workspace_bytes, int num_segments,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, bool zoh = false) {
     axon_status st = check_shape(B, L, E, N, K, io);
     if (st != AXON_OK) return st;
     if (num_segments < 0) return AXON_ERR_INVALID_ARG;
@@ -259,8 +259,9 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
         cp.conv_w = conv_w; cp.conv_b = conv_b; cp.dt_bias = dt_bias; cp.A_log = A_log; cp.D = D;
         cp.conv_cache_in = conv_cache_in; cp.ssm_state_in = ssm_state_in;
         cp.y = y; cp.conv_cache_out = conv_cache_out; cp.ssm_state_out = ssm_state_out;
-        return io == AXON_BF16 ? launch_chunked<IoBF16>(cp, cplan, stream)
-                               : launch_chunked<IoF32>(cp, cplan, stream);
+        if (io == AXON_BF16) return zoh ? launch_chunked<IoBF16, true>(cp, cplan, stream)
+                                        : launch_chunked<IoBF16, false>(cp, cplan, stream);
+        return zoh ? launch_chunked<IoF32, true>(cp, cplan, stream) : launch_chunked<IoF32, false>(cp, cplan, stream);
     }
 
     ScanParams prm;
@@ -274,7 +275,8 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
     prm.ws_h = P > 1 ? static_cast<float*>(workspace) : nullptr;
     prm.ws_sdt = P > 1 ? static_cast<float*>(workspace) + (size_t)(P - 1) * B * E * kN : nullptr;
 
-    return io == AXON_BF16 ? launch_scan<IoBF16>(prm, stream) : launch_scan<IoF32>(prm, stream);
+    if (io == AXON_BF16) return zoh ? launch_scan<IoBF16, true>(prm, stream) : launch_scan<IoBF16, false>(prm, stream);
+    return zoh ? launch_scan<IoF32, true>(prm, stream) : launch_scan<IoF32, false>(prm, stream);
 }
 
 // ---- scratch for axon_ssm_scan_fwd_noalloc --------------------------------
@@ -371,12 +373,13 @@ axon_status axon_ssm_scan_fwd_segments(int B, int L, int E, int N, int K, axon_d
                      reinterpret_cast<cudaStream_t>(stream));
 }
 
-axon_status axon_ssm_step(int B, int E, int N, int K, axon_dtype io,
-                          const void* x, const void* z, const void* dt_raw,
-                          const void* Bm, const void* Cm,
-                          const float* conv_w, const float* conv_b,
-                          const float* dt_bias, const float* A_log, const float* D,
-                          void* conv_cache, float* ssm_state, void* y, axon_stream_t stream) {
+namespace {
+axon_status step_impl(int B, int E, int N, int K, axon_dtype io,
+                      const void* x, const void* z, const void* dt_raw,
+                      const void* Bm, const void* Cm,
+                      const float* conv_w, const float* conv_b,
+                      const float* dt_bias, const float* A_log, const float* D,
+                      void* conv_cache, float* ssm_state, void* y, axon_stream_t stream, bool zoh) {
     axon_status st = check_shape(B, 1, E, N, K, io);
     if (st != AXON_OK) return st;
     if (B == 0 || E == 0) return AXON_OK;
@@ -416,9 +419,53 @@ axon_status axon_ssm_step(int B, int E, int N, int K, axon_dtype io,
     while (rows < kStepMaxRows && rows < B && bx * ((B + rows - 1) / rows) > 8LL * sms) rows *= 2;
     const dim3 grid((unsigned)bx, (unsigned)((B + rows - 1) / rows));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (io == AXON_BF16) step_kernel<IoBF16><<<grid, kStepThreads, 0, s>>>(prm, rows);
-    else step_kernel<IoF32><<<grid, kStepThreads, 0, s>>>(prm, rows);
+    if (io == AXON_BF16) {
+        if (zoh) step_kernel<IoBF16, true><<<grid, kStepThreads, 0, s>>>(prm, rows);
+        else step_kernel<IoBF16, false><<<grid, kStepThreads, 0, s>>>(prm, rows);
+    } else {
+        if (zoh) step_kernel<IoF32, true><<<grid, kStepThreads, 0, s>>>(prm, rows);
+        else step_kernel<IoF32, false><<<grid, kStepThreads, 0, s>>>(prm, rows);
+    }
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+}
+}  // namespace
+
+axon_status axon_ssm_step(int B, int E, int N, int K, axon_dtype io,
+                          const void* x, const void* z, const void* dt_raw,
+                          const void* Bm, const void* Cm,
+                          const float* conv_w, const float* conv_b,
+                          const float* dt_bias, const float* A_log, const float* D,
+                          void* conv_cache, float* ssm_state, void* y, axon_stream_t stream) {
+    return step_impl(B, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
+                     conv_cache, ssm_state, y, stream, false);
+}
+
+axon_status axon_ssm_step_ex(int B, int E, int N, int K, axon_dtype io, axon_discretization disc,
+                             const void* x, const void* z, const void* dt_raw,
+                             const void* Bm, const void* Cm,
+                             const float* conv_w, const float* conv_b,
+                             const float* dt_bias, const float* A_log, const float* D,
+                             void* conv_cache, float* ssm_state, void* y, axon_stream_t stream) {
+    if (disc != AXON_DISC_FIRST_ORDER && disc != AXON_DISC_ZOH) return AXON_ERR_UNSUPPORTED;
+    return step_impl(B, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
+                     conv_cache, ssm_state, y, stream, disc == AXON_DISC_ZOH);
+}
+
+axon_status axon_ssm_scan_fwd_ex(int B, int L, int E, int N, int K, axon_dtype io,
+                                 axon_discretization disc,
+                                 const void* x, const void* z, const void* dt_raw,
+                                 const void* Bm, const void* Cm,
+                                 const float* conv_w, const float* conv_b,
+                                 const float* dt_bias, const float* A_log, const float* D,
+                                 const void* conv_cache_in, const float* ssm_state_in,
+                                 void* y, void* conv_cache_out, float* ssm_state_out,
+                                 void* workspace, size_t workspace_bytes, int num_segments,
+                                 axon_stream_t stream) {
+    if (disc != AXON_DISC_FIRST_ORDER && disc != AXON_DISC_ZOH) return AXON_ERR_UNSUPPORTED;
+    return scan_impl(B, L, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
+                     conv_cache_in, ssm_state_in, y, conv_cache_out, ssm_state_out,
+                     workspace, workspace_bytes, num_segments,
+                     reinterpret_cast<cudaStream_t>(stream), disc == AXON_DISC_ZOH);
 }
 
 axon_status axon_ssm_scan_fwd_noalloc(int B, int L, int E, int N, int K, axon_dtype io,

@@ -64,6 +64,20 @@ __device__ __forceinline__ float dt_from_raw(float v) {
     return fminf(fmaxf(softplus(v), kDtMin), kDtMax);
 }
 
+// Exact zero-order-hold input factor (Axon-SSM page, "ZOH discretisation"):
+// Bbar = (exp(dt A) - 1) / A * B.  With x = dt*A <= 0 and a = exp(x) already
+// evaluated, this returns Bbar / B = dt * phi(x), phi(x) = expm1(x) / x:
+//   |x| < 1/16: dt * (1 + x/2 + x^2/6 + x^3/24 + x^4/120)  (Taylor; the
+//               truncation x^5/720 stays below 2e-9 relative), so the
+//               cancellation in a - 1 for small |x| never enters;
+//   otherwise:  (a - 1) * (1/A), where a - 1 <= -0.06 keeps its relative error
+//               near that of a.
+__device__ __forceinline__ float zoh_bbar(float dt, float x, float a, float invA) {
+    const float series = dt * fmaf(x, fmaf(x, fmaf(x, fmaf(x, 1.0f / 120.0f, 1.0f / 24.0f), 1.0f / 6.0f), 0.5f), 1.0f);
+    const float direct = (a - 1.0f) * invA;
+    return fabsf(x) < 0.0625f ? series : direct;
+}
+
 // ---------------------------------------------------------------- io dtypes
 struct IoF32 {
     using T = float;

@@ -161,7 +161,7 @@ struct PieceWalk {
     }
 };
 
-template <class Io, int W, int R, int kMinBlocks = 1>
+template <class Io, int W, int R, bool kZoh = false, int kMinBlocks = 1>
 __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkParams p) {
     static_assert(R % 4 == 0 && (R & (R - 1)) == 0, "R: power of two, multiple of 4");
     using T = typename Io::T;
@@ -255,11 +255,13 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
     // registers (state pairs) for the direct walk, in shared memory otherwise.
     float2 s2[W == 1 ? kN / 2 : 1];
     float2 h2[W == 1 ? kN / 2 : 1];
+    float2 iA2[(W == 1 && kZoh) ? kN / 2 : 1];    // 1/A per state pair (ZOH only)
     if constexpr (W == 1) {
 #pragma unroll
         for (int q = 0; q < kN / 2; ++q) {
             s2[q] = f2(-expf(__ldg(p.A_log + (size_t)e * kN + 2 * q)) * kLog2e,
                        -expf(__ldg(p.A_log + (size_t)e * kN + 2 * q + 1)) * kLog2e);
+            if constexpr (kZoh) iA2[q] = f2(kLog2e / s2[q].x, kLog2e / s2[q].y);
             h2[q] = (p.ssm_state_in && active)
                         ? f2(p.ssm_state_in[((size_t)b * p.E + e) * kN + 2 * q],
                              p.ssm_state_in[((size_t)b * p.E + e) * kN + 2 * q + 1])
@@ -335,8 +337,9 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
                 const bool live = (t0 + i) < p.L;
                 const float dtl = live ? dt : 0.0f;     // dt = 0: decay 1, no input
                 const float2 dt2 = f2(dtl, dtl);
-                const float dtu = live ? dt * u : 0.0f;
-                const float2 dtu2 = f2(dtu, dtu);
+                // first-order: Bbar u = (dt u) B;  ZOH: Bbar u = (u zoh_bbar) B
+                const float uin = live ? (kZoh ? u : dt * u) : 0.0f;
+                const float2 dtu2 = f2(uin, uin);
                 float2 yacc = f2(Dv * u, 0.0f);
                 const float4* bq = reinterpret_cast<const float4*>(bf + i * kN);
                 const float4* cq = reinterpret_cast<const float4*>(cf + i * kN);
@@ -351,7 +354,11 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
                         const float2 a = f2(ex2_approx(arg.x), ex2_approx(arg.y));
                         const float2 bb = hh ? f2(bv.z, bv.w) : f2(bv.x, bv.y);
                         const float2 cc = hh ? f2(cv.z, cv.w) : f2(cv.x, cv.y);
-                        h2[pq] = __ffma2_rn(a, h2[pq], __fmul2_rn(dtu2, bb));
+                        float2 uin2 = dtu2;
+                        if constexpr (kZoh)
+                            uin2 = __fmul2_rn(dtu2, f2(zoh_bbar(dtl, arg.x * kLn2, a.x, iA2[pq].x),
+                                                       zoh_bbar(dtl, arg.y * kLn2, a.y, iA2[pq].y)));
+                        h2[pq] = __ffma2_rn(a, h2[pq], __fmul2_rn(uin2, bb));
                         yacc = __ffma2_rn(cc, h2[pq], yacc);
                     }
                 }
@@ -379,7 +386,7 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
                     const float dt = dt_from_raw(dr + db);
                     const bool live = (t0 + i0 + i) < p.L;
                     const float dtl = live ? dt : 0.0f;
-                    const float dtul = live ? dt * u : 0.0f;
+                    const float dtul = live ? (kZoh ? u : dt * u) : 0.0f;   // input factor of Bbar u
                     if (i & 1) { dtv[i / 2].y = dtl; dtu[i / 2].y = dtul; yv[i / 2].y = Dv * u; }
                     else       { dtv[i / 2].x = dtl; dtu[i / 2].x = dtul; yv[i / 2].x = Dv * u; }
                 }
@@ -390,6 +397,7 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
             for (int n = 0; n < kN; ++n) {
                 const float s = a2s[n * ET + c];
                 const float2 ss = f2(s, s);
+                const float iA = kZoh ? kLog2e * rcp_approx(s) : 0.0f;   // 1/A (ZOH only)
                 const float4* brow = reinterpret_cast<const float4*>(bf + n * tpad + r * (R + 4));
                 const float4* crow = reinterpret_cast<const float4*>(cf + n * tpad + r * (R + 4));
                 // first pass from a zero state: cumulative decay Acum_i and local
@@ -404,7 +412,11 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
                         const int ip = 2 * i4 + hh;
                         const float2 arg = __fmul2_rn(dtv[ip], ss);
                         const float a0 = ex2_approx(arg.x), a1 = ex2_approx(arg.y);
-                        const float2 bu = __fmul2_rn(dtu[ip], hh ? f2(bv.z, bv.w) : f2(bv.x, bv.y));
+                        float2 uin = dtu[ip];
+                        if constexpr (kZoh)
+                            uin = __fmul2_rn(uin, f2(zoh_bbar(dtv[ip].x, arg.x * kLn2, a0, iA),
+                                                     zoh_bbar(dtv[ip].y, arg.y * kLn2, a1, iA)));
+                        const float2 bu = __fmul2_rn(uin, hh ? f2(bv.z, bv.w) : f2(bv.x, bv.y));
                         const float A0 = A * a0, H0 = fmaf(a0, H, bu.x);
                         A = A0 * a1;
                         H = fmaf(a1, H0, bu.y);

@@ -14,8 +14,10 @@
 // carry structure of the chunked associative scan described in the SSD article;
 // it costs a second walk of the middle segments.
 //
-// Recurrence (Axon-SSM page, recurrence equation, first-order discretisation):
-//   h_n <- exp(dt * A_n) h_n + dt * u * B_n,   y = (sum_n C_n h_n + D u) * SiLU(z)
+// Recurrence (Axon-SSM page, recurrence equation; first-order discretisation,
+// or the exact zero-order hold when kZoh):
+//   h_n <- exp(dt * A_n) h_n + Bbar_n u,   y = (sum_n C_n h_n + D u) * SiLU(z)
+//   Bbar_n = dt B_n (first order)  or  (exp(dt A_n) - 1) / A_n B_n (ZOH)
 #pragma once
 
 #include "device_math.cuh"
@@ -57,7 +59,7 @@ __device__ __forceinline__ float xpad_at(const ScanParams& p, int b, int e, int 
 
 // Walk tokens [t0, t1) of channel (b, e) starting from state h.
 //   kWriteY: produce y (else only the state and the dt sum are tracked).
-template <class Io, bool kWriteY>
+template <class Io, bool kWriteY, bool kZoh>
 __device__ __forceinline__ void walk(const ScanParams& p, int b, int e, int t0, int t1,
                                      const float (&A2)[kN], float (&h)[kN], float& sdt,
                                      float (&win)[kK - 1]) {
@@ -93,6 +95,11 @@ __device__ __forceinline__ void walk(const ScanParams& p, int b, int e, int t0, 
         const float dt = dt_from_raw(dr + db);
         const float dtu = dt * u;
         sdt += dt;
+        // input term Bbar_n u: (dt u) B_n first-order; u zoh_bbar(...) B_n for ZOH
+        auto input = [&](int n, float a) {
+            if constexpr (kZoh) return u * zoh_bbar(dt, dt * A2[n] * kLn2, a, kLog2e / A2[n]) * Bv[n];
+            else return dtu * Bv[n];
+        };
         if constexpr (kWriteY) {
             const float zt = Io::load(zs + o);
             float Cv[kN];
@@ -101,7 +108,7 @@ __device__ __forceinline__ void walk(const ScanParams& p, int b, int e, int t0, 
 #pragma unroll
             for (int n = 0; n < kN; ++n) {
                 const float a = ex2_approx(dt * A2[n]);
-                h[n] = fmaf(a, h[n], dtu * Bv[n]);
+                h[n] = fmaf(a, h[n], input(n, a));
                 acc[n & 3] = fmaf(Cv[n], h[n], acc[n & 3]);
             }
             const float yv = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * silu(zt);
@@ -110,7 +117,7 @@ __device__ __forceinline__ void walk(const ScanParams& p, int b, int e, int t0, 
 #pragma unroll
             for (int n = 0; n < kN; ++n) {
                 const float a = ex2_approx(dt * A2[n]);
-                h[n] = fmaf(a, h[n], dtu * Bv[n]);
+                h[n] = fmaf(a, h[n], input(n, a));
             }
         }
     }
@@ -136,7 +143,7 @@ __device__ __forceinline__ void write_final(const ScanParams& p, int b, int e,
 }
 
 // Phase 1 (or the whole scan when num_seg == 1).  grid = (ceil(E/128), B, max(P-1, 1)).
-template <class Io>
+template <class Io, bool kZoh>
 __global__ void __launch_bounds__(128) scan_seq_phase1(ScanParams p) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     const int b = blockIdx.y;
@@ -163,7 +170,7 @@ __global__ void __launch_bounds__(128) scan_seq_phase1(ScanParams p) {
 #pragma unroll
             for (int n = 0; n < kN; ++n) h[n] = 0.0f;
         }
-        walk<Io, true>(p, b, e, t0, t1, A2, h, sdt, win);
+        walk<Io, true, kZoh>(p, b, e, t0, t1, A2, h, sdt, win);
         if (p.num_seg == 1) {
             write_final<Io>(p, b, e, h, win);
         } else {
@@ -174,7 +181,7 @@ __global__ void __launch_bounds__(128) scan_seq_phase1(ScanParams p) {
     } else {
 #pragma unroll
         for (int n = 0; n < kN; ++n) h[n] = 0.0f;
-        walk<Io, false>(p, b, e, t0, t1, A2, h, sdt, win);
+        walk<Io, false, kZoh>(p, b, e, t0, t1, A2, h, sdt, win);
         const size_t slot = ((size_t)s * p.B + b) * p.E + e;
         float4* wo = reinterpret_cast<float4*>(p.ws_h + slot * kN);
 #pragma unroll
@@ -184,7 +191,7 @@ __global__ void __launch_bounds__(128) scan_seq_phase1(ScanParams p) {
 }
 
 // Phase 2: segments 1..P-1 fold the carry and walk again.  grid = (ceil(E/128), B, P-1).
-template <class Io>
+template <class Io, bool kZoh>
 __global__ void __launch_bounds__(128) scan_seq_phase2(ScanParams p) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     const int b = blockIdx.y;
@@ -222,7 +229,7 @@ __global__ void __launch_bounds__(128) scan_seq_phase2(ScanParams p) {
 #pragma unroll
     for (int j = 0; j < kK - 1; ++j) win[j] = xpad_at<Io>(p, b, e, t0 - (kK - 1) + j);
     float sdt = 0.0f;
-    walk<Io, true>(p, b, e, t0, t1, A2, h, sdt, win);
+    walk<Io, true, kZoh>(p, b, e, t0, t1, A2, h, sdt, win);
     if (s == p.num_seg - 1) write_final<Io>(p, b, e, h, win);
 }
 

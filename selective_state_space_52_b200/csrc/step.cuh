@@ -54,7 +54,7 @@ constexpr int kStepMaxRows = 32;   // batch rows per block
 //  - A = -exp(A_log) is formed once per lane.
 // The conv/SiLU/dt prologue of four consecutive rows is spread over the four
 // lanes of a channel; C . h is finished with two shuffles.
-template <class Io>
+template <class Io, bool kZoh>
 __global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int rows) {
     using T = typename Io::T;
     constexpr int S = Io::kBytes;
@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int ro
             xc = fmaf(w.w, x_t, xc);
             uq = silu(xc);
             dtq = dt_from_raw(Io::sload(&small[jq][2][co]) + db);
-            dtuq = dtq * uq;
+            dtuq = kZoh ? uq : dtq * uq;                  // input factor of Bbar u
             gzq = silu(Io::sload(&small[jq][1][co]));
         }
 #pragma unroll
@@ -161,7 +161,10 @@ __global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int ro
             float acc = 0.0f;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                h[i] = fmaf(ex2_approx(dt * A2[i]), h[i], dtu * Bq[i]);
+                const float a = ex2_approx(dt * A2[i]);
+                // first-order: (dt u) B;  ZOH: u ((exp(dt A) - 1) / A) B
+                const float uin = kZoh ? dtu * zoh_bbar(dt, dt * A2[i] * kLn2, a, kLog2e / A2[i]) : dtu;
+                h[i] = fmaf(a, h[i], uin * Bq[i]);
                 acc = fmaf(Cq[i], h[i], acc);
             }
             acc += __shfl_xor_sync(0xffffffffu, acc, 1);

@@ -176,6 +176,21 @@ def test_step_noop_sizes(lib):
     assert _step(lib, E=0) == OK
 
 
+def test_discretization_enum_is_checked(lib):
+    f = lib.axon_ssm_scan_fwd_ex
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int] * 7 + [ctypes.c_void_p] * 15 + [ctypes.c_void_p, ctypes.c_size_t,
+                                                               ctypes.c_int, ctypes.c_void_p]
+    ptrs = [FAKE + 0x10000 * i for i in range(15)]
+    assert f(1, 64, 32, 16, 4, 0, 2, *ptrs, None, 0, 0, None) == UNSUPPORTED
+    assert f(1, 64, 32, 8, 4, 0, 1, *ptrs, None, 0, 0, None) == UNSUPPORTED    # N checked as usual
+    g = lib.axon_ssm_step_ex
+    g.restype = ctypes.c_int
+    g.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 14
+    assert g(2, 16, 16, 4, 1, -1, *ptrs[:13], None) == UNSUPPORTED
+    assert g(2, 16, 16, 4, 1, 1, None, *ptrs[1:13], None) == INVALID
+
+
 def test_binding_module_exposes_c_names():
     from selective_state_space_52_b200 import axon_ssm
     for name in declared_symbols():
