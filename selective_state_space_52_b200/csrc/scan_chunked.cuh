@@ -5,8 +5,8 @@
 // the tiles cover B*E channels with about one CTA per SM).  The sequence is
 // walked in chunks of kT = W*R tokens; the ET*W threads of the CTA split each
 // chunk into W runs of R consecutive tokens.  All W runs of a channel sit in
-// one warp (lane = channel-in-warp * W + run; a warp holds 32/W channels), so
-// runs exchange their partial results with warp shuffles, never with a CTA
+// one warp (lane = run * 32/W + channel-in-warp; a warp holds 32/W channels),
+// so runs exchange their partial results with warp shuffles, never with a CTA
 // barrier.  Per chunk:
 //
 //   1. x (with a 3-token halo), z, dt_raw rows of the tile's byte window and
@@ -174,8 +174,11 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
     const int tid = threadIdx.x;
     const int ET = p.ET;
     constexpr int CPW = 32 / W;                 // channels per warp (W > 1)
-    const int c = (W == 1) ? tid : (tid >> 5) * CPW + (tid & 31) / W;
-    const int r = (W == 1) ? 0 : (tid & (W - 1));
+    // lane = run * CPW + channel-in-warp: the 8 lanes of a quarter warp span
+    // at most two runs, so a float4 read of a transposed B/C row touches at
+    // most two addresses per quarter warp (two shared-memory wavefronts, not four)
+    const int c = (W == 1) ? tid : (tid >> 5) * CPW + (tid & (CPW - 1));
+    const int r = (W == 1) ? 0 : (tid & 31) / CPW;
     const int b = blockIdx.x / p.tiles_per_b;
     const int e0 = (blockIdx.x - b * p.tiles_per_b) * ET;
     const int ne = min(ET, p.E - e0);
@@ -425,17 +428,17 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
                     }
                 }
                 // inclusive scan of the run aggregates (A, H) over the W runs of this
-                // channel (W consecutive lanes); later o earlier = (A A', A H' + H)
+                // channel (lanes CPW apart); later o earlier = (A A', A H' + H)
                 float As = A, Hs = H;
 #pragma unroll
                 for (int d = 1; d < W; d <<= 1) {
-                    const float Ap = __shfl_up_sync(0xffffffffu, As, d, W);
-                    const float Hp = __shfl_up_sync(0xffffffffu, Hs, d, W);
+                    const float Ap = __shfl_up_sync(0xffffffffu, As, d * CPW);
+                    const float Hp = __shfl_up_sync(0xffffffffu, Hs, d * CPW);
                     if (r >= d) { Hs = fmaf(As, Hp, Hs); As *= Ap; }
                 }
                 // exclusive prefix (the runs before this one) applied to the carry-in
-                float Ae = __shfl_up_sync(0xffffffffu, As, 1, W);
-                float He = __shfl_up_sync(0xffffffffu, Hs, 1, W);
+                float Ae = __shfl_up_sync(0xffffffffu, As, CPW);
+                float He = __shfl_up_sync(0xffffffffu, Hs, CPW);
                 if (r == 0) { Ae = 1.0f; He = 0.0f; }
                 const float hc = cin[n * ET + c];
                 const float hin = fmaf(Ae, hc, He);
