@@ -539,11 +539,21 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-bench", action="store_true",
                     help="skip the separate cached-decode measurement (decode workload shapes)")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the cached-decode measurement and print it as one JSON line "
+                         "(for profiling the step kernel alone)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     wl = W.WORKLOAD_BY_NAME[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.decode_only:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA GPU for --decode-only")
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps({"decode": bench_decode(dev)}), flush=True)
+        return 0
     return run_axon(args, wl)
 
 

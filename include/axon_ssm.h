@@ -169,8 +169,9 @@ AXON_API axon_status axon_ssm_scan_fwd(
  * chunk carry passed through `workspace` (which must then hold at least
  * (num_segments-1) * B * E * (N+1) floats; num_segments <= 64 and every
  * segment at least K tokens long, else AXON_ERR_INVALID_ARG).
- * num_segments == 1 runs the sequence unsplit (the chunked kernel, no
- * workspace); num_segments == 0 lets the library choose, exactly as
+ * num_segments == 1 runs the sequence unsplit (one kernel walks every
+ * channel's whole sequence, no workspace); num_segments == 0 lets the
+ * library choose, exactly as
  * axon_ssm_scan_fwd does.  Same arguments and errors as axon_ssm_scan_fwd
  * otherwise.  Intended for tests and tuning; results agree with the library's
  * own plan to float32 rounding.

@@ -10,6 +10,7 @@
 #include "axon_ssm.h"
 #include "device_math.cuh"
 #include "scan_chunked.cuh"
+#include "scan_quad.cuh"
 #include "scan_seq.cuh"
 #include "step.cuh"
 
@@ -134,6 +135,29 @@ bool plan_chunked(int B, int E, int io_bytes, int sms, int max_smem, ChunkPlan* 
     return true;
 }
 
+// Warp-per-8-channels scan with the states split in quadrants.  Measured on
+// B200: it beats the run-split chunked kernel from 48 channels per SM (first
+// order; from 128 with exact ZOH, whose heavier input factor favours the
+// chunked kernel's wider tiles a little longer) and the one-thread-per-channel
+// walk up to 512 channels per SM.  The per-chunk byte offsets it keeps are
+// 32-bit.
+constexpr int kQuadT = 32;
+bool use_quad(int B, int E, int io_bytes, int sms, bool zoh) {
+    const long long channels = (long long)B * E;
+    if (channels < (long long)sms * (zoh ? 128 : 48) || channels >= (long long)sms * 512) return false;
+    return (long long)(kQuadT + kK) * E * io_bytes < (1LL << 31);
+}
+
+template <class Io, bool Z>
+axon_status launch_quad(const ChunkParams& prm, cudaStream_t st) {
+    auto kern = scan_quad_kernel<Io, kQuadT, Z>;
+    const int smem = QuadSmem(kQuadT, Io::kBytes).total;       // one warp per CTA
+    const long long warps = (long long)prm.B * ((prm.E + kQuadCh - 1) / kQuadCh);
+    if (warps > 0x7fffffffLL) return AXON_ERR_UNSUPPORTED;
+    kern<<<(unsigned)warps, 32, smem, st>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+}
+
 template <class Io, int W, int R, bool Z>
 axon_status launch_chunked_t(const ChunkParams& prm, int smem, cudaStream_t st) {
     auto kern = scan_chunked_kernel<Io, W, R, Z>;
@@ -218,7 +242,7 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
 
     int P = 1;
     int seg = L > 0 ? L : 1;
-    bool chunked = false;
+    bool chunked = false, quad = false;
     ChunkPlan cplan{};
     if (L > 0) {
         if (num_segments > kMaxSegments) return AXON_ERR_INVALID_ARG;
@@ -229,6 +253,8 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
             if (sms <= 0) return AXON_ERR_CUDA;
             if (num_segments == 0 && use_time_split(B, L, E, sms)) {
                 P = plan_segments(B, L, E, sms);
+            } else if (use_quad(B, E, (int)io_bytes(io), sms, zoh)) {
+                quad = true;                   // unsplit: the quadrant scan
             } else {
                 // unsplit: the chunked kernel (the channel walk is the fallback)
                 const int max_smem = device_max_smem_optin();
@@ -251,14 +277,20 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
             return AXON_ERR_INVALID_ARG;
     }
 
-    if (chunked) {
+    if (chunked || quad) {
         ChunkParams cp;
         cp.B = B; cp.L = L; cp.E = E;
-        cp.ET = cplan.ET; cp.tiles_per_b = cplan.tiles_per_b; cp.pitch = cplan.pitch;
+        cp.ET = quad ? kQuadCh : cplan.ET;
+        cp.tiles_per_b = quad ? (E + kQuadCh - 1) / kQuadCh : cplan.tiles_per_b;
+        cp.pitch = quad ? 0 : cplan.pitch;
         cp.x = x; cp.z = z; cp.dt_raw = dt_raw; cp.Bm = Bm; cp.Cm = Cm;
         cp.conv_w = conv_w; cp.conv_b = conv_b; cp.dt_bias = dt_bias; cp.A_log = A_log; cp.D = D;
         cp.conv_cache_in = conv_cache_in; cp.ssm_state_in = ssm_state_in;
         cp.y = y; cp.conv_cache_out = conv_cache_out; cp.ssm_state_out = ssm_state_out;
+        if (quad) {
+            if (io == AXON_BF16) return zoh ? launch_quad<IoBF16, true>(cp, stream) : launch_quad<IoBF16, false>(cp, stream);
+            return zoh ? launch_quad<IoF32, true>(cp, stream) : launch_quad<IoF32, false>(cp, stream);
+        }
         if (io == AXON_BF16) return zoh ? launch_chunked<IoBF16, true>(cp, cplan, stream)
                                         : launch_chunked<IoBF16, false>(cp, cplan, stream);
         return zoh ? launch_chunked<IoF32, true>(cp, cplan, stream) : launch_chunked<IoF32, false>(cp, cplan, stream);

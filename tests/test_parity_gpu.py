@@ -42,16 +42,21 @@ def test_chunked_kernel_small_shapes(cuda_lib, io, B, E, L):
     compare_scan(inp, io, num_segments=1, with_state=(L % 2 == 1), what=f"chunked B{B} L{L} E{E} {io}")
 
 
-# Shapes that steer the planner to each run count W (channels per tile ET =
-# ceil(E / (148 / B)); W is the largest of 16/8/4/2/1 with ET*W <= 512 whose
-# shared memory fits), including partial last tiles (E % ET != 0).
+# Shapes that steer the planner to each unsplit kernel on a 148-SM B200: the
+# run-split chunked kernel below 48 channels per SM (channels per tile ET =
+# ceil(E / (148 / B)), W the largest of 16/8/4/2 with ET*W <= 512 whose shared
+# memory fits, partial last tiles when E % ET != 0), the quadrant scan from 48
+# to 511 channels per SM (first order; with ZOH from 128, so that the 52 and
+# 100 channel shapes take the chunked kernel's W = 8 and 4 plans, covered in
+# test_zoh_gpu.py), the direct walk above.
 PLANNER_SHAPES = [
     (1, 1000, 300),     # ET 7, partial last tile, W 16
-    (1, 7680, 200),     # ET 52 (the Bit-Axon tiling), W 8
+    (1, 7680, 200),     # 52 channels per SM: quadrant scan
     (2, 2048, 300),     # ET 28, two batch rows, W 16 (bf16) / 8 (fp32)
-    (1, 14800, 100),    # ET 100, W 4 (bf16)
-    (1, 29600, 40),     # ET 200, W 2 (bf16) / 1 (fp32)
-    (8, 4800, 40),      # 38400 channels: direct walk, W 1
+    (1, 14800, 100),    # 100 channels per SM: quadrant scan
+    (1, 29600, 40),     # 200 channels per SM: quadrant scan
+    (8, 4800, 40),      # 259 channels per SM: quadrant scan
+    (16, 4800, 24),     # 519 channels per SM: direct walk, W 1
 ]
 
 
@@ -61,6 +66,53 @@ def test_chunked_kernel_planner_shapes(cuda_lib, io, B, E, L):
     wl = W.custom(B, L, E, io=io, seed=4000 + E + L)
     inp = W.make_inputs(wl, with_state=True)
     compare_scan(inp, io, num_segments=1, with_state=True, what=f"planner B{B} E{E} L{L} {io}")
+
+
+# The quadrant scan (one warp per 8 channels, chunks of 32 tokens): single
+# tokens, ragged last chunks, several batch rows, both ends of its planner range.
+QUAD_SHAPES = [
+    (1, 7680, 1), (1, 7680, 33), (1, 7680, 257), (2, 3584, 100), (3, 2400, 65), (1, 37000, 40),
+    (8, 9440, 20),
+]
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("B,E,L", QUAD_SHAPES)
+def test_quadrant_scan_shapes(cuda_lib, io, B, E, L):
+    wl = W.custom(B, L, E, io=io, seed=4500 + E + L)
+    inp = W.make_inputs(wl, with_state=True)
+    compare_scan(inp, io, with_state=(L % 2 == 1), what=f"quad B{B} E{E} L{L} {io}")
+
+
+@pytest.mark.parametrize("B,E,L", [(1, 7684, 97), (2, 3596, 40)])
+def test_quadrant_scan_fp32_tail_tile(cuda_lib, B, E, L):
+    """E % 8 == 4 (fp32 only): the last warp of every batch row owns 4 channels."""
+    inp = W.make_inputs(W.custom(B, L, E, io="f32", seed=4600 + E), with_state=True)
+    compare_scan(inp, "f32", what=f"quad tail B{B} E{E} L{L}")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_quadrant_scan_continues_in_place(cuda_lib, io):
+    """Streaming prefill on a quadrant-scan shape with the caches updated in
+    place: scan(0:1), scan(1:3), scan(3:40), scan(40:100) == one scan."""
+    from selective_state_space_52_b200 import axon_ssm
+    wl = W.custom(1, 100, 7680, io=io, seed=4700)
+    inp = W.make_inputs(wl, with_state=True)
+    d = to_dev(inp)
+    params = {k: d[k] for k in axon_ssm.PARAM_KEYS}
+    cc, ss = d["conv_cache"].clone(), d["ssm_state"].clone()
+    ys = []
+    for lo, hi in [(0, 1), (1, 3), (3, 40), (40, 100)]:
+        sl = {k: d[k][:, lo:hi].contiguous() for k in ("x", "z", "dt_raw", "B", "C")}
+        y = torch.empty_like(sl["x"])
+        axon_ssm.scan_fwd(sl["x"], sl["z"], sl["dt_raw"], sl["B"], sl["C"], params, (cc, ss), out=(y, cc, ss))
+        ys.append(y)
+    torch.cuda.synchronize()
+    y = torch.cat(ys, dim=1).float().cpu().numpy()
+    y_ref, cc_ref, ss_ref = oracle_scan(inp)
+    check_close(y, y_ref, tol_for(io, y_ref), "quad streamed y")
+    check_close(ss.cpu().numpy(), ss_ref, state_tol(ss_ref), "quad streamed state")
+    assert torch.equal(cc.cpu(), torch.from_numpy(cc_ref).to(cc.dtype))
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
