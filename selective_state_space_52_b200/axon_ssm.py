@@ -89,8 +89,13 @@ def _p(t):
     return t.data_ptr()
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream):
     if stream is None:
+        if _raw_stream is not None:
+            return _raw_stream(torch.cuda.current_device())
         return torch.cuda.current_stream().cuda_stream
     if isinstance(stream, int):
         return stream
@@ -224,12 +229,13 @@ def scan_fwd(x, z, dt_raw, Bm, Cm, params: dict, cache=None, *, num_segments=Non
         ss_out = torch.empty(Bsz, E, N, dtype=torch.float32, device=dev)
     else:
         y, cc_out, ss_out = out
-    if num_segments is None:
-        nbytes = axon_ssm_scan_workspace_bytes(Bsz, L, E, N, K, io)
-    else:
-        nbytes = max(num_segments - 1, 0) * Bsz * E * (N + 1) * 4
-    if workspace is None and nbytes > 0:
-        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    if workspace is None:
+        if num_segments is None:
+            nbytes = axon_ssm_scan_workspace_bytes(Bsz, L, E, N, K, io)
+        else:
+            nbytes = max(num_segments - 1, 0) * Bsz * E * (N + 1) * 4
+        if nbytes > 0:
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
     args = (Bsz, L, E, N, K, io, x, z, dt_raw, Bm, Cm, *(params[k] for k in PARAM_KEYS),
             cc_in, ss_in, y, cc_out, ss_out, workspace, wsz)

@@ -3,6 +3,7 @@
 // kernel launches on the caller's stream.  The library allocates nothing.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -56,12 +57,25 @@ size_t ws_bytes_for(int B, int E, int P) {
     return (size_t)(P - 1) * (size_t)B * (size_t)E * (kN + 1) * sizeof(float);
 }
 
-int device_sm_count() {
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-    return sms;
+// Per-device attributes, queried once per device (the values never change).
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sms[kMaxDevices];
+std::atomic<int> g_max_smem[kMaxDevices];
+
+int cached_attribute(std::atomic<int>* table, cudaDeviceAttr attr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return -1;
+    if (dev < kMaxDevices) {
+        const int v = table[dev].load(std::memory_order_relaxed);
+        if (v > 0) return v;
+    }
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, attr, dev) != cudaSuccess) return -1;
+    if (dev < kMaxDevices && v > 0) table[dev].store(v, std::memory_order_relaxed);
+    return v;
 }
+
+int device_sm_count() { return cached_attribute(g_sms, cudaDevAttrMultiProcessorCount); }
 
 // Channel-parallel scan: one thread per (b, e).  Split the sequence only when
 // the channels alone cannot give every SM a few warps.
@@ -81,11 +95,22 @@ bool use_time_split(int B, int L, int E, int sms) {
     return (long long)B * E < (long long)sms * 4 && L >= 2 * kMinSegLen;
 }
 
-int device_max_smem_optin() {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return -1;
-    return v;
+int device_max_smem_optin() { return cached_attribute(g_max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin); }
+
+// Raises a kernel's dynamic shared-memory limit to the device's opt-in maximum
+// once per device (the limit only permits; each launch asks for what it uses).
+template <class Kern>
+bool allow_max_smem(Kern kern, std::atomic<unsigned long long>& done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    const unsigned long long bit = dev < kMaxDevices ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return true;
+    const int max_smem = device_max_smem_optin();
+    if (max_smem <= 0) return false;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem) != cudaSuccess)
+        return false;
+    if (bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return true;
 }
 
 struct ChunkPlan {
@@ -161,8 +186,8 @@ axon_status launch_quad(const ChunkParams& prm, cudaStream_t st) {
 template <class Io, int W, int R, bool Z>
 axon_status launch_chunked_t(const ChunkParams& prm, int smem, cudaStream_t st) {
     auto kern = scan_chunked_kernel<Io, W, R, Z>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return AXON_ERR_CUDA;
+    static std::atomic<unsigned long long> smem_set{0};
+    if (!allow_max_smem(kern, smem_set)) return AXON_ERR_CUDA;
     const unsigned grid = (unsigned)((long long)prm.B * prm.tiles_per_b);
     kern<<<grid, prm.ET * W, smem, st>>>(prm);
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;

@@ -226,91 +226,79 @@ __global__ void __launch_bounds__(256) scan_quad_kernel(ChunkParams p) {
         h23 = f2(h0.z, h0.w);
     }
 
-    float2* pf = reinterpret_cast<float2*>(ws + lay.pf);   // [padded token][channel] (dt, f)
     // y of token t0 + g*TQ + j, channel e: ybase + (t0 + j) * row_bytes
     unsigned char* ybase = static_cast<unsigned char*>(p.y) + tile_off + (size_t)(g * TQ) * row_bytes + c * S;
     const int nck = (p.L + T - 1) / T;
-    prefetch(0, 0);
-    cp_async_commit();
-    for (int k = 0; k < nck; ++k) {
-        const int st = k & 1;
-        const int t0 = k * T;
-        const bool full = t0 + T <= p.L;
-        __syncwarp();                        // every lane is done with the stage refilled below and with pf
-        if (k + 1 < nck) prefetch(k + 1, st ^ 1);
-        cp_async_commit();
-        cp_async_wait_1();                   // this lane's copies of chunk k have landed
-        __syncwarp();                        // ... and every lane's
-        const unsigned char* sb = ws + st * lay.stage;
 
-        // ---- prologue: tokens g*TQ .. g*TQ + TQ - 1 of channel c
-        float Du[TQ], gz[TQ];
-        {
-            const int tb = g * TQ;
-            const unsigned char* xc = sb + lay.xs + c * S;
-            float xm3 = SI::ld(xc + QuadSmem::pad(tb + 0, TQ) * XB);
-            float xm2 = SI::ld(xc + QuadSmem::pad(tb + 1, TQ) * XB);
-            float xm1 = SI::ld(xc + QuadSmem::pad(tb + 2, TQ) * XB);
-#pragma unroll
-            for (int i = 0; i < TQ; ++i) {
-                const int t = tb + i;
-                const float xt = SI::ld(xc + QuadSmem::pad(t + 3, TQ) * XB);
-                float xv = fmaf(w0, xm3, cb);
-                xv = fmaf(w1, xm2, xv);
-                xv = fmaf(w2, xm1, xv);
-                xv = fmaf(w3, xt, xv);
-                xm3 = xm2; xm2 = xm1; xm1 = xt;
-                const float u = silu(xv);
-                const int tp = t + g;        // padded row of token t (t / TQ == g)
-                const float dt = dt_from_raw(SI::ld(sb + lay.ds + tp * XB + c * S) + db);
-                const bool live = full || (t0 + t) < p.L;
-                const float dtl = live ? dt : 0.0f;          // dt = 0: decay 1, no input
-                const float f = live ? (kZoh ? u : dt * u) : 0.0f;
-                pf[tp * kQuadCh + c] = make_float2(dtl, f);
-                Du[i] = Dv * u;
-                gz[i] = silu(SI::ld(sb + lay.zs + tp * XB + c * S));
-            }
+    // ---- prologue, one token at a time: lane (g, c) takes tokens g*TQ ..
+    // g*TQ + TQ - 1 of channel c; the conv window slides in registers
+    struct Window { float xm3, xm2, xm1; };
+    auto pro_begin = [&](const unsigned char* sb) {
+        const int tb = g * TQ;
+        const unsigned char* xc = sb + lay.xs + c * S;
+        return Window{SI::ld(xc + QuadSmem::pad(tb + 0, TQ) * XB), SI::ld(xc + QuadSmem::pad(tb + 1, TQ) * XB),
+                      SI::ld(xc + QuadSmem::pad(tb + 2, TQ) * XB)};
+    };
+    auto pro_token = [&](Window& wd, const unsigned char* sb, float2* pfb, int t0, bool full, int i,
+                         float& du, float& gzv) {
+        const int t = g * TQ + i;
+        const float xt = SI::ld(sb + lay.xs + c * S + QuadSmem::pad(t + 3, TQ) * XB);
+        float xv = fmaf(w0, wd.xm3, cb);
+        xv = fmaf(w1, wd.xm2, xv);
+        xv = fmaf(w2, wd.xm1, xv);
+        xv = fmaf(w3, xt, xv);
+        wd.xm3 = wd.xm2; wd.xm2 = wd.xm1; wd.xm1 = xt;
+        const float u = silu(xv);
+        const int tp = t + g;            // padded row of token t (t / TQ == g)
+        const float dt = dt_from_raw(SI::ld(sb + lay.ds + tp * XB + c * S) + db);
+        const bool live = full || (t0 + t) < p.L;
+        const float dtl = live ? dt : 0.0f;          // dt = 0: decay 1, no input
+        const float f = live ? (kZoh ? u : dt * u) : 0.0f;
+        pfb[tp * kQuadCh + c] = make_float2(dtl, f);
+        du = Dv * u;
+        gzv = silu(SI::ld(sb + lay.zs + tp * XB + c * S));
+    };
+
+    // ---- walk pieces: decays and inputs of token t (state-independent), then
+    // the state update and the quadrant's partial C . h
+    float part[T];
+    auto decay_input = [&](const unsigned char* sb, const float2* pfb, int t,
+                           float2& a01, float2& a23, float2& u01, float2& u23) {
+        const float2 v = pfb[(t + t / TQ) * kQuadCh + c];
+        const float2 dd = f2(v.x, v.x), ff = f2(v.y, v.y);
+        float Bq[4];
+        QuadRow<Io>::ld(sb + lay.bs + t * (kN * S), g, Bq);
+        const float2 arg01 = __fmul2_rn(dd, s01);
+        const float2 arg23 = __fmul2_rn(dd, s23);
+        a01 = f2(ex2_approx(arg01.x), ex2_approx(arg01.y));
+        a23 = f2(ex2_approx(arg23.x), ex2_approx(arg23.y));
+        u01 = __fmul2_rn(ff, f2(Bq[0], Bq[1]));
+        u23 = __fmul2_rn(ff, f2(Bq[2], Bq[3]));
+        if constexpr (kZoh) {
+            u01 = __fmul2_rn(u01, f2(zoh_bbar(v.x, arg01.x * kLn2, a01.x, iA01.x),
+                                     zoh_bbar(v.x, arg01.y * kLn2, a01.y, iA01.y)));
+            u23 = __fmul2_rn(u23, f2(zoh_bbar(v.x, arg23.x * kLn2, a23.x, iA23.x),
+                                     zoh_bbar(v.x, arg23.y * kLn2, a23.y, iA23.y)));
         }
-        __syncwarp();
+    };
+    auto update = [&](const unsigned char* sb, int t, float2 a01, float2 a23, float2 u01, float2 u23) {
+        float Cq[4];
+        QuadRow<Io>::ld(sb + lay.cs + t * (kN * S), g, Cq);
+        h01 = __ffma2_rn(a01, h01, u01);
+        h23 = __ffma2_rn(a23, h23, u23);
+        const float2 pq = __ffma2_rn(f2(Cq[2], Cq[3]), h23, __fmul2_rn(f2(Cq[0], Cq[1]), h01));
+        part[t] = pq.x + pq.y;
+    };
+    auto walk_block = [&](const unsigned char* sb, const float2* pfb, int tb) {
+        float2 a01[kBlk], a23[kBlk], u01[kBlk], u23[kBlk];
+#pragma unroll
+        for (int i = 0; i < kBlk; ++i) decay_input(sb, pfb, tb + i, a01[i], a23[i], u01[i], u23[i]);
+#pragma unroll
+        for (int i = 0; i < kBlk; ++i) update(sb, tb + i, a01[i], a23[i], u01[i], u23[i]);
+    };
 
-        // ---- walk: 4 states per lane, partial C . h per token
-        float part[T];
-        auto decay_input = [&](int t, float2& a01, float2& a23, float2& u01, float2& u23) {
-            const float2 v = pf[(t + t / TQ) * kQuadCh + c];
-            const float2 dd = f2(v.x, v.x), ff = f2(v.y, v.y);
-            float Bq[4];
-            QuadRow<Io>::ld(sb + lay.bs + t * (kN * S), g, Bq);
-            const float2 arg01 = __fmul2_rn(dd, s01);
-            const float2 arg23 = __fmul2_rn(dd, s23);
-            a01 = f2(ex2_approx(arg01.x), ex2_approx(arg01.y));
-            a23 = f2(ex2_approx(arg23.x), ex2_approx(arg23.y));
-            u01 = __fmul2_rn(ff, f2(Bq[0], Bq[1]));
-            u23 = __fmul2_rn(ff, f2(Bq[2], Bq[3]));
-            if constexpr (kZoh) {
-                u01 = __fmul2_rn(u01, f2(zoh_bbar(v.x, arg01.x * kLn2, a01.x, iA01.x),
-                                         zoh_bbar(v.x, arg01.y * kLn2, a01.y, iA01.y)));
-                u23 = __fmul2_rn(u23, f2(zoh_bbar(v.x, arg23.x * kLn2, a23.x, iA23.x),
-                                         zoh_bbar(v.x, arg23.y * kLn2, a23.y, iA23.y)));
-            }
-        };
-        auto update = [&](int t, float2 a01, float2 a23, float2 u01, float2 u23) {
-            float Cq[4];
-            QuadRow<Io>::ld(sb + lay.cs + t * (kN * S), g, Cq);
-            h01 = __ffma2_rn(a01, h01, u01);
-            h23 = __ffma2_rn(a23, h23, u23);
-            const float2 pq = __ffma2_rn(f2(Cq[2], Cq[3]), h23, __fmul2_rn(f2(Cq[0], Cq[1]), h01));
-            part[t] = pq.x + pq.y;
-        };
-#pragma unroll
-        for (int tb = 0; tb < T; tb += kBlk) {
-            float2 a01[kBlk], a23[kBlk], u01[kBlk], u23[kBlk];
-#pragma unroll
-            for (int i = 0; i < kBlk; ++i) decay_input(tb + i, a01[i], a23[i], u01[i], u23[i]);
-#pragma unroll
-            for (int i = 0; i < kBlk; ++i) update(tb + i, a01[i], a23[i], u01[i], u23[i]);
-        }
-
-        // ---- reduce-scatter over the quadrants (lanes 8 and 16 apart) and store y
+    // ---- reduce-scatter over the quadrants (lanes 8 and 16 apart) and store y
+    auto finish = [&](int t0, bool full, const float (&Du)[TQ], const float (&gz)[TQ]) {
         const bool hi = (g & 2) != 0, lo = (g & 1) != 0;
         unsigned char* yrow = ybase + (size_t)t0 * row_bytes;
 #pragma unroll
@@ -325,6 +313,29 @@ __global__ void __launch_bounds__(256) scan_quad_kernel(ChunkParams p) {
             if (active && (full || t0 + g * TQ + j < p.L))
                 Io::store(reinterpret_cast<TT*>(yrow + j * row_bytes), (tot + Du[j]) * gz[j]);
         }
+    };
+
+    float2* pf = reinterpret_cast<float2*>(ws + lay.pf);   // [padded token][channel] (dt, f)
+    prefetch(0, 0);
+    cp_async_commit();
+    for (int k = 0; k < nck; ++k) {
+        const int st = k & 1;
+        const int t0 = k * T;
+        const bool full = t0 + T <= p.L;
+        __syncwarp();                        // every lane is done with the stage refilled below and with pf
+        if (k + 1 < nck) prefetch(k + 1, st ^ 1);
+        cp_async_commit();
+        cp_async_wait_1();                   // this lane's copies of chunk k have landed
+        __syncwarp();                        // ... and every lane's
+        const unsigned char* sb = ws + st * lay.stage;
+        float Du[TQ], gz[TQ];
+        Window wd = pro_begin(sb);
+#pragma unroll
+        for (int i = 0; i < TQ; ++i) pro_token(wd, sb, pf, t0, full, i, Du[i], gz[i]);
+        __syncwarp();
+#pragma unroll
+        for (int tb = 0; tb < T; tb += kBlk) walk_block(sb, pf, tb);
+        finish(t0, full, Du, gz);
     }
 
     // ---- final caches
