@@ -43,16 +43,17 @@ def test_chunked_kernel_small_shapes(cuda_lib, io, B, E, L):
 
 
 # Shapes that steer the planner to each unsplit kernel on a 148-SM B200: the
-# run-split chunked kernel below 48 channels per SM (channels per tile ET =
-# ceil(E / (148 / B)), W the largest of 16/8/4/2 with ET*W <= 512 whose shared
-# memory fits, partial last tiles when E % ET != 0), the quadrant scan from 48
-# to 511 channels per SM (first order; with ZOH from 128, so that the 52 and
-# 100 channel shapes take the chunked kernel's W = 8 and 4 plans, covered in
-# test_zoh_gpu.py), the direct walk above.
+# run-split chunked kernel below 8 channels per SM (channels per tile ET =
+# ceil(E / (148 / B)), W the largest of 32/16/8 with ET*W <= 512 whose shared
+# memory fits, partial last tiles when E % ET != 0), the eighths scan from 8
+# to 47 channels per SM (to 127 with exact ZOH), the quadrant scan from 48 to
+# 511 (first order; from 128 with ZOH), the direct walk above.
 PLANNER_SHAPES = [
     (1, 1000, 300),     # ET 7, partial last tile, W 16
     (1, 7680, 200),     # 52 channels per SM: quadrant scan
-    (2, 2048, 300),     # ET 28, two batch rows, W 16 (bf16) / 8 (fp32)
+    (2, 2048, 300),     # 28 channels per SM: eighths scan
+    (1, 1100, 200),     # ET 8, W 32
+    (1, 1600, 200),     # 10.8 channels per SM: eighths scan
     (1, 14800, 100),    # 100 channels per SM: quadrant scan
     (1, 29600, 40),     # 200 channels per SM: quadrant scan
     (8, 4800, 40),      # 259 channels per SM: quadrant scan
@@ -84,6 +85,19 @@ def test_quadrant_scan_shapes(cuda_lib, io, B, E, L):
     compare_scan(inp, io, with_state=(L % 2 == 1), what=f"quad B{B} E{E} L{L} {io}")
 
 
+# The eighths scan (one warp per 4 channels, two states per lane).
+OCTO_SHAPES = [(1, 4096, 1), (1, 4096, 33), (1, 4096, 257), (2, 2048, 100), (1, 3072, 65), (3, 2000, 40),
+               (1, 1800, 130)]
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("B,E,L", OCTO_SHAPES)
+def test_eighths_scan_shapes(cuda_lib, io, B, E, L):
+    wl = W.custom(B, L, E, io=io, seed=4800 + E + L)
+    inp = W.make_inputs(wl, with_state=True)
+    compare_scan(inp, io, with_state=(L % 2 == 1), what=f"octo B{B} E{E} L{L} {io}")
+
+
 @pytest.mark.parametrize("B,E,L", [(1, 7684, 97), (2, 3596, 40)])
 def test_quadrant_scan_fp32_tail_tile(cuda_lib, B, E, L):
     """E % 8 == 4 (fp32 only): the last warp of every batch row owns 4 channels."""
@@ -92,11 +106,13 @@ def test_quadrant_scan_fp32_tail_tile(cuda_lib, B, E, L):
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
-def test_quadrant_scan_continues_in_place(cuda_lib, io):
-    """Streaming prefill on a quadrant-scan shape with the caches updated in
-    place: scan(0:1), scan(1:3), scan(3:40), scan(40:100) == one scan."""
+@pytest.mark.parametrize("E", [7680, 4096])
+def test_warp_scans_continue_in_place(cuda_lib, io, E):
+    """Streaming prefill on a quadrant-scan (E 7680) and an eighths-scan (E
+    4096) shape with the caches updated in place: scan(0:1), scan(1:3),
+    scan(3:40), scan(40:100) == one scan."""
     from selective_state_space_52_b200 import axon_ssm
-    wl = W.custom(1, 100, 7680, io=io, seed=4700)
+    wl = W.custom(1, 100, E, io=io, seed=4700 + E)
     inp = W.make_inputs(wl, with_state=True)
     d = to_dev(inp)
     params = {k: d[k] for k in axon_ssm.PARAM_KEYS}

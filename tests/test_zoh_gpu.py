@@ -2,10 +2,11 @@
 Axon-SSM page, "ZOH discretisation"), selected through axon_ssm_scan_fwd_ex /
 axon_ssm_step_ex, against the fp64 oracle run with zoh=True.
 
-Covers the direct walk (many channels), the quadrant scan and the run-split
-chunked kernel (fewer channels), the segment-carry split, the decode step,
-decode == prefill, and dt at both clips (dt = 1e-4 makes dt*A tiny: the series branch of the input
-factor; dt = 100 makes exp(dt A) vanish: Bbar = B / |A|).
+Covers the direct walk (many channels), the quadrant and eighths scans and
+the run-split chunked kernel (fewer channels), the segment-carry split, the
+decode step, decode == prefill, and dt at both clips (dt = 1e-4 makes dt*A
+tiny: the series branch of the input factor; dt = 100 makes exp(dt A) vanish:
+Bbar = B / |A|).
 """
 import numpy as np
 import pytest
@@ -46,7 +47,8 @@ def _compare(inp, io, what, num_segments=None):
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 @pytest.mark.parametrize("B,E,L", [(1, 8, 300), (2, 264, 1000), (1, 1000, 257), (1, 7680, 96),
-                                   (8, 4800, 40), (1, 14800, 100), (1, 29600, 40), (16, 4800, 24)])
+                                   (8, 4800, 40), (1, 14800, 100), (1, 29600, 40), (16, 4800, 24),
+                                   (2, 2048, 130)])
 def test_zoh_chunked_kernel(cuda_lib, io, B, E, L):
     inp = W.make_inputs(W.custom(B, L, E, io=io, seed=7000 + E + L), with_state=True)
     _compare(inp, io, f"zoh B{B} E{E} L{L} {io}", num_segments=1)
