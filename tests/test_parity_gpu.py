@@ -52,7 +52,7 @@ PLANNER_SHAPES = [
     (1, 1000, 300),     # ET 7, partial last tile, W 16
     (1, 7680, 200),     # 52 channels per SM: quadrant scan
     (2, 2048, 300),     # 28 channels per SM: eighths scan
-    (1, 1100, 200),     # ET 8, W 32
+    (1, 1096, 200),     # ET 8, W 32
     (1, 1600, 200),     # 10.8 channels per SM: eighths scan
     (1, 14800, 100),    # 100 channels per SM: quadrant scan
     (1, 29600, 40),     # 200 channels per SM: quadrant scan
