@@ -11,7 +11,8 @@ State Space Model for Apple Silicon" (or the wiki page "Selective State Space
 Models (Mamba)") that it follows; see the C source for the step list.
 
 Parity pins (tests/test_oracle_pins.py) tie every function here to something
-other than itself: the recurrence == convolution identity and the worked
+other than itself (for the conv stage: numpy.correlate and scipy's expit; for
+the whole layer: closed forms with W_x = 0 and with dt at its upper clip): the recurrence == convolution identity and the worked
 example of the Ultralytics glossary page "State Space Models (SSM)", the
 geometric-series closed form, the A_log = log(1..N) initialisation, a brute
 force of the unrolled (attention-like) form, and decode == prefill.
@@ -69,6 +70,8 @@ def _load():
             lib.oracle_ssm_scan_fwd.argtypes = [ctypes.c_int] * 5 + [_dp] * 12 + [_dp] * 3 + [ctypes.c_int]
             lib.oracle_ssm_step.restype = ctypes.c_int
             lib.oracle_ssm_step.argtypes = [ctypes.c_int] * 4 + [_dp] * 10 + [_dp] * 3 + [ctypes.c_int]
+            lib.oracle_conv_silu.restype = ctypes.c_int
+            lib.oracle_conv_silu.argtypes = [ctypes.c_int] * 4 + [_dp] * 5
             _lib = lib
     return _lib
 
@@ -164,6 +167,53 @@ def step(x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
     if rc != 0:
         raise RuntimeError("oracle_ssm_step failed")
     return y, cc, ss
+
+
+def conv_silu(x, conv_w, conv_b, conv_cache=None):
+    """u = SiLU(causal depthwise conv1d(x)) over (B,L,E), fp64: the conv output
+    that feeds the projection f_proj of the full layer (Axon-SSM page,
+    "Selective mechanism")."""
+    x, conv_w, conv_b = (_f64(v) for v in (x, conv_w, conv_b))
+    Bsz, L, E = x.shape
+    K = conv_w.shape[1]
+    cc = None if conv_cache is None else _f64(conv_cache)
+    u = np.zeros((Bsz, L, E))
+    rc = _load().oracle_conv_silu(Bsz, L, E, K, _ptr(x), _ptr(conv_w), _ptr(conv_b), _ptr(cc), _ptr(u))
+    if rc != 0:
+        raise RuntimeError("oracle_conv_silu failed")
+    return u
+
+
+def block_fwd(X, W_in, W_x, W_out, conv_w, conv_b, dt_bias, A_log, D,
+              conv_cache=None, ssm_state=None, zoh=False):
+    """The whole Axon-SSM layer, fp64, in the page's order:
+
+      (x, z) = split(X W_in)                 ("Gating": the input projection makes
+                                              the two branches; W_in is (Dm, 2E),
+                                              x = first E columns)
+      u = SiLU(conv(x))                      (conv output)
+      (dt_raw, B, C) = split(u W_x)          ("Selective mechanism": f_proj is a
+                                              linear map of the conv output; W_x is
+                                              (E, E + 2N): dt_raw, then B, then C)
+      y = scan(x, z, dt_raw, B, C)           (the layer core: recurrence, D skip,
+                                              SiLU(z) gate -- ``scan_fwd``)
+      out = y W_out                          ("Gating": y_out = W_out (y_ssm * SiLU(z)))
+
+    The matrix products are numpy's (fp64); the scan is the C oracle.
+    Returns (out (B,L,Dm), conv_cache_out, ssm_state_out).
+    """
+    X, W_in, W_x, W_out = (_f64(v) for v in (X, W_in, W_x, W_out))
+    E = W_in.shape[1] // 2
+    N = _f64(A_log).shape[1]
+    assert W_in.shape[1] == 2 * E and W_x.shape == (E, E + 2 * N) and W_out.shape[0] == E
+    xz = X @ W_in
+    x, z = xz[..., :E], xz[..., E:]
+    u = conv_silu(x, conv_w, conv_b, conv_cache)
+    p = u @ W_x
+    dt_raw, Bm, Cm = p[..., :E], p[..., E:E + N], p[..., E + N:]
+    y, cc, ss = scan_fwd(x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
+                         conv_cache, ssm_state, zoh=zoh)
+    return y @ W_out, cc, ss
 
 
 def scan_channels(inputs: dict, channels, zoh=False):

@@ -157,3 +157,33 @@ int oracle_ssm_step(int B, int E, int N, int K,
                                dt_bias, A_log, D, conv_cache, ssm_state,
                                y, conv_cache, ssm_state, zoh);
 }
+
+/*
+ * The conv + SiLU stage alone (steps 1-2 above without the recurrence):
+ * u[b,t,e] = SiLU(conv_b[e] + sum_k conv_w[e,k] * x[b, t+k-(K-1), e]), with
+ * times before 0 read from conv_cache_in (or zeros).  In the full layer this
+ * u is the input of the projection f_proj that produces dt, B and C (Axon-SSM
+ * page, "Selective mechanism": the projection starts from the conv output).
+ */
+int oracle_conv_silu(int B, int L, int E, int K, const double *x, const double *conv_w,
+                     const double *conv_b, const double *conv_cache_in, double *u)
+{
+    if (B < 0 || L < 0 || E < 0 || K <= 0) return -1;
+    const int KM1 = K - 1;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < L; ++t)
+            for (int e = 0; e < E; ++e) {
+                double acc = conv_b[e];
+                for (int k = 0; k < K; ++k) {
+                    const int s = t + k - KM1;          /* input time met by tap k */
+                    double xv = 0.0;
+                    if (s >= 0)
+                        xv = x[((size_t)b * L + s) * E + e];
+                    else if (conv_cache_in)
+                        xv = conv_cache_in[((size_t)b * KM1 + (KM1 + s)) * E + e];
+                    acc += conv_w[(size_t)e * K + k] * xv;
+                }
+                u[((size_t)b * L + t) * E + e] = oracle_silu(acc);
+            }
+    return 0;
+}

@@ -31,6 +31,10 @@ MUTANTS = {
     "input_before_decay": ("h[n] = abar * h[n] + bbar * u;", "h[n] = abar * (h[n] + bbar * u);"),
     "silu_as_sigmoid": ("double oracle_silu(double v) { return v / (1.0 + exp(-v)); }",
                         "double oracle_silu(double v) { return 1.0 / (1.0 + exp(-v)); }"),
+    "conv_stage_taps_reversed": ("acc += conv_w[(size_t)e * K + k] * xv;",
+                                 "acc += conv_w[(size_t)e * K + (K - 1 - k)] * xv;"),
+    "conv_stage_cache_order": ("xv = conv_cache_in[((size_t)b * KM1 + (KM1 + s)) * E + e];",
+                               "xv = conv_cache_in[((size_t)b * KM1 + (-1 - s)) * E + e];"),
     "zoh_missing_A_division": ("double bbar = zoh ? expm1(dt * A[n]) / A[n] * Bm[bn] : dt * Bm[bn];",
                                "double bbar = zoh ? expm1(dt * A[n]) * Bm[bn] : dt * Bm[bn];"),
 }

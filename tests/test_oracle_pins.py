@@ -15,7 +15,10 @@ Sources of truth used here (none re-types the oracle's own loop):
   * prefill == prefill + cached steps == chunked prefill (the streaming
     `model.step(chunk, state)` pattern of the wiki page "Selective State Space
     Models (Mamba)");
-  * causality and zero-input decay.
+  * causality and zero-input decay;
+  * for the conv stage alone, numpy.correlate; for the whole layer (input
+    projection, conv, f_proj, scan, output projection), closed forms with the
+    projection to the SSM parameters zeroed or reduced to its dt, B or C part.
 """
 import json
 import os
@@ -387,3 +390,108 @@ def test_sampled_channels_match_full_run():
         np.testing.assert_array_equal(s["y"][i], y[b, :, e])
         np.testing.assert_array_equal(s["conv_cache"][i], cc[b, :, e])
         np.testing.assert_array_equal(s["ssm_state"][i], ss[b, e])
+
+
+# ---------------------------------------------------------------- full layer
+def ref_conv_silu(x, conv_w, conv_b, cache):
+    """SiLU(causal depthwise conv) by numpy.correlate on the padded stream."""
+    B, L, E = x.shape
+    K = conv_w.shape[1]
+    u = np.zeros((B, L, E))
+    for b in range(B):
+        for e in range(E):
+            xpad = np.concatenate([cache[b, :, e] if cache is not None else np.zeros(K - 1), x[b, :, e]])
+            u[b, :, e] = ref_silu(conv_b[e] + np.correlate(xpad, conv_w[e], mode="valid"))
+    return u
+
+
+@pytest.mark.parametrize("with_cache", [False, True])
+def test_conv_silu_matches_correlate(with_cache):
+    rng = np.random.default_rng(71)
+    B, L, E, K = 2, 9, 3, 4
+    x = rng.standard_normal((B, L, E))
+    w = rng.standard_normal((E, K))
+    cb = rng.standard_normal(E)
+    cache = rng.standard_normal((B, K - 1, E)) if with_cache else None
+    np.testing.assert_allclose(oracle.conv_silu(x, w, cb, cache), ref_conv_silu(x, w, cb, cache),
+                               rtol=1e-13, atol=1e-13)
+
+
+def rand_block(rng, B=2, L=6, Dm=5, E=4, N=16, K=4):
+    return {
+        "X": rng.standard_normal((B, L, Dm)),
+        "W_in": rng.standard_normal((Dm, 2 * E)) / np.sqrt(Dm),
+        "W_x": rng.standard_normal((E, E + 2 * N)) / np.sqrt(E),
+        "W_out": rng.standard_normal((E, Dm)) / np.sqrt(E),
+        "conv_w": rng.standard_normal((E, K)) * 0.5,
+        "conv_b": rng.standard_normal(E) * 0.1,
+        "dt_bias": np.log(np.expm1(rng.uniform(1e-3, 1e-1, E))),
+        "A_log": np.log(np.tile(np.arange(1, N + 1, dtype=np.float64), (E, 1))),
+        "D": rng.standard_normal(E),
+        "conv_cache": rng.standard_normal((B, K - 1, E)),
+        "ssm_state": rng.standard_normal((B, E, N)),
+    }
+
+
+def run_block(d, **over):
+    d = {**d, **over}
+    return oracle.block_fwd(d["X"], d["W_in"], d["W_x"], d["W_out"], d["conv_w"], d["conv_b"],
+                            d["dt_bias"], d["A_log"], d["D"], d["conv_cache"], d["ssm_state"])
+
+
+def test_block_without_projection_to_ssm_is_gated_skip():
+    """W_x = 0: dt_raw = B = C = 0, so y_ssm = D u and the state only decays
+    with dt = softplus(dt_bias): out = (D u SiLU(z)) W_out, h_L = h0 exp(L dt A)."""
+    rng = np.random.default_rng(72)
+    d = rand_block(rng)
+    E, N, L = d["W_out"].shape[0], d["A_log"].shape[1], d["X"].shape[1]
+    W_x = np.zeros_like(d["W_x"])
+    out, _, ss = run_block(d, W_x=W_x)
+    xz = d["X"] @ d["W_in"]
+    x, z = xz[..., :E], xz[..., E:]
+    u = ref_conv_silu(x, d["conv_w"], d["conv_b"], d["conv_cache"])
+    np.testing.assert_allclose(out, (d["D"] * u * ref_silu(z)) @ d["W_out"], rtol=1e-11, atol=1e-12)
+    dt = ref_dt(d["dt_bias"])                                     # (E,)
+    A = -np.arange(1, N + 1, dtype=np.float64)
+    np.testing.assert_allclose(ss, d["ssm_state"] * np.exp(L * dt[:, None] * A[None, :]),
+                               rtol=1e-11, atol=1e-14)
+
+
+def test_block_dt_columns_set_the_decay():
+    """B = C = 0 (their columns of W_x zeroed): the state decays by
+    exp(A sum_t dt_t) with dt_t = clip(softplus(dt_raw_t + dt_bias)) and dt_raw
+    = u W_x[:, :E]; the output is still the gated skip."""
+    rng = np.random.default_rng(73)
+    d = rand_block(rng)
+    E, N = d["W_out"].shape[0], d["A_log"].shape[1]
+    W_x = d["W_x"].copy()
+    W_x[:, E:] = 0.0
+    out, _, ss = run_block(d, W_x=W_x)
+    xz = d["X"] @ d["W_in"]
+    x, z = xz[..., :E], xz[..., E:]
+    u = ref_conv_silu(x, d["conv_w"], d["conv_b"], d["conv_cache"])
+    dt = ref_dt(u @ W_x[:, :E] + d["dt_bias"])                     # (B, L, E)
+    A = -np.arange(1, N + 1, dtype=np.float64)
+    np.testing.assert_allclose(ss, d["ssm_state"] * np.exp(dt.sum(axis=1)[..., None] * A),
+                               rtol=1e-11, atol=1e-14)
+    np.testing.assert_allclose(out, (d["D"] * u * ref_silu(z)) @ d["W_out"], rtol=1e-11, atol=1e-12)
+
+
+def test_block_upper_clip_reads_B_then_C():
+    """dt at its upper clip (dt_bias = 200, dt columns zero): abar = exp(-100 n)
+    vanishes, so h_t = 100 B_t u_t -- the final state names the B columns of
+    W_x -- and y = u (100 sum_n C_t,n B_t,n + D) SiLU(z)."""
+    rng = np.random.default_rng(74)
+    d = rand_block(rng)
+    E, N = d["W_out"].shape[0], d["A_log"].shape[1]
+    W_x = d["W_x"].copy()
+    W_x[:, :E] = 0.0
+    out, _, ss = run_block(d, W_x=W_x, dt_bias=np.full(E, 200.0))
+    xz = d["X"] @ d["W_in"]
+    x, z = xz[..., :E], xz[..., E:]
+    u = ref_conv_silu(x, d["conv_w"], d["conv_b"], d["conv_cache"])
+    Bt = u @ W_x[:, E:E + N]                                      # (B, L, N)
+    Ct = u @ W_x[:, E + N:]
+    np.testing.assert_allclose(ss, 100.0 * u[:, -1, :, None] * Bt[:, -1, None, :], rtol=1e-11, atol=1e-12)
+    y = u * (100.0 * (Ct * Bt).sum(-1, keepdims=True) + d["D"]) * ref_silu(z)
+    np.testing.assert_allclose(out, y @ d["W_out"], rtol=1e-10, atol=1e-11)
