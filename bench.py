@@ -47,6 +47,7 @@ UNIT = "G token·channel/s"
 MUFU_PER_TOKEN_CH = 16 + 6
 MUFU_LANES_PER_SM_CLK = 16
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -102,9 +103,10 @@ def measured_peaks():
         with open(path) as f:
             d = json.load(f)
         return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
-                "source": "measured"}
+                "bf16_tflops": float(d.get("bf16_tflops", FALLBACK_BF16_TFLOPS)), "source": "measured"}
     except Exception:
-        return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0, "source": "fallback"}
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "source": "fallback"}
 
 
 def scan_model(wl) -> dict:
@@ -358,6 +360,46 @@ def bench_zoh_prefill(wl, sets, params, out, ws, dev, launches: int = 20) -> dic
     return {"kernel_ms": ms, "value": T / (ms / 1e3) / 1e9, "unit": UNIT, "launches": launches}
 
 
+def bench_block(dev, launches: int = 10) -> dict:
+    """The whole Axon-SSM layer (input projection, conv stage, projection to
+    dt/B/C, fused scan, output projection; axon_ssm_block_fwd) on the Bit-Axon
+    layer (B1 L2048 D2560 E7680, bf16): mean event time of `launches` calls."""
+    from selective_state_space_52_b200 import axon_ssm
+    bw = W.BLOCK_WORKLOAD_BY_NAME["bit_axon_block"]
+    inp = {k: v.to(dev) for k, v in W.make_block_inputs(bw).items()}
+    weights = {k: inp[k] for k in axon_ssm.WEIGHT_KEYS}
+    params = {k: inp[k] for k in axon_ssm.PARAM_KEYS}
+    M, Dm, E, N = bw.B * bw.L, bw.Dm, bw.E, bw.N
+    out = torch.empty(bw.B, bw.L, Dm, dtype=torch.bfloat16, device=dev)
+    cc = torch.empty(bw.B, bw.K - 1, E, dtype=torch.bfloat16, device=dev)
+    ss = torch.empty(bw.B, E, N, dtype=torch.float32, device=dev)
+    ws = torch.empty(axon_ssm.axon_ssm_block_workspace_bytes(bw.B, bw.L, Dm, E, N, bw.K), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call():
+        axon_ssm.block_fwd(inp["X"], weights, params, None, out=(out, cc, ss), workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    times = []
+    for _ in range(launches):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream); call(); b.record(stream)
+        torch.cuda.synchronize(dev)
+        times.append(a.elapsed_time(b))
+    ms = statistics.mean(times)
+    flops = 2 * M * (Dm * 2 * E + E * (E + 2 * N) + E * Dm)
+    peaks = measured_peaks()
+    return {"workload": "Axon-SSM layer: B1 L2048 D2560 E7680 N16 K4, bf16, weights and input resident",
+            "ms": ms, "tokens_per_s": M / (ms / 1e3),
+            "gemm_flops": flops, "gemm_tflops_over_layer_time": flops / (ms / 1e3) / 1e12,
+            "bf16_peak_tflops": peaks.get("bf16_tflops"),
+            "note": "four bf16 GEMMs (cuBLASLt, fp32 accumulate) + conv stage + fused scan; "
+                    "the scan alone is the prefill kernel of this line's roofline"}
+
+
 def workload_desc(wl) -> str:
     return (f"{wl.name}: B{wl.B} L{wl.L} E{wl.E} N{wl.N} K{wl.K}, {wl.io} io, fp32 state; "
             "step = prefill + 1 cached decode token")
@@ -514,6 +556,8 @@ def run_axon(args, wl):
     if not args.no_decode_bench:
         line["decode"] = bench_decode(dev)
         line["prefill_zoh"] = bench_zoh_prefill(wl, sets, params, (y, cc, ss), ws, dev)
+    if not args.no_block_bench and world == 1:
+        line["block"] = bench_block(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inp_cpu = {**params_cpu, **{k: v.cpu() for k, v in sets[0].items()}}
         rate, units, secs, ch = time_oracle(wl, inp_cpu, args.cpu_budget)
@@ -539,6 +583,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-bench", action="store_true",
                     help="skip the separate cached-decode measurement (decode workload shapes)")
+    ap.add_argument("--no-block-bench", action="store_true",
+                    help="skip the whole-layer measurement (input/output projections around the scan)")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the cached-decode measurement and print it as one JSON line "
                          "(for profiling the step kernel alone)")

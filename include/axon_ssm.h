@@ -3,7 +3,8 @@
  *
  * The operation is the Axon-SSM layer core of the page "Axon-SSM: Selective
  * State Space Model for Apple Silicon" (bit-axon docs), between its input and
- * output projections (which are not part of this library):
+ * output projections (axon_ssm_block_fwd, at the end of this file, adds the
+ * projections around it):
  *
  *   xc_t  = conv_b + sum_{k<K} conv_w[k] * xpad[t+k]     causal depthwise conv1d,
  *           xpad = conv_cache ++ x, tap K-1 meets x_t    (section "Implementation
@@ -45,7 +46,8 @@
  *    even on output).  Arithmetic is float32 throughout; the state is float32.
  *  - Pointers are DEVICE pointers owned by the caller.  The library never
  *    allocates, frees or retains them; scratch memory comes from the caller
- *    through `workspace`.  Every pointer must be 16-byte aligned, and E must be
+ *    through `workspace` (axon_ssm_block_fwd's cuBLASLt handle is the one
+ *    library-owned object).  Every pointer must be 16-byte aligned, and E must be
  *    a multiple of 8 (bf16) or 4 (f32), else AXON_ERR_ALIGNMENT.  There is no
  *    fallback path.
  *  - Work is enqueued on `stream` and runs asynchronously.  Arguments are
@@ -281,6 +283,43 @@ AXON_API axon_status axon_ssm_step_ex(
     const float *conv_w, const float *conv_b,
     const float *dt_bias, const float *A_log, const float *D,
     void *conv_cache, float *ssm_state, void *y, axon_stream_t stream);
+
+/*
+ * The whole Axon-SSM layer around the layer core (Axon-SSM page, sections
+ * "Gating" and "Selective mechanism"), bf16 io only:
+ *
+ *   (x, z)          = split(X W_in)       X (B,L,Dm); W_in (Dm, 2E): x = columns
+ *                                         [0, E), z = columns [E, 2E)
+ *   u               = SiLU(conv(x))       the conv output (conv_w, conv_b, cache)
+ *   (dt_raw, B, C)  = split(u W_x)        f_proj, one linear map of the conv
+ *                                         output; W_x (E, E+2N): dt_raw = columns
+ *                                         [0, E), B = [E, E+N), C = [E+N, E+2N)
+ *   y               = layer core          axon_ssm_scan_fwd on (x, z, dt_raw, B, C)
+ *   out             = y W_out             W_out (E, Dm); out (B,L,Dm)
+ *
+ * Weights are row-major bf16 ("activations times weights").  The four matrix
+ * products are plain bf16 GEMMs with float32 accumulation run by cuBLASLt
+ * (one handle per device, created on first use); the conv stage and the layer
+ * core run in this library's kernels.  The intermediates x, z, u, dt_raw, B,
+ * C and y are stored in bf16 inside `workspace`, which must hold at least
+ * axon_ssm_block_workspace_bytes(...) bytes (16-byte aligned; it also serves
+ * as the GEMMs' and the scan's scratch).  Caches and parameters as for
+ * axon_ssm_scan_fwd (in == out allowed); conv_cache_out receives the last K-1
+ * rows of x.  Dm and E must be multiples of 8 (AXON_ERR_ALIGNMENT); io other
+ * than AXON_BF16, N != 16 or K != 4 return AXON_ERR_UNSUPPORTED; out and the
+ * workspace must not overlap each other, X, the weights or the caches
+ * (AXON_ERR_INVALID_ARG).  L == 0 copies the caches in -> out.
+ */
+AXON_API size_t axon_ssm_block_workspace_bytes(int B, int L, int Dm, int E, int N, int K, axon_dtype io);
+
+AXON_API axon_status axon_ssm_block_fwd(
+    int B, int L, int Dm, int E, int N, int K, axon_dtype io,
+    const void *X, const void *W_in, const void *W_x, const void *W_out,
+    const float *conv_w, const float *conv_b,
+    const float *dt_bias, const float *A_log, const float *D,
+    const void *conv_cache_in, const float *ssm_state_in,
+    void *out, void *conv_cache_out, float *ssm_state_out,
+    void *workspace, size_t workspace_bytes, axon_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -184,8 +184,14 @@ def conv_silu(x, conv_w, conv_b, conv_cache=None):
     return u
 
 
+def _round_bf16(a: np.ndarray) -> np.ndarray:
+    """Round to the nearest bfloat16 (ties to even), returned as float64."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).double().numpy()
+
+
 def block_fwd(X, W_in, W_x, W_out, conv_w, conv_b, dt_bias, A_log, D,
-              conv_cache=None, ssm_state=None, zoh=False):
+              conv_cache=None, ssm_state=None, zoh=False, bf16_intermediates=False):
     """The whole Axon-SSM layer, fp64, in the page's order:
 
       (x, z) = split(X W_in)                 ("Gating": the input projection makes
@@ -199,21 +205,25 @@ def block_fwd(X, W_in, W_x, W_out, conv_w, conv_b, dt_bias, A_log, D,
                                               SiLU(z) gate -- ``scan_fwd``)
       out = y W_out                          ("Gating": y_out = W_out (y_ssm * SiLU(z)))
 
-    The matrix products are numpy's (fp64); the scan is the C oracle.
+    The matrix products are numpy's (fp64); the scan is the C oracle.  With
+    ``bf16_intermediates`` the values a bf16 layer stores between its stages
+    (x, z, u, dt_raw, B, C and y) are rounded to bf16 where it stores them;
+    everything else stays fp64.
     Returns (out (B,L,Dm), conv_cache_out, ssm_state_out).
     """
     X, W_in, W_x, W_out = (_f64(v) for v in (X, W_in, W_x, W_out))
     E = W_in.shape[1] // 2
     N = _f64(A_log).shape[1]
     assert W_in.shape[1] == 2 * E and W_x.shape == (E, E + 2 * N) and W_out.shape[0] == E
+    rnd = _round_bf16 if bf16_intermediates else (lambda a: a)
     xz = X @ W_in
-    x, z = xz[..., :E], xz[..., E:]
-    u = conv_silu(x, conv_w, conv_b, conv_cache)
+    x, z = rnd(xz[..., :E]), rnd(xz[..., E:])
+    u = rnd(conv_silu(x, conv_w, conv_b, conv_cache))
     p = u @ W_x
-    dt_raw, Bm, Cm = p[..., :E], p[..., E:E + N], p[..., E + N:]
+    dt_raw, Bm, Cm = rnd(p[..., :E]), rnd(p[..., E:E + N]), rnd(p[..., E + N:])
     y, cc, ss = scan_fwd(x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
                          conv_cache, ssm_state, zoh=zoh)
-    return y @ W_out, cc, ss
+    return rnd(y) @ W_out, cc, ss
 
 
 def scan_channels(inputs: dict, channels, zoh=False):

@@ -62,6 +62,10 @@ AXON_DISC_ZOH = 1
 _DISC = {"first_order": AXON_DISC_FIRST_ORDER, "zoh": AXON_DISC_ZOH}
 _lib.axon_ssm_step.restype = _i
 _lib.axon_ssm_step.argtypes = [_i] * 5 + [_vp] * 13 + [_vp]
+_lib.axon_ssm_block_workspace_bytes.restype = _sz
+_lib.axon_ssm_block_workspace_bytes.argtypes = [_i] * 7
+_lib.axon_ssm_block_fwd.restype = _i
+_lib.axon_ssm_block_fwd.argtypes = [_i] * 7 + [_vp] * 14 + [_vp, _sz, _vp]
 
 
 class AxonError(RuntimeError):
@@ -204,8 +208,26 @@ def axon_ssm_step(B, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias,
     return rc
 
 
+def axon_ssm_block_workspace_bytes(B, L, Dm, E, N=16, K=4, io=AXON_BF16) -> int:
+    return int(_lib.axon_ssm_block_workspace_bytes(B, L, Dm, E, N, K, io))
+
+
+def axon_ssm_block_fwd(B, L, Dm, E, N, K, io, X, W_in, W_x, W_out, conv_w, conv_b, dt_bias,
+                       A_log, D, conv_cache_in, ssm_state_in, out, conv_cache_out, ssm_state_out,
+                       workspace, workspace_bytes, stream=None, *, raise_on_error=True) -> int:
+    rc = _lib.axon_ssm_block_fwd(B, L, Dm, E, N, K, io, _p(X), _p(W_in), _p(W_x), _p(W_out),
+                                 _p(conv_w), _p(conv_b), _p(dt_bias), _p(A_log), _p(D),
+                                 _p(conv_cache_in), _p(ssm_state_in), _p(out), _p(conv_cache_out),
+                                 _p(ssm_state_out), _p(workspace), int(workspace_bytes),
+                                 _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_ssm_block_fwd")
+    return rc
+
+
 # ------------------------------------------------------------ conveniences
 PARAM_KEYS = ("conv_w", "conv_b", "dt_bias", "A_log", "D")
+WEIGHT_KEYS = ("W_in", "W_x", "W_out")
 
 
 def scan_fwd(x, z, dt_raw, Bm, Cm, params: dict, cache=None, *, num_segments=None,
@@ -265,3 +287,33 @@ def step(x, z, dt_raw, Bm, Cm, params: dict, cache, *, y=None, stream=None,
     else:
         axon_ssm_step(Bsz, E, N, K, _dtype_code(x.dtype), *args, stream=stream)
     return y
+
+
+def block_fwd(X, weights: dict, params: dict, cache=None, *, out=None, workspace=None, stream=None):
+    """The whole Axon-SSM layer on (B, L, Dm) bf16 input ``X``.
+
+    ``weights`` holds W_in (Dm, 2E), W_x (E, E+2N), W_out (E, Dm) in bf16;
+    ``params`` and ``cache`` as for ``scan_fwd``.  Returns
+    ``(out, (conv_cache, ssm_state))``.
+    """
+    Bsz, L, Dm = X.shape
+    E = weights["W_in"].shape[1] // 2
+    K = params["conv_w"].shape[1]
+    N = params["A_log"].shape[1]
+    dev = X.device
+    cc_in, ss_in = (None, None) if cache is None else cache
+    if out is None:
+        y = torch.empty_like(X)
+        cc_out = torch.empty(Bsz, K - 1, E, dtype=X.dtype, device=dev)
+        ss_out = torch.empty(Bsz, E, N, dtype=torch.float32, device=dev)
+    else:
+        y, cc_out, ss_out = out
+    io = _dtype_code(X.dtype)
+    nbytes = axon_ssm_block_workspace_bytes(Bsz, L, Dm, E, N, K, io)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    wsz = workspace.numel() * workspace.element_size()
+    axon_ssm_block_fwd(Bsz, L, Dm, E, N, K, io, X, weights["W_in"], weights["W_x"], weights["W_out"],
+                       *(params[k] for k in PARAM_KEYS), cc_in, ss_in, y, cc_out, ss_out,
+                       workspace, wsz, stream=stream)
+    return y, (cc_out, ss_out)

@@ -3,7 +3,8 @@
     python -m selective_state_space_52_b200.build [--force] [--verbose]
 
 The shared library is written next to this file, so it ships with the source
-tree; nothing is installed into site-packages.  cudart is linked statically.
+tree; nothing is installed into site-packages.  cudart is linked statically,
+cuBLASLt (the whole-layer entry point's GEMMs) dynamically from the toolkit.
 """
 from __future__ import annotations
 
@@ -23,6 +24,7 @@ LIB = os.path.join(PKG, "libaxon_ssm.so")
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--use_fast_math", "-Xcompiler", "-fPIC",
               "-Xcompiler", "-fvisibility=hidden", "-shared", "-cudart", "static"]
+LINK_LIBS = ["-lcublasLt"]    # the block's plain GEMMs
 
 
 def _nvcc() -> str:
@@ -53,7 +55,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [_nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, f"-I{INCLUDE}", f"-I{CSRC}",
-           *extra, *sources(), "-o", tmp]
+           *extra, *sources(), *LINK_LIBS, "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)

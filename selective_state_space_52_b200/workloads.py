@@ -16,6 +16,12 @@ Distributions ("config-0 distributions"), for every workload below:
   D = 1
 The Mamba-block workload adds a bimodal dt: even channels u = 1e-4 (long
 memory), odd channels u = 1.0 (fast forgetting), same dt_raw noise.
+
+The whole-layer workloads (``BLOCK_WORKLOADS``) draw the layer input
+X ~ N(0, 1) and the projection weights with fan-in scaling, W_in ~ N(0, 1/Dm),
+W_x ~ N(0, 1/E), W_out ~ N(0, 1/E), all rounded to bf16 once; the per-channel
+parameters are those above (drawn for E channels).  dt_raw, B and C then come
+out of the projection with standard deviation about 0.6.
 """
 from __future__ import annotations
 
@@ -147,3 +153,47 @@ def make_decode_inputs(wl: Workload, steps: int, g: torch.Generator | None = Non
         "B": torch.randn(S, Bsz, N, generator=g, dtype=torch.float32).to(io),
         "C": torch.randn(S, Bsz, N, generator=g, dtype=torch.float32).to(io),
     }
+
+
+# ------------------------------------------------------------ whole layer
+@dataclass(frozen=True)
+class BlockWorkload:
+    name: str
+    B: int
+    L: int
+    Dm: int          # hidden size D of the layer configuration table
+    E: int           # d_inner = expand * D
+    seed: int
+    note: str = ""
+    N: int = N_STATE
+    K: int = K_CONV
+
+    def core(self) -> Workload:
+        """The layer-core workload with the same per-channel parameters."""
+        return Workload(self.name, self.B, self.L, self.E, "bf16", self.seed)
+
+
+BLOCK_WORKLOADS = [
+    BlockWorkload("bit_axon_block", 1, 2048, 2560, 7680, 11,
+                  note="the Bit-Axon layer: D=2560, expand 3 -> E=7680, bf16"),
+    BlockWorkload("small_block", 2, 100, 256, 768, 12, note="small layer for parity tests"),
+]
+BLOCK_WORKLOAD_BY_NAME = {w.name: w for w in BLOCK_WORKLOADS}
+
+
+def make_block_inputs(bw: BlockWorkload, with_state: bool = False, L: int | None = None,
+                      B: int | None = None) -> dict:
+    """X (B,L,Dm), W_in (Dm,2E), W_x (E,E+2N), W_out (E,Dm) in bf16, plus the
+    per-channel parameters (and an initial cache pair with ``with_state``)."""
+    g = _gen(bw.seed + 5000)
+    Bsz = bw.B if B is None else B
+    L = bw.L if L is None else L
+    Dm, E, N = bw.Dm, bw.E, bw.N
+    out = make_params(bw.core())
+    out["X"] = torch.randn(Bsz, L, Dm, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    out["W_in"] = (torch.randn(Dm, 2 * E, generator=g, dtype=torch.float32) / math.sqrt(Dm)).to(torch.bfloat16)
+    out["W_x"] = (torch.randn(E, E + 2 * N, generator=g, dtype=torch.float32) / math.sqrt(E)).to(torch.bfloat16)
+    out["W_out"] = (torch.randn(E, Dm, generator=g, dtype=torch.float32) / math.sqrt(E)).to(torch.bfloat16)
+    if with_state:
+        out.update(make_state(bw.core(), B=Bsz))
+    return out

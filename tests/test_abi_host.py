@@ -195,3 +195,46 @@ def test_binding_module_exposes_c_names():
     from selective_state_space_52_b200 import axon_ssm
     for name in declared_symbols():
         assert callable(getattr(axon_ssm, name)), name
+
+
+def _block(lib, **over):
+    a = dict(B=1, L=64, Dm=256, E=768, N=16, K=4, io=1, ws_bytes=1 << 34)
+    ptr_names = ["X", "W_in", "W_x", "W_out", "conv_w", "conv_b", "dt_bias", "A_log", "D",
+                 "cc_in", "ss_in", "out", "cc_out", "ss_out", "ws"]
+    for i, n in enumerate(ptr_names):
+        a[n] = FAKE + (i << 32)          # far apart: no overlaps unless a case makes one
+    a["cc_in"] = a["ss_in"] = None
+    a.update(over)
+    f = lib.axon_ssm_block_fwd
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int] * 7 + [ctypes.c_void_p] * 14 + [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    return f(a["B"], a["L"], a["Dm"], a["E"], a["N"], a["K"], a["io"], *(a[n] for n in ptr_names[:14]),
+             a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(B=-1), INVALID),
+    (dict(io=0), UNSUPPORTED),                     # the whole layer is bf16 only
+    (dict(N=8), UNSUPPORTED),
+    (dict(Dm=260), ALIGNMENT),
+    (dict(E=772), ALIGNMENT),
+    (dict(X=None), INVALID),
+    (dict(W_x=None), INVALID),
+    (dict(ws=None), INVALID),
+    (dict(W_in=FAKE + 8), ALIGNMENT),
+    (dict(ws_bytes=1024), WORKSPACE),
+    (dict(out=FAKE), INVALID),                     # out overlaps X
+    (dict(ws=FAKE + (2 << 32)), INVALID),          # workspace overlaps W_x
+])
+def test_block_rejects_bad_arguments(lib, over, status):
+    assert _block(lib, **over) == status
+
+
+def test_block_workspace_query(lib):
+    q = lib.axon_ssm_block_workspace_bytes
+    q.restype = ctypes.c_size_t
+    q.argtypes = [ctypes.c_int] * 7
+    need = q(1, 2048, 2560, 7680, 16, 4, 1)
+    assert need >= 5 * 2048 * 7680 * 2 + (32 << 20)      # five (M, E) bf16 intermediates + GEMM scratch
+    assert q(1, 2048, 2560, 7680, 16, 4, 0) == 0          # fp32 io: not supported
+    assert _block(lib, ws_bytes=need - 1, L=2048, Dm=2560, E=7680) == WORKSPACE

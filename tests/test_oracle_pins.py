@@ -495,3 +495,10 @@ def test_block_upper_clip_reads_B_then_C():
     np.testing.assert_allclose(ss, 100.0 * u[:, -1, :, None] * Bt[:, -1, None, :], rtol=1e-11, atol=1e-12)
     y = u * (100.0 * (Ct * Bt).sum(-1, keepdims=True) + d["D"]) * ref_silu(z)
     np.testing.assert_allclose(out, y @ d["W_out"], rtol=1e-10, atol=1e-11)
+
+
+def test_bf16_rounding_of_intermediates():
+    """The oracle's bf16 model rounds to nearest, ties to even (8 significant
+    bits): 1 + 2^-8 is a tie -> 1, 1 + 3*2^-8 a tie -> 1 + 2^-6, 1 + 2^-9 -> 1."""
+    v = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -9, -3.0, 0.15625])
+    np.testing.assert_array_equal(oracle._round_bf16(v), [1.0, 1.0 + 2.0 ** -6, 1.0, -3.0, 0.15625])
