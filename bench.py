@@ -481,38 +481,60 @@ def run_axon(args, wl):
     units_step = B * (L + 1) * E
     value = rank_units(units_step, world) * args.steps / (ms / 1e3) / 1e9
 
-    # ---- end to end through the public API with host buffers (pinned)
+    # ---- end to end through the public API with host buffers (pinned).  The
+    # steps are pipelined the way a serving loop runs them: step i's upload
+    # (its own stream) overlaps step i-1's compute and download (another
+    # stream); device inputs, outputs and caches are double-buffered.
     host = {k: v.cpu().pin_memory() for k, v in sets[0].items()}
     host_tok = {k: v.cpu().pin_memory() for k, v in tok.items()}
-    dev_in = {k: torch.empty_like(v) for k, v in sets[0].items()}
-    dev_tok = {k: torch.empty_like(v) for k, v in tok.items()}
-    y_host = torch.empty(y.shape, dtype=io).pin_memory()
-    ytok_host = torch.empty(y_tok.shape, dtype=io).pin_memory()
+    nbuf = 2
+    dev_in = [{k: torch.empty_like(v) for k, v in sets[0].items()} for _ in range(nbuf)]
+    dev_tok = [{k: torch.empty_like(v) for k, v in tok.items()} for _ in range(nbuf)]
+    y_dev = [y] + [torch.empty_like(y) for _ in range(nbuf - 1)]
+    ytok_dev = [y_tok] + [torch.empty_like(y_tok) for _ in range(nbuf - 1)]
+    caches = [(cc, ss)] + [(torch.empty_like(cc), torch.empty_like(ss)) for _ in range(nbuf - 1)]
+    y_host = [torch.empty(y.shape, dtype=io).pin_memory() for _ in range(nbuf)]
+    ytok_host = [torch.empty(y_tok.shape, dtype=io).pin_memory() for _ in range(nbuf)]
     h2d = sum(v.numel() * v.element_size() for v in host.values()) + \
         sum(v.numel() * v.element_size() for v in host_tok.values())
-    d2h = y_host.numel() * y_host.element_size() + ytok_host.numel() * ytok_host.element_size()
+    d2h = y_host[0].numel() * y_host[0].element_size() + ytok_host[0].numel() * ytok_host[0].element_size()
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {name: [torch.cuda.Event() for _ in range(nbuf)] for name in ("in_ready", "in_free", "out_ready", "out_free")}
 
-    def e2e_step():
-        for k in host:
-            dev_in[k].copy_(host[k], non_blocking=True)
-        for k in host_tok:
-            dev_tok[k].copy_(host_tok[k], non_blocking=True)
-        axon_ssm.scan_fwd(dev_in["x"], dev_in["z"], dev_in["dt_raw"], dev_in["B"], dev_in["C"],
-                          params, None, out=(y, cc, ss), workspace=ws)
-        axon_ssm.step(dev_tok["x"], dev_tok["z"], dev_tok["dt_raw"], dev_tok["B"], dev_tok["C"],
-                      params, (cc, ss), y=y_tok)
-        y_host.copy_(y, non_blocking=True)
-        ytok_host.copy_(y_tok, non_blocking=True)
+    def e2e_step(i):
+        k = i % nbuf
+        with torch.cuda.stream(up):
+            up.wait_event(ev["in_free"][k])          # step i-2's compute is done with these buffers
+            for kk in host:
+                dev_in[k][kk].copy_(host[kk], non_blocking=True)
+            for kk in host_tok:
+                dev_tok[k][kk].copy_(host_tok[kk], non_blocking=True)
+            ev["in_ready"][k].record(up)
+        stream.wait_event(ev["in_ready"][k])
+        stream.wait_event(ev["out_free"][k])         # step i-2's download has read y_dev[k]
+        d, t = dev_in[k], dev_tok[k]
+        axon_ssm.scan_fwd(d["x"], d["z"], d["dt_raw"], d["B"], d["C"], params, None,
+                          out=(y_dev[k], *caches[k]), workspace=ws)
+        axon_ssm.step(t["x"], t["z"], t["dt_raw"], t["B"], t["C"], params, caches[k], y=ytok_dev[k])
+        ev["in_free"][k].record(stream)
+        ev["out_ready"][k].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(ev["out_ready"][k])
+            y_host[k].copy_(y_dev[k], non_blocking=True)
+            ytok_host[k].copy_(ytok_dev[k], non_blocking=True)
+            ev["out_free"][k].record(down)
 
     e2e_steps = max(3, min(args.steps, 50))
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     barrier(dev)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    up.wait_event(a)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    stream.wait_event(ev["out_free"][(e2e_steps - 1) % nbuf])   # the last download is inside the region
     b.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = reduce_max(a.elapsed_time(b), dev)
@@ -548,7 +570,9 @@ def run_axon(args, wl):
         "decode_step": {"us": step_ms * 1e3, "algorithmic_bytes": stm["bytes"],
                         "hbm_gbs": stm["bytes"] / (step_ms / 1e3) / 1e9},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "pipeline": "pinned host buffers; step i's upload overlaps step i-1's compute and "
+                            "download (separate streams, two device buffer sets)"},
         "clocks": clk,
         "gpu_launches": args.steps * (scan_launches + 1),
     }
