@@ -285,6 +285,37 @@ AXON_API axon_status axon_ssm_step_ex(
     void *conv_cache, float *ssm_state, void *y, axon_stream_t stream);
 
 /*
+ * A sequence split by time across P devices (slice r = tokens [r*L/P, ...)),
+ * with one exchange of per-slice summaries (the chunked associative scan of
+ * the SSD article, devices as blocks; the recurrence's decay over a run of
+ * tokens is exp(A * sum dt), Axon-SSM page, recurrence equation):
+ *   1. every slice r >= 1 runs axon_ssm_scan_fwd from a ZERO state (its conv
+ *      cache = the last K-1 inputs of slice r-1) for its end state h_loc_r,
+ *      and axon_ssm_dt_sum for dt_sum_r; slice 0 runs from the true initial
+ *      state, its end state is h_loc_0 and its output is final;
+ *   2. the P (h_loc, dt_sum) pairs are exchanged (one all-gather);
+ *   3. axon_ssm_carry_fold gives slice r its entering state
+ *      h = h_loc_0; h = exp(A * dt_sum_j) * h + h_loc_j for j = 1 .. r-1;
+ *   4. slice r runs axon_ssm_scan_fwd again from that state: its y and end
+ *      caches are final (the last slice's caches are the sequence's).
+ *
+ * axon_ssm_dt_sum: dt_sum (B,E) float32 = sum over t of clip(softplus(dt_raw
+ * + dt_bias), 1e-4, 100) (section "Selective mechanism"); dt_raw (B,L,E) io.
+ * dt_sum is zeroed on the stream first and accumulated with atomic adds, so
+ * its last bits may vary from run to run.
+ * axon_ssm_carry_fold: h_loc (P,B,E,N) and dt_sum (P,B,E) float32 as
+ * gathered (index = slice), A_log (E,N); writes h_in (B,E,N) for slice r,
+ * 1 <= r < P (AXON_ERR_INVALID_ARG otherwise).  Conventions as above; h_in
+ * must not overlap the inputs.
+ */
+AXON_API axon_status axon_ssm_dt_sum(int B, int L, int E, axon_dtype io, const void *dt_raw,
+                                     const float *dt_bias, float *dt_sum, axon_stream_t stream);
+
+AXON_API axon_status axon_ssm_carry_fold(int P, int r, int B, int E, int N, const float *A_log,
+                                         const float *h_loc, const float *dt_sum, float *h_in,
+                                         axon_stream_t stream);
+
+/*
  * The whole Axon-SSM layer around the layer core (Axon-SSM page, sections
  * "Gating" and "Selective mechanism"), bf16 io only:
  *

@@ -62,6 +62,10 @@ AXON_DISC_ZOH = 1
 _DISC = {"first_order": AXON_DISC_FIRST_ORDER, "zoh": AXON_DISC_ZOH}
 _lib.axon_ssm_step.restype = _i
 _lib.axon_ssm_step.argtypes = [_i] * 5 + [_vp] * 13 + [_vp]
+_lib.axon_ssm_dt_sum.restype = _i
+_lib.axon_ssm_dt_sum.argtypes = [_i] * 4 + [_vp] * 3 + [_vp]
+_lib.axon_ssm_carry_fold.restype = _i
+_lib.axon_ssm_carry_fold.argtypes = [_i] * 5 + [_vp] * 4 + [_vp]
 _lib.axon_ssm_block_workspace_bytes.restype = _sz
 _lib.axon_ssm_block_workspace_bytes.argtypes = [_i] * 7
 _lib.axon_ssm_block_fwd.restype = _i
@@ -208,6 +212,22 @@ def axon_ssm_step(B, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias,
     return rc
 
 
+def axon_ssm_dt_sum(B, L, E, io, dt_raw, dt_bias, dt_sum, stream=None, *, raise_on_error=True) -> int:
+    rc = _lib.axon_ssm_dt_sum(B, L, E, io, _p(dt_raw), _p(dt_bias), _p(dt_sum), _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_ssm_dt_sum")
+    return rc
+
+
+def axon_ssm_carry_fold(P, r, B, E, N, A_log, h_loc, dt_sum, h_in, stream=None, *,
+                        raise_on_error=True) -> int:
+    rc = _lib.axon_ssm_carry_fold(P, r, B, E, N, _p(A_log), _p(h_loc), _p(dt_sum), _p(h_in),
+                                  _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_ssm_carry_fold")
+    return rc
+
+
 def axon_ssm_block_workspace_bytes(B, L, Dm, E, N=16, K=4, io=AXON_BF16) -> int:
     return int(_lib.axon_ssm_block_workspace_bytes(B, L, Dm, E, N, K, io))
 
@@ -317,3 +337,20 @@ def block_fwd(X, weights: dict, params: dict, cache=None, *, out=None, workspace
                        *(params[k] for k in PARAM_KEYS), cc_in, ss_in, y, cc_out, ss_out,
                        workspace, wsz, stream=stream)
     return y, (cc_out, ss_out)
+
+
+def dt_sum(dt_raw, dt_bias, *, stream=None):
+    """(B, E) float32: the sum over the sequence of clip(softplus(dt_raw + dt_bias))."""
+    Bsz, L, E = dt_raw.shape
+    out = torch.empty(Bsz, E, dtype=torch.float32, device=dt_raw.device)
+    axon_ssm_dt_sum(Bsz, L, E, _dtype_code(dt_raw.dtype), dt_raw, dt_bias, out, stream=stream)
+    return out
+
+
+def carry_fold(r, A_log, h_loc_all, dt_sum_all, *, stream=None):
+    """The state entering slice r of a time-split sequence from the stacked
+    (P,B,E,N) end states and (P,B,E) dt sums of all slices."""
+    P, Bsz, E, N = h_loc_all.shape
+    out = torch.empty(Bsz, E, N, dtype=torch.float32, device=h_loc_all.device)
+    axon_ssm_carry_fold(P, r, Bsz, E, N, A_log, h_loc_all, dt_sum_all, out, stream=stream)
+    return out

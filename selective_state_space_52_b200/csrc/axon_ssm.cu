@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "axon_ssm.h"
+#include "carry.cuh"
 #include "device_math.cuh"
 #include "scan_chunked.cuh"
 #include "scan_octo.cuh"
@@ -582,6 +583,46 @@ axon_status axon_ssm_scan_fwd_noalloc(int B, int L, int E, int N, int K, axon_dt
                      conv_cache_in, ssm_state_in, y, conv_cache_out, ssm_state_out,
                      scratch, scratch ? kStaticScratchBytes : 0, num_segments,
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+axon_status axon_ssm_dt_sum(int B, int L, int E, axon_dtype io, const void* dt_raw,
+                            const float* dt_bias, float* dt_sum, axon_stream_t stream) {
+    if (B < 0 || L < 0 || E < 0) return AXON_ERR_INVALID_ARG;
+    if (io != AXON_F32 && io != AXON_BF16) return AXON_ERR_UNSUPPORTED;
+    if (B > 65535 || (long long)B * E > (1LL << 31)) return AXON_ERR_UNSUPPORTED;
+    if (B == 0 || E == 0) return AXON_OK;
+    if (!dt_bias || !dt_sum || (L > 0 && !dt_raw)) return AXON_ERR_INVALID_ARG;
+    if ((dt_raw && !aligned16(dt_raw)) || !aligned16(dt_bias) || !aligned16(dt_sum)) return AXON_ERR_ALIGNMENT;
+    if (L > 0 && overlaps(dt_raw, (size_t)B * L * E * io_bytes(io), dt_sum, (size_t)B * E * 4))
+        return AXON_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(dt_sum, 0, (size_t)B * E * sizeof(float), st) != cudaSuccess) return AXON_ERR_CUDA;
+    if (L == 0) return AXON_OK;
+    const dim3 grid((unsigned)((E + kDtSumThreads - 1) / kDtSumThreads),
+                    (unsigned)((L + kDtSumRun - 1) / kDtSumRun), (unsigned)B);
+    if (grid.y > 65535u) return AXON_ERR_UNSUPPORTED;
+    if (io == AXON_BF16) dt_sum_kernel<IoBF16><<<grid, kDtSumThreads, 0, st>>>(L, E, dt_raw, dt_bias, dt_sum);
+    else dt_sum_kernel<IoF32><<<grid, kDtSumThreads, 0, st>>>(L, E, dt_raw, dt_bias, dt_sum);
+    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+}
+
+axon_status axon_ssm_carry_fold(int P, int r, int B, int E, int N, const float* A_log,
+                                const float* h_loc, const float* dt_sum, float* h_in,
+                                axon_stream_t stream) {
+    if (P < 1 || r < 1 || r >= P || B < 0 || E < 0) return AXON_ERR_INVALID_ARG;
+    if (N != kN) return AXON_ERR_UNSUPPORTED;
+    if ((long long)B * E > (1LL << 31) / kN) return AXON_ERR_UNSUPPORTED;
+    if (B == 0 || E == 0) return AXON_OK;
+    if (!A_log || !h_loc || !dt_sum || !h_in) return AXON_ERR_INVALID_ARG;
+    if (!aligned16(A_log) || !aligned16(h_loc) || !aligned16(dt_sum) || !aligned16(h_in))
+        return AXON_ERR_ALIGNMENT;
+    const size_t state = (size_t)B * E * kN * 4;
+    if (overlaps(h_in, state, h_loc, (size_t)P * state) || overlaps(h_in, state, dt_sum, (size_t)P * B * E * 4))
+        return AXON_ERR_INVALID_ARG;
+    const size_t total = (size_t)B * E * kN;
+    carry_fold_kernel<<<(unsigned)((total + 127) / 128), 128, 0, static_cast<cudaStream_t>(stream)>>>(
+        r, B, E, A_log, h_loc, dt_sum, h_in);
+    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -238,3 +238,25 @@ def test_block_workspace_query(lib):
     assert need >= 5 * 2048 * 7680 * 2 + (32 << 20)      # five (M, E) bf16 intermediates + GEMM scratch
     assert q(1, 2048, 2560, 7680, 16, 4, 0) == 0          # fp32 io: not supported
     assert _block(lib, ws_bytes=need - 1, L=2048, Dm=2560, E=7680) == WORKSPACE
+
+
+def test_time_split_pieces_reject_bad_arguments(lib):
+    s = lib.axon_ssm_dt_sum
+    s.restype = ctypes.c_int
+    s.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p] * 4
+    assert s(-1, 8, 16, 1, FAKE, FAKE + 0x10000, FAKE + 0x20000, None) == INVALID
+    assert s(1, 8, 16, 5, FAKE, FAKE + 0x10000, FAKE + 0x20000, None) == UNSUPPORTED
+    assert s(1, 8, 16, 1, FAKE, None, FAKE + 0x20000, None) == INVALID
+    assert s(1, 8, 16, 1, FAKE + 2, FAKE + 0x10000, FAKE + 0x20000, None) == ALIGNMENT
+    assert s(1, 8, 16, 1, FAKE, FAKE + 0x10000, FAKE + 16, None) == INVALID      # sum overlaps dt_raw
+    assert s(0, 8, 16, 1, FAKE, FAKE + 0x10000, FAKE + 0x20000, None) == OK       # nothing to do
+    f = lib.axon_ssm_carry_fold
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 5
+    args = (FAKE, FAKE + 0x100000, FAKE + 0x200000, FAKE + 0x300000, None)
+    assert f(4, 0, 1, 16, 16, *args) == INVALID          # slice 0 has no carry to fold
+    assert f(4, 4, 1, 16, 16, *args) == INVALID          # r < P
+    assert f(0, 1, 1, 16, 16, *args) == INVALID
+    assert f(4, 1, 1, 16, 8, *args) == UNSUPPORTED
+    assert f(4, 1, 1, 16, 16, FAKE, FAKE + 0x100000, FAKE + 0x200000, FAKE + 0x100000, None) == INVALID
+    assert f(4, 1, 1, 16, 16, FAKE, FAKE + 0x100004, FAKE + 0x200000, FAKE + 0x300000, None) == ALIGNMENT
