@@ -400,6 +400,52 @@ def bench_block(dev, launches: int = 10) -> dict:
                     "the scan alone is the prefill kernel of this line's roofline"}
 
 
+def bench_time_split(wl, s, params, dev, P: int = 4, launches: int = 10) -> dict:
+    """The time-split protocol (shard.py) on the bench workload's sequence cut
+    into P slices, all on this one GPU: the whole protocol, and one rank's own
+    work (slice 1: scan from a zero state + dt sum, then fold + scan again),
+    which is what each of P GPUs would run besides the two small exchanges."""
+    from selective_state_space_52_b200 import shard
+    L = wl.L
+    cut = [L * r // P for r in range(P + 1)]
+    slices = [{k: s[k][:, cut[r]:cut[r + 1]].contiguous() for k in ("x", "z", "dt_raw", "B", "C")}
+              for r in range(P)]
+    ops = shard.cuda_ops()
+    K = wl.K
+    stream = torch.cuda.current_stream(dev)
+
+    def whole():
+        shard.sliced_scan_local(slices, params, None, ops)
+
+    tails = [shard.slice_tail(sl["x"], K) for sl in slices]
+    firsts = [shard.first_pass(r, sl, params, tails[r - 1] if r else None, None, ops) for r, sl in enumerate(slices)]
+    h_all = torch.stack([f[2] for f in firsts])
+    dts_all = torch.stack([f[3] for f in firsts])
+
+    def one_rank():
+        shard.first_pass(1, slices[1], params, tails[0], None, ops)
+        shard.second_pass(1, slices[1], params, tails[0], h_all, dts_all, ops)
+
+    res = {}
+    for name, fn in (("protocol_ms", whole), ("one_rank_ms", one_rank)):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(launches):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = a.elapsed_time(b) / launches
+    exch = P * (wl.B * wl.E * (wl.N + 1) * 4 + wl.B * (wl.K - 1) * wl.E * 2)
+    return {"workload": f"prefill of B{wl.B} L{L} E{wl.E} N{wl.N} K{wl.K} {wl.io}, cut into {P} slices "
+                        f"of {L // P} tokens", "slices": P,
+            **res, "exchange_bytes_per_rank": exch,
+            "note": "all slices on one GPU (one GPU per call here); on P GPUs each rank runs one_rank_ms "
+                    "of work plus two all-gathers of the listed bytes"}
+
+
 def workload_desc(wl) -> str:
     return (f"{wl.name}: B{wl.B} L{wl.L} E{wl.E} N{wl.N} K{wl.K}, {wl.io} io, fp32 state; "
             "step = prefill + 1 cached decode token")
@@ -582,6 +628,7 @@ def run_axon(args, wl):
         line["prefill_zoh"] = bench_zoh_prefill(wl, sets, params, (y, cc, ss), ws, dev)
     if not args.no_block_bench and world == 1:
         line["block"] = bench_block(dev)
+        line["time_split"] = bench_time_split(wl, sets[0], params, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inp_cpu = {**params_cpu, **{k: v.cpu() for k, v in sets[0].items()}}
         rate, units, secs, ch = time_oracle(wl, inp_cpu, args.cpu_budget)
