@@ -55,9 +55,12 @@
  *    nothing was launched and no output was touched.  AXON_ERR_CUDA reports a
  *    failed launch; faults that occur later surface at the caller's next
  *    synchronisation, as for any CUDA kernel.
- *  - Apart from axon_ssm_scan_fwd_noalloc (below), the library holds no
- *    mutable global state; concurrent calls on different streams with
- *    disjoint outputs are safe.
+ *  - Global state: per-device caches of read-only facts (SM count, shared-
+ *    memory limit, each kernel's raised shared-memory limit) and, for
+ *    axon_ssm_block_fwd, one cuBLASLt handle per device, all set up once under
+ *    a lock or with atomics; and the scratch array of
+ *    axon_ssm_scan_fwd_noalloc (below).  Otherwise concurrent calls on
+ *    different streams with disjoint outputs are safe.
  *  - `axon_stream_t` is the CUDA runtime's cudaStream_t (a CUstream_st
  *    pointer); NULL means the legacy default stream.
  */

@@ -1,6 +1,7 @@
 // axon_ssm.cu -- host side of the C ABI declared in include/axon_ssm.h:
 // argument checks (nothing is launched on any error), the launch plan, and the
-// kernel launches on the caller's stream.  The library allocates nothing.
+// kernel launches on the caller's stream.  The library allocates no device
+// memory: scratch comes from the caller's workspace.
 #include <cuda_runtime.h>
 
 #include <atomic>
