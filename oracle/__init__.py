@@ -72,6 +72,8 @@ def _load():
             lib.oracle_ssm_step.argtypes = [ctypes.c_int] * 4 + [_dp] * 10 + [_dp] * 3 + [ctypes.c_int]
             lib.oracle_conv_silu.restype = ctypes.c_int
             lib.oracle_conv_silu.argtypes = [ctypes.c_int] * 4 + [_dp] * 5
+            lib.oracle_ssd_scan.restype = ctypes.c_int
+            lib.oracle_ssd_scan.argtypes = [ctypes.c_int] * 5 + [_dp] * 10
             _lib = lib
     return _lib
 
@@ -224,6 +226,27 @@ def block_fwd(X, W_in, W_x, W_out, conv_w, conv_b, dt_bias, A_log, D,
     y, cc, ss = scan_fwd(x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
                          conv_cache, ssm_state, zoh=zoh)
     return rnd(y) @ W_out, cc, ss
+
+
+def ssd_scan(x, dt_raw, dt_bias, A_log, Bm, Cm, D, h0=None):
+    """The Mamba-2 (SSD) layer core with one scalar decay per head, fp64 (wiki
+    page "Selective State Space Models (Mamba)", section "Mamba-2 block (SSD)").
+
+    x (B,L,H,P); dt_raw (B,L,H); dt_bias, A_log, D (H,); Bm, Cm (B,L,N) shared
+    by all heads; h0 (B,H,P,N) or None.  Returns (y (B,L,H,P), h_out (B,H,P,N)).
+    """
+    x, dt_raw, Bm, Cm = (_f64(v) for v in (x, dt_raw, Bm, Cm))
+    dt_bias, A_log, D = (_f64(v) for v in (dt_bias, A_log, D))
+    Bsz, L, H, P = x.shape
+    N = Bm.shape[2]
+    hh = None if h0 is None else _f64(h0)
+    y = np.zeros((Bsz, L, H, P))
+    h_out = np.zeros((Bsz, H, P, N))
+    rc = _load().oracle_ssd_scan(Bsz, L, H, P, N, _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A_log),
+                                 _ptr(Bm), _ptr(Cm), _ptr(D), _ptr(hh), _ptr(y), _ptr(h_out))
+    if rc != 0:
+        raise RuntimeError("oracle_ssd_scan failed")
+    return y, h_out
 
 
 def scan_channels(inputs: dict, channels, zoh=False):

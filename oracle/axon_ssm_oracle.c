@@ -187,3 +187,49 @@ int oracle_conv_silu(int B, int L, int E, int K, const double *x, const double *
             }
     return 0;
 }
+
+/*
+ * The Mamba-2 (SSD) layer core, one scalar decay per head (wiki page
+ * "Selective State Space Models (Mamba)", section "Mamba-2 block (SSD)":
+ * d_state 128, headdim 64; the SSD article: a structured SSM whose state is
+ * carried token to token).  Per batch row b and head h, state S (P x N):
+ *   dt  = clip(softplus(dt_raw[b,t,h] + dt_bias[h]), 1e-4, 100)
+ *   a   = exp(dt * A_h),  A_h = -exp(A_log[h])
+ *   S[p][n] = a * S[p][n] + dt * x[b,t,h,p] * B[b,t,n]
+ *   y[b,t,h,p] = sum_n S[p][n] * C[b,t,n] + D[h] * x[b,t,h,p]
+ * Layouts: x, y (B,L,H,P); dt_raw (B,L,H); B, C (B,L,N) shared by all heads;
+ * dt_bias, A_log, D (H); h0, h_out (B,H,P,N), h0 may be NULL (zeros).
+ */
+int oracle_ssd_scan(int B, int L, int H, int P, int N, const double *x, const double *dt_raw,
+                    const double *dt_bias, const double *A_log, const double *Bm, const double *Cm,
+                    const double *D, const double *h0, double *y, double *h_out)
+{
+    if (B < 0 || L < 0 || H < 0 || P <= 0 || N <= 0) return -1;
+    double *S = (double *)malloc(sizeof(double) * (size_t)P * N);
+    if (!S) return -1;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const double A = -exp(A_log[h]);
+            for (int i = 0; i < P * N; ++i) S[i] = h0 ? h0[((size_t)b * H + h) * P * N + i] : 0.0;
+            for (int t = 0; t < L; ++t) {
+                const double dt = oracle_dt(dt_raw[((size_t)b * L + t) * H + h] + dt_bias[h]);
+                const double a = exp(dt * A);
+                const double *xv = x + (((size_t)b * L + t) * H + h) * P;
+                const double *Bt = Bm + ((size_t)b * L + t) * N;
+                const double *Ct = Cm + ((size_t)b * L + t) * N;
+                double *yv = y + (((size_t)b * L + t) * H + h) * P;
+                for (int p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (int n = 0; n < N; ++n) {
+                        double *s = S + (size_t)p * N + n;
+                        *s = a * *s + dt * xv[p] * Bt[n];
+                        acc += *s * Ct[n];
+                    }
+                    yv[p] = acc + D[h] * xv[p];
+                }
+            }
+            for (int i = 0; i < P * N; ++i) h_out[((size_t)b * H + h) * P * N + i] = S[i];
+        }
+    free(S);
+    return 0;
+}

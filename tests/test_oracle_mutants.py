@@ -35,6 +35,9 @@ MUTANTS = {
                                  "acc += conv_w[(size_t)e * K + (K - 1 - k)] * xv;"),
     "conv_stage_cache_order": ("xv = conv_cache_in[((size_t)b * KM1 + (KM1 + s)) * E + e];",
                                "xv = conv_cache_in[((size_t)b * KM1 + (-1 - s)) * E + e];"),
+    "ssd_input_without_dt": ("*s = a * *s + dt * xv[p] * Bt[n];", "*s = a * *s + xv[p] * Bt[n];"),
+    "ssd_decay_sign": ("const double A = -exp(A_log[h]);", "const double A = exp(A_log[h]);"),
+    "ssd_C_replaced_by_B": ("acc += *s * Ct[n];", "acc += *s * Bt[n];"),
     "zoh_missing_A_division": ("double bbar = zoh ? expm1(dt * A[n]) / A[n] * Bm[bn] : dt * Bm[bn];",
                                "double bbar = zoh ? expm1(dt * A[n]) * Bm[bn] : dt * Bm[bn];"),
 }

@@ -502,3 +502,52 @@ def test_bf16_rounding_of_intermediates():
     bits): 1 + 2^-8 is a tie -> 1, 1 + 3*2^-8 a tie -> 1 + 2^-6, 1 + 2^-9 -> 1."""
     v = np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -9, -3.0, 0.15625])
     np.testing.assert_array_equal(oracle._round_bf16(v), [1.0, 1.0 + 2.0 ** -6, 1.0, -3.0, 0.15625])
+
+
+# ---------------------------------------------------------------- Mamba-2 SSD core
+def rand_ssd(rng, B=2, L=23, H=3, P=4, N=5):
+    return {"x": rng.standard_normal((B, L, H, P)), "dt_raw": rng.standard_normal((B, L, H)) * 0.7,
+            "dt_bias": np.log(np.expm1(rng.uniform(1e-2, 0.3, H))), "A_log": rng.uniform(-1.0, 1.5, H),
+            "Bm": rng.standard_normal((B, L, N)), "Cm": rng.standard_normal((B, L, N)),
+            "D": rng.standard_normal(H), "h0": rng.standard_normal((B, H, P, N))}
+
+
+@pytest.mark.parametrize("with_state", [False, True])
+def test_ssd_matches_its_attention_form(with_state):
+    """The state-space duality of the SSD article, written with numpy.einsum:
+    y_i = sum_{j<=i} (C_i . B_j) exp(A (S_i - S_j)) dt_j x_j + exp(A S_i) h0 C_i + D x_i,
+    S = cumsum(dt); and h_L = exp(A S_L) h0 + sum_j exp(A (S_L - S_j)) dt_j x_j B_j^T."""
+    rng = np.random.default_rng(81)
+    d = rand_ssd(rng)
+    h0 = d["h0"] if with_state else None
+    y, hL = oracle.ssd_scan(d["x"], d["dt_raw"], d["dt_bias"], d["A_log"], d["Bm"], d["Cm"], d["D"], h0)
+    dt = ref_dt(d["dt_raw"] + d["dt_bias"])                          # (B,L,H)
+    A = -np.exp(d["A_log"])                                           # (H,)
+    S = np.cumsum(dt, axis=1)                                         # (B,L,H)
+    L = dt.shape[1]
+    G = np.einsum("bin,bjn->bij", d["Cm"], d["Bm"])                   # (B,L,L)
+    decay = np.exp(A[None, None, None, :] * (S[:, :, None, :] - S[:, None, :, :]))   # (B,i,j,H)
+    mask = np.tril(np.ones((L, L)))[None, :, :, None]
+    W_ = G[..., None] * decay * mask * dt[:, None, :, :]              # (B,i,j,H)
+    y_ref = np.einsum("bijh,bjhp->bihp", W_, d["x"]) + d["D"][None, None, :, None] * d["x"]
+    h_ref = np.einsum("bjh,bjhp,bjn->bhpn", np.exp(A * (S[:, -1:, :] - S)) * dt, d["x"], d["Bm"])
+    if with_state:
+        y_ref += np.einsum("bih,bhpn,bin->bihp", np.exp(A * S), h0, d["Cm"])
+        h_ref += np.exp(A * S[:, -1, :])[:, :, None, None] * h0
+    np.testing.assert_allclose(y, y_ref, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(hL, h_ref, rtol=1e-10, atol=1e-10)
+
+
+def test_ssd_upper_clip_forgets_at_once():
+    """dt at its upper clip (dt_bias = 200) with A = -1: exp(-100) removes the
+    past, so y_t = 100 (C_t . B_t) x_t + D x_t and h_L = 100 x_L B_L^T."""
+    rng = np.random.default_rng(82)
+    d = rand_ssd(rng)
+    H = d["D"].shape[0]
+    y, hL = oracle.ssd_scan(d["x"], d["dt_raw"], np.full(H, 200.0), np.zeros(H), d["Bm"], d["Cm"],
+                            d["D"], d["h0"])
+    cb = (d["Cm"] * d["Bm"]).sum(-1)                                  # (B,L)
+    np.testing.assert_allclose(y, (100.0 * cb[..., None, None] + d["D"][None, None, :, None]) * d["x"],
+                               rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(hL, 100.0 * np.einsum("bhp,bn->bhpn", d["x"][:, -1], d["Bm"][:, -1]),
+                               rtol=1e-10, atol=1e-10)
