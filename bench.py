@@ -446,6 +446,54 @@ def bench_time_split(wl, s, params, dev, P: int = 4, launches: int = 10) -> dict
                     "of work plus two all-gathers of the listed bytes"}
 
 
+def bench_ssd(dev, launches: int = 20) -> dict:
+    """The Mamba-2 (SSD) layer core (axon_ssd_scan_fwd) on the Mamba-2 block's
+    heads: B1 L4096, 64 heads of 64, d_state 128, bf16; mean event time, with
+    its HBM and tensor-core rooflines."""
+    from selective_state_space_52_b200 import axon_ssm
+    sw = W.SSD_WORKLOAD_BY_NAME["mamba2_ssd"]
+    inp = {k: v.to(dev) for k, v in W.make_ssd_inputs(sw).items()}
+    params = {k: inp[k] for k in ("dt_bias", "A_log", "D")}
+    y = torch.empty_like(inp["x"])
+    h = torch.empty(sw.B, sw.H, sw.P, sw.N, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(axon_ssm.axon_ssd_workspace_bytes(sw.B, sw.L, sw.H, sw.P, sw.N), 16),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call():
+        axon_ssm.ssd_scan(inp["x"], inp["dt_raw"], inp["B"], inp["C"], params, None, out=(y, h), workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    times = []
+    for _ in range(launches):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream); call(); b.record(stream)
+        torch.cuda.synchronize(dev)
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    Q, P, N, H, L, B = 64, sw.P, sw.N, sw.H, sw.L, sw.B
+    nC = (L + Q - 1) // Q
+    # per chunk: C B^T once; per chunk and head: exp(acum) C S_in, the causal
+    # half of the masked Gram times x, and x^T (w B)
+    flops = B * nC * (2 * Q * Q * N + H * (2 * Q * N * P + Q * Q * P + 2 * P * N * Q))
+    nbytes = B * L * H * P * 2 * 2 + B * L * (H * 2 + 2 * N * 2) + B * H * P * N * 4
+    peaks = measured_peaks()
+    hbm = nbytes / (ms / 1e3) / 1e9
+    tfl = flops / (ms / 1e3) / 1e12
+    return {"workload": "Mamba-2 (SSD) core: B1 L4096, 64 heads x 64, d_state 128, bf16; L2 flushed",
+            "ms": ms, "algorithmic_bytes": nbytes, "flops": flops,
+            "hbm": {"achieved": hbm, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": hbm / peaks["hbm_gbs"]},
+            "tensor": {"achieved": tfl, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                       "frac": tfl / peaks["bf16_tflops"],
+                       "note": "bf16 mma.sync (m16n8k16) tensor path; the carried-state product runs twice "
+                               "(hi and lo parts), counted once"},
+            "token_head_per_s": B * L * H / (ms / 1e3)}
+
+
 def workload_desc(wl) -> str:
     return (f"{wl.name}: B{wl.B} L{wl.L} E{wl.E} N{wl.N} K{wl.K}, {wl.io} io, fp32 state; "
             "step = prefill + 1 cached decode token")
@@ -629,6 +677,7 @@ def run_axon(args, wl):
     if not args.no_block_bench and world == 1:
         line["block"] = bench_block(dev)
         line["time_split"] = bench_time_split(wl, sets[0], params, dev)
+        line["ssd"] = bench_ssd(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inp_cpu = {**params_cpu, **{k: v.cpu() for k, v in sets[0].items()}}
         rate, units, secs, ch = time_oracle(wl, inp_cpu, args.cpu_budget)

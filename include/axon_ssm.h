@@ -319,6 +319,33 @@ AXON_API axon_status axon_ssm_carry_fold(int P, int r, int B, int E, int N, cons
                                          axon_stream_t stream);
 
 /*
+ * The Mamba-2 (SSD) layer core: one scalar decay per head (wiki page
+ * "Selective State Space Models (Mamba)", section "Mamba-2 block (SSD)":
+ * d_state 128, headdim 64), computed as a chunked scan on the tensor cores
+ * (the SSD article: masked matrix products inside 64-token chunks, a carried
+ * state between them).  Per batch row b and head h, state S (P x N):
+ *   dt = clip(softplus(dt_raw[b,t,h] + dt_bias[h]), 1e-4, 100),
+ *   S  = exp(dt * A_h) S + dt * x[b,t,h,:] B[b,t,:]^T,  A_h = -exp(A_log[h]),
+ *   y[b,t,h,:] = S C[b,t,:] + D[h] x[b,t,h,:].
+ * Layouts: x, y (B,L,H,P) bf16; dt_raw (B,L,H) bf16; Bm, Cm (B,L,N) bf16,
+ * shared by all heads; dt_bias, A_log, D (H) float32; h0 (B,H,P,N) float32 or
+ * NULL (zeros); h_out (B,H,P,N) float32, may be h0 itself.  P == 64, N == 128
+ * and io == AXON_BF16 only (else AXON_ERR_UNSUPPORTED).  The products take
+ * bf16 operands (the decayed chunk Gram matrix, dt-weighted B, and the
+ * carried state split in two bf16 parts) with float32 accumulation; the
+ * carried state itself is float32.  `workspace` holds axon_ssd_workspace_bytes(...) bytes (the chunk
+ * Gram matrices C B^T, B * ceil(L/64) * 64 * 64 floats).  Other conventions
+ * as above.
+ */
+AXON_API size_t axon_ssd_workspace_bytes(int B, int L, int H, int P, int N);
+
+AXON_API axon_status axon_ssd_scan_fwd(
+    int B, int L, int H, int P, int N, axon_dtype io,
+    const void *x, const void *dt_raw, const float *dt_bias, const float *A_log,
+    const void *Bm, const void *Cm, const float *D, const float *h0,
+    void *y, float *h_out, void *workspace, size_t workspace_bytes, axon_stream_t stream);
+
+/*
  * The whole Axon-SSM layer around the layer core (Axon-SSM page, sections
  * "Gating" and "Selective mechanism"), bf16 io only:
  *

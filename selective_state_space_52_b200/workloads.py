@@ -17,6 +17,11 @@ Distributions ("config-0 distributions"), for every workload below:
 The Mamba-block workload adds a bimodal dt: even channels u = 1e-4 (long
 memory), odd channels u = 1.0 (fast forgetting), same dt_raw noise.
 
+The Mamba-2 (SSD) workloads (``SSD_WORKLOADS``): x ~ N(0, 1) (B,L,H,64),
+dt_raw ~ N(0, 0.5), B, C ~ N(0, 1) (B,L,128) in bf16; per head dt_bias =
+log(expm1(u)), u ~ logUniform[1e-3, 1e-1], A_log = log(Uniform[1, 16]) and
+D = 1; an initial state h0 ~ N(0, 1/4).
+
 The whole-layer workloads (``BLOCK_WORKLOADS``) draw the layer input
 X ~ N(0, 1) and the projection weights with fan-in scaling, W_in ~ N(0, 1/Dm),
 W_x ~ N(0, 1/E), W_out ~ N(0, 1/E), all rounded to bf16 once; the per-channel
@@ -196,4 +201,46 @@ def make_block_inputs(bw: BlockWorkload, with_state: bool = False, L: int | None
     out["W_out"] = (torch.randn(E, Dm, generator=g, dtype=torch.float32) / math.sqrt(E)).to(torch.bfloat16)
     if with_state:
         out.update(make_state(bw.core(), B=Bsz))
+    return out
+
+
+# ------------------------------------------------------------ Mamba-2 (SSD) core
+@dataclass(frozen=True)
+class SsdWorkload:
+    name: str
+    B: int
+    L: int
+    H: int
+    seed: int
+    P: int = 64
+    N: int = 128
+    note: str = ""
+
+
+SSD_WORKLOADS = [
+    SsdWorkload("mamba2_ssd", 1, 4096, 64, 21,
+                note="Mamba-2 block: d_model 2048, expand 2 -> 64 heads of 64, d_state 128, bf16"),
+    SsdWorkload("small_ssd", 2, 130, 3, 22, note="small SSD case for parity tests"),
+]
+SSD_WORKLOAD_BY_NAME = {w.name: w for w in SSD_WORKLOADS}
+
+
+def make_ssd_inputs(sw: SsdWorkload, with_state: bool = False, L: int | None = None) -> dict:
+    g = _gen(sw.seed + 7000)
+    L = sw.L if L is None else L
+    B, H, P, N = sw.B, sw.H, sw.P, sw.N
+    bf = torch.bfloat16
+    lo, hi = math.log(1e-3), math.log(1e-1)
+    u = torch.exp(lo + (hi - lo) * torch.rand(H, generator=g, dtype=torch.float64))
+    out = {
+        "x": torch.randn(B, L, H, P, generator=g, dtype=torch.float32).to(bf),
+        "dt_raw": (torch.randn(B, L, H, generator=g, dtype=torch.float32) * math.sqrt(0.5)).to(bf),
+        "B": torch.randn(B, L, N, generator=g, dtype=torch.float32).to(bf),
+        "C": torch.randn(B, L, N, generator=g, dtype=torch.float32).to(bf),
+        "dt_bias": torch.log(torch.expm1(u)).to(torch.float32),
+        "A_log": torch.log(1.0 + 15.0 * torch.rand(H, generator=g, dtype=torch.float64)).to(torch.float32),
+        "D": torch.ones(H, dtype=torch.float32),
+    }
+    if with_state:
+        out["h0"] = torch.randn(B, H, P, N, generator=g, dtype=torch.float32) * 0.5
     return out

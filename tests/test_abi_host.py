@@ -260,3 +260,34 @@ def test_time_split_pieces_reject_bad_arguments(lib):
     assert f(4, 1, 1, 16, 8, *args) == UNSUPPORTED
     assert f(4, 1, 1, 16, 16, FAKE, FAKE + 0x100000, FAKE + 0x200000, FAKE + 0x100000, None) == INVALID
     assert f(4, 1, 1, 16, 16, FAKE, FAKE + 0x100004, FAKE + 0x200000, FAKE + 0x300000, None) == ALIGNMENT
+
+
+def test_ssd_rejects_bad_arguments(lib):
+    f = lib.axon_ssd_scan_fwd
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 10 + [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    ptrs = [FAKE + (i << 32) for i in range(10)]      # x, dt_raw, dt_bias, A_log, B, C, D, h0, y, h_out
+    ws = FAKE + (10 << 32)
+
+    def call(B=1, L=128, H=2, P=64, N=128, io=1, ws_ptr=ws, ws_bytes=1 << 30, **over):
+        p = list(ptrs)
+        for i, v in over.items():
+            p[int(i[1:])] = v
+        return f(B, L, H, P, N, io, *p, ws_ptr, ws_bytes, None)
+
+    assert call(B=-1) == INVALID
+    assert call(P=32) == UNSUPPORTED
+    assert call(N=64) == UNSUPPORTED
+    assert call(io=0) == UNSUPPORTED                            # bf16 only
+    assert call(p0=None) == INVALID
+    assert call(p9=None) == INVALID
+    assert call(p2=FAKE + 8) == ALIGNMENT
+    assert call(ws_bytes=100) == WORKSPACE
+    assert call(p8=ptrs[0]) == INVALID                          # y overlaps x
+    assert call(p9=ptrs[7] + 16) == INVALID                     # h_out partly overlaps h0
+    assert call(B=0) == OK
+    q = lib.axon_ssd_workspace_bytes
+    q.restype = ctypes.c_size_t
+    q.argtypes = [ctypes.c_int] * 5
+    assert q(2, 130, 3, 64, 128) == 2 * 3 * 64 * 64 * 4     # three 64-token chunks per batch row
+    assert q(1, 128, 1, 32, 128) == 0

@@ -1,0 +1,75 @@
+"""GPU parity of the Mamba-2 (SSD) layer core (axon_ssd_scan_fwd: chunk Gram
+matrices, then one chunk-walking kernel per (batch row, head, 16 head
+columns) with the products on bf16 tensor-core MMAs) against the fp64
+oracle's ``ssd_scan`` on the same bf16 inputs.
+
+Tolerance.  The tensor-core products take bf16 operands: the decayed chunk
+Gram matrix G_ij exp(acum_i - acum_j) dt_j and the dt-weighted B rows
+(relative rounding 2^-9 each); the carried state enters the inter-chunk term
+as two bf16 parts (about 2^-17); accumulation and the carried state are
+float32.  The errors of the
+many products summed into each output are independent, so the error is a
+fraction of a percent of the output's rms scale: elementwise |got - ref| <=
+3e-2 * max(rms(ref), |ref|) and normwise ||got - ref|| / ||ref|| <= 1e-2, for
+y and for the final state.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from selective_state_space_52_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def close(got, ref, what):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (what, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), what + ": non-finite"
+    scale = max(float(np.sqrt(np.mean(ref ** 2))), 1e-30)
+    err = np.abs(got - ref) / np.maximum(scale, np.abs(ref))
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
+    assert err.max() <= 3e-2, f"{what}: worst {err.max():.3g} of scale, {int((err > 3e-2).sum())} elements; normwise {rel:.3g}"
+    assert rel <= 1e-2, f"{what}: normwise {rel:.3g}"
+
+
+def run(inp, with_state):
+    from selective_state_space_52_b200 import axon_ssm
+    d = {k: v.cuda() for k, v in inp.items()}
+    params = {k: d[k] for k in ("dt_bias", "A_log", "D")}
+    y, h = axon_ssm.ssd_scan(d["x"], d["dt_raw"], d["B"], d["C"], params, d["h0"] if with_state else None)
+    torch.cuda.synchronize()
+    return y.float().cpu().numpy(), h.cpu().numpy()
+
+
+def ref(inp, with_state):
+    return oracle.ssd_scan(inp["x"], inp["dt_raw"], inp["dt_bias"], inp["A_log"], inp["B"], inp["C"],
+                           inp["D"], inp["h0"] if with_state else None)
+
+
+@pytest.mark.parametrize("L", [1, 64, 130, 1000])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_ssd_small(cuda_lib, L, with_state):
+    inp = W.make_ssd_inputs(W.SSD_WORKLOAD_BY_NAME["small_ssd"], with_state=True, L=L)
+    y, h = run(inp, with_state)
+    y_ref, h_ref = ref(inp, with_state)
+    close(y, y_ref, f"ssd y L{L}")
+    close(h, h_ref, f"ssd state L{L}")
+
+
+def test_ssd_mamba2_heads(cuda_lib):
+    """The Mamba-2 block's 64 heads on a sequence of several chunks."""
+    inp = W.make_ssd_inputs(W.SSD_WORKLOAD_BY_NAME["mamba2_ssd"], with_state=True, L=320)
+    y, h = run(inp, True)
+    y_ref, h_ref = ref(inp, True)
+    close(y, y_ref, "mamba2 y")
+    close(h, h_ref, "mamba2 state")
+
+
+def test_ssd_empty_sequence_copies_state(cuda_lib):
+    inp = W.make_ssd_inputs(W.SSD_WORKLOAD_BY_NAME["small_ssd"], with_state=True, L=0)
+    y, h = run(inp, True)
+    assert y.shape[1] == 0
+    np.testing.assert_array_equal(h, inp["h0"].numpy())
