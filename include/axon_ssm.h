@@ -331,19 +331,26 @@ AXON_API axon_status axon_ssm_carry_fold(int P, int r, int B, int E, int N, cons
  * shared by all heads; dt_bias, A_log, D (H) float32; h0 (B,H,P,N) float32 or
  * NULL (zeros); h_out (B,H,P,N) float32, may be h0 itself.  P == 64, N == 128
  * and io == AXON_BF16 only (else AXON_ERR_UNSUPPORTED).  The products take
- * bf16 operands (the decayed chunk Gram matrix, dt-weighted B, and the
- * carried state split in two bf16 parts) with float32 accumulation; the
- * carried state itself is float32.  `workspace` holds axon_ssd_workspace_bytes(...) bytes (the chunk
- * Gram matrices C B^T, B * ceil(L/64) * 64 * 64 floats).  Other conventions
- * as above.
+ * bf16 operands (the decayed chunk Gram matrix with D on its diagonal, the
+ * dt-weighted x, and the carried state split in two bf16 parts) with float32
+ * accumulation; the carried state itself is float32.  To fill the GPU when
+ * B * H is small the sequence is cut into `segments` runs of whole 64-token
+ * chunks (0: chosen for the current device, about two walks per SM; capped at
+ * one per chunk and 64): a first walk of every segment but the last gives its
+ * local end state from a zero state, and the full walk of each segment starts
+ * from the fold of those.  `workspace` (16-byte aligned; may be NULL when the
+ * size is 0) holds axon_ssd_workspace_bytes(B, L, H, P, N, segments) bytes for
+ * the same `segments` on the current device: the chunk Gram matrices C B^T,
+ * the per-chunk decays and weights, and the segments' local states.  Other
+ * conventions as above.
  */
-AXON_API size_t axon_ssd_workspace_bytes(int B, int L, int H, int P, int N);
+AXON_API size_t axon_ssd_workspace_bytes(int B, int L, int H, int P, int N, int segments);
 
 AXON_API axon_status axon_ssd_scan_fwd(
     int B, int L, int H, int P, int N, axon_dtype io,
     const void *x, const void *dt_raw, const float *dt_bias, const float *A_log,
     const void *Bm, const void *Cm, const float *D, const float *h0,
-    void *y, float *h_out, void *workspace, size_t workspace_bytes, axon_stream_t stream);
+    void *y, float *h_out, int segments, void *workspace, size_t workspace_bytes, axon_stream_t stream);
 
 /*
  * The whole Axon-SSM layer around the layer core (Axon-SSM page, sections

@@ -67,9 +67,9 @@ _lib.axon_ssm_dt_sum.argtypes = [_i] * 4 + [_vp] * 3 + [_vp]
 _lib.axon_ssm_carry_fold.restype = _i
 _lib.axon_ssm_carry_fold.argtypes = [_i] * 5 + [_vp] * 4 + [_vp]
 _lib.axon_ssd_workspace_bytes.restype = _sz
-_lib.axon_ssd_workspace_bytes.argtypes = [_i] * 5
+_lib.axon_ssd_workspace_bytes.argtypes = [_i] * 6
 _lib.axon_ssd_scan_fwd.restype = _i
-_lib.axon_ssd_scan_fwd.argtypes = [_i] * 6 + [_vp] * 10 + [_vp, _sz, _vp]
+_lib.axon_ssd_scan_fwd.argtypes = [_i] * 6 + [_vp] * 10 + [_i, _vp, _sz, _vp]
 _lib.axon_ssm_block_workspace_bytes.restype = _sz
 _lib.axon_ssm_block_workspace_bytes.argtypes = [_i] * 7
 _lib.axon_ssm_block_fwd.restype = _i
@@ -232,14 +232,14 @@ def axon_ssm_carry_fold(P, r, B, E, N, A_log, h_loc, dt_sum, h_in, stream=None, 
     return rc
 
 
-def axon_ssd_workspace_bytes(B, L, H, P=64, N=128) -> int:
-    return int(_lib.axon_ssd_workspace_bytes(B, L, H, P, N))
+def axon_ssd_workspace_bytes(B, L, H, P=64, N=128, segments=0) -> int:
+    return int(_lib.axon_ssd_workspace_bytes(B, L, H, P, N, segments))
 
 
-def axon_ssd_scan_fwd(B, L, H, P, N, io, x, dt_raw, dt_bias, A_log, Bm, Cm, D, h0, y, h_out,
+def axon_ssd_scan_fwd(B, L, H, P, N, io, x, dt_raw, dt_bias, A_log, Bm, Cm, D, h0, y, h_out, segments,
                       workspace, workspace_bytes, stream=None, *, raise_on_error=True) -> int:
     rc = _lib.axon_ssd_scan_fwd(B, L, H, P, N, io, _p(x), _p(dt_raw), _p(dt_bias), _p(A_log), _p(Bm),
-                                _p(Cm), _p(D), _p(h0), _p(y), _p(h_out), _p(workspace),
+                                _p(Cm), _p(D), _p(h0), _p(y), _p(h_out), int(segments), _p(workspace),
                                 int(workspace_bytes), _stream(stream))
     if raise_on_error:
         _check(rc, "axon_ssd_scan_fwd")
@@ -374,9 +374,10 @@ def carry_fold(r, A_log, h_loc_all, dt_sum_all, *, stream=None):
     return out
 
 
-def ssd_scan(x, dt_raw, Bm, Cm, params: dict, h0=None, *, out=None, workspace=None, stream=None):
+def ssd_scan(x, dt_raw, Bm, Cm, params: dict, h0=None, *, out=None, workspace=None, stream=None, segments=0):
     """The Mamba-2 (SSD) layer core on x (B,L,H,P) bf16; ``params`` holds
-    dt_bias, A_log, D (H,) float32.  Returns (y, h_out (B,H,P,N))."""
+    dt_bias, A_log, D (H,) float32; ``segments`` = 0 lets the library cut the
+    sequence for the current device.  Returns (y, h_out (B,H,P,N))."""
     Bsz, L, H, P = x.shape
     N = Bm.shape[2]
     if out is None:
@@ -385,9 +386,10 @@ def ssd_scan(x, dt_raw, Bm, Cm, params: dict, h0=None, *, out=None, workspace=No
     else:
         y, h_out = out
     if workspace is None:
-        workspace = torch.empty(max(axon_ssd_workspace_bytes(Bsz, L, H, P, N), 16), dtype=torch.uint8,
-                                device=x.device)
+        with torch.cuda.device(x.device):
+            nbytes = axon_ssd_workspace_bytes(Bsz, L, H, P, N, segments)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=x.device)
     axon_ssd_scan_fwd(Bsz, L, H, P, N, _dtype_code(x.dtype), x, dt_raw, params["dt_bias"], params["A_log"],
-                      Bm, Cm, params["D"], h0, y, h_out, workspace,
+                      Bm, Cm, params["D"], h0, y, h_out, segments, workspace,
                       workspace.numel() * workspace.element_size(), stream=stream)
     return y, h_out

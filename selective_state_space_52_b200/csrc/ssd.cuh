@@ -10,10 +10,24 @@
 //   y_i      = exp(acum_i) C_i . S_in                  (the carried state)
 //            + sum_{j<=i} G_ij exp(acum_i - acum_j) dt_j x_j  + D_h x_i
 //   S_out    = exp(acum_{Q-1}) S_in + sum_j exp(acum_{Q-1} - acum_j) dt_j x_j B_j^T
-// The three products run as bf16 m16n8k16 tensor-core MMAs with float32
-// accumulation (mma.sync); the carried state stays float32 in registers, and
-// its product with C uses it split in two bf16 parts (hi + lo, about 16
-// significant bits), because C . S_in can cancel heavily for long-memory heads.
+//
+// Launches: ssd_gram_kernel (G per chunk), ssd_prep_kernel (per chunk and
+// head: acum, log2(dt_j) - acum_j and the state weights w_j), then the chunk
+// walk.  To fill the GPU when B * H is small, the sequence is cut into
+// segments of whole chunks, and the carried state crosses them as in the
+// chunked associative scan of the SSD article: a first walk of every segment
+// but the last from a zero state (state products only) gives its local end
+// state and total decay; the full walk of segment k starts from the fold
+// S_end(j) = exp(sum a over segment j) S_end(j-1) + S_loc(j) for j < k.
+//
+// The products run as bf16 m16n8k16 tensor-core MMAs (mma.sync) with float32
+// accumulation; operands reach them by ldmatrix from XOR-swizzled shared
+// tiles (x and B rows are read transposed, so no transposed copies are built).
+// The carried state stays float32 in registers: warp w owns head columns
+// 16w .. 16w+15 and all 128 state columns, and its accumulator layout is the
+// B-operand layout of the C . S_in product, which therefore reads the state
+// straight from registers, split in two bf16 parts (hi + lo, about 16
+// significant bits) because C . S_in can cancel heavily for long-memory heads.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -26,11 +40,13 @@ namespace axon {
 constexpr int kSsdQ = 64;     // tokens per chunk
 constexpr int kSsdP = 64;     // head dimension
 constexpr int kSsdN = 128;    // state size
-constexpr int kSsdPB = 16;    // head-dimension columns per CTA of the scan
 constexpr int kSsdThreads = 128;
+constexpr int kSsdMaxSegs = 64;
 
 struct SsdParams {
     int B, L, H;
+    int nC;                      // chunks
+    int segs, cps;               // segments of the sequence, chunks per segment
     const __nv_bfloat16* x;      // (B, L, H, P)
     const __nv_bfloat16* dt_raw; // (B, L, H)
     const float* dt_bias;        // (H)
@@ -42,6 +58,10 @@ struct SsdParams {
     __nv_bfloat16* y;            // (B, L, H, P)
     float* h_out;                // (B, H, P, N)
     float* G;                    // (B, nC, Q, Q) workspace
+    float* prep;                 // (B, H, nC, 3, Q): acum (log2 units), log2(dt) - acum, w
+    float* sloc;                 // (segs - 1, B, H, P, N): local end states
+    float* sega;                 // (segs - 1, B, H): total decay of a segment (log2 units)
+    float* h0c;                  // (B, H, P, N): copy of h0 (h_out may overwrite h0) when segs > 1
 };
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -52,20 +72,36 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Four 8x8 bf16 matrices from shared memory; lane l gives the address of row
+// l % 8 of matrix l / 8.  ldsm_x4_t delivers them transposed.
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], unsigned addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], unsigned addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&v);
 }
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
 __device__ __forceinline__ uint32_t ld32(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
-// Stores the pair (v0, v1) as bf16 hi parts at hi and the rounding remainders
-// v - hi as bf16 lo parts at lo.
-__device__ __forceinline__ void store_split(__nv_bfloat16* hi, __nv_bfloat16* lo, float v0, float v1) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(v0, v1);
-    *reinterpret_cast<__nv_bfloat162*>(hi) = h;
-    *reinterpret_cast<uint32_t*>(lo) = pack_bf16(v0 - __low2float(h), v1 - __high2float(h));
-}
+// Byte offsets inside the swizzled shared tiles: rows of 16-byte chunks with
+// the chunk index XORed by the row (mod 8), so the eight rows one ldmatrix
+// phase reads fall in distinct banks.
+__device__ __forceinline__ int sw256(int row, int chunk) { return row * 256 + ((chunk ^ (row & 7)) << 4); }   // 128 bf16
+__device__ __forceinline__ int sw128(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }   // 64 bf16
+// 64 floats per row; odd rows swap the two 64-byte halves of each 128 bytes,
+// so two consecutive rows read as float2 by half a warp use all 32 banks.
+__device__ __forceinline__ int swg(int row, int chunk) { return row * 256 + ((chunk ^ ((row & 1) << 2)) << 4); }
 
 // Copies rows [t0, t0 + 64) of a (B, L, N) bf16 matrix into shared memory rows
 // of `stride` elements (zeros past L).  All threads of the CTA take part.
@@ -117,273 +153,313 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_gram_kernel(SsdParams p) {
     }
 }
 
-// Dynamic shared-memory layout of the scan kernel (bytes).  Staged with
-// cp.async: G (float rows), C rows (padded for fragment loads), raw B rows and
-// raw x rows (16 head columns, both double-buffered: the next chunk's arrive
-// while this one computes); built from them: w*B as [n][j] and x as [p][j]
-// (stride 33 words: the pair stores that build them hit distinct banks).
-struct SsdSmem {
-    static constexpr int kGs = kSsdQ + 4;            // float row stride of G
-    static constexpr int kCs = kSsdN + 8;            // bf16 row stride of C
-    static constexpr int kWs = kSsdQ + 2;            // bf16 row stride of w*B^T and x^T
-    static constexpr int kSs = kSsdN + 8;            // bf16 row stride of the carried state
-    static constexpr int G = 0;
-    static constexpr int C = G + kSsdQ * kGs * 4;
-    static constexpr int BR = C + kSsdQ * kCs * 2;            // two buffers (this chunk, the next)
-    static constexpr int XR = BR + 2 * kSsdQ * kSsdN * 2;     // two buffers
-    static constexpr int WB = XR + 2 * kSsdQ * kSsdPB * 2;
-    static constexpr int XT = WB + kSsdN * kWs * 2;
-    static constexpr int SS = XT + kSsdPB * kWs * 2;          // hi part, then lo part
-    static constexpr int ACUM = SS + 2 * kSsdPB * kSs * 2;    // cumulative decay, in log2 units
-    static constexpr int DTV = ACUM + kSsdQ * 4;
-    static constexpr int WV = DTV + kSsdQ * 4;                // w_j = exp(acum_last - acum_j) dt_j
-    static constexpr int TOTAL = WV + kSsdQ * 4;
+// Per (b, chunk, head): dt_j, acum_j (log2 units: exp(acum) = 2^acum2),
+// e_j = log2(dt_j) - acum2_j (so dt_j exp(acum_i - acum_j) = 2^(acum2_i + e_j),
+// whose exponent never exceeds log2(dt_j) for j <= i), and the state weights
+// w_j = dt_j 2^(acum2_{Q-1} - acum2_j).  Tokens past L get dt = 0, e = -inf.
+// grid = (nC, ceil(H / 4), B), 128 threads: warp -> head, lane -> 2 tokens.
+__global__ void __launch_bounds__(kSsdThreads) ssd_prep_kernel(SsdParams p) {
+    const int c = blockIdx.x, b = blockIdx.z;
+    const int lane = threadIdx.x & 31;
+    const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
+    if (h >= p.H) return;                      // whole warps
+    const int L = p.L, H = p.H;
+    const float A2 = -expf(__ldg(p.A_log + h)) * kLog2e;
+    const float bias = __ldg(p.dt_bias + h);
+    float dt[2], a2[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int t = c * kSsdQ + 2 * lane + k;
+        dt[k] = t < L ? dt_from_raw(__bfloat162float(p.dt_raw[((size_t)b * L + t) * H + h]) + bias) : 0.f;
+        a2[k] = dt[k] * A2;
+    }
+    float s = a2[0] + a2[1];
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const float o = __shfl_up_sync(0xffffffffu, s, d);
+        if (lane >= d) s += o;
+    }
+    const float alast = __shfl_sync(0xffffffffu, s, 31);
+    const float c0 = s - a2[1], c1 = s;
+    const int t0 = c * kSsdQ + 2 * lane;
+    const float e0 = t0 < L ? lg2_approx(dt[0]) - c0 : -INFINITY;
+    const float e1 = t0 + 1 < L ? lg2_approx(dt[1]) - c1 : -INFINITY;
+    float* out = p.prep + (((size_t)b * H + h) * p.nC + c) * 3 * kSsdQ;
+    *reinterpret_cast<float2*>(out + 2 * lane) = make_float2(c0, c1);
+    *reinterpret_cast<float2*>(out + kSsdQ + 2 * lane) = make_float2(e0, e1);
+    *reinterpret_cast<float2*>(out + 2 * kSsdQ + 2 * lane) =
+        make_float2(dt[0] * ex2_approx(alast - c0), dt[1] * ex2_approx(alast - c1));
+}
+
+// Shared memory of the chunk walk (bytes).  Two stages of per-chunk rows (C,
+// B, x of this head, the prep values), filled by cp.async one chunk ahead;
+// the full walk adds G (float32) and the decayed, masked Gram matrix M (bf16).
+template <bool kFull> struct SsdSmem;
+template <> struct SsdSmem<true> {
+    static constexpr int CS = 0, BS = 16384, XS = 32768, PR = 40960, STAGE = 41728;
+    static constexpr int GS = 2 * STAGE, MS = GS + 16384, TOTAL = MS + 8192;
+};
+template <> struct SsdSmem<false> {
+    static constexpr int CS = -1, BS = 0, XS = 16384, PR = 24576, STAGE = 25344;
+    static constexpr int GS = -1, MS = -1, TOTAL = 2 * STAGE;
 };
 
-// grid = (H, P / 16, B), 128 threads; walks the chunks of one sequence in
-// order for one head and 16 head-dimension columns, carrying the state
-// (16 x 128, float32) in registers: warp w owns state columns 32w .. 32w+31
-// and output rows 16w .. 16w+15 of every chunk.
-__global__ void __launch_bounds__(kSsdThreads) ssd_scan_kernel(SsdParams p) {
+// The chunk walk of one (head h, segment, batch row b): grid = (H, segs (or
+// segs - 1 for the first walk), B), 128 threads.  kFull = false: the first
+// walk (state products only, from h0 for segment 0 and zeros otherwise),
+// writing the local end state and the segment's total decay.  kFull = true:
+// the outputs y and, for the last segment, the final state.
+template <bool kFull>
+__global__ void __launch_bounds__(kSsdThreads, 2) ssd_chunk_scan_kernel(SsdParams p) {
+    using Lay = SsdSmem<kFull>;
+    constexpr int Q = kSsdQ, P = kSsdP, N = kSsdN;
     extern __shared__ __align__(16) unsigned char smem[];
-    float* Gs = reinterpret_cast<float*>(smem + SsdSmem::G);
-    __nv_bfloat16* Cs = reinterpret_cast<__nv_bfloat16*>(smem + SsdSmem::C);
-    __nv_bfloat16* Br = reinterpret_cast<__nv_bfloat16*>(smem + SsdSmem::BR);    // [j][n]
-    __nv_bfloat16* Xr = reinterpret_cast<__nv_bfloat16*>(smem + SsdSmem::XR);    // [j][p]
-    __nv_bfloat16* WBt = reinterpret_cast<__nv_bfloat16*>(smem + SsdSmem::WB);   // [n][j]
-    __nv_bfloat16* Xt = reinterpret_cast<__nv_bfloat16*>(smem + SsdSmem::XT);    // [p][j]
-    __nv_bfloat16* Ss = reinterpret_cast<__nv_bfloat16*>(smem + SsdSmem::SS);    // [p][n], hi part
-    __nv_bfloat16* Sl = Ss + kSsdPB * SsdSmem::kSs;                                // [p][n], lo part
-    float* acum2 = reinterpret_cast<float*>(smem + SsdSmem::ACUM);
-    float* dtv = reinterpret_cast<float*>(smem + SsdSmem::DTV);
-    float* wv = reinterpret_cast<float*>(smem + SsdSmem::WV);
+    const unsigned sbase = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    const int h = blockIdx.x, seg = blockIdx.y, b = blockIdx.z;
+    const int H = p.H, L = p.L, nC = p.nC;
+    const int c_begin = seg * p.cps, c_end = min(nC, c_begin + p.cps);
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, tq = lane & 3;
 
-    const int h = blockIdx.x, pb = blockIdx.y * kSsdPB, b = blockIdx.z;
-    const int H = p.H, L = p.L;
-    const int nC = (L + kSsdQ - 1) / kSsdQ;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int g = lane >> 2, tq = lane & 3;
-    const int tid = threadIdx.x;
-    const float A2 = -expf(__ldg(p.A_log + h)) * kLog2e;     // exp(dt A) = 2^(dt A2)
-    const float bias = __ldg(p.dt_bias + h);
-    const float Dh = __ldg(p.D + h);
+    auto issue_stage = [&](int c, int s) {
+        unsigned char* st = smem + s * Lay::STAGE;
+        const int t0 = c * Q;
+        for (int v = tid; v < Q * 16; v += kSsdThreads) {          // B (and C) rows: 16 chunks each
+            const int r = v >> 4, ch = v & 15;
+            const bool ok = t0 + r < L;
+            const size_t go = ok ? ((size_t)b * L + t0 + r) * N + ch * 8 : 0;
+            cp_async16(st + Lay::BS + sw256(r, ch), p.Bm + go, ok);
+            if constexpr (kFull) cp_async16(st + Lay::CS + sw256(r, ch), p.Cm + go, ok);
+        }
+        for (int v = tid; v < Q * 8; v += kSsdThreads) {           // x rows of head h: 8 chunks each
+            const int r = v >> 3, ch = v & 7;
+            const bool ok = t0 + r < L;
+            const size_t go = ok ? (((size_t)b * L + t0 + r) * H + h) * P + ch * 8 : 0;
+            cp_async16(st + Lay::XS + sw128(r, ch), p.x + go, ok);
+        }
+        if (tid < 3 * Q / 4)
+            cp_async16(st + Lay::PR + tid * 16, p.prep + (((size_t)b * H + h) * nC + c) * 3 * Q + tid * 4, true);
+    };
+    auto issue_g = [&](int c) {
+        const float* Gc = p.G + ((size_t)b * nC + c) * Q * Q;
+        for (int v = tid; v < Q * 16; v += kSsdThreads) {
+            const int r = v >> 4, ch = v & 15;
+            cp_async16(smem + Lay::GS + swg(r, ch), Gc + r * Q + ch * 4, true);
+        }
+    };
 
-    // carried state: rows p = g, g+8 (of the CTA's 16), columns n = 32w + 8nt + 2tq (+1)
-    float S[4][4];
-    const float* h0 = p.h0 ? p.h0 + (((size_t)b * H + h) * kSsdP + pb) * kSsdN : nullptr;
+    // ---- the carried state: rows p = 16w + g (+8), columns n = 8t + 2tq (+1)
+    float S[16][4];
+    const size_t hoff = (((size_t)b * H + h) * P + 16 * w) * N;
+    auto load_state = [&](const float* src) {
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-        const int n = 32 * w + 8 * nt + 2 * tq;
-        S[nt][0] = h0 ? h0[g * kSsdN + n] : 0.f;
-        S[nt][1] = h0 ? h0[g * kSsdN + n + 1] : 0.f;
-        S[nt][2] = h0 ? h0[(g + 8) * kSsdN + n] : 0.f;
-        S[nt][3] = h0 ? h0[(g + 8) * kSsdN + n + 1] : 0.f;
-        store_split(Ss + g * SsdSmem::kSs + n, Sl + g * SsdSmem::kSs + n, S[nt][0], S[nt][1]);
-        store_split(Ss + (g + 8) * SsdSmem::kSs + n, Sl + (g + 8) * SsdSmem::kSs + n, S[nt][2], S[nt][3]);
+        for (int t = 0; t < 16; ++t) {
+            const float2 u = *reinterpret_cast<const float2*>(src + hoff + g * N + 8 * t + 2 * tq);
+            const float2 v = *reinterpret_cast<const float2*>(src + hoff + (g + 8) * N + 8 * t + 2 * tq);
+            S[t][0] = u.x; S[t][1] = u.y; S[t][2] = v.x; S[t][3] = v.y;
+        }
+    };
+    auto store_state = [&](float* dst) {
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            *reinterpret_cast<float2*>(dst + hoff + g * N + 8 * t + 2 * tq) = make_float2(S[t][0], S[t][1]);
+            *reinterpret_cast<float2*>(dst + hoff + (g + 8) * N + 8 * t + 2 * tq) = make_float2(S[t][2], S[t][3]);
+        }
+    };
+    const size_t BHPN = (size_t)p.B * H * P * N;
+    bool s_nonzero;
+    if constexpr (!kFull) {
+        s_nonzero = seg == 0 && p.h0 != nullptr;
+        if (s_nonzero) {
+            load_state(p.h0);
+            if (p.h0c) store_state(p.h0c);
+        } else {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) S[t][0] = S[t][1] = S[t][2] = S[t][3] = 0.f;
+        }
+    } else {
+        if (seg == 0) {
+            const float* src = p.h0c ? p.h0c : p.h0;
+            s_nonzero = src != nullptr;
+            if (s_nonzero) {
+                load_state(src);
+            } else {
+#pragma unroll
+                for (int t = 0; t < 16; ++t) S[t][0] = S[t][1] = S[t][2] = S[t][3] = 0.f;
+            }
+        } else {
+            s_nonzero = true;
+            load_state(p.sloc);                                      // segment 0 ran from h0
+            for (int j = 1; j < seg; ++j) {
+                const float dj = ex2_approx(p.sega[((size_t)j * p.B + b) * H + h]);
+                const float* src = p.sloc + (size_t)j * BHPN;
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const float2 u = *reinterpret_cast<const float2*>(src + hoff + g * N + 8 * t + 2 * tq);
+                    const float2 v = *reinterpret_cast<const float2*>(src + hoff + (g + 8) * N + 8 * t + 2 * tq);
+                    S[t][0] = fmaf(dj, S[t][0], u.x); S[t][1] = fmaf(dj, S[t][1], u.y);
+                    S[t][2] = fmaf(dj, S[t][2], v.x); S[t][3] = fmaf(dj, S[t][3], v.y);
+                }
+            }
+        }
     }
-    const bool has_h0 = p.h0 != nullptr;
 
-    // ---- copies of chunk c: G and C (one buffer), raw B and x rows (buffer c % 2)
-    auto copy_gc = [&](int c) {
-        const int t0 = c * kSsdQ;
-        const float* Gc = p.G + ((size_t)b * nC + c) * kSsdQ * kSsdQ;
-        for (int v = tid; v < kSsdQ * (kSsdQ / 4); v += kSsdThreads) {
-            const int i = v / (kSsdQ / 4), pc = v % (kSsdQ / 4);
-            cp_async16(Gs + i * SsdSmem::kGs + 4 * pc, Gc + i * kSsdQ + 4 * pc, true);
-        }
-        for (int v = tid; v < kSsdQ * (kSsdN / 8); v += kSsdThreads) {
-            const int r = v / (kSsdN / 8), pc = v % (kSsdN / 8);
-            const int t = t0 + r;
-            const bool ok = t < L;
-            cp_async16(Cs + r * SsdSmem::kCs + 8 * pc, p.Cm + (ok ? ((size_t)b * L + t) * kSsdN + 8 * pc : 0), ok);
-        }
-    };
-    auto copy_bx = [&](int c) {
-        const int t0 = c * kSsdQ;
-        __nv_bfloat16* br = Br + (c & 1) * kSsdQ * kSsdN;
-        __nv_bfloat16* xr = Xr + (c & 1) * kSsdQ * kSsdPB;
-        for (int v = tid; v < kSsdQ * (kSsdN / 8); v += kSsdThreads) {
-            const int r = v / (kSsdN / 8), pc = v % (kSsdN / 8);
-            const int t = t0 + r;
-            const bool ok = t < L;
-            cp_async16(br + r * kSsdN + 8 * pc, p.Bm + (ok ? ((size_t)b * L + t) * kSsdN + 8 * pc : 0), ok);
-        }
-        for (int v = tid; v < kSsdQ * (kSsdPB / 8); v += kSsdThreads) {
-            const int j = v / (kSsdPB / 8), half = v % (kSsdPB / 8);
-            const int t = t0 + j;
-            const bool ok = t < L;
-            cp_async16(xr + j * kSsdPB + 8 * half,
-                       p.x + (ok ? (((size_t)b * L + t) * H + h) * kSsdP + pb + 8 * half : 0), ok);
-        }
-    };
-    // warp 0: the raw dt of chunk c into registers (two tokens per lane)
-    auto load_dt = [&](int c, float (&d)[2]) {
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const int t = c * kSsdQ + 2 * lane + k;
-            d[k] = t < L ? __bfloat162float(p.dt_raw[((size_t)b * L + t) * H + h]) : 0.f;
-        }
-    };
-
-    float dtraw[2] = {0.f, 0.f};
-    if (nC > 0) {
-        copy_gc(0);
-        copy_bx(0);
+    float seg_decay = 0.f;
+    if (c_begin < c_end) {
+        issue_stage(c_begin, 0);
+        if constexpr (kFull) issue_g(c_begin);
         cp_async_commit();
-        if (w == 0) load_dt(0, dtraw);
     }
-    for (int c = 0; c < nC; ++c) {
-        const int t0 = c * kSsdQ;
-        const __nv_bfloat16* br = Br + (c & 1) * kSsdQ * kSsdN;
-        const __nv_bfloat16* xr = Xr + (c & 1) * kSsdQ * kSsdPB;
-        if (w == 0) {
-            // dt, the inclusive cumulative decay (log2 units) and w_j of this chunk
-            float dt2[2], a2[2];
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int t = t0 + 2 * lane + k;
-                dt2[k] = t < L ? dt_from_raw(dtraw[k] + bias) : 0.f;
-                a2[k] = dt2[k] * A2;
-            }
-            float sacc = a2[0] + a2[1];
-#pragma unroll
-            for (int d = 1; d < 32; d <<= 1) {
-                const float o = __shfl_up_sync(0xffffffffu, sacc, d);
-                if (lane >= d) sacc += o;
-            }
-            const float alast = __shfl_sync(0xffffffffu, sacc, 31);
-            const float c0 = sacc - a2[1], c1 = sacc;
-            acum2[2 * lane] = c0;
-            acum2[2 * lane + 1] = c1;
-            dtv[2 * lane] = dt2[0];
-            dtv[2 * lane + 1] = dt2[1];
-            wv[2 * lane] = ex2_approx(alast - c0) * dt2[0];
-            wv[2 * lane + 1] = ex2_approx(alast - c1) * dt2[1];
-        }
-        cp_async_wait_0();                     // this chunk's copies (this thread's share)
-        __syncthreads();                       // ... everyone's; acum, dtv, wv written
-        if (c + 1 < nC) {
-            copy_bx(c + 1);                    // its buffers were last read before the previous barrier
-            cp_async_commit();
-            if (w == 0) load_dt(c + 1, dtraw);
-        }
-        // ---- x as [p][j] and w*B as [n][j], one bf16 pair (j, j+1) per store
-        for (int v = tid; v < kSsdPB * (kSsdQ / 2); v += kSsdThreads) {
-            const int pp = v % kSsdPB, jp = v / kSsdPB;
-            *reinterpret_cast<uint32_t*>(Xt + pp * SsdSmem::kWs + 2 * jp) =
-                pack_bf16(__bfloat162float(xr[(2 * jp) * kSsdPB + pp]), __bfloat162float(xr[(2 * jp + 1) * kSsdPB + pp]));
-        }
-        for (int v = tid; v < kSsdN * (kSsdQ / 2); v += kSsdThreads) {
-            const int n = v % kSsdN, jp = v / kSsdN;
-            *reinterpret_cast<uint32_t*>(WBt + n * SsdSmem::kWs + 2 * jp) =
-                pack_bf16(wv[2 * jp] * __bfloat162float(br[(2 * jp) * kSsdN + n]),
-                          wv[2 * jp + 1] * __bfloat162float(br[(2 * jp + 1) * kSsdN + n]));
-        }
-        __syncthreads();
+    float Dh = 0.f;
+    if constexpr (kFull) Dh = __ldg(p.D + h);
 
-        // ---- outputs of rows 16w .. 16w+15, columns pb .. pb+15
-        float acc[2][4] = {};
-        const int i0 = 16 * w + g, i1 = i0 + 8;
-        const float ai0 = acum2[i0], ai1 = acum2[i1];
-        if (c > 0 || has_h0) {
-            // exp(acum_i) C_i . S_in: K = N, the state as hi + lo bf16 parts
+    for (int c = c_begin; c < c_end; ++c) {
+        const int s = (c - c_begin) & 1;
+        const unsigned st = sbase + s * Lay::STAGE;
+        const float* pr = reinterpret_cast<const float*>(smem + s * Lay::STAGE + Lay::PR);  // acum, e, w
+        cp_async_wait_0();
+        __syncthreads();                       // this chunk's rows landed; chunk c-1 is done everywhere
+        if (c + 1 < c_end) {
+            issue_stage(c + 1, s ^ 1);
+            cp_async_commit();
+        }
+
+        if constexpr (kFull) {
+            // ---- M = mask(G_ij 2^(acum_i + e_j)) + D on the diagonal, bf16: the ten 16x16
+            // blocks on or below the diagonal; thread -> row tid/8 of a block, column pair tid%8
+            const int rr = tid >> 3, k2 = 2 * (tid & 7);
+            float2 ej[4];
 #pragma unroll
-            for (int ks = 0; ks < kSsdN / 16; ++ks) {
-                const int k0 = ks * 16 + 2 * tq;
-                const uint32_t a[4] = {ld32(Cs + i0 * SsdSmem::kCs + k0), ld32(Cs + i1 * SsdSmem::kCs + k0),
-                                       ld32(Cs + i0 * SsdSmem::kCs + k0 + 8), ld32(Cs + i1 * SsdSmem::kCs + k0 + 8)};
+            for (int jb = 0; jb < 4; ++jb) ej[jb] = *reinterpret_cast<const float2*>(pr + Q + 16 * jb + k2);
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    const __nv_bfloat16* sr = Ss + (8 * nt + g) * SsdSmem::kSs;
-                    const __nv_bfloat16* lr = Sl + (8 * nt + g) * SsdSmem::kSs;
-                    mma_16816(acc[nt], a, ld32(sr + k0), ld32(sr + k0 + 8));
-                    mma_16816(acc[nt], a, ld32(lr + k0), ld32(lr + k0 + 8));
+            for (int ib = 0; ib < 4; ++ib) {
+                const int i = 16 * ib + rr;
+                const float ai = pr[i];
+#pragma unroll
+                for (int jb = 0; jb <= ib; ++jb) {
+                    const int j = 16 * jb + k2;
+                    const float2 gv = *reinterpret_cast<const float2*>(smem + Lay::GS + swg(i, j >> 2) + (j & 3) * 4);
+                    float m0 = gv.x * ex2_approx(ai + ej[jb].x);
+                    float m1 = gv.y * ex2_approx(ai + ej[jb].y);
+                    if (jb == ib) {
+                        m0 = j < i ? m0 : (j == i ? m0 + Dh : 0.f);
+                        m1 = j + 1 < i ? m1 : (j + 1 == i ? m1 + Dh : 0.f);
+                    }
+                    *reinterpret_cast<uint32_t*>(smem + Lay::MS + sw128(i, j >> 3) + (j & 7) * 2) = pack_bf16(m0, m1);
                 }
             }
-            const float e0 = ex2_approx(ai0), e1 = ex2_approx(ai1);
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                acc[nt][0] *= e0; acc[nt][1] *= e0; acc[nt][2] *= e1; acc[nt][3] *= e1;
-            }
-        }
-        // masked, decayed G times dt x: K = the chunk's tokens, only blocks on or below the diagonal
-#pragma unroll
-        for (int ks = 0; ks < kSsdQ / 16; ++ks) {
-            if (ks > w) break;                 // j >= 16 ks > i for every row of this warp
-            uint32_t a[4];
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-                const int i = (q4 & 1) ? i1 : i0;
-                const float ai = (q4 & 1) ? ai1 : ai0;
-                const int j = ks * 16 + 2 * tq + ((q4 & 2) ? 8 : 0);
-                const float m0 = j <= i ? Gs[i * SsdSmem::kGs + j] * ex2_approx(ai - acum2[j]) * dtv[j] : 0.f;
-                const float m1 =
-                    j + 1 <= i ? Gs[i * SsdSmem::kGs + j + 1] * ex2_approx(ai - acum2[j + 1]) * dtv[j + 1] : 0.f;
-                a[q4] = pack_bf16(m0, m1);
-            }
-            const int k0 = ks * 16 + 2 * tq;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const __nv_bfloat16* xr = Xt + (8 * nt + g) * SsdSmem::kWs;
-                mma_16816(acc[nt], a, ld32(xr + k0), ld32(xr + k0 + 8));
-            }
-        }
-        // + D x, store rows inside the sequence
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int pc = 8 * nt + 2 * tq;
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int i = r ? i1 : i0;
-                const int t = t0 + i;
-                if (t < L) {
-                    const float x0 = __bfloat162float(xr[i * kSsdPB + pc]);
-                    const float x1 = __bfloat162float(xr[i * kSsdPB + pc + 1]);
-                    const float y0 = fmaf(Dh, x0, acc[nt][2 * r]), y1 = fmaf(Dh, x1, acc[nt][2 * r + 1]);
-                    *reinterpret_cast<uint32_t*>(p.y + (((size_t)b * L + t) * H + h) * kSsdP + pb + pc) =
-                        pack_bf16(y0, y1);
-                }
+            __syncthreads();                   // M complete; G free
+            if (c + 1 < c_end) {
+                issue_g(c + 1);
+                cp_async_commit();
             }
         }
 
-        // ---- G and C of the next chunk, in flight during the state update
-        const float el = ex2_approx(acum2[kSsdQ - 1]);
-        __syncthreads();                       // every warp is done with G, C and this chunk's acum
-        if (c + 1 < nC) {
-            copy_gc(c + 1);
-            cp_async_commit();
+        // ---- x of this warp's 16 head columns: ks -> tokens 16ks .. 16ks+15
+        uint32_t xr[4][4];
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            ldsm_x4_t(xr[ks], st + Lay::XS + sw128(16 * ks + ((lane >> 4) << 3) + (lane & 7), 2 * w + ((lane >> 3) & 1)));
+
+        if constexpr (kFull) {
+            float yacc[4][2][4];
+#pragma unroll
+            for (int rb = 0; rb < 4; ++rb)
+#pragma unroll
+                for (int pt = 0; pt < 2; ++pt) yacc[rb][pt][0] = yacc[rb][pt][1] = yacc[rb][pt][2] = yacc[rb][pt][3] = 0.f;
+            if (s_nonzero || c > c_begin) {
+                // exp(acum_i) C_i . S_in: K = the state columns, B operand = the state registers
+#pragma unroll
+                for (int ks = 0; ks < N / 16; ++ks) {
+                    uint32_t bh[2][2], bl[2][2];
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const float* v = S[2 * ks + half];
+                        const uint32_t u0 = pack_bf16(v[0], v[1]), u1 = pack_bf16(v[2], v[3]);
+                        bh[0][half] = u0;
+                        bh[1][half] = u1;
+                        bl[0][half] = pack_bf16(v[0] - bf16_lo(u0), v[1] - bf16_hi(u0));
+                        bl[1][half] = pack_bf16(v[2] - bf16_lo(u1), v[3] - bf16_hi(u1));
+                    }
+#pragma unroll
+                    for (int rb = 0; rb < 4; ++rb) {
+                        uint32_t a[4];
+                        ldsm_x4(a, st + Lay::CS + sw256(16 * rb + (((lane >> 3) & 1) << 3) + (lane & 7), 2 * ks + (lane >> 4)));
+#pragma unroll
+                        for (int pt = 0; pt < 2; ++pt) {
+                            mma_16816(yacc[rb][pt], a, bl[pt][0], bl[pt][1]);
+                            mma_16816(yacc[rb][pt], a, bh[pt][0], bh[pt][1]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int rb = 0; rb < 4; ++rb) {
+                    const float e0 = ex2_approx(pr[16 * rb + g]), e1 = ex2_approx(pr[16 * rb + g + 8]);
+#pragma unroll
+                    for (int pt = 0; pt < 2; ++pt) {
+                        yacc[rb][pt][0] *= e0; yacc[rb][pt][1] *= e0;
+                        yacc[rb][pt][2] *= e1; yacc[rb][pt][3] *= e1;
+                    }
+                }
+            }
+            // + M x: K = the chunk's tokens, blocks on or below the diagonal
+#pragma unroll
+            for (int rb = 0; rb < 4; ++rb) {
+#pragma unroll
+                for (int kb = 0; kb <= rb; ++kb) {
+                    uint32_t a[4];
+                    ldsm_x4(a, sbase + Lay::MS + sw128(16 * rb + (((lane >> 3) & 1) << 3) + (lane & 7), 2 * kb + (lane >> 4)));
+                    mma_16816(yacc[rb][0], a, xr[kb][0], xr[kb][2]);
+                    mma_16816(yacc[rb][1], a, xr[kb][1], xr[kb][3]);
+                }
+            }
+            // ---- y rows inside the sequence
+            const int t0 = c * Q;
+#pragma unroll
+            for (int rb = 0; rb < 4; ++rb)
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int t = t0 + 16 * rb + g + 8 * r;
+                    if (t < L) {
+                        __nv_bfloat16* yo = p.y + (((size_t)b * L + t) * H + h) * P + 16 * w + 2 * tq;
+#pragma unroll
+                        for (int pt = 0; pt < 2; ++pt)
+                            *reinterpret_cast<uint32_t*>(yo + 8 * pt) = pack_bf16(yacc[rb][pt][2 * r], yacc[rb][pt][2 * r + 1]);
+                    }
+                }
         }
-        // ---- carried state: S = exp(acum_last) S + x^T (w B): K = the chunk's tokens
+
+        // ---- S = exp(acum_last) S + (w x)^T B: K = the chunk's tokens
+        const float alast = pr[Q - 1];
+        seg_decay += alast;
+        const float el = ex2_approx(alast);
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int t = 0; t < 16; ++t) {
+            S[t][0] *= el; S[t][1] *= el; S[t][2] *= el; S[t][3] *= el;
+        }
 #pragma unroll
-            for (int k = 0; k < 4; ++k) S[nt][k] *= el;
+        for (int ks = 0; ks < 4; ++ks) {
+            const float2 wa = *reinterpret_cast<const float2*>(pr + 2 * Q + 16 * ks + 2 * tq);
+            const float2 wb = *reinterpret_cast<const float2*>(pr + 2 * Q + 16 * ks + 8 + 2 * tq);
+            const uint32_t a[4] = {
+                pack_bf16(bf16_lo(xr[ks][0]) * wa.x, bf16_hi(xr[ks][0]) * wa.y),
+                pack_bf16(bf16_lo(xr[ks][1]) * wa.x, bf16_hi(xr[ks][1]) * wa.y),
+                pack_bf16(bf16_lo(xr[ks][2]) * wb.x, bf16_hi(xr[ks][2]) * wb.y),
+                pack_bf16(bf16_lo(xr[ks][3]) * wb.x, bf16_hi(xr[ks][3]) * wb.y)};
 #pragma unroll
-        for (int ks = 0; ks < kSsdQ / 16; ++ks) {
-            const int k0 = ks * 16 + 2 * tq;
-            const uint32_t a[4] = {ld32(Xt + g * SsdSmem::kWs + k0), ld32(Xt + (g + 8) * SsdSmem::kWs + k0),
-                                   ld32(Xt + g * SsdSmem::kWs + k0 + 8), ld32(Xt + (g + 8) * SsdSmem::kWs + k0 + 8)};
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const __nv_bfloat16* wr = WBt + (32 * w + 8 * nt + g) * SsdSmem::kWs;
-                mma_16816(S[nt], a, ld32(wr + k0), ld32(wr + k0 + 8));
+            for (int q = 0; q < 8; ++q) {
+                uint32_t bb[4];
+                ldsm_x4_t(bb, st + Lay::BS + sw256(16 * ks + (((lane >> 3) & 1) << 3) + (lane & 7), 2 * q + (lane >> 4)));
+                mma_16816(S[2 * q], a, bb[0], bb[1]);
+                mma_16816(S[2 * q + 1], a, bb[2], bb[3]);
             }
         }
-        __syncthreads();                       // every warp has read the old carried state
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            const int n = 32 * w + 8 * nt + 2 * tq;
-            store_split(Ss + g * SsdSmem::kSs + n, Sl + g * SsdSmem::kSs + n, S[nt][0], S[nt][1]);
-            store_split(Ss + (g + 8) * SsdSmem::kSs + n, Sl + (g + 8) * SsdSmem::kSs + n, S[nt][2], S[nt][3]);
-        }
     }
-    // ---- final state
-    float* ho = p.h_out + (((size_t)b * H + h) * kSsdP + pb) * kSsdN;
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-        const int n = 32 * w + 8 * nt + 2 * tq;
-        *reinterpret_cast<float2*>(ho + g * kSsdN + n) = make_float2(S[nt][0], S[nt][1]);
-        *reinterpret_cast<float2*>(ho + (g + 8) * kSsdN + n) = make_float2(S[nt][2], S[nt][3]);
+
+    if constexpr (kFull) {
+        if (seg == p.segs - 1) store_state(p.h_out);
+    } else {
+        store_state(p.sloc + (size_t)seg * BHPN);
+        if (tid == 0) p.sega[((size_t)seg * p.B + b) * H + h] = seg_decay;
     }
 }
 

@@ -265,17 +265,20 @@ def test_time_split_pieces_reject_bad_arguments(lib):
 def test_ssd_rejects_bad_arguments(lib):
     f = lib.axon_ssd_scan_fwd
     f.restype = ctypes.c_int
-    f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 10 + [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    f.argtypes = ([ctypes.c_int] * 6 + [ctypes.c_void_p] * 10 +
+                  [ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p])
     ptrs = [FAKE + (i << 32) for i in range(10)]      # x, dt_raw, dt_bias, A_log, B, C, D, h0, y, h_out
     ws = FAKE + (10 << 32)
 
-    def call(B=1, L=128, H=2, P=64, N=128, io=1, ws_ptr=ws, ws_bytes=1 << 30, **over):
+    def call(B=1, L=128, H=2, P=64, N=128, io=1, segments=1, ws_ptr=ws, ws_bytes=1 << 30, **over):
         p = list(ptrs)
         for i, v in over.items():
             p[int(i[1:])] = v
-        return f(B, L, H, P, N, io, *p, ws_ptr, ws_bytes, None)
+        return f(B, L, H, P, N, io, *p, segments, ws_ptr, ws_bytes, None)
 
     assert call(B=-1) == INVALID
+    assert call(segments=-1) == INVALID
+    assert call(ws_ptr=None) == INVALID                         # a workspace is needed when L > 0
     assert call(P=32) == UNSUPPORTED
     assert call(N=64) == UNSUPPORTED
     assert call(io=0) == UNSUPPORTED                            # bf16 only
@@ -288,6 +291,16 @@ def test_ssd_rejects_bad_arguments(lib):
     assert call(B=0) == OK
     q = lib.axon_ssd_workspace_bytes
     q.restype = ctypes.c_size_t
-    q.argtypes = [ctypes.c_int] * 5
-    assert q(2, 130, 3, 64, 128) == 2 * 3 * 64 * 64 * 4     # three 64-token chunks per batch row
-    assert q(1, 128, 1, 32, 128) == 0
+    q.argtypes = [ctypes.c_int] * 6
+    # one segment: the chunk Gram matrices (three 64-token chunks per batch row)
+    # and the per-chunk decays, each rounded up to 256 bytes
+    gram, prep = 2 * 3 * 64 * 64 * 4, 2 * 3 * 3 * 3 * 64 * 4
+    assert q(2, 130, 3, 64, 128, 1) == gram + (prep + 255) // 256 * 256
+    # two segments (chunks 0-1, 2) add one local end state per (b, h), its decay
+    # and the copy of h0
+    state = 2 * 3 * 64 * 128 * 4
+    assert q(2, 130, 3, 64, 128, 2) == gram + (prep + 255) // 256 * 256 + state + 256 + state
+    assert q(2, 130, 3, 64, 128, 5) == q(2, 130, 3, 64, 128, 3)     # at most one segment per chunk
+    assert q(2, 0, 3, 64, 128, 0) == 0
+    assert q(1, 128, 1, 32, 128, 0) == 0
+    assert q(1, 128, 1, 64, 128, -1) == 0

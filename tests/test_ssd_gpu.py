@@ -1,13 +1,14 @@
 """GPU parity of the Mamba-2 (SSD) layer core (axon_ssd_scan_fwd: chunk Gram
-matrices, then one chunk-walking kernel per (batch row, head, 16 head
-columns) with the products on bf16 tensor-core MMAs) against the fp64
-oracle's ``ssd_scan`` on the same bf16 inputs.
+matrices, per-chunk decays, then chunk walks per (batch row, head, segment of
+the sequence) with the products on bf16 tensor-core MMAs) against the fp64
+oracle's ``ssd_scan`` on the same bf16 inputs, for one segment, forced
+segment counts and the automatic plan.
 
 Tolerance.  The tensor-core products take bf16 operands: the decayed chunk
-Gram matrix G_ij exp(acum_i - acum_j) dt_j and the dt-weighted B rows
-(relative rounding 2^-9 each); the carried state enters the inter-chunk term
-as two bf16 parts (about 2^-17); accumulation and the carried state are
-float32.  The errors of the
+Gram matrix G_ij exp(acum_i - acum_j) dt_j (plus D on its diagonal) and the
+weighted x rows w_j x_j (relative rounding 2^-9 each); the carried state
+enters the inter-chunk term as two bf16 parts (about 2^-17); accumulation and
+the carried state are float32.  The errors of the
 many products summed into each output are independent, so the error is a
 fraction of a percent of the output's rms scale: elementwise |got - ref| <=
 3e-2 * max(rms(ref), |ref|) and normwise ||got - ref|| / ||ref|| <= 1e-2, for
@@ -35,11 +36,13 @@ def close(got, ref, what):
     assert rel <= 1e-2, f"{what}: normwise {rel:.3g}"
 
 
-def run(inp, with_state):
+def run(inp, with_state, segments=0, in_place=False):
     from selective_state_space_52_b200 import axon_ssm
     d = {k: v.cuda() for k, v in inp.items()}
     params = {k: d[k] for k in ("dt_bias", "A_log", "D")}
-    y, h = axon_ssm.ssd_scan(d["x"], d["dt_raw"], d["B"], d["C"], params, d["h0"] if with_state else None)
+    h0 = d["h0"] if with_state else None
+    out = (torch.empty_like(d["x"]), h0) if in_place else None
+    y, h = axon_ssm.ssd_scan(d["x"], d["dt_raw"], d["B"], d["C"], params, h0, out=out, segments=segments)
     torch.cuda.synchronize()
     return y.float().cpu().numpy(), h.cpu().numpy()
 
@@ -57,6 +60,28 @@ def test_ssd_small(cuda_lib, L, with_state):
     y_ref, h_ref = ref(inp, with_state)
     close(y, y_ref, f"ssd y L{L}")
     close(h, h_ref, f"ssd state L{L}")
+
+
+@pytest.mark.parametrize("segments", [1, 2, 3, 16])
+def test_ssd_segments(cuda_lib, segments):
+    """The same answer for any cut of the sequence into segments (1000 tokens:
+    16 chunks, the last one ragged)."""
+    inp = W.make_ssd_inputs(W.SSD_WORKLOAD_BY_NAME["small_ssd"], with_state=True, L=1000)
+    y, h = run(inp, True, segments=segments)
+    y_ref, h_ref = ref(inp, True)
+    close(y, y_ref, f"ssd y, {segments} segments")
+    close(h, h_ref, f"ssd state, {segments} segments")
+
+
+@pytest.mark.parametrize("segments", [1, 4])
+def test_ssd_state_in_place(cuda_lib, segments):
+    """h_out = h0: the final state overwrites the initial one, which the walks
+    of the first segment read."""
+    inp = W.make_ssd_inputs(W.SSD_WORKLOAD_BY_NAME["small_ssd"], with_state=True, L=520)
+    y_ref, h_ref = ref(inp, True)
+    y, h = run(inp, True, segments=segments, in_place=True)
+    close(y, y_ref, f"ssd y in place, {segments} segments")
+    close(h, h_ref, f"ssd state in place, {segments} segments")
 
 
 def test_ssd_mamba2_heads(cuda_lib):
