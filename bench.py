@@ -130,14 +130,24 @@ def step_model(wl) -> dict:
     return {"bytes": bytes_, "mufu": MUFU_PER_TOKEN_CH * BE, "token_ch": BE}
 
 
-def kernel_source_hash() -> str:
+# The sources each profiled kernel is built from: its own headers and the
+# translation unit that plans and launches it.  A committed ncu figure counts
+# only while these files are unchanged.
+KERNEL_SOURCES = {
+    "scan": ("axon_ssm.cu", "device_math.cuh", "scan_chunked.cuh", "scan_octo.cuh", "scan_quad.cuh",
+             "scan_seq.cuh"),
+    "step": ("axon_ssm.cu", "device_math.cuh", "step.cuh"),
+    "ssd": ("axon_ssd.cu", "device_math.cuh", "scan_chunked.cuh", "ssd.cuh"),
+}
+
+
+def kernel_source_hash(kernel_key: str = "scan") -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_state_space_52_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode())
-                h.update(f.read())
+    for fn in sorted(KERNEL_SOURCES[kernel_key]):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -151,7 +161,7 @@ def ncu_traffic(kernel_key: str, workload: str, units: int):
     except Exception:
         return None
     ent = d.get(kernel_key, {}).get(workload)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel_key):
         return None
     per_unit = ent["dram_bytes"] / ent["units"]
     return per_unit * units
@@ -708,6 +718,9 @@ def main(argv=None):
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the cached-decode measurement and print it as one JSON line "
                          "(for profiling the step kernel alone)")
+    ap.add_argument("--ssd-only", action="store_true",
+                    help="run only the Mamba-2 (SSD) layer-core measurement and print it as one JSON line "
+                         "(for profiling its kernels alone)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     wl = W.WORKLOAD_BY_NAME[args.workload]
@@ -719,6 +732,13 @@ def main(argv=None):
         dev = torch.device("cuda", 0)
         torch.cuda.set_device(dev)
         print(json.dumps({"decode": bench_decode(dev)}), flush=True)
+        return 0
+    if args.ssd_only:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA GPU for --ssd-only")
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps({"ssd": bench_ssd(dev)}), flush=True)
         return 0
     return run_axon(args, wl)
 
