@@ -1,6 +1,6 @@
 // axon_ssd.cu -- C ABI of the Mamba-2 (SSD) layer core (include/axon_ssm.h):
 // argument checks, the segment plan, the workspace, and the launches of
-// ssd.cuh (chunk Gram matrices, per-chunk decays, the chunk walks).
+// ssd.cuh (chunk Gram matrices and per-chunk decays, the chunk walks).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -21,8 +21,10 @@ bool ovl(const void* a, size_t na, const void* b, size_t nb) {
 }
 size_t up256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Resident chunk walks per SM (shared memory and registers allow two).
+// Resident chunk walks per SM: two full walks (shared memory and registers),
+// three state-only walks.
 constexpr int kWalksPerSm = 2;
+constexpr int kStateWalksPerSm = 3;
 
 int sm_count() {
     static std::atomic<int> cached[64];   // zero-initialised (static storage)
@@ -54,16 +56,30 @@ void plan_segments(int B, int H, int nC, int requested, int& segs, int& cps) {
     segs = (nC + cps - 1) / cps;
 }
 
+// Pieces per segment for the first (state-only) walk: enough walks over the
+// segments but the last to give every SM kStateWalksPerSm of them.  Returns
+// pieces per segment and chunks per piece (no piece is empty).
+void plan_pieces(int B, int H, int segs, int cps, int& pcs, int& cpp) {
+    pcs = 1;
+    if (segs > 1) {
+        const long long walks = (long long)(segs - 1) * B * H;
+        pcs = (int)std::max<long long>(1, (long long)kStateWalksPerSm * sm_count() / walks);
+        pcs = std::min(pcs, cps);
+    }
+    cpp = (cps + pcs - 1) / pcs;
+    pcs = (cps + cpp - 1) / cpp;
+}
+
 struct SsdWs {
     size_t g, prep, sloc, sega, h0c, total;
 };
-SsdWs ws_layout(int B, int L, int H, int segs) {
+SsdWs ws_layout(int B, int L, int H, int segs, int pcs) {
     const size_t nC = ((size_t)L + kSsdQ - 1) / kSsdQ;
     SsdWs w{};
     w.g = 0;
     w.prep = w.g + up256((size_t)B * nC * kSsdQ * kSsdQ * 4);
     w.sloc = w.prep + up256((size_t)B * H * nC * 3 * kSsdQ * 4);
-    const size_t extra = segs > 1 ? (size_t)(segs - 1) : 0;
+    const size_t extra = segs > 1 ? (size_t)(segs - 1) * pcs : 0;
     w.sega = w.sloc + up256(extra * B * H * kSsdP * kSsdN * 4);
     w.h0c = w.sega + up256(extra * B * H * 4);
     w.total = w.h0c + (segs > 1 ? up256((size_t)B * H * kSsdP * kSsdN * 4) : 0);
@@ -93,9 +109,10 @@ extern "C" {
 
 size_t axon_ssd_workspace_bytes(int B, int L, int H, int P, int N, int segments) {
     if (B < 0 || L < 0 || H < 0 || segments < 0 || P != kSsdP || N != kSsdN) return 0;
-    int segs = 1, cps = 1;
+    int segs = 1, cps = 1, pcs = 1, cpp = 1;
     plan_segments(B, H, (L + kSsdQ - 1) / kSsdQ, segments, segs, cps);
-    return ws_layout(B, L, H, segs).total;
+    plan_pieces(B, H, segs, cps, pcs, cpp);
+    return ws_layout(B, L, H, segs, pcs).total;
 }
 
 axon_status axon_ssd_scan_fwd(int B, int L, int H, int P, int N, axon_dtype io,
@@ -105,7 +122,7 @@ axon_status axon_ssd_scan_fwd(int B, int L, int H, int P, int N, axon_dtype io,
                               axon_stream_t stream) {
     if (B < 0 || L < 0 || H < 0 || segments < 0) return AXON_ERR_INVALID_ARG;
     if (P != kSsdP || N != kSsdN || io != AXON_BF16) return AXON_ERR_UNSUPPORTED;
-    if (B > 65535 || H > 65535 || (long long)B * L * H > (1LL << 31)) return AXON_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 4 * (65535 - kGramBlocks) || (long long)B * L * H > (1LL << 31)) return AXON_ERR_UNSUPPORTED;
     if (B == 0 || H == 0) return AXON_OK;
     if (!dt_bias || !A_log || !D || !h_out) return AXON_ERR_INVALID_ARG;
     if (L > 0 && (!x || !dt_raw || !Bm || !Cm || !y)) return AXON_ERR_INVALID_ARG;
@@ -113,9 +130,10 @@ axon_status axon_ssd_scan_fwd(int B, int L, int H, int P, int N, axon_dtype io,
     for (const void* q : ptrs)
         if (q && !al16(q)) return AXON_ERR_ALIGNMENT;
     const int nC = (L + kSsdQ - 1) / kSsdQ;
-    int segs = 1, cps = 1;
+    int segs = 1, cps = 1, pcs = 1, cpp = 1;
     plan_segments(B, H, nC, segments, segs, cps);
-    const SsdWs lay = ws_layout(B, L, H, segs);
+    plan_pieces(B, H, segs, cps, pcs, cpp);
+    const SsdWs lay = ws_layout(B, L, H, segs, pcs);
     const size_t n_x = (size_t)B * L * H * kSsdP * 2, n_dt = (size_t)B * L * H * 2, n_bc = (size_t)B * L * kSsdN * 2;
     const size_t n_h = (size_t)B * H * kSsdP * kSsdN * 4, n_ws = lay.total;
     if (workspace_bytes < n_ws) return AXON_ERR_WORKSPACE;
@@ -134,7 +152,7 @@ axon_status axon_ssd_scan_fwd(int B, int L, int H, int P, int N, axon_dtype io,
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     SsdParams p;
     p.B = B; p.L = L; p.H = H;
-    p.nC = nC; p.segs = segs; p.cps = cps;
+    p.nC = nC; p.segs = segs; p.cps = cps; p.pcs = pcs; p.cpp = cpp;
     p.x = static_cast<const __nv_bfloat16*>(x);
     p.dt_raw = static_cast<const __nv_bfloat16*>(dt_raw);
     p.dt_bias = dt_bias; p.A_log = A_log;
@@ -150,14 +168,13 @@ axon_status axon_ssd_scan_fwd(int B, int L, int H, int P, int N, axon_dtype io,
     p.h0c = (segs > 1 && h0) ? reinterpret_cast<float*>(ws + lay.h0c) : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (nC > 0) {
-        ssd_gram_kernel<<<dim3((unsigned)nC, (unsigned)B), kSsdThreads, 0, st>>>(p);
-        if (cudaGetLastError() != cudaSuccess) return AXON_ERR_CUDA;
-        ssd_prep_kernel<<<dim3((unsigned)nC, (unsigned)((H + 3) / 4), (unsigned)B), kSsdThreads, 0, st>>>(p);
+        ssd_chunk_prep_kernel<<<dim3((unsigned)nC, (unsigned)B, (unsigned)kGramBlocks + (unsigned)((H + 3) / 4)),
+                                kSsdThreads, 0, st>>>(p);
         if (cudaGetLastError() != cudaSuccess) return AXON_ERR_CUDA;
     }
     if (!allow_smem<true>() || !allow_smem<false>()) return AXON_ERR_CUDA;
     if (segs > 1) {
-        ssd_chunk_scan_kernel<false><<<dim3((unsigned)H, (unsigned)(segs - 1), (unsigned)B), kSsdThreads,
+        ssd_chunk_scan_kernel<false><<<dim3((unsigned)H, (unsigned)((segs - 1) * pcs), (unsigned)B), kSsdThreads,
                                        SsdSmem<false>::TOTAL, st>>>(p);
         if (cudaGetLastError() != cudaSuccess) return AXON_ERR_CUDA;
     }

@@ -46,6 +46,7 @@ struct SsdParams {
     int B, L, H;
     int nC;                      // chunks
     int segs, cps;               // segments of the sequence, chunks per segment
+    int pcs, cpp;                // first walk: pieces per segment, chunks per piece
     const __nv_bfloat16* x;      // (B, L, H, P)
     const __nv_bfloat16* dt_raw; // (B, L, H)
     const float* dt_bias;        // (H)
@@ -58,8 +59,8 @@ struct SsdParams {
     float* h_out;                // (B, H, P, N)
     float* G;                    // (B, nC, Q, Q) workspace
     float* prep;                 // (B, H, nC, 3, Q): acum (log2 units), log2(dt) - acum, w
-    float* sloc;                 // (segs - 1, B, H, P, N): local end states
-    float* sega;                 // (segs - 1, B, H): total decay of a segment (log2 units)
+    float* sloc;                 // ((segs - 1) pcs, B, H, P, N): local end states of the pieces
+    float* sega;                 // ((segs - 1) pcs, B, H): total decay of a piece (log2 units)
     float* h0c;                  // (B, H, P, N): copy of h0 (h_out may overwrite h0) when segs > 1
 };
 
@@ -96,62 +97,68 @@ __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v 
 __device__ __forceinline__ uint32_t ld32(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
 
-// One launch for the two per-chunk preliminaries.  grid = (nC, B, 1 + ceil(H/4)),
-// 128 threads; blockIdx.z == 0: the chunk's Gram matrix, else the per-head
-// decays of heads 4 (z - 1) .. 4 (z - 1) + 3.
+// One launch for the two per-chunk preliminaries.  grid = (nC, B, 4 +
+// ceil(H/4)), 128 threads; blockIdx.z < 4: rows 16z .. 16z+15 of the chunk's
+// Gram matrix, else the per-head decays of heads 4 (z - 4) .. 4 (z - 4) + 3.
 //
-// Gram: G[b, c] = C_c B_c^T (float32); warp w owns rows 16w .. 16w+15 and
-// all 64 columns.
+// Gram: G[b, c] = C_c B_c^T (float32); warp w owns columns 16w .. 16w+15 of
+// the CTA's 16 rows.
 //
 // Decays, per head: dt_j, acum_j (log2 units: exp(acum) = 2^acum2),
 // e_j = log2(dt_j) - acum2_j (so dt_j exp(acum_i - acum_j) = 2^(acum2_i + e_j),
 // whose exponent never exceeds log2(dt_j) for j <= i), and the state weights
 // w_j = dt_j 2^(acum2_{Q-1} - acum2_j).  Tokens past L get dt = 0, e = -inf.
 // Warp -> head, lane -> 2 tokens.
+constexpr int kGramBlocks = 4;
 __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_prep_kernel(SsdParams p) {
     constexpr int kS = kSsdN + 8;            // padded row stride (bf16 elements)
-    __shared__ __align__(16) __nv_bfloat16 Cs[kSsdQ * kS];
+    constexpr int kRows = kSsdQ / kGramBlocks;
+    __shared__ __align__(16) __nv_bfloat16 Cs[kRows * kS];
     __shared__ __align__(16) __nv_bfloat16 Bs[kSsdQ * kS];
     const int c = blockIdx.x, b = blockIdx.y;
     const int L = p.L, H = p.H, nC = p.nC;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int t0 = c * kSsdQ;
-    if (blockIdx.z == 0) {
+    if (blockIdx.z < kGramBlocks) {
+        const int r0 = blockIdx.z * kRows;
         constexpr int kPieces = kSsdN * 2 / 16;   // 16-byte pieces per row
         for (int v = threadIdx.x; v < kSsdQ * kPieces; v += kSsdThreads) {
             const int r = v / kPieces, pc = v % kPieces;
             const bool ok = t0 + r < L;
-            const size_t go = ok ? ((size_t)b * L + t0 + r) * kSsdN + pc * 8 : 0;
-            cp_async16(Cs + r * kS + pc * 8, p.Cm + go, ok);
-            cp_async16(Bs + r * kS + pc * 8, p.Bm + go, ok);
+            cp_async16(Bs + r * kS + pc * 8, p.Bm + (ok ? ((size_t)b * L + t0 + r) * kSsdN + pc * 8 : 0), ok);
+        }
+        for (int v = threadIdx.x; v < kRows * kPieces; v += kSsdThreads) {
+            const int r = v / kPieces, pc = v % kPieces;
+            const bool ok = t0 + r0 + r < L;
+            cp_async16(Cs + r * kS + pc * 8, p.Cm + (ok ? ((size_t)b * L + t0 + r0 + r) * kSsdN + pc * 8 : 0), ok);
         }
         cp_async_commit();
         cp_async_wait_0();
         __syncthreads();
         const int g = lane >> 2, tq = lane & 3;
-        float acc[8][4] = {};
+        float acc[2][4] = {};
 #pragma unroll
         for (int ks = 0; ks < kSsdN / 16; ++ks) {
             const int k0 = ks * 16 + 2 * tq;
-            const __nv_bfloat16* r0 = Cs + (16 * w + g) * kS;
-            const __nv_bfloat16* r1 = r0 + 8 * kS;
-            const uint32_t a[4] = {ld32(r0 + k0), ld32(r1 + k0), ld32(r0 + k0 + 8), ld32(r1 + k0 + 8)};
+            const __nv_bfloat16* a0 = Cs + g * kS;
+            const __nv_bfloat16* a1 = a0 + 8 * kS;
+            const uint32_t a[4] = {ld32(a0 + k0), ld32(a1 + k0), ld32(a0 + k0 + 8), ld32(a1 + k0 + 8)};
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                const __nv_bfloat16* br = Bs + (8 * nt + g) * kS;     // B^T column j = B row j
+            for (int nt = 0; nt < 2; ++nt) {
+                const __nv_bfloat16* br = Bs + (16 * w + 8 * nt + g) * kS;     // B^T column j = B row j
                 mma_16816(acc[nt], a, ld32(br + k0), ld32(br + k0 + 8));
             }
         }
         float* Gc = p.G + ((size_t)b * nC + c) * kSsdQ * kSsdQ;
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const int i = 16 * w + g, j = 8 * nt + 2 * tq;
+        for (int nt = 0; nt < 2; ++nt) {
+            const int i = r0 + g, j = 16 * w + 8 * nt + 2 * tq;
             *reinterpret_cast<float2*>(Gc + i * kSsdQ + j) = make_float2(acc[nt][0], acc[nt][1]);
             *reinterpret_cast<float2*>(Gc + (i + 8) * kSsdQ + j) = make_float2(acc[nt][2], acc[nt][3]);
         }
         return;
     }
-    const int h = (blockIdx.z - 1) * 4 + w;
+    const int h = (blockIdx.z - kGramBlocks) * 4 + w;
     if (h >= H) return;                        // whole warps
     const float A2 = -expf(__ldg(p.A_log + h)) * kLog2e;
     const float bias = __ldg(p.dt_bias + h);
@@ -229,20 +236,30 @@ template <> struct SsdSmem<false> {
     static constexpr int GS = -1, MS = -1, TOTAL = 2 * STAGE;
 };
 
-// The chunk walk of one (head h, segment, batch row b): grid = (H, segs (or
-// segs - 1 for the first walk), B), 128 threads.  kFull = false: the first
-// walk (state products only, from h0 for segment 0 and zeros otherwise),
-// writing the local end state and the segment's total decay.  kFull = true:
-// the outputs y and, for the last segment, the final state.
+// The chunk walk of one (head h, run of chunks, batch row b), 128 threads.
+// kFull = false, the first walk: grid = (H, (segs - 1) pcs, B), one piece of
+// cpp chunks of a segment but the last, state products only, from h0 for the
+// first piece and zeros otherwise, writing the piece's local end state and
+// total decay.  kFull = true: grid = (H, segs, B), one segment, entering
+// with the fold of the pieces before it; the outputs y and, for the last
+// segment, the final state.
 template <bool kFull>
-__global__ void __launch_bounds__(kSsdThreads, 2) ssd_chunk_scan_kernel(SsdParams p) {
+__global__ void __launch_bounds__(kSsdThreads, kFull ? 2 : 3) ssd_chunk_scan_kernel(SsdParams p) {
     using Lay = SsdSmem<kFull>;
     constexpr int Q = kSsdQ, P = kSsdP, N = kSsdN;
     extern __shared__ __align__(16) unsigned char smem[];
     const unsigned sbase = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-    const int h = blockIdx.x, seg = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.x, seg = blockIdx.y, b = blockIdx.z;     // seg: segment, or piece of the first walk
     const int H = p.H, L = p.L, nC = p.nC;
-    const int c_begin = seg * p.cps, c_end = min(nC, c_begin + p.cps);
+    int c_begin, c_end;
+    if constexpr (kFull) {
+        c_begin = seg * p.cps;
+        c_end = min(nC, c_begin + p.cps);
+    } else {
+        const int k = seg / p.pcs, m = seg - k * p.pcs;
+        c_begin = k * p.cps + m * p.cpp;
+        c_end = min(min(nC, (k + 1) * p.cps), c_begin + p.cpp);
+    }
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, tq = lane & 3;
 
     // ---- per-thread parts of the copy addresses: B/C rows r = tid/16 + 8k, 16-byte
@@ -324,8 +341,8 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ssd_chunk_scan_kernel(SsdParam
             else zero_state();
         } else {
             s_nonzero = true;
-            load_state(p.sloc);                                      // segment 0 ran from h0
-            for (int j = 1; j < seg; ++j) {
+            load_state(p.sloc);                                      // the first piece ran from h0
+            for (int j = 1; j < seg * p.pcs; ++j) {
                 const float dj = ex2_approx(p.sega[((size_t)j * p.B + b) * H + h]);
                 const float* src = p.sloc + (size_t)j * BHPN;
 #pragma unroll
@@ -491,13 +508,18 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ssd_chunk_scan_kernel(SsdParam
                 const unsigned long long xv = f2_mul(f2_pack(bf16_lo(xr[ks][r]), bf16_hi(xr[ks][r])), r < 2 ? wa : wb);
                 a[r] = pack_bf16(f2_lo(xv), f2_hi(xv));
             }
-            uint32_t bb[8][4];
+            constexpr int kBatch = kFull ? 8 : 4;             // fragments loaded ahead of their MMAs
 #pragma unroll
-            for (int q = 0; q < 8; ++q) ldsm_x4_t(bb[q], st + Lay::BS + offCB + ks * 16 * kRowCB + q * 32);
+            for (int q0 = 0; q0 < 8; q0 += kBatch) {
+                uint32_t bb[kBatch][4];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                mma_16816(S[2 * q], a, bb[q][0], bb[q][1]);
-                mma_16816(S[2 * q + 1], a, bb[q][2], bb[q][3]);
+                for (int q = 0; q < kBatch; ++q)
+                    ldsm_x4_t(bb[q], st + Lay::BS + offCB + ks * 16 * kRowCB + (q0 + q) * 32);
+#pragma unroll
+                for (int q = 0; q < kBatch; ++q) {
+                    mma_16816(S[2 * (q0 + q)], a, bb[q][0], bb[q][1]);
+                    mma_16816(S[2 * (q0 + q) + 1], a, bb[q][2], bb[q][3]);
+                }
             }
         }
     }

@@ -296,10 +296,11 @@ def test_ssd_rejects_bad_arguments(lib):
     # and the per-chunk decays, each rounded up to 256 bytes
     gram, prep = 2 * 3 * 64 * 64 * 4, 2 * 3 * 3 * 3 * 64 * 4
     assert q(2, 130, 3, 64, 128, 1) == gram + (prep + 255) // 256 * 256
-    # two segments (chunks 0-1, 2) add one local end state per (b, h), its decay
-    # and the copy of h0
+    # two segments (chunks 0-1, 2): the state-only walk over the first segment
+    # runs in one-chunk pieces (few heads), each adding a local end state per
+    # (b, h) and its decay; plus the copy of h0
     state = 2 * 3 * 64 * 128 * 4
-    assert q(2, 130, 3, 64, 128, 2) == gram + (prep + 255) // 256 * 256 + state + 256 + state
+    assert q(2, 130, 3, 64, 128, 2) == gram + (prep + 255) // 256 * 256 + 2 * state + 256 + state
     assert q(2, 130, 3, 64, 128, 5) == q(2, 130, 3, 64, 128, 3)     # at most one segment per chunk
     assert q(2, 0, 3, 64, 128, 0) == 0
     assert q(1, 128, 1, 32, 128, 0) == 0

@@ -98,3 +98,15 @@ def test_ssd_empty_sequence_copies_state(cuda_lib):
     y, h = run(inp, True)
     assert y.shape[1] == 0
     np.testing.assert_array_equal(h, inp["h0"].numpy())
+
+
+def test_ssd_full_size(cuda_lib):
+    """The benchmark's shape (B1 L4096, 64 heads, the automatic segment plan,
+    as bench.py times it), every output against the oracle."""
+    sw = W.SSD_WORKLOAD_BY_NAME["mamba2_ssd"]
+    inp = W.make_ssd_inputs(sw, with_state=True)
+    for with_state in (False, True):
+        y, h = run(inp, with_state)
+        y_ref, h_ref = ref(inp, with_state)
+        close(y, y_ref, f"mamba2 full-size y, h0 {with_state}")
+        close(h, h_ref, f"mamba2 full-size state, h0 {with_state}")
