@@ -485,7 +485,7 @@ def bench_ssd(dev, launches: int = 20) -> dict:
         torch.cuda.synchronize(dev)
         times.append(a.elapsed_time(b))
     ms = statistics.median(times)
-    Q, P, N, H, L, B = 64, sw.P, sw.N, sw.H, sw.L, sw.B
+    Q, P, N, H, L, B = 128, sw.P, sw.N, sw.H, sw.L, sw.B     # Q: tokens per chunk of the kernels
     nC = (L + Q - 1) // Q
     # per chunk: C B^T once; per chunk and head: exp(acum) C S_in, the causal
     # half of the masked Gram times x, and x^T (w B)
@@ -499,8 +499,9 @@ def bench_ssd(dev, launches: int = 20) -> dict:
             "hbm": {"achieved": hbm, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": hbm / peaks["hbm_gbs"]},
             "tensor": {"achieved": tfl, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                        "frac": tfl / peaks["bf16_tflops"],
-                       "note": "bf16 mma.sync (m16n8k16) tensor path; the carried-state product runs twice "
-                               "(hi and lo parts), counted once"},
+                       "note": "bf16 tcgen05 MMAs (M = 128, float32 accumulators in tensor memory); the "
+                               "carried-state product runs twice (hi and lo parts) and C B^T once per head, "
+                               "both counted once"},
             "token_head_per_s": B * L * H / (ms / 1e3)}
 
 

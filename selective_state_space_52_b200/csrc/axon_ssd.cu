@@ -1,6 +1,6 @@
 // axon_ssd.cu -- C ABI of the Mamba-2 (SSD) layer core (include/axon_ssm.h):
 // argument checks, the segment plan, the workspace, and the launches of
-// ssd.cuh (chunk Gram matrices and per-chunk decays, the chunk walks).
+// ssd.cuh (per-chunk decays, the chunk walks).
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -21,9 +21,9 @@ bool ovl(const void* a, size_t na, const void* b, size_t nb) {
 }
 size_t up256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Resident chunk walks per SM: two full walks (shared memory and registers),
-// three state-only walks.
-constexpr int kWalksPerSm = 2;
+// Resident chunk walks per SM: one full walk (164 KB of shared memory, 256
+// tensor-memory columns), three state-only walks.
+constexpr int kWalksPerSm = 1;
 constexpr int kStateWalksPerSm = 3;
 
 int sm_count() {
@@ -71,18 +71,19 @@ void plan_pieces(int B, int H, int segs, int cps, int& pcs, int& cpp) {
 }
 
 struct SsdWs {
-    size_t g, prep, sloc, sega, h0c, total;
+    size_t err, prep, sloc, sega, h0c, total;
 };
 SsdWs ws_layout(int B, int L, int H, int segs, int pcs) {
     const size_t nC = ((size_t)L + kSsdQ - 1) / kSsdQ;
     SsdWs w{};
-    w.g = 0;
-    w.prep = w.g + up256((size_t)B * nC * kSsdQ * kSsdQ * 4);
+    w.err = 0;
+    w.prep = w.err + 256;
     w.sloc = w.prep + up256((size_t)B * H * nC * 3 * kSsdQ * 4);
     const size_t extra = segs > 1 ? (size_t)(segs - 1) * pcs : 0;
     w.sega = w.sloc + up256(extra * B * H * kSsdP * kSsdN * 4);
     w.h0c = w.sega + up256(extra * B * H * 4);
     w.total = w.h0c + (segs > 1 ? up256((size_t)B * H * kSsdP * kSsdN * 4) : 0);
+    if (nC == 0) w.total = 0;                  // an empty sequence only copies the state
     return w;
 }
 
@@ -122,7 +123,7 @@ axon_status axon_ssd_scan_fwd(int B, int L, int H, int P, int N, axon_dtype io,
                               axon_stream_t stream) {
     if (B < 0 || L < 0 || H < 0 || segments < 0) return AXON_ERR_INVALID_ARG;
     if (P != kSsdP || N != kSsdN || io != AXON_BF16) return AXON_ERR_UNSUPPORTED;
-    if (B > 65535 || H > 4 * (65535 - kGramBlocks) || (long long)B * L * H > (1LL << 31)) return AXON_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535 || (long long)B * L * H > (1LL << 31)) return AXON_ERR_UNSUPPORTED;
     if (B == 0 || H == 0) return AXON_OK;
     if (!dt_bias || !A_log || !D || !h_out) return AXON_ERR_INVALID_ARG;
     if (L > 0 && (!x || !dt_raw || !Bm || !Cm || !y)) return AXON_ERR_INVALID_ARG;
@@ -161,15 +162,14 @@ axon_status axon_ssd_scan_fwd(int B, int L, int H, int P, int N, axon_dtype io,
     p.D = D; p.h0 = h0;
     p.y = static_cast<__nv_bfloat16*>(y);
     p.h_out = h_out;
-    p.G = reinterpret_cast<float*>(ws + lay.g);
+    p.err = reinterpret_cast<int*>(ws + lay.err);
     p.prep = reinterpret_cast<float*>(ws + lay.prep);
     p.sloc = reinterpret_cast<float*>(ws + lay.sloc);
     p.sega = reinterpret_cast<float*>(ws + lay.sega);
     p.h0c = (segs > 1 && h0) ? reinterpret_cast<float*>(ws + lay.h0c) : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (nC > 0) {
-        ssd_chunk_prep_kernel<<<dim3((unsigned)nC, (unsigned)B, (unsigned)kGramBlocks + (unsigned)((H + 3) / 4)),
-                                kSsdThreads, 0, st>>>(p);
+        ssd_chunk_prep_kernel<<<dim3((unsigned)nC, (unsigned)((H + 3) / 4), (unsigned)B), kSsdThreads, 0, st>>>(p);
         if (cudaGetLastError() != cudaSuccess) return AXON_ERR_CUDA;
     }
     if (!allow_smem<true>() || !allow_smem<false>()) return AXON_ERR_CUDA;
@@ -178,7 +178,7 @@ axon_status axon_ssd_scan_fwd(int B, int L, int H, int P, int N, axon_dtype io,
                                        SsdSmem<false>::TOTAL, st>>>(p);
         if (cudaGetLastError() != cudaSuccess) return AXON_ERR_CUDA;
     }
-    ssd_chunk_scan_kernel<true><<<dim3((unsigned)H, (unsigned)segs, (unsigned)B), kSsdThreads,
+    ssd_chunk_scan_kernel<true><<<dim3((unsigned)H, (unsigned)segs, (unsigned)B), kSsdFullThreads,
                                   SsdSmem<true>::TOTAL, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }

@@ -1,32 +1,38 @@
 // ssd.cuh -- the Mamba-2 (SSD) layer core, one scalar decay per head, as a
-// chunked scan on the tensor cores (the SSD article: inside a chunk the
-// recurrence is a masked matrix product on fast on-chip memory, between chunks
-// a carried state; wiki page "Selective State Space Models (Mamba)", section
-// "Mamba-2 block (SSD)": d_state 128, headdim 64).
+// chunked scan on the tcgen05 tensor cores (the SSD article: inside a chunk
+// the recurrence is a masked matrix product on fast on-chip memory, between
+// chunks a carried state; wiki page "Selective State Space Models (Mamba)",
+// section "Mamba-2 block (SSD)": d_state 128, headdim 64).
 //
-// Per batch row b, head h, chunk of Q = 64 tokens starting at t0, with
+// Per batch row b, head h, chunk of Q = 128 tokens starting at t0, with
 // a_t = dt_t A_h and acum_i = sum_{k<=i} a_k inside the chunk:
-//   G        = C B^T                                   (Q x Q, shared by all heads)
-//   y_i      = exp(acum_i) C_i . S_in                  (the carried state)
-//            + sum_{j<=i} G_ij exp(acum_i - acum_j) dt_j x_j  + D_h x_i
-//   S_out    = exp(acum_{Q-1}) S_in + sum_j exp(acum_{Q-1} - acum_j) dt_j x_j B_j^T
+//   G        = C B^T                                   (Q x Q)
+//   M        = mask(G_ij exp(acum_i - acum_j) dt_j) + D_h I
+//   y        = diag(exp(acum)) C S_in^T + M x
+//   S_out^T  = exp(acum_{Q-1}) S_in^T + B^T (w x),    w_j = exp(acum_{Q-1} - acum_j) dt_j
 //
-// Launches: ssd_chunk_prep_kernel (G per chunk; per chunk and head: acum,
-// log2(dt_j) - acum_j and the state weights w_j), then the chunk walk.  To fill the GPU when B * H is small, the sequence is cut into
-// segments of whole chunks, and the carried state crosses them as in the
-// chunked associative scan of the SSD article: a first walk of every segment
-// but the last from a zero state (state products only) gives its local end
-// state and total decay; the full walk of segment k starts from the fold
-// S_end(j) = exp(sum a over segment j) S_end(j-1) + S_loc(j) for j < k.
+// Launches: ssd_chunk_prep_kernel (per chunk and head: acum, log2(dt_j) -
+// acum_j and w_j), then the chunk walk.  To fill the GPU when B * H is small,
+// the sequence is cut into segments of whole chunks and the carried state
+// crosses them as in the chunked associative scan of the SSD article: a first
+// walk over pieces of every segment but the last, from a zero state (state
+// products only), gives each piece's local end state and total decay; the full
+// walk of segment k starts from the fold S_end(j) = exp(sum a over piece j)
+// S_end(j-1) + S_loc(j) over the pieces before it.
 //
-// The products run as bf16 m16n8k16 tensor-core MMAs (mma.sync) with float32
-// accumulation; operands reach them by ldmatrix from padded shared tiles (x
-// and B rows are read transposed, so no transposed copies are built).
-// The carried state stays float32 in registers: warp w owns head columns
-// 16w .. 16w+15 and all 128 state columns, and its accumulator layout is the
-// B-operand layout of the C . S_in product, which therefore reads the state
-// straight from registers, split in two bf16 parts (hi + lo, about 16
-// significant bits) because C . S_in can cancel heavily for long-memory heads.
+// The four products of a chunk are tcgen05 MMAs (kind::f16, bf16 operands,
+// float32 accumulators in tensor memory, M = 128), issued by one thread and
+// tracked by mbarriers.  Operands sit in shared memory as 128-byte-swizzled
+// tiles of 64-element rows; one copy of each input tile serves every product
+// (the B rows are the K-major B operand of C B^T and the MN-major A operand of
+// B^T (w x); the x rows are the MN-major B operand of M x), except M, which
+// each thread writes as its row into tensor memory, the A operand of M x.
+// Thread i of the 128 owns tensor-memory lane i: row i of G, M, y and of the
+// transposed state.  The full walk double-buffers its input rows: chunk c+1's
+// copies are in flight while chunk c computes.
+// The carried state stays float32 in registers (thread n: S[:, n]) and enters
+// C S^T as two bf16 parts (hi + lo, about 16 significant bits), because that
+// product can cancel heavily for long-memory heads.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -36,11 +42,14 @@
 
 namespace axon {
 
-constexpr int kSsdQ = 64;     // tokens per chunk
+constexpr int kSsdQ = 128;    // tokens per chunk
 constexpr int kSsdP = 64;     // head dimension
 constexpr int kSsdN = 128;    // state size
-constexpr int kSsdThreads = 128;
+constexpr int kSsdThreads = 128;      // the preliminary launch and the state-only walk
+constexpr int kSsdFullThreads = 256;  // the full walk: two threads per tensor-memory lane
 constexpr int kSsdMaxSegs = 64;
+// Iterations of an mbarrier poll before a walk gives up and records an error.
+constexpr int kSsdWaitLimit = 1 << 22;
 
 struct SsdParams {
     int B, L, H;
@@ -57,35 +66,12 @@ struct SsdParams {
     const float* h0;             // (B, H, P, N) or null
     __nv_bfloat16* y;            // (B, L, H, P)
     float* h_out;                // (B, H, P, N)
-    float* G;                    // (B, nC, Q, Q) workspace
     float* prep;                 // (B, H, nC, 3, Q): acum (log2 units), log2(dt) - acum, w
     float* sloc;                 // ((segs - 1) pcs, B, H, P, N): local end states of the pieces
     float* sega;                 // ((segs - 1) pcs, B, H): total decay of a piece (log2 units)
     float* h0c;                  // (B, H, P, N): copy of h0 (h_out may overwrite h0) when segs > 1
+    int* err;                    // set to 1 when a wait gave up
 };
-
-// No side effects beyond its operands: not volatile, so the scheduler may
-// interleave independent MMAs with the loads that feed later ones.
-__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};\n"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Four 8x8 bf16 matrices from shared memory; lane l gives the address of row
-// l % 8 of matrix l / 8.  ldsm_x4_t delivers them transposed.
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], unsigned addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], unsigned addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -94,163 +80,187 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
-__device__ __forceinline__ uint32_t ld32(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
+// ---- tcgen05 / mbarrier primitives (inline PTX)
+// Shared-memory matrix descriptor for a 128-byte-swizzled tile: start address,
+// leading and stride byte offsets (16-byte units), version 1, layout 2.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor, kind::f16: bf16 A and B, float32 D, operand majors
+// (0 = K-major, 1 = MN-major), N / 8, M / 16.
+__host__ __device__ constexpr uint32_t umma_idesc(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+                 ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+// The same with A (K-major, two bf16 per column) in tensor memory.
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+                 ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void umma_commit(uint32_t mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+// Polls the mbarrier's phase `parity` at most kSsdWaitLimit times; false when it gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
+    for (int it = 0; it < kSsdWaitLimit; ++it) {
+        uint32_t done;
+        asm volatile("{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
+                     "selp.b32 %0, 1, 0, P1;\n\t}\n"
+                     : "=r"(done) : "r"(mbar), "r"(parity) : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+// 16 consecutive float32 columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(r[q]);
+}
 
+// 16 consecutive 32-bit columns into this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+                   "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]));
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// One launch for the two per-chunk preliminaries.  grid = (nC, B, 4 +
-// ceil(H/4)), 128 threads; blockIdx.z < 4: rows 16z .. 16z+15 of the chunk's
-// Gram matrix, else the per-head decays of heads 4 (z - 4) .. 4 (z - 4) + 3.
-//
-// Gram: G[b, c] = C_c B_c^T (float32); warp w owns columns 16w .. 16w+15 of
-// the CTA's 16 rows.
-//
-// Decays, per head: dt_j, acum_j (log2 units: exp(acum) = 2^acum2),
+// Byte offset of the 16-byte piece `pc` (8 bf16) of row r in a tile of 128
+// rows stored as 64-column blocks of 128-byte rows, 128-byte swizzle (the
+// piece index XORed by the row mod 8; the tile base is 1024-byte aligned).
+__device__ __forceinline__ int tile_off(int r, int pc) {
+    return (pc >> 3) * (128 * 128) + r * 128 + (((pc & 7) ^ (r & 7)) << 4);
+}
+
+// Per (b, chunk, head): dt_j, acum_j (log2 units: exp(acum) = 2^acum2),
 // e_j = log2(dt_j) - acum2_j (so dt_j exp(acum_i - acum_j) = 2^(acum2_i + e_j),
 // whose exponent never exceeds log2(dt_j) for j <= i), and the state weights
 // w_j = dt_j 2^(acum2_{Q-1} - acum2_j).  Tokens past L get dt = 0, e = -inf.
-// Warp -> head, lane -> 2 tokens.
-constexpr int kGramBlocks = 4;
+// grid = (nC, ceil(H / 4), B), 128 threads: warp -> head, lane -> 4 tokens.
 __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_prep_kernel(SsdParams p) {
-    constexpr int kS = kSsdN + 8;            // padded row stride (bf16 elements)
-    constexpr int kRows = kSsdQ / kGramBlocks;
-    __shared__ __align__(16) __nv_bfloat16 Cs[kRows * kS];
-    __shared__ __align__(16) __nv_bfloat16 Bs[kSsdQ * kS];
-    const int c = blockIdx.x, b = blockIdx.y;
-    const int L = p.L, H = p.H, nC = p.nC;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int t0 = c * kSsdQ;
-    if (blockIdx.z < kGramBlocks) {
-        const int r0 = blockIdx.z * kRows;
-        constexpr int kPieces = kSsdN * 2 / 16;   // 16-byte pieces per row
-        for (int v = threadIdx.x; v < kSsdQ * kPieces; v += kSsdThreads) {
-            const int r = v / kPieces, pc = v % kPieces;
-            const bool ok = t0 + r < L;
-            cp_async16(Bs + r * kS + pc * 8, p.Bm + (ok ? ((size_t)b * L + t0 + r) * kSsdN + pc * 8 : 0), ok);
-        }
-        for (int v = threadIdx.x; v < kRows * kPieces; v += kSsdThreads) {
-            const int r = v / kPieces, pc = v % kPieces;
-            const bool ok = t0 + r0 + r < L;
-            cp_async16(Cs + r * kS + pc * 8, p.Cm + (ok ? ((size_t)b * L + t0 + r0 + r) * kSsdN + pc * 8 : 0), ok);
-        }
-        cp_async_commit();
-        cp_async_wait_0();
-        __syncthreads();
-        const int g = lane >> 2, tq = lane & 3;
-        float acc[2][4] = {};
-#pragma unroll
-        for (int ks = 0; ks < kSsdN / 16; ++ks) {
-            const int k0 = ks * 16 + 2 * tq;
-            const __nv_bfloat16* a0 = Cs + g * kS;
-            const __nv_bfloat16* a1 = a0 + 8 * kS;
-            const uint32_t a[4] = {ld32(a0 + k0), ld32(a1 + k0), ld32(a0 + k0 + 8), ld32(a1 + k0 + 8)};
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                const __nv_bfloat16* br = Bs + (16 * w + 8 * nt + g) * kS;     // B^T column j = B row j
-                mma_16816(acc[nt], a, ld32(br + k0), ld32(br + k0 + 8));
-            }
-        }
-        float* Gc = p.G + ((size_t)b * nC + c) * kSsdQ * kSsdQ;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int i = r0 + g, j = 16 * w + 8 * nt + 2 * tq;
-            *reinterpret_cast<float2*>(Gc + i * kSsdQ + j) = make_float2(acc[nt][0], acc[nt][1]);
-            *reinterpret_cast<float2*>(Gc + (i + 8) * kSsdQ + j) = make_float2(acc[nt][2], acc[nt][3]);
-        }
-        return;
-    }
-    const int h = (blockIdx.z - kGramBlocks) * 4 + w;
-    if (h >= H) return;                        // whole warps
+    const int c = blockIdx.x, b = blockIdx.z;
+    const int lane = threadIdx.x & 31;
+    const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
+    if (c == 0 && b == 0 && threadIdx.x == 0 && blockIdx.y == 0) *p.err = 0;
+    if (h >= p.H) return;                      // whole warps
+    const int L = p.L, H = p.H;
     const float A2 = -expf(__ldg(p.A_log + h)) * kLog2e;
     const float bias = __ldg(p.dt_bias + h);
-    float dt[2], a2[2];
+    const int t0 = c * kSsdQ + 4 * lane;
+    float dt[4], cum[4];
+    float run = 0.f;
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const int t = t0 + 2 * lane + k;
+    for (int k = 0; k < 4; ++k) {
+        const int t = t0 + k;
         dt[k] = t < L ? dt_from_raw(__bfloat162float(p.dt_raw[((size_t)b * L + t) * H + h]) + bias) : 0.f;
-        a2[k] = dt[k] * A2;
+        run += dt[k] * A2;
+        cum[k] = run;
     }
-    float s = a2[0] + a2[1];
+    float s = run;                             // inclusive scan of the lanes' totals
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
         const float o = __shfl_up_sync(0xffffffffu, s, d);
         if (lane >= d) s += o;
     }
+    const float before = s - run;
     const float alast = __shfl_sync(0xffffffffu, s, 31);
-    const float c0 = s - a2[1], c1 = s;
-    const int tl = t0 + 2 * lane;
-    const float e0 = tl < L ? lg2_approx(dt[0]) - c0 : -INFINITY;
-    const float e1 = tl + 1 < L ? lg2_approx(dt[1]) - c1 : -INFINITY;
-    float* out = p.prep + (((size_t)b * H + h) * nC + c) * 3 * kSsdQ;
-    *reinterpret_cast<float2*>(out + 2 * lane) = make_float2(c0, c1);
-    *reinterpret_cast<float2*>(out + kSsdQ + 2 * lane) = make_float2(e0, e1);
-    *reinterpret_cast<float2*>(out + 2 * kSsdQ + 2 * lane) =
-        make_float2(dt[0] * ex2_approx(alast - c0), dt[1] * ex2_approx(alast - c1));
+    float a[4], e[4], wv[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        a[k] = before + cum[k];
+        e[k] = t0 + k < L ? lg2_approx(dt[k]) - a[k] : -INFINITY;
+        wv[k] = dt[k] * ex2_approx(alast - a[k]);
+    }
+    float* out = p.prep + (((size_t)b * H + h) * p.nC + c) * 3 * kSsdQ + 4 * lane;
+    *reinterpret_cast<float4*>(out) = make_float4(a[0], a[1], a[2], a[3]);
+    *reinterpret_cast<float4*>(out + kSsdQ) = make_float4(e[0], e[1], e[2], e[3]);
+    *reinterpret_cast<float4*>(out + 2 * kSsdQ) = make_float4(wv[0], wv[1], wv[2], wv[3]);
 }
 
-// Packed float pairs (one instruction for two lanes of arithmetic).
-__device__ __forceinline__ unsigned long long f2_pack(float a, float b) {
-    return (unsigned long long)__float_as_uint(a) | ((unsigned long long)__float_as_uint(b) << 32);
-}
-__device__ __forceinline__ float f2_lo(unsigned long long v) { return __uint_as_float((uint32_t)v); }
-__device__ __forceinline__ float f2_hi(unsigned long long v) { return __uint_as_float((uint32_t)(v >> 32)); }
-__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
-    unsigned long long d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ unsigned long long f2_sub(unsigned long long a, unsigned long long b) {
-    unsigned long long d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
-// The pair (v0, v1) as bf16 pairs hi + lo: hi = the top 16 bits of each value
-// (truncation), lo = the remainder v - hi (exact in float32), rounded to bf16;
-// together about 16 significant bits.
-__device__ __forceinline__ void split_bf16(float v0, float v1, uint32_t& hi, uint32_t& lo) {
-    hi = __byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x7632);
-    const unsigned long long v = f2_pack(v0, v1);
-    const unsigned long long t = f2_pack(__uint_as_float(__float_as_uint(v0) & 0xffff0000u),
-                                         __uint_as_float(__float_as_uint(v1) & 0xffff0000u));
-    const unsigned long long r = f2_sub(v, t);
-    lo = pack_bf16(f2_lo(r), f2_hi(r));
-}
-
-// Shared memory of the chunk walk (bytes).  Two stages of per-chunk rows (C,
-// B, x of this head, the prep values), filled by cp.async one chunk ahead;
-// the full walk adds G (float32) and the decayed, masked Gram matrix M (bf16).
-// bf16 tiles have padded rows (128 columns: 272 bytes, 64 columns: 144
-// bytes), so the eight rows of an ldmatrix phase fall in distinct banks and
-// every fragment address is a per-lane base plus a constant.
-constexpr int kRowCB = 272;   // bytes per row of the C and B tiles
-constexpr int kRowX = 144;    // bytes per row of the x and M tiles
+// Shared memory of the chunk walk (bytes from a 1024-byte-aligned base).
+// STAGES copies of the input rows (C, B, x), STAGE bytes apart.
 template <bool kFull> struct SsdSmem;
 template <> struct SsdSmem<true> {
-    static constexpr int CS = 0, BS = CS + 64 * kRowCB, XS = BS + 64 * kRowCB, PR = XS + 64 * kRowX;
-    static constexpr int STAGE = PR + 3 * kSsdQ * 4;
-    static constexpr int GS = 2 * STAGE, MS = GS + kSsdQ * kSsdQ * 4, TOTAL = MS + 64 * kRowX;
+    static constexpr int STAGES = 2;
+    static constexpr int CT = 0;                 // C rows: 128 x 128 bf16
+    static constexpr int BT = CT + 32768;        // B rows: 128 x 128 bf16
+    static constexpr int XT = BT + 32768;        // x rows of this head: 128 x 64 bf16
+    static constexpr int STAGE = XT + 16384 - CT;
+    static constexpr int XW = STAGES * STAGE;    // w_j x_j rows
+    static constexpr int SH = XW + 16384;        // S^T rows, hi part: 128 (n) x 64 (p) bf16
+    static constexpr int SL = SH + 16384;        // lo part
+    static constexpr int PR = SL + 16384;        // two buffers of (acum, e, w) x 128 floats
+    static constexpr int MB = PR + 2 * 3 * kSsdQ * 4;   // mbarriers: Gram, state, outputs
+    static constexpr int SLOT = MB + 24;         // tensor-memory address
+    static constexpr int BYTES = SLOT + 8;
+    static constexpr int TOTAL = BYTES + 1024;   // with the alignment pad
+    // tensor memory: G (0..127); the state product (128..191); M as the A
+    // operand, two bf16 per column (192..255); C S^T, hi part (256..319) and lo
+    // part (320..383); M x (384..447)
+    static constexpr int TMEM_COLS = 512;
 };
 template <> struct SsdSmem<false> {
-    static constexpr int CS = -1, BS = 0, XS = BS + 64 * kRowCB, PR = XS + 64 * kRowX;
-    static constexpr int STAGE = PR + 3 * kSsdQ * 4;
-    static constexpr int GS = -1, MS = -1, TOTAL = 2 * STAGE;
+    static constexpr int STAGES = 1;
+    static constexpr int CT = -1;
+    static constexpr int BT = 0;
+    static constexpr int XT = BT + 32768;
+    static constexpr int STAGE = XT + 16384 - BT;
+    static constexpr int XW = STAGES * STAGE;
+    static constexpr int SH = -1, SL = -1;
+    static constexpr int PR = XW + 16384;
+    static constexpr int MB = PR + 2 * 3 * kSsdQ * 4;
+    static constexpr int SLOT = MB + 24;
+    static constexpr int BYTES = SLOT + 8;
+    static constexpr int TOTAL = BYTES + 1024;
+    static constexpr int TMEM_COLS = 64;
 };
 
-// The chunk walk of one (head h, run of chunks, batch row b), 128 threads.
-// kFull = false, the first walk: grid = (H, (segs - 1) pcs, B), one piece of
-// cpp chunks of a segment but the last, state products only, from h0 for the
-// first piece and zeros otherwise, writing the piece's local end state and
-// total decay.  kFull = true: grid = (H, segs, B), one segment, entering
-// with the fold of the pieces before it; the outputs y and, for the last
-// segment, the final state.
+// The chunk walk of one (head h, run of chunks, batch row b).
+// kFull = false, the first walk (128 threads): grid = (H, (segs - 1) pcs, B),
+// one piece of cpp chunks of a segment but the last, state products only, from
+// h0 for the first piece and zeros otherwise, writing the piece's local end
+// state and total decay.  kFull = true (256 threads): grid = (H, segs, B), one
+// segment, entering with the fold of the pieces before it; the outputs y and,
+// for the last segment, the final state.  Thread t serves row r = t % 128
+// (tensor-memory lane r, reachable from warps r/32 and r/32 + 4) and half
+// hf = t / 128 of that row's work: head columns 32 hf .. 32 hf + 31 of the
+// state, w x and y, and the column blocks jb = hf, hf + 2 of M.
 template <bool kFull>
-__global__ void __launch_bounds__(kSsdThreads, kFull ? 2 : 3) ssd_chunk_scan_kernel(SsdParams p) {
+__global__ void __launch_bounds__(kFull ? kSsdFullThreads : kSsdThreads, kFull ? 1 : 3)
+    ssd_chunk_scan_kernel(SsdParams p) {
     using Lay = SsdSmem<kFull>;
     constexpr int Q = kSsdQ, P = kSsdP, N = kSsdN;
-    extern __shared__ __align__(16) unsigned char smem[];
-    const unsigned sbase = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+    constexpr int NT = kFull ? kSsdFullThreads : kSsdThreads;
+    constexpr int HALVES = NT / 128;
+    constexpr int PH = P / HALVES;             // head columns per thread
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
+    const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+    unsigned char* sm = smem_raw + pad;
+    const uint32_t sb = raw + pad;
     const int h = blockIdx.x, seg = blockIdx.y, b = blockIdx.z;     // seg: segment, or piece of the first walk
     const int H = p.H, L = p.L, nC = p.nC;
+    const int tid = threadIdx.x, w = tid >> 5;
+    const int r = tid & 127, hf = tid >> 7, qd = w & 3;             // row, half, lane quadrant
     int c_begin, c_end;
     if constexpr (kFull) {
         c_begin = seg * p.cps;
@@ -260,276 +270,286 @@ __global__ void __launch_bounds__(kSsdThreads, kFull ? 2 : 3) ssd_chunk_scan_ker
         c_begin = k * p.cps + m * p.cpp;
         c_end = min(min(nC, (k + 1) * p.cps), c_begin + p.cpp);
     }
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, tq = lane & 3;
+    const uint32_t mbG = sb + Lay::MB, mbS = sb + Lay::MB + 8, mbY = sb + Lay::MB + 16;
 
-    // ---- per-thread parts of the copy addresses: B/C rows r = tid/16 + 8k, 16-byte
-    // piece tid%16; x rows r = tid/8 + 16k, piece tid%8; G rows as B/C
+    // ---- copies of chunk c's rows: B/C rows rBC + (NT/16) k, piece tid%16; x rows
+    // rX + (NT/8) k, piece tid%8; the prep values into buffer `slot`
     const int rBC = tid >> 4, pBC = tid & 15, rX = tid >> 3, pX = tid & 7;
-    const int sBC = rBC * kRowCB + pBC * 16, sX = rX * kRowX + pX * 16;
-    const int sG = rBC * 256 + ((pBC ^ ((rBC & 1) << 2)) << 4);
-    const size_t HP = (size_t)H * P;
-    auto issue_stage = [&](int c, int s) {
-        unsigned char* st = smem + s * Lay::STAGE;
+    const int sBC = tile_off(rBC, pBC), sX = tile_off(rX, pX);
+    auto issue_chunk = [&](int c, int slot) {
+        unsigned char* st = sm + (Lay::STAGES > 1 ? slot : 0) * Lay::STAGE;   // input rows of this chunk
         const int t0 = c * Q;
-        const int left = L - t0;               // rows of this chunk inside the sequence
-        const __nv_bfloat16* gB = p.Bm + ((size_t)b * L + t0 + rBC) * N + pBC * 8;
-        const __nv_bfloat16* gC = p.Cm + ((size_t)b * L + t0 + rBC) * N + pBC * 8;
+        const int left = L - t0;
+        const size_t rowBC = (size_t)b * L + t0 + rBC;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const bool ok = rBC + 8 * k < left;
-            cp_async16(st + Lay::BS + sBC + k * 8 * kRowCB, ok ? gB + (size_t)k * 8 * N : p.Bm, ok);
-            if constexpr (kFull) cp_async16(st + Lay::CS + sBC + k * 8 * kRowCB, ok ? gC + (size_t)k * 8 * N : p.Cm, ok);
+        for (int k = 0; k < 128 * 16 / NT; ++k) {
+            const int dr = (NT / 16) * k;
+            const bool ok = rBC + dr < left;
+            const size_t go = (rowBC + dr) * N + pBC * 8;
+            cp_async16(st + Lay::BT + sBC + dr * 128, ok ? p.Bm + go : p.Bm, ok);
+            if constexpr (kFull) cp_async16(st + Lay::CT + sBC + dr * 128, ok ? p.Cm + go : p.Cm, ok);
         }
-        const __nv_bfloat16* gX = p.x + (((size_t)b * L + t0 + rX) * H + h) * P + pX * 8;
+        const size_t rowX = (size_t)b * L + t0 + rX;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const bool ok = rX + 16 * k < left;
-            cp_async16(st + Lay::XS + sX + k * 16 * kRowX, ok ? gX + (size_t)k * 16 * HP : p.x, ok);
+        for (int k = 0; k < 128 * 8 / NT; ++k) {
+            const int dr = (NT / 8) * k;
+            const bool ok = rX + dr < left;
+            cp_async16(st + Lay::XT + sX + dr * 128, ok ? p.x + ((rowX + dr) * H + h) * P + pX * 8 : p.x, ok);
         }
         if (tid < 3 * Q / 4)
-            cp_async16(st + Lay::PR + tid * 16, p.prep + (((size_t)b * H + h) * nC + c) * 3 * Q + tid * 4, true);
-    };
-    auto issue_g = [&](int c) {
-        const float* gG = p.G + ((size_t)b * nC + c) * Q * Q + rBC * Q + pBC * 4;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) cp_async16(smem + Lay::GS + sG + k * 8 * 256, gG + k * 8 * Q, true);
+            cp_async16(sm + Lay::PR + slot * 3 * Q * 4 + tid * 16,
+                       p.prep + (((size_t)b * H + h) * nC + c) * 3 * Q + tid * 4, true);
+        cp_async_commit();
     };
 
-    // ---- per-lane parts of the ldmatrix addresses
-    const int rowL = (((lane >> 3) & 1) << 3) + (lane & 7), chL = lane >> 4;
-    const unsigned offCB = rowL * kRowCB + chL * 16;                 // C (A operand), B (transposed B operand)
-    const unsigned offM = rowL * kRowX + chL * 16;                   // M (A operand)
-    const unsigned offX = ((((lane >> 4) << 3) + (lane & 7)) * kRowX) + (2 * w + ((lane >> 3) & 1)) * 16;
+    // ---- tensor memory and mbarriers
+    if (tid == 0) {
+        mbar_init(mbG, 1);
+        mbar_init(mbS, 1);
+        mbar_init(mbY, 1);
+    }
+    if (w == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sb + Lay::SLOT),
+                     "r"(Lay::TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (c_begin < c_end) issue_chunk(c_begin, 0);
 
-    // ---- the carried state: rows p = 16w + g (+8), columns n = 8t + 2tq (+1)
-    float S[16][4];
-    const size_t hoff = (((size_t)b * H + h) * P + 16 * w) * N;
-    auto load_state = [&](const float* src) {
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const float2 u = *reinterpret_cast<const float2*>(src + hoff + g * N + 8 * t + 2 * tq);
-            const float2 v = *reinterpret_cast<const float2*>(src + hoff + (g + 8) * N + 8 * t + 2 * tq);
-            S[t][0] = u.x; S[t][1] = u.y; S[t][2] = v.x; S[t][3] = v.y;
-        }
-    };
-    auto store_state = [&](float* dst) {
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            *reinterpret_cast<float2*>(dst + hoff + g * N + 8 * t + 2 * tq) = make_float2(S[t][0], S[t][1]);
-            *reinterpret_cast<float2*>(dst + hoff + (g + 8) * N + 8 * t + 2 * tq) = make_float2(S[t][2], S[t][3]);
-        }
-    };
-    auto zero_state = [&]() {
-#pragma unroll
-        for (int t = 0; t < 16; ++t) S[t][0] = S[t][1] = S[t][2] = S[t][3] = 0.f;
-    };
+    // ---- the carried state, transposed: thread (n, hf) holds S[p][n] for its PH head columns
+    float S[PH];
+    const size_t hoff = ((size_t)b * H + h) * P * N + (size_t)(PH * hf) * N + r;
     const size_t BHPN = (size_t)p.B * H * P * N;
     bool s_nonzero;
     if constexpr (!kFull) {
         s_nonzero = seg == 0 && p.h0 != nullptr;
-        if (s_nonzero) {
-            load_state(p.h0);
-            if (p.h0c) store_state(p.h0c);
-        } else {
-            zero_state();
+#pragma unroll
+        for (int q = 0; q < PH; ++q) S[q] = s_nonzero ? p.h0[hoff + (size_t)q * N] : 0.f;
+        if (s_nonzero && p.h0c) {
+#pragma unroll
+            for (int q = 0; q < PH; ++q) p.h0c[hoff + (size_t)q * N] = S[q];
         }
     } else {
         if (seg == 0) {
             const float* src = p.h0c ? p.h0c : p.h0;
             s_nonzero = src != nullptr;
-            if (s_nonzero) load_state(src);
-            else zero_state();
+#pragma unroll
+            for (int q = 0; q < PH; ++q) S[q] = s_nonzero ? src[hoff + (size_t)q * N] : 0.f;
         } else {
             s_nonzero = true;
-            load_state(p.sloc);                                      // the first piece ran from h0
+#pragma unroll
+            for (int q = 0; q < PH; ++q) S[q] = p.sloc[hoff + (size_t)q * N];     // the first piece ran from h0
             for (int j = 1; j < seg * p.pcs; ++j) {
                 const float dj = ex2_approx(p.sega[((size_t)j * p.B + b) * H + h]);
-                const float* src = p.sloc + (size_t)j * BHPN;
+                const float* src = p.sloc + (size_t)j * BHPN + hoff;
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const float2 u = *reinterpret_cast<const float2*>(src + hoff + g * N + 8 * t + 2 * tq);
-                    const float2 v = *reinterpret_cast<const float2*>(src + hoff + (g + 8) * N + 8 * t + 2 * tq);
-                    S[t][0] = fmaf(dj, S[t][0], u.x); S[t][1] = fmaf(dj, S[t][1], u.y);
-                    S[t][2] = fmaf(dj, S[t][2], v.x); S[t][3] = fmaf(dj, S[t][3], v.y);
-                }
+                for (int q = 0; q < PH; ++q) S[q] = fmaf(dj, S[q], src[(size_t)q * N]);
             }
         }
     }
-
-    float seg_decay = 0.f;
-    if (c_begin < c_end) {
-        issue_stage(c_begin, 0);
-        if constexpr (kFull) issue_g(c_begin);
-        cp_async_commit();
-    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(sm + Lay::SLOT);
+    const uint32_t tlane = tbase + ((uint32_t)(qd * 32) << 16);     // this warp's lanes
+    bool ok_all = true;
     float Dh = 0.f;
     if constexpr (kFull) Dh = __ldg(p.D + h);
-    // M build: thread -> row tid/8 of a 16x16 block, column pair tid%8
-    const int rr = tid >> 3, k2 = 2 * (tid & 7);
-    int gcol[4];                               // byte offset of G[rr][16jb + k2] within a row pair
-#pragma unroll
-    for (int jb = 0; jb < 4; ++jb) gcol[jb] = ((((jb ^ (rr & 1)) << 2) + (k2 >> 2)) << 4) + (k2 & 3) * 4;
+    float seg_decay = 0.f;
+    // instruction descriptors
+    constexpr uint32_t kIdGram = umma_idesc(128, 128, 0, 0);     // C (K-major) x B rows (K-major)
+    constexpr uint32_t kIdState = umma_idesc(128, 64, 1, 1);     // B rows as B^T (MN-major) x w x (MN-major)
+    constexpr uint32_t kIdOff = umma_idesc(128, 128, 0, 1);      // C (K-major) x [S^T hi | S^T lo] (MN-major)
+    constexpr uint32_t kIdDiag = umma_idesc(128, 64, 0, 1);      // M (tensor memory, K-major) x x (MN-major)
+    constexpr uint32_t kColState = kFull ? 128 : 0;
 
     for (int c = c_begin; c < c_end; ++c) {
-        const int s = (c - c_begin) & 1;
-        const unsigned st = sbase + s * Lay::STAGE;
-        const float* pr = reinterpret_cast<const float*>(smem + s * Lay::STAGE + Lay::PR);  // acum, e, w
+        const int k = c - c_begin;
+        const uint32_t par = (uint32_t)(k & 1);
+        const float* pr = reinterpret_cast<const float*>(sm + Lay::PR + (k & 1) * 3 * Q * 4);   // acum, e, w
+        const int so = (Lay::STAGES > 1 ? (k & 1) : 0) * Lay::STAGE;                              // this chunk's rows
         cp_async_wait_0();
-        __syncthreads();                       // this chunk's rows landed; chunk c-1 is done everywhere
-        if (c + 1 < c_end) {
-            issue_stage(c + 1, s ^ 1);
-            cp_async_commit();
-        }
-
+        fence_async_smem();
+        tc_fence_before();
+        // chunk c's rows landed; the previous chunk's tensor reads done; a wait that
+        // gave up anywhere ends the walk for the whole CTA
+        if (__syncthreads_or(!ok_all)) break;
+        tc_fence_after();
         if constexpr (kFull) {
-            // ---- M = mask(G_ij 2^(acum_i + e_j)) + D on the diagonal, bf16: the ten 16x16
-            // blocks on or below the diagonal
-            float2 ej[4];
+            // the other stage was last read by the previous chunk, whose products are done
+            if (c + 1 < c_end) issue_chunk(c + 1, (k + 1) & 1);
+            if (tid == 0) {
 #pragma unroll
-            for (int jb = 0; jb < 4; ++jb) ej[jb] = *reinterpret_cast<const float2*>(pr + Q + 16 * jb + k2);
-#pragma unroll
-            for (int ib = 0; ib < 4; ++ib) {
-                const int i = 16 * ib + rr;
-                const float ai = pr[i];
-#pragma unroll
-                for (int jb = 0; jb <= ib; ++jb) {
-                    const int j = 16 * jb + k2;
-                    const float2 gv = *reinterpret_cast<const float2*>(smem + Lay::GS + i * 256 + gcol[jb]);
-                    float m0 = gv.x * ex2_approx(ai + ej[jb].x);
-                    float m1 = gv.y * ex2_approx(ai + ej[jb].y);
-                    if (jb == ib) {
-                        m0 = j < i ? m0 : (j == i ? m0 + Dh : 0.f);
-                        m1 = j + 1 < i ? m1 : (j + 1 == i ? m1 + Dh : 0.f);
-                    }
-                    *reinterpret_cast<uint32_t*>(smem + Lay::MS + i * kRowX + j * 2) = pack_bf16(m0, m1);
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t off = so + (ks >> 2) * 16384 + (ks & 3) * 32;
+                    umma(tbase, umma_desc(sb + Lay::CT + off, 16, 1024), umma_desc(sb + Lay::BT + off, 16, 1024),
+                         kIdGram, ks > 0);
                 }
-            }
-            __syncthreads();                   // M complete; G free
-            if (c + 1 < c_end) {
-                issue_g(c + 1);
-                cp_async_commit();
+                umma_commit(mbG);
             }
         }
-
-        // ---- x of this warp's 16 head columns: ks -> tokens 16ks .. 16ks+15
-        uint32_t xr[4][4];
+        // ---- w_j x_j (thread (j, hf): its 16-byte pieces of row j)
+        {
+            const float wj = pr[2 * Q + r];
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) ldsm_x4_t(xr[ks], st + Lay::XS + offX + ks * 16 * kRowX);
-
+            for (int pc = (8 / HALVES) * hf; pc < (8 / HALVES) * (hf + 1); ++pc) {
+                const uint4 v = *reinterpret_cast<const uint4*>(sm + so + Lay::XT + tile_off(r, pc));
+                uint4 o;
+                o.x = pack_bf16(bf16_lo(v.x) * wj, bf16_hi(v.x) * wj);
+                o.y = pack_bf16(bf16_lo(v.y) * wj, bf16_hi(v.y) * wj);
+                o.z = pack_bf16(bf16_lo(v.z) * wj, bf16_hi(v.z) * wj);
+                o.w = pack_bf16(bf16_lo(v.w) * wj, bf16_hi(v.w) * wj);
+                *reinterpret_cast<uint4*>(sm + Lay::XW + tile_off(r, pc)) = o;
+            }
+        }
         if constexpr (kFull) {
-            float yacc[4][2][4];
+            // ---- S_in^T row n as hi + lo bf16 parts (thread (n, hf): its head columns), when nonzero
+            if (s_nonzero || k > 0) {
 #pragma unroll
-            for (int rb = 0; rb < 4; ++rb)
+                for (int pq = 0; pq < PH / 8; ++pq) {
+                    const int pc = (PH / 8) * hf + pq;
+                    uint32_t hi[4], lo[4];
 #pragma unroll
-                for (int pt = 0; pt < 2; ++pt) yacc[rb][pt][0] = yacc[rb][pt][1] = yacc[rb][pt][2] = yacc[rb][pt][3] = 0.f;
-            if (s_nonzero || c > c_begin) {
-                // exp(acum_i) C_i . S_in: K = the state columns, B operand = the state registers
-#pragma unroll
-                for (int ks = 0; ks < N / 16; ++ks) {
-                    uint32_t bh[2][2], bl[2][2];
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const float* v = S[2 * ks + half];
-                        split_bf16(v[0], v[1], bh[0][half], bl[0][half]);
-                        split_bf16(v[2], v[3], bh[1][half], bl[1][half]);
+                    for (int q = 0; q < 4; ++q) {
+                        const float v0 = S[8 * pq + 2 * q], v1 = S[8 * pq + 2 * q + 1];
+                        hi[q] = __byte_perm(__float_as_uint(v0), __float_as_uint(v1), 0x7632);
+                        lo[q] = pack_bf16(v0 - bf16_lo(hi[q]), v1 - bf16_hi(hi[q]));
                     }
-                    uint32_t a[4][4];
-#pragma unroll
-                    for (int rb = 0; rb < 4; ++rb) ldsm_x4(a[rb], st + Lay::CS + offCB + rb * 16 * kRowCB + ks * 32);
-#pragma unroll
-                    for (int rb = 0; rb < 4; ++rb)
-#pragma unroll
-                        for (int pt = 0; pt < 2; ++pt) mma_16816(yacc[rb][pt], a[rb], bl[pt][0], bl[pt][1]);
-#pragma unroll
-                    for (int rb = 0; rb < 4; ++rb)
-#pragma unroll
-                        for (int pt = 0; pt < 2; ++pt) mma_16816(yacc[rb][pt], a[rb], bh[pt][0], bh[pt][1]);
-                }
-#pragma unroll
-                for (int rb = 0; rb < 4; ++rb) {
-                    const unsigned long long e =
-                        f2_pack(ex2_approx(pr[16 * rb + g]), ex2_approx(pr[16 * rb + g + 8]));
-#pragma unroll
-                    for (int pt = 0; pt < 2; ++pt) {
-                        const unsigned long long u = f2_mul(f2_pack(yacc[rb][pt][0], yacc[rb][pt][2]), e);
-                        const unsigned long long v = f2_mul(f2_pack(yacc[rb][pt][1], yacc[rb][pt][3]), e);
-                        yacc[rb][pt][0] = f2_lo(u); yacc[rb][pt][2] = f2_hi(u);
-                        yacc[rb][pt][1] = f2_lo(v); yacc[rb][pt][3] = f2_hi(v);
-                    }
+                    *reinterpret_cast<uint4*>(sm + Lay::SH + tile_off(r, pc)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4*>(sm + Lay::SL + tile_off(r, pc)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                 }
             }
-            // + M x: K = the chunk's tokens, blocks on or below the diagonal
+            // ---- M row i from G row i into tensor memory (the A operand of M x): thread
+            // (i, hf) takes the 32-column blocks jb = hf, hf + 2; zeros above the diagonal
+            ok_all &= mbar_wait(mbG, par);
+            tc_fence_after();
+            const int i = r;
+            const float ai = pr[i];
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-                uint32_t a[4][4];
+            for (int bb = 0; bb < 2; ++bb) {
+                const int jb = hf + 2 * bb;
+                uint32_t m[16];
+                if (jb <= qd) {                // warp-uniform: rows 32 qd .. 32 qd + 31
 #pragma unroll
-                for (int rb = kb; rb < 4; ++rb) ldsm_x4(a[rb], sbase + Lay::MS + offM + rb * 16 * kRowX + kb * 32);
+                    for (int hb = 0; hb < 2; ++hb) {
+                        float g[16];
+                        tmem_ld16(tlane + 32 * jb + 16 * hb, g);
+                        const int j0 = 32 * jb + 16 * hb;
 #pragma unroll
-                for (int rb = kb; rb < 4; ++rb) {
-                    mma_16816(yacc[rb][0], a[rb], xr[kb][0], xr[kb][2]);
-                    mma_16816(yacc[rb][1], a[rb], xr[kb][1], xr[kb][3]);
-                }
-            }
-            // ---- y rows inside the sequence
-            const int left = L - c * Q;
-            __nv_bfloat16* yb = p.y + (((size_t)b * L + (size_t)c * Q + g) * H + h) * P + 16 * w + 2 * tq;
-#pragma unroll
-            for (int rb = 0; rb < 4; ++rb)
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    if (16 * rb + g + 8 * r < left) {
-                        __nv_bfloat16* yo = yb + (size_t)(16 * rb + 8 * r) * HP;
-#pragma unroll
-                        for (int pt = 0; pt < 2; ++pt)
-                            *reinterpret_cast<uint32_t*>(yo + 8 * pt) = pack_bf16(yacc[rb][pt][2 * r], yacc[rb][pt][2 * r + 1]);
+                        for (int q = 0; q < 8; ++q) {
+                            const int j = j0 + 2 * q;
+                            const float2 e2 = *reinterpret_cast<const float2*>(pr + Q + j);
+                            float m0 = g[2 * q] * ex2_approx(ai + e2.x);
+                            float m1 = g[2 * q + 1] * ex2_approx(ai + e2.y);
+                            if (jb == qd) {
+                                m0 = j < i ? m0 : (j == i ? m0 + Dh : 0.f);
+                                m1 = j + 1 < i ? m1 : (j + 1 == i ? m1 + Dh : 0.f);
+                            }
+                            m[8 * hb + q] = pack_bf16(m0, m1);
+                        }
                     }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) m[q] = 0u;
                 }
+                tmem_st16(tlane + 192 + 16 * jb, m);
+            }
+            tmem_st_wait();
         }
-
-        // ---- S = exp(acum_last) S + (w x)^T B: K = the chunk's tokens
+        fence_async_smem();
+        tc_fence_before();
+        if (__syncthreads_or(!ok_all)) break;  // w x, S parts and M written; G read
+        tc_fence_after();
+        if (tid == 0) {
+            // state: S^T += B^T (w x): A = B rows (MN-major, two 64-column blocks), K = the tokens
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                umma(tbase + kColState, umma_desc(sb + so + Lay::BT + ks * 2048, 16384, 1024),
+                     umma_desc(sb + Lay::XW + ks * 2048, 16384, 1024), kIdState, ks > 0);
+            umma_commit(mbS);
+            if constexpr (kFull) {
+                // outputs: C [S_in^T hi | lo] (N = 128, the lo part 16 KB after the hi part)
+                // into columns 256..383, M x into 384..447
+                if (s_nonzero || k > 0) {
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t off = so + (ks >> 2) * 16384 + (ks & 3) * 32;
+                        umma(tbase + 256, umma_desc(sb + Lay::CT + off, 16, 1024),
+                             umma_desc(sb + Lay::SH + ks * 2048, 16384, 1024), kIdOff, ks > 0);
+                    }
+                }
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_ts(tbase + 384, tbase + 192 + 8 * ks, umma_desc(sb + so + Lay::XT + ks * 2048, 16384, 1024),
+                            kIdDiag, ks > 0);
+                umma_commit(mbY);
+            }
+        }
+        // ---- state update (thread (n, hf): its head columns of row n of S^T)
+        ok_all &= mbar_wait(mbS, par);
+        tc_fence_after();
         const float alast = pr[Q - 1];
         seg_decay += alast;
         const float el = ex2_approx(alast);
-        const unsigned long long el2 = f2_pack(el, el);
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const unsigned long long u = f2_mul(f2_pack(S[t][0], S[t][1]), el2);
-            const unsigned long long v = f2_mul(f2_pack(S[t][2], S[t][3]), el2);
-            S[t][0] = f2_lo(u); S[t][1] = f2_hi(u); S[t][2] = f2_lo(v); S[t][3] = f2_hi(v);
+        if constexpr (!kFull) {
+            if (c + 1 < c_end) issue_chunk(c + 1, (k + 1) & 1);     // every tensor read of this chunk is done
         }
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const float4 wv = make_float4(pr[2 * Q + 16 * ks + 2 * tq], pr[2 * Q + 16 * ks + 2 * tq + 1],
-                                          pr[2 * Q + 16 * ks + 8 + 2 * tq], pr[2 * Q + 16 * ks + 9 + 2 * tq]);
-            const unsigned long long wa = f2_pack(wv.x, wv.y), wb = f2_pack(wv.z, wv.w);
-            uint32_t a[4];
+        for (int q0 = 0; q0 < PH; q0 += 16) {
+            float d[16];
+            tmem_ld16(tlane + kColState + PH * hf + q0, d);
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const unsigned long long xv = f2_mul(f2_pack(bf16_lo(xr[ks][r]), bf16_hi(xr[ks][r])), r < 2 ? wa : wb);
-                a[r] = pack_bf16(f2_lo(xv), f2_hi(xv));
-            }
-            constexpr int kBatch = kFull ? 8 : 4;             // fragments loaded ahead of their MMAs
+            for (int q = 0; q < 16; ++q) S[q0 + q] = fmaf(el, S[q0 + q], d[q]);
+        }
+        if constexpr (kFull) {
+            // ---- y row i, head columns of this half: 2^acum_i (C S_in^T)_i + (M x)_i
+            ok_all &= mbar_wait(mbY, par);
+            tc_fence_after();
+            const int i = r;
+            const bool with_state = s_nonzero || k > 0;
+            const float ea = ex2_approx(pr[i]);
+            const bool inside = c * Q + i < L;
+            __nv_bfloat16* yo = p.y + (((size_t)b * L + (size_t)c * Q + i) * H + h) * P + PH * hf;
 #pragma unroll
-            for (int q0 = 0; q0 < 8; q0 += kBatch) {
-                uint32_t bb[kBatch][4];
+            for (int q0 = 0; q0 < PH; q0 += 16) {
+                float yd[16], yh[16], yl[16];
+                tmem_ld16(tlane + 384 + PH * hf + q0, yd);     // warp-wide: rows past L take part too
+                if (with_state) {
+                    tmem_ld16(tlane + 256 + PH * hf + q0, yh);
+                    tmem_ld16(tlane + 320 + PH * hf + q0, yl);
+                }
+                uint32_t o[8];
 #pragma unroll
-                for (int q = 0; q < kBatch; ++q)
-                    ldsm_x4_t(bb[q], st + Lay::BS + offCB + ks * 16 * kRowCB + (q0 + q) * 32);
-#pragma unroll
-                for (int q = 0; q < kBatch; ++q) {
-                    mma_16816(S[2 * (q0 + q)], a, bb[q][0], bb[q][1]);
-                    mma_16816(S[2 * (q0 + q) + 1], a, bb[q][2], bb[q][3]);
+                for (int q = 0; q < 8; ++q) {
+                    const float y0 = with_state ? fmaf(ea, yh[2 * q] + yl[2 * q], yd[2 * q]) : yd[2 * q];
+                    const float y1 = with_state ? fmaf(ea, yh[2 * q + 1] + yl[2 * q + 1], yd[2 * q + 1]) : yd[2 * q + 1];
+                    o[q] = pack_bf16(y0, y1);
+                }
+                if (inside) {
+                    *reinterpret_cast<uint4*>(yo + q0) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4*>(yo + q0 + 8) = make_uint4(o[4], o[5], o[6], o[7]);
                 }
             }
         }
     }
 
+    cp_async_wait_0();                         // this thread's copies in flight
+    if (!ok_all) atomicExch(p.err, 1);
     if constexpr (kFull) {
-        if (seg == p.segs - 1) store_state(p.h_out);
+        if (seg == p.segs - 1) {
+#pragma unroll
+            for (int q = 0; q < PH; ++q) p.h_out[hoff + (size_t)q * N] = S[q];
+        }
     } else {
-        store_state(p.sloc + (size_t)seg * BHPN);
+        float* dst = p.sloc + (size_t)seg * BHPN + hoff;
+#pragma unroll
+        for (int q = 0; q < PH; ++q) dst[(size_t)q * N] = S[q];
         if (tid == 0) p.sega[((size_t)seg * p.B + b) * H + h] = seg_decay;
     }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (w == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(Lay::TMEM_COLS));
 }
 
 }  // namespace axon

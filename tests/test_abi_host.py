@@ -292,16 +292,15 @@ def test_ssd_rejects_bad_arguments(lib):
     q = lib.axon_ssd_workspace_bytes
     q.restype = ctypes.c_size_t
     q.argtypes = [ctypes.c_int] * 6
-    # one segment: the chunk Gram matrices (three 64-token chunks per batch row)
-    # and the per-chunk decays, each rounded up to 256 bytes
-    gram, prep = 2 * 3 * 64 * 64 * 4, 2 * 3 * 3 * 3 * 64 * 4
-    assert q(2, 130, 3, 64, 128, 1) == gram + (prep + 255) // 256 * 256
-    # two segments (chunks 0-1, 2): the state-only walk over the first segment
-    # runs in one-chunk pieces (few heads), each adding a local end state per
-    # (b, h) and its decay; plus the copy of h0
+    # one segment: a 256-byte error flag and the per-chunk decays (two
+    # 128-token chunks per batch row: acum, log2 dt - acum, w per token and head)
+    prep = 2 * 3 * 2 * 3 * 128 * 4
+    assert q(2, 130, 3, 64, 128, 1) == 256 + prep
+    # two segments (one chunk each): the state-only walk over the first segment
+    # adds one local end state per (b, h) and its decay, plus the copy of h0
     state = 2 * 3 * 64 * 128 * 4
-    assert q(2, 130, 3, 64, 128, 2) == gram + (prep + 255) // 256 * 256 + 2 * state + 256 + state
-    assert q(2, 130, 3, 64, 128, 5) == q(2, 130, 3, 64, 128, 3)     # at most one segment per chunk
+    assert q(2, 130, 3, 64, 128, 2) == 256 + prep + state + 256 + state
+    assert q(2, 130, 3, 64, 128, 5) == q(2, 130, 3, 64, 128, 2)     # at most one segment per chunk
     assert q(2, 0, 3, 64, 128, 0) == 0
     assert q(1, 128, 1, 32, 128, 0) == 0
     assert q(1, 128, 1, 64, 128, -1) == 0
