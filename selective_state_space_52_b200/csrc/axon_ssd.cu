@@ -78,7 +78,7 @@ SsdWs ws_layout(int B, int L, int H, int segs, int pcs) {
     SsdWs w{};
     w.err = 0;
     w.prep = w.err + 256;
-    w.sloc = w.prep + up256((size_t)B * H * nC * 3 * kSsdQ * 4);
+    w.sloc = w.prep + up256((size_t)B * H * nC * 4 * kSsdQ * 4);
     const size_t extra = segs > 1 ? (size_t)(segs - 1) * pcs : 0;
     w.sega = w.sloc + up256(extra * B * H * kSsdP * kSsdN * 4);
     w.h0c = w.sega + up256(extra * B * H * 4);

@@ -66,7 +66,7 @@ struct SsdParams {
     const float* h0;             // (B, H, P, N) or null
     __nv_bfloat16* y;            // (B, L, H, P)
     float* h_out;                // (B, H, P, N)
-    float* prep;                 // (B, H, nC, 3, Q): acum (log2 units), log2(dt) - acum, w
+    float* prep;                 // (B, H, nC, 4, Q): acum (log2 units), log2(dt) - acum, w, v
     float* sloc;                 // ((segs - 1) pcs, B, H, P, N): local end states of the pieces
     float* sega;                 // ((segs - 1) pcs, B, H): total decay of a piece (log2 units)
     float* h0c;                  // (B, H, P, N): copy of h0 (h_out may overwrite h0) when segs > 1
@@ -153,8 +153,12 @@ __device__ __forceinline__ int tile_off(int r, int pc) {
 
 // Per (b, chunk, head): dt_j, acum_j (log2 units: exp(acum) = 2^acum2),
 // e_j = log2(dt_j) - acum2_j (so dt_j exp(acum_i - acum_j) = 2^(acum2_i + e_j),
-// whose exponent never exceeds log2(dt_j) for j <= i), and the state weights
-// w_j = dt_j 2^(acum2_{Q-1} - acum2_j).  Tokens past L get dt = 0, e = -inf.
+// whose exponent never exceeds log2(dt_j) for j <= i), the state weights
+// w_j = dt_j 2^(acum2_{Q-1} - acum2_j), and v_j = dt_j 2^(acum2_r - acum2_j)
+// with r the last token of j's 32-token block: below the diagonal blocks,
+// dt_j exp(acum_i - acum_j) = 2^(acum2_i - acum2_r) v_j, both factors at most
+// 1 (acum decreases), so neither overflows and an underflow only drops a term
+// below 2^-126 of G_ij dt_j.  Tokens past L get dt = 0, e = -inf, v = 0.
 // grid = (nC, ceil(H / 4), B), 128 threads: warp -> head, lane -> 4 tokens.
 __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_prep_kernel(SsdParams p) {
     const int c = blockIdx.x, b = blockIdx.z;
@@ -183,17 +187,20 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_prep_kernel(SsdParams p
     }
     const float before = s - run;
     const float alast = __shfl_sync(0xffffffffu, s, 31);
-    float a[4], e[4], wv[4];
+    const float ablock = __shfl_sync(0xffffffffu, s, lane | 7);   // acum2 at the last token of this 32-token block
+    float a[4], e[4], wv[4], vv[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         a[k] = before + cum[k];
         e[k] = t0 + k < L ? lg2_approx(dt[k]) - a[k] : -INFINITY;
         wv[k] = dt[k] * ex2_approx(alast - a[k]);
+        vv[k] = dt[k] * ex2_approx(ablock - a[k]);
     }
-    float* out = p.prep + (((size_t)b * H + h) * p.nC + c) * 3 * kSsdQ + 4 * lane;
+    float* out = p.prep + (((size_t)b * H + h) * p.nC + c) * 4 * kSsdQ + 4 * lane;
     *reinterpret_cast<float4*>(out) = make_float4(a[0], a[1], a[2], a[3]);
     *reinterpret_cast<float4*>(out + kSsdQ) = make_float4(e[0], e[1], e[2], e[3]);
     *reinterpret_cast<float4*>(out + 2 * kSsdQ) = make_float4(wv[0], wv[1], wv[2], wv[3]);
+    *reinterpret_cast<float4*>(out + 3 * kSsdQ) = make_float4(vv[0], vv[1], vv[2], vv[3]);
 }
 
 // Shared memory of the chunk walk (bytes from a 1024-byte-aligned base).
@@ -208,8 +215,8 @@ template <> struct SsdSmem<true> {
     static constexpr int XW = STAGES * STAGE;    // w_j x_j rows
     static constexpr int SH = XW + 16384;        // S^T rows, hi part: 128 (n) x 64 (p) bf16
     static constexpr int SL = SH + 16384;        // lo part
-    static constexpr int PR = SL + 16384;        // two buffers of (acum, e, w) x 128 floats
-    static constexpr int MB = PR + 2 * 3 * kSsdQ * 4;   // mbarriers: Gram, state, outputs
+    static constexpr int PR = SL + 16384;        // two buffers of (acum, e, w, v) x 128 floats
+    static constexpr int MB = PR + 2 * 4 * kSsdQ * 4;   // mbarriers: Gram, state, outputs
     static constexpr int SLOT = MB + 24;         // tensor-memory address
     static constexpr int BYTES = SLOT + 8;
     static constexpr int TOTAL = BYTES + 1024;   // with the alignment pad
@@ -227,7 +234,7 @@ template <> struct SsdSmem<false> {
     static constexpr int XW = STAGES * STAGE;
     static constexpr int SH = -1, SL = -1;
     static constexpr int PR = XW + 16384;
-    static constexpr int MB = PR + 2 * 3 * kSsdQ * 4;
+    static constexpr int MB = PR + 2 * 4 * kSsdQ * 4;
     static constexpr int SLOT = MB + 24;
     static constexpr int BYTES = SLOT + 8;
     static constexpr int TOTAL = BYTES + 1024;
@@ -296,9 +303,9 @@ __global__ void __launch_bounds__(kFull ? kSsdFullThreads : kSsdThreads, kFull ?
             const bool ok = rX + dr < left;
             cp_async16(st + Lay::XT + sX + dr * 128, ok ? p.x + ((rowX + dr) * H + h) * P + pX * 8 : p.x, ok);
         }
-        if (tid < 3 * Q / 4)
-            cp_async16(sm + Lay::PR + slot * 3 * Q * 4 + tid * 16,
-                       p.prep + (((size_t)b * H + h) * nC + c) * 3 * Q + tid * 4, true);
+        if (tid < Q)
+            cp_async16(sm + Lay::PR + slot * 4 * Q * 4 + tid * 16,
+                       p.prep + (((size_t)b * H + h) * nC + c) * 4 * Q + tid * 4, true);
         cp_async_commit();
     };
 
@@ -366,7 +373,7 @@ __global__ void __launch_bounds__(kFull ? kSsdFullThreads : kSsdThreads, kFull ?
     for (int c = c_begin; c < c_end; ++c) {
         const int k = c - c_begin;
         const uint32_t par = (uint32_t)(k & 1);
-        const float* pr = reinterpret_cast<const float*>(sm + Lay::PR + (k & 1) * 3 * Q * 4);   // acum, e, w
+        const float* pr = reinterpret_cast<const float*>(sm + Lay::PR + (k & 1) * 4 * Q * 4);   // acum, e, w, v
         const int so = (Lay::STAGES > 1 ? (k & 1) : 0) * Lay::STAGE;                              // this chunk's rows
         cp_async_wait_0();
         fence_async_smem();
@@ -403,6 +410,18 @@ __global__ void __launch_bounds__(kFull ? kSsdFullThreads : kSsdThreads, kFull ?
             }
         }
         if constexpr (kFull) {
+            // the state product needs only w x: issue it now, to run during the M build
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            if (tid == 0) {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    umma(tbase + kColState, umma_desc(sb + so + Lay::BT + ks * 2048, 16384, 1024),
+                         umma_desc(sb + Lay::XW + ks * 2048, 16384, 1024), kIdState, ks > 0);
+                umma_commit(mbS);
+            }
             // ---- S_in^T row n as hi + lo bf16 parts (thread (n, hf): its head columns), when nonzero
             if (s_nonzero || k > 0) {
 #pragma unroll
@@ -435,17 +454,24 @@ __global__ void __launch_bounds__(kFull ? kSsdFullThreads : kSsdThreads, kFull ?
                         float g[16];
                         tmem_ld16(tlane + 32 * jb + 16 * hb, g);
                         const int j0 = 32 * jb + 16 * hb;
+                        if (jb < qd) {         // below the diagonal: G u_i v_j
+                            const float ui = ex2_approx(ai - pr[32 * jb + 31]);
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            const int j = j0 + 2 * q;
-                            const float2 e2 = *reinterpret_cast<const float2*>(pr + Q + j);
-                            float m0 = g[2 * q] * ex2_approx(ai + e2.x);
-                            float m1 = g[2 * q + 1] * ex2_approx(ai + e2.y);
-                            if (jb == qd) {
+                            for (int q = 0; q < 8; ++q) {
+                                const float2 v2 = *reinterpret_cast<const float2*>(pr + 3 * Q + j0 + 2 * q);
+                                m[8 * hb + q] = pack_bf16(g[2 * q] * ui * v2.x, g[2 * q + 1] * ui * v2.y);
+                            }
+                        } else {               // the diagonal block: masked, D on the diagonal
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const int j = j0 + 2 * q;
+                                const float2 e2 = *reinterpret_cast<const float2*>(pr + Q + j);
+                                float m0 = g[2 * q] * ex2_approx(ai + e2.x);
+                                float m1 = g[2 * q + 1] * ex2_approx(ai + e2.y);
                                 m0 = j < i ? m0 : (j == i ? m0 + Dh : 0.f);
                                 m1 = j + 1 < i ? m1 : (j + 1 == i ? m1 + Dh : 0.f);
+                                m[8 * hb + q] = pack_bf16(m0, m1);
                             }
-                            m[8 * hb + q] = pack_bf16(m0, m1);
                         }
                     }
                 } else {
@@ -461,13 +487,14 @@ __global__ void __launch_bounds__(kFull ? kSsdFullThreads : kSsdThreads, kFull ?
         if (__syncthreads_or(!ok_all)) break;  // w x, S parts and M written; G read
         tc_fence_after();
         if (tid == 0) {
-            // state: S^T += B^T (w x): A = B rows (MN-major, two 64-column blocks), K = the tokens
+            if constexpr (!kFull) {
+                // state: S^T += B^T (w x): A = B rows (MN-major, two 64-column blocks), K = the tokens
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                umma(tbase + kColState, umma_desc(sb + so + Lay::BT + ks * 2048, 16384, 1024),
-                     umma_desc(sb + Lay::XW + ks * 2048, 16384, 1024), kIdState, ks > 0);
-            umma_commit(mbS);
-            if constexpr (kFull) {
+                for (int ks = 0; ks < 8; ++ks)
+                    umma(tbase + kColState, umma_desc(sb + so + Lay::BT + ks * 2048, 16384, 1024),
+                         umma_desc(sb + Lay::XW + ks * 2048, 16384, 1024), kIdState, ks > 0);
+                umma_commit(mbS);
+            } else {
                 // outputs: C [S_in^T hi | lo] (N = 128, the lo part 16 KB after the hi part)
                 // into columns 256..383, M x into 384..447
                 if (s_nonzero || k > 0) {

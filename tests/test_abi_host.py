@@ -293,8 +293,8 @@ def test_ssd_rejects_bad_arguments(lib):
     q.restype = ctypes.c_size_t
     q.argtypes = [ctypes.c_int] * 6
     # one segment: a 256-byte error flag and the per-chunk decays (two
-    # 128-token chunks per batch row: acum, log2 dt - acum, w per token and head)
-    prep = 2 * 3 * 2 * 3 * 128 * 4
+    # 128-token chunks per batch row: acum, log2 dt - acum, w, v per token and head)
+    prep = 2 * 3 * 2 * 4 * 128 * 4
     assert q(2, 130, 3, 64, 128, 1) == 256 + prep
     # two segments (one chunk each): the state-only walk over the first segment
     # adds one local end state per (b, h) and its decay, plus the copy of h0
