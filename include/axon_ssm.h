@@ -330,18 +330,22 @@ AXON_API axon_status axon_ssm_carry_fold(int P, int r, int B, int E, int N, cons
  * Layouts: x, y (B,L,H,P) bf16; dt_raw (B,L,H) bf16; Bm, Cm (B,L,N) bf16,
  * shared by all heads; dt_bias, A_log, D (H) float32; h0 (B,H,P,N) float32 or
  * NULL (zeros); h_out (B,H,P,N) float32, may be h0 itself.  P == 64, N == 128
- * and io == AXON_BF16 only (else AXON_ERR_UNSUPPORTED).  The products take
- * bf16 operands (the decayed chunk Gram matrix with D on its diagonal, the
- * dt-weighted x, and the carried state split in two bf16 parts) with float32
- * accumulation; the carried state itself is float32.  To fill the GPU when
- * B * H is small the sequence is cut into `segments` runs of whole 64-token
- * chunks (0: chosen for the current device, about two walks per SM; capped at
- * one per chunk and 64): a first walk of every segment but the last gives its
- * local end state from a zero state, and the full walk of each segment starts
- * from the fold of those.  `workspace` (16-byte aligned; may be NULL when the
- * size is 0) holds axon_ssd_workspace_bytes(B, L, H, P, N, segments) bytes for
- * the same `segments` on the current device: the chunk Gram matrices C B^T,
- * the per-chunk decays and weights, and the segments' local states.  Other
+ * and io == AXON_BF16 only (else AXON_ERR_UNSUPPORTED).  The products run on
+ * the tcgen05 tensor cores with bf16 operands (the decayed chunk Gram matrix
+ * with D on its diagonal, the dt-weighted x, and the carried state split in
+ * two bf16 parts) and float32 accumulators; the carried state itself is
+ * float32.  To fill the GPU when B * H is small the sequence is cut into
+ * `segments` runs of whole 128-token chunks (0: chosen for the current
+ * device, about one walk per SM; capped at one per chunk and 64): a first
+ * walk over pieces of every segment but the last gives their local end
+ * states from a zero state, and the full walk of each segment starts from
+ * the fold of those.  `workspace` (16-byte aligned; may be NULL when the size
+ * is 0) holds axon_ssd_workspace_bytes(B, L, H, P, N, segments) bytes for the
+ * same `segments` on the current device: an error flag (its first 4 bytes,
+ * an int), the per-chunk decays and weights, and the pieces' local states.
+ * The flag is cleared by each call and set to 1 if a wait of the walk for its
+ * tensor-core products gave up (the outputs are then undefined); it is
+ * written on the stream, so read it after the call completes.  Other
  * conventions as above.
  */
 AXON_API size_t axon_ssd_workspace_bytes(int B, int L, int H, int P, int N, int segments);

@@ -1,6 +1,6 @@
-"""GPU parity of the Mamba-2 (SSD) layer core (axon_ssd_scan_fwd: chunk Gram
-matrices, per-chunk decays, then chunk walks per (batch row, head, segment of
-the sequence) with the products on bf16 tensor-core MMAs) against the fp64
+"""GPU parity of the Mamba-2 (SSD) layer core (axon_ssd_scan_fwd: per-chunk
+decays, then chunk walks per (batch row, head, segment of the sequence) with
+the products on tcgen05 tensor-core MMAs into tensor memory) against the fp64
 oracle's ``ssd_scan`` on the same bf16 inputs, for one segment, forced
 segment counts and the automatic plan.
 
@@ -110,3 +110,18 @@ def test_ssd_full_size(cuda_lib):
         y_ref, h_ref = ref(inp, with_state)
         close(y, y_ref, f"mamba2 full-size y, h0 {with_state}")
         close(h, h_ref, f"mamba2 full-size state, h0 {with_state}")
+
+
+def test_ssd_wait_flag_stays_clear(cuda_lib):
+    """The workspace's first 4 bytes are the walk's error flag: every wait for
+    a tensor-core product completed, so it reads 0 after the call."""
+    from selective_state_space_52_b200 import axon_ssm
+    sw = W.SSD_WORKLOAD_BY_NAME["small_ssd"]
+    inp = W.make_ssd_inputs(sw, with_state=True, L=1000)
+    d = {k: v.cuda() for k, v in inp.items()}
+    params = {k: d[k] for k in ("dt_bias", "A_log", "D")}
+    nbytes = axon_ssm.axon_ssd_workspace_bytes(sw.B, 1000, sw.H, sw.P, sw.N, 3)
+    ws = torch.full((nbytes,), 0xA5, dtype=torch.uint8, device="cuda")   # a nonzero flag beforehand
+    axon_ssm.ssd_scan(d["x"], d["dt_raw"], d["B"], d["C"], params, d["h0"], workspace=ws, segments=3)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
