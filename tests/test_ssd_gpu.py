@@ -14,6 +14,8 @@ fraction of a percent of the output's rms scale: elementwise |got - ref| <=
 3e-2 * max(rms(ref), |ref|) and normwise ||got - ref|| / ||ref|| <= 1e-2, for
 y and for the final state.
 """
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -125,3 +127,27 @@ def test_ssd_wait_flag_stays_clear(cuda_lib):
     axon_ssm.ssd_scan(d["x"], d["dt_raw"], d["B"], d["C"], params, d["h0"], workspace=ws, segments=3)
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0
+
+
+def extreme_inputs(L=300):
+    """Three heads at the edges of the dt clip: head 0 at the lower bound with
+    A = -1 (a memory of ~10^4 tokens), head 1 at the upper bound with A = -16
+    (exp(-1600): every token forgets the past), head 2 as drawn; D ~ N(0, 1)."""
+    inp = W.make_ssd_inputs(W.SSD_WORKLOAD_BY_NAME["small_ssd"], with_state=True, L=L)
+    g = torch.Generator().manual_seed(23)
+    inp["dt_bias"] = torch.tensor([-30.0, 200.0, float(inp["dt_bias"][2])], dtype=torch.float32)
+    inp["A_log"] = torch.tensor([0.0, math.log(16.0), float(inp["A_log"][2])], dtype=torch.float32)
+    inp["D"] = torch.randn(3, generator=g, dtype=torch.float32)
+    return inp
+
+
+def test_ssd_extreme_decays_per_head(cuda_lib):
+    """Both dt clip bounds and a random D, with an initial state, over three
+    chunks (the last ragged) and the automatic segment plan; each head is held
+    to its own scale."""
+    inp = extreme_inputs()
+    y, h = run(inp, True)
+    y_ref, h_ref = ref(inp, True)
+    for hd in range(3):
+        close(y[:, :, hd], y_ref[:, :, hd], f"ssd y, extreme head {hd}")
+        close(h[:, hd], h_ref[:, hd], f"ssd state, extreme head {hd}")
