@@ -551,3 +551,34 @@ def test_ssd_upper_clip_forgets_at_once():
                                rtol=1e-10, atol=1e-10)
     np.testing.assert_allclose(hL, 100.0 * np.einsum("bhp,bn->bhpn", d["x"][:, -1], d["Bm"][:, -1]),
                                rtol=1e-10, atol=1e-10)
+
+
+def test_ssd_split_sequence_carries_state():
+    """Cutting the sequence anywhere and passing the final state on gives the
+    same outputs and final state as one pass (the recurrence is a scan)."""
+    rng = np.random.default_rng(83)
+    d = rand_ssd(rng, L=29)
+    full_y, full_h = oracle.ssd_scan(d["x"], d["dt_raw"], d["dt_bias"], d["A_log"], d["Bm"], d["Cm"], d["D"], d["h0"])
+    for cut in (1, 13, 28):
+        y1, h1 = oracle.ssd_scan(d["x"][:, :cut], d["dt_raw"][:, :cut], d["dt_bias"], d["A_log"], d["Bm"][:, :cut],
+                                 d["Cm"][:, :cut], d["D"], d["h0"])
+        y2, h2 = oracle.ssd_scan(d["x"][:, cut:], d["dt_raw"][:, cut:], d["dt_bias"], d["A_log"], d["Bm"][:, cut:],
+                                 d["Cm"][:, cut:], d["D"], h1)
+        np.testing.assert_allclose(np.concatenate([y1, y2], axis=1), full_y, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(h2, full_h, rtol=1e-12, atol=1e-12)
+
+
+def test_ssd_without_input_only_decays_the_state():
+    """B = 0: nothing enters the state, so h_t = exp(A S_t) h0 and
+    y_t = exp(A S_t) h0 C_t + D x_t, S_t = the running sum of dt."""
+    rng = np.random.default_rng(84)
+    d = rand_ssd(rng)
+    Bz = np.zeros_like(d["Bm"])
+    y, hL = oracle.ssd_scan(d["x"], d["dt_raw"], d["dt_bias"], d["A_log"], Bz, d["Cm"], d["D"], d["h0"])
+    dt = ref_dt(d["dt_raw"] + d["dt_bias"])
+    A = -np.exp(d["A_log"])
+    S = np.cumsum(dt, axis=1)                                         # (B,L,H)
+    dec = np.exp(A * S)                                               # (B,L,H)
+    y_ref = np.einsum("blh,bhpn,bln->blhp", dec, d["h0"], d["Cm"]) + d["D"][None, None, :, None] * d["x"]
+    np.testing.assert_allclose(y, y_ref, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(hL, dec[:, -1][:, :, None, None] * d["h0"], rtol=1e-11, atol=1e-11)
