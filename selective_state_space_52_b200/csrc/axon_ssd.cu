@@ -21,8 +21,8 @@ bool ovl(const void* a, size_t na, const void* b, size_t nb) {
 }
 size_t up256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Resident chunk walks per SM: one full walk (164 KB of shared memory, 256
-// tensor-memory columns), three state-only walks.
+// Resident chunk walks per SM: one full walk (217 KB of shared memory, 512
+// tensor-memory columns), three state-only walks (70 KB, 64 columns each).
 constexpr int kWalksPerSm = 1;
 constexpr int kStateWalksPerSm = 3;
 
