@@ -304,3 +304,51 @@ def test_ssd_rejects_bad_arguments(lib):
     assert q(2, 0, 3, 64, 128, 0) == 0
     assert q(1, 128, 1, 32, 128, 0) == 0
     assert q(1, 128, 1, 64, 128, -1) == 0
+
+
+def _ceil(a, b):
+    return -(-a // b)
+
+
+def _up256(n):
+    return _ceil(n, 256) * 256
+
+
+def ssd_plan_bytes(B, L, H, segments, sms=148):
+    """The SSD call's plan restated: 128-token chunks; segments so that the
+    full walks give one per SM (or as requested), at most one per chunk and 64;
+    the first walk's pieces so that it gives three per SM; the workspace is an
+    error flag, four floats per token and head, and per piece a local state and
+    its decay plus a copy of h0."""
+    nC = _ceil(L, 128)
+    if nC <= 1:
+        segs, cps = 1, max(nC, 1)
+    else:
+        want = segments if segments > 0 else max(1, sms // (B * H))
+        want = min(want, nC, 64)
+        cps = _ceil(nC, want)
+        segs = _ceil(nC, cps)
+    pcs = 1
+    if segs > 1:
+        pcs = min(max(1, 3 * sms // ((segs - 1) * B * H)), cps)
+    cpp = _ceil(cps, pcs)
+    pcs = _ceil(cps, cpp)
+    if nC == 0:
+        return 0, segs, pcs
+    total = 256 + _up256(B * H * nC * 4 * 128 * 4)
+    if segs > 1:
+        extra = (segs - 1) * pcs
+        total += _up256(extra * B * H * 64 * 128 * 4) + _up256(extra * B * H * 4) + _up256(B * H * 64 * 128 * 4)
+    return total, segs, pcs
+
+
+@pytest.mark.parametrize("B,L,H", [(1, 4096, 64), (2, 1000, 3), (1, 65536, 1), (8, 2048, 32), (1, 129, 2),
+                                   (4, 128, 8), (1, 300000, 2)])
+@pytest.mark.parametrize("segments", [0, 1, 2, 5, 100])
+def test_ssd_plan_and_workspace(lib, B, L, H, segments):
+    q = lib.axon_ssd_workspace_bytes
+    q.restype = ctypes.c_size_t
+    q.argtypes = [ctypes.c_int] * 6
+    want, segs, pcs = ssd_plan_bytes(B, L, H, segments)
+    assert q(B, L, H, 64, 128, segments) == want, (segs, pcs)
+    assert segs <= 64 and segs <= max(1, _ceil(L, 128))
