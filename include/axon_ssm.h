@@ -350,6 +350,15 @@ AXON_API axon_status axon_ssm_carry_fold(int P, int r, int B, int E, int N, cons
  */
 AXON_API size_t axon_ssd_workspace_bytes(int B, int L, int H, int P, int N, int segments);
 
+/*
+ * A check of the SSD walks' failure path, for tests: one warp polls, `limit`
+ * times (1 .. 65536), an mbarrier that nothing arrives on, exactly as a walk
+ * waits for its tensor-core products, and writes 1 to *status (a device int,
+ * 4-byte aligned) when the wait gave up.  AXON_ERR_INVALID_ARG for a NULL or
+ * misaligned status or a limit out of range.  Enqueued on `stream`.
+ */
+AXON_API axon_status axon_ssd_wait_probe(int *status, int limit, axon_stream_t stream);
+
 AXON_API axon_status axon_ssd_scan_fwd(
     int B, int L, int H, int P, int N, axon_dtype io,
     const void *x, const void *dt_raw, const float *dt_bias, const float *A_log,

@@ -66,6 +66,8 @@ _lib.axon_ssm_dt_sum.restype = _i
 _lib.axon_ssm_dt_sum.argtypes = [_i] * 4 + [_vp] * 3 + [_vp]
 _lib.axon_ssm_carry_fold.restype = _i
 _lib.axon_ssm_carry_fold.argtypes = [_i] * 5 + [_vp] * 4 + [_vp]
+_lib.axon_ssd_wait_probe.restype = _i
+_lib.axon_ssd_wait_probe.argtypes = [_vp, _i, _vp]
 _lib.axon_ssd_workspace_bytes.restype = _sz
 _lib.axon_ssd_workspace_bytes.argtypes = [_i] * 6
 _lib.axon_ssd_scan_fwd.restype = _i
@@ -229,6 +231,13 @@ def axon_ssm_carry_fold(P, r, B, E, N, A_log, h_loc, dt_sum, h_in, stream=None, 
                                   _stream(stream))
     if raise_on_error:
         _check(rc, "axon_ssm_carry_fold")
+    return rc
+
+
+def axon_ssd_wait_probe(status, limit, stream=None, *, raise_on_error=True) -> int:
+    rc = _lib.axon_ssd_wait_probe(_p(status), int(limit), _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_ssd_wait_probe")
     return rc
 
 

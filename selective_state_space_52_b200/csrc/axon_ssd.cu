@@ -108,6 +108,13 @@ using namespace axon;
 
 extern "C" {
 
+axon_status axon_ssd_wait_probe(int* status, int limit, axon_stream_t stream) {
+    if (!status || (reinterpret_cast<uintptr_t>(status) & 3u) || limit < 1 || limit > (1 << 16))
+        return AXON_ERR_INVALID_ARG;
+    ssd_wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status, limit);
+    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+}
+
 size_t axon_ssd_workspace_bytes(int B, int L, int H, int P, int N, int segments) {
     if (B < 0 || L < 0 || H < 0 || segments < 0 || P != kSsdP || N != kSsdN) return 0;
     int segs = 1, cps = 1, pcs = 1, cpp = 1;

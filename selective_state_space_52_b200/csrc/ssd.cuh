@@ -113,9 +113,9 @@ __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.a
 __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
 }
-// Polls the mbarrier's phase `parity` at most kSsdWaitLimit times; false when it gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
-    for (int it = 0; it < kSsdWaitLimit; ++it) {
+// Polls the mbarrier's phase `parity` at most `limit` times; false when it gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, int limit = kSsdWaitLimit) {
+    for (int it = 0; it < limit; ++it) {
         uint32_t done;
         asm volatile("{\n\t.reg .pred P1;\n\tmbarrier.try_wait.parity.shared::cta.b64 P1, [%1], %2;\n\t"
                      "selp.b32 %0, 1, 0, P1;\n\t}\n"
@@ -143,6 +143,19 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
                    "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]));
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// The walks' failure path in isolation: one warp polls, `limit` times, an
+// mbarrier that nothing arrives on, as a walk does when a product never
+// completes, and thread 0 writes 1 to *status when the wait gave up (0 if it
+// completed, which cannot happen here).  grid = 1, 32 threads.
+__global__ void __launch_bounds__(32) ssd_wait_probe_kernel(int* status, int limit) {
+    __shared__ __align__(8) unsigned long long bar;
+    const uint32_t mbar = static_cast<uint32_t>(__cvta_generic_to_shared(&bar));
+    if (threadIdx.x == 0) mbar_init(mbar, 1);
+    __syncwarp();
+    const bool done = mbar_wait(mbar, 0u, limit);
+    if (threadIdx.x == 0) *status = done ? 0 : 1;
+}
 
 // Byte offset of the 16-byte piece `pc` (8 bf16) of row r in a tile of 128
 // rows stored as 64-column blocks of 128-byte rows, 128-byte swizzle (the

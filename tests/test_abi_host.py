@@ -352,3 +352,13 @@ def test_ssd_plan_and_workspace(lib, B, L, H, segments):
     want, segs, pcs = ssd_plan_bytes(B, L, H, segments)
     assert q(B, L, H, 64, 128, segments) == want, (segs, pcs)
     assert segs <= 64 and segs <= max(1, _ceil(L, 128))
+
+
+def test_ssd_wait_probe_rejects_bad_arguments(lib):
+    f = lib.axon_ssd_wait_probe
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    assert f(None, 64, None) == INVALID
+    assert f(FAKE + 2, 64, None) == INVALID                     # not 4-byte aligned
+    assert f(FAKE, 0, None) == INVALID
+    assert f(FAKE, (1 << 16) + 1, None) == INVALID

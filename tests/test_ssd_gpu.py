@@ -151,3 +151,16 @@ def test_ssd_extreme_decays_per_head(cuda_lib):
     for hd in range(3):
         close(y[:, :, hd], y_ref[:, :, hd], f"ssd y, extreme head {hd}")
         close(h[:, hd], h_ref[:, hd], f"ssd state, extreme head {hd}")
+
+
+def test_ssd_wait_gives_up_and_reports(cuda_lib):
+    """The walks' failure path: a wait on an mbarrier that nothing arrives on
+    gives up after its bounded polls and reports it in the status word, and
+    the device stays usable."""
+    from selective_state_space_52_b200 import axon_ssm
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    axon_ssm.axon_ssd_wait_probe(status, 64)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 1
+    # the device still runs the SSD core afterwards
+    test_ssd_small(cuda_lib, 130, True)
