@@ -12,7 +12,7 @@
 //   S_out^T  = exp(acum_{Q-1}) S_in^T + B^T (w x),    w_j = exp(acum_{Q-1} - acum_j) dt_j
 //
 // Launches: ssd_chunk_prep_kernel (per chunk and head: acum, log2(dt_j) -
-// acum_j and w_j), then the chunk walk.  To fill the GPU when B * H is small,
+// acum_j, w_j, and the in-block decay factors v_j), then the chunk walks.  To fill the GPU when B * H is small,
 // the sequence is cut into segments of whole chunks and the carried state
 // crosses them as in the chunked associative scan of the SSD article: a first
 // walk over pieces of every segment but the last, from a zero state (state
@@ -27,12 +27,16 @@
 // (the B rows are the K-major B operand of C B^T and the MN-major A operand of
 // B^T (w x); the x rows are the MN-major B operand of M x), except M, which
 // each thread writes as its row into tensor memory, the A operand of M x.
-// Thread i of the 128 owns tensor-memory lane i: row i of G, M, y and of the
-// transposed state.  The full walk double-buffers its input rows: chunk c+1's
-// copies are in flight while chunk c computes.
-// The carried state stays float32 in registers (thread n: S[:, n]) and enters
-// C S^T as two bf16 parts (hi + lo, about 16 significant bits), because that
-// product can cancel heavily for long-memory heads.
+// Tensor-memory lane i holds row i of G, M, y and of the transposed state; the
+// full walk gives each lane two threads, each taking half of the row's head
+// columns and of M's column blocks.  M's entries below the diagonal 32-token
+// blocks come from the factorised decay (one exponential per row and block);
+// only the diagonal block takes one per entry.  The full walk double-buffers
+// its input rows: chunk c+1's copies are in flight while chunk c computes.
+// The carried state stays float32 in registers (row n of S^T with the threads
+// of lane n) and enters C S^T as two bf16 parts (hi + lo, about 16
+// significant bits), because that product can cancel heavily for long-memory
+// heads.
 #pragma once
 
 #include <cuda_bf16.h>
