@@ -38,6 +38,11 @@ MUTANTS = {
     "ssd_input_without_dt": ("*s = a * *s + dt * xv[p] * Bt[n];", "*s = a * *s + xv[p] * Bt[n];"),
     "ssd_decay_sign": ("const double A = -exp(A_log[h]);", "const double A = exp(A_log[h]);"),
     "ssd_C_replaced_by_B": ("acc += *s * Ct[n];", "acc += *s * Bt[n];"),
+    "ssd_dropped_D": ("yv[p] = acc + D[h] * xv[p];", "yv[p] = acc;"),
+    "ssd_h0_ignored": ("S[i] = h0 ? h0[((size_t)b * H + h) * P * N + i] : 0.0;", "S[i] = 0.0;"),
+    "ssd_input_before_decay": ("*s = a * *s + dt * xv[p] * Bt[n];", "*s = a * (*s + dt * xv[p] * Bt[n]);"),
+    "ssd_output_before_update": ("*s = a * *s + dt * xv[p] * Bt[n];\n                        acc += *s * Ct[n];",
+                                 "acc += *s * Ct[n];\n                        *s = a * *s + dt * xv[p] * Bt[n];"),
     "zoh_missing_A_division": ("double bbar = zoh ? expm1(dt * A[n]) / A[n] * Bm[bn] : dt * Bm[bn];",
                                "double bbar = zoh ? expm1(dt * A[n]) * Bm[bn] : dt * Bm[bn];"),
 }
