@@ -6,10 +6,12 @@
 
 One step = one pass of the whole hot path over one batch of synthetic input:
 the prefill (conv1d + SiLU + dt + selective recurrence + C/D epilogue + SiLU(z)
-gate, returning the (conv_cache, ssm_state) pair) of the Bit-Axon layer shape
-(B1 L2048 E7680 N16 K4, bf16 io, fp32 state), followed by one cached decode step
-on the returned caches.  Throughput is counted in token x channel units:
-B*(L+1)*E per step.
+gate, returning the (conv_cache, ssm_state) pair) of the long-sequence workload
+(B1 L65536 E2048 N16 K4, bf16 io, fp32 state: the largest of the five measured
+workloads that fits one GPU), followed by one cached decode step on the
+returned caches.  Throughput is counted in token x channel units: B*(L+1)*E
+per step.  The other workloads' prefills are measured beside it (key
+``workloads``), each with its own roofline fraction.
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own independent
 sequences (different seeds); the path has no data exchange, so there is no
@@ -175,7 +177,7 @@ class ClockSampler:
                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
                0x2: "applications_clocks_setting", 0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.period = period_s
         self.samples = []
         self.reasons = set()
@@ -234,26 +236,44 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------- CPU oracle
-def time_oracle(wl, inp, budget_s: float, block: int = 256):
+def time_oracle(wl, inp, budget_s: float, block: int = 256, parallel: bool = False):
     """Time the fp64 oracle on the first channels of the workload until the
-    budget is spent; returns (token_ch/s, token_ch done, seconds, channels)."""
+    budget is spent; returns (token_ch/s, token_ch done, seconds, channels,
+    threads).  ``parallel`` runs the OpenMP build of the same source on all
+    host cores (blocks of ``block`` channels per thread)."""
     import oracle
-    oracle.build()
+    threads = oracle.threads(parallel)
+    blk = block * threads
     done_ch, t_total = 0, 0.0
     E = wl.E
     while done_ch < E and t_total < budget_s:
-        e0, e1 = done_ch, min(E, done_ch + block)
+        e0, e1 = done_ch, min(E, done_ch + blk)
         sl = slice(e0, e1)
         args = [inp["x"][:, :, sl].contiguous(), inp["z"][:, :, sl].contiguous(),
                 inp["dt_raw"][:, :, sl].contiguous(), inp["B"], inp["C"],
                 inp["conv_w"][sl], inp["conv_b"][sl], inp["dt_bias"][sl], inp["A_log"][sl],
                 inp["D"][sl]]
         t0 = time.perf_counter()
-        oracle.scan_fwd(*args)
+        oracle.scan_fwd(*args, parallel=parallel)
         t_total += time.perf_counter() - t0
         done_ch = e1
     units = done_ch * wl.B * wl.L
-    return units / t_total, units, t_total, done_ch
+    return units / t_total, units, t_total, done_ch, threads
+
+
+def cpu_baselines(wl, inp, budget_s: float) -> dict:
+    """The oracle on one host core and (its OpenMP build) on all of them."""
+    import oracle
+    oracle.build()
+    oracle.build(openmp=True)
+    rate1, _, secs1, ch1, _ = time_oracle(wl, inp, budget_s, block=64)
+    rate, _, secs, ch, thr = time_oracle(wl, inp, budget_s, block=16, parallel=True)
+    return {"value": rate / 1e9, "unit": UNIT, "cores": thr, "kind": "oracle",
+            "sample": f"{ch} of {wl.E} channels x {wl.L} tokens (prefill), {secs:.1f} s, fp64 C oracle, "
+                      f"OpenMP build over channels on {thr} host threads",
+            "single_core": {"value": rate1 / 1e9, "unit": UNIT, "cores": 1,
+                            "sample": f"{ch1} of {wl.E} channels x {wl.L} tokens (prefill), {secs1:.1f} s, "
+                                      "fp64 C oracle, single thread"}}
 
 
 def run_reference(args, wl):
@@ -261,11 +281,14 @@ def run_reference(args, wl):
     if rank != 0:
         return 0
     inp = W.make_inputs(wl)
+    import oracle
+    oracle.build(openmp=True)
     per_step_budget = max(0.5, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
     channels = None
+    threads = 1
     rates = []
     for i in range(args.warmup + args.steps):
-        rate, units, secs, ch = time_oracle(wl, inp, per_step_budget, block=64)
+        rate, units, secs, ch, threads = time_oracle(wl, inp, per_step_budget, block=16, parallel=True)
         channels = ch
         if i >= args.warmup:
             rates.append((units, secs))
@@ -278,9 +301,9 @@ def run_reference(args, wl):
         "ms_per_step": 1000.0 * secs / max(1, args.steps), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_desc(wl), "sample": f"first {channels} channels x {wl.L} tokens per step"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"{channels} of {wl.E} channels x {wl.L} tokens per step, "
-                                   "fp64 C oracle, single thread"},
+                                   f"fp64 C oracle, OpenMP build over channels on {threads} host threads"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -471,7 +494,8 @@ def bench_ssd(dev, launches: int = 20) -> dict:
     stream = torch.cuda.current_stream(dev)
 
     def call():
-        axon_ssm.ssd_scan(inp["x"], inp["dt_raw"], inp["B"], inp["C"], params, None, out=(y, h), workspace=ws)
+        axon_ssm.ssd_scan(inp["x"], inp["dt_raw"], inp["B"], inp["C"], params, None, out=(y, h), workspace=ws,
+                          check=False)
 
     for _ in range(3):
         call()
@@ -484,6 +508,8 @@ def bench_ssd(dev, launches: int = 20) -> dict:
         a.record(stream); call(); b.record(stream)
         torch.cuda.synchronize(dev)
         times.append(a.elapsed_time(b))
+        if axon_ssm.ssd_error_flag(ws) != 0:
+            raise RuntimeError("axon_ssd_scan_fwd: a wait for a tensor-core product gave up")
     ms = statistics.median(times)
     Q, P, N, H, L, B = 128, sw.P, sw.N, sw.H, sw.L, sw.B     # Q: tokens per chunk of the kernels
     nC = (L + Q - 1) // Q
@@ -503,6 +529,50 @@ def bench_ssd(dev, launches: int = 20) -> dict:
                                "carried-state product runs twice (hi and lo parts) and C B^T once per head, "
                                "both counted once"},
             "token_head_per_s": B * L * H / (ms / 1e3)}
+
+
+def bench_prefill_workload(wl, dev, launches: int = 20) -> dict:
+    """One workload's prefill alone (the library's own plan, inputs resident):
+    CUDA-event mean over `launches` calls with the L2 flushed (a buffer of
+    twice its size written) before each, and its MUFU and HBM rooflines."""
+    from selective_state_space_52_b200 import axon_ssm
+    inp = {k: v.to(dev) for k, v in W.make_inputs(wl).items()}
+    params = {k: inp[k] for k in axon_ssm.PARAM_KEYS}
+    io_code = axon_ssm.AXON_BF16 if wl.io == "bf16" else axon_ssm.AXON_F32
+    y = torch.empty(wl.B, wl.L, wl.E, dtype=wl.torch_io, device=dev)
+    cc = torch.empty(wl.B, wl.K - 1, wl.E, dtype=wl.torch_io, device=dev)
+    ss = torch.empty(wl.B, wl.E, wl.N, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(axon_ssm.axon_ssm_scan_workspace_bytes(wl.B, wl.L, wl.E, wl.N, wl.K, io_code), 16),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call():
+        axon_ssm.scan_fwd(inp["x"], inp["z"], inp["dt_raw"], inp["B"], inp["C"], params, None,
+                          out=(y, cc, ss), workspace=ws)
+
+    for _ in range(3):
+        call()
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    times = []
+    for _ in range(launches):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream); call(); b.record(stream)
+        torch.cuda.synchronize(dev)
+        times.append(a.elapsed_time(b))
+    ms = statistics.mean(times)
+    peaks = measured_peaks()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mufu_peak = sms * MUFU_LANES_PER_SM_CLK * peaks["sm_max_mhz"] * 1e6 / 1e9
+    m = scan_model(wl)
+    mufu = m["mufu"] / (ms / 1e3) / 1e9
+    hbm = m["bytes"] / (ms / 1e3) / 1e9
+    return {"shape": f"B{wl.B} L{wl.L} E{wl.E} {wl.io}", "prefill_us": ms * 1e3,
+            "value": m["token_ch"] / (ms / 1e3) / 1e9, "unit": UNIT,
+            "mufu_frac": mufu / mufu_peak, "hbm_gbs": hbm, "hbm_frac": hbm / peaks["hbm_gbs"],
+            "launches": axon_ssm.axon_ssm_scan_launch_count(wl.B, wl.L, wl.E, wl.N, wl.K, io_code),
+            "note": "L2 flushed before every call; mufu_frac = 22 transcendentals per token x channel "
+                    "over the MUFU peak"}
 
 
 def workload_desc(wl) -> str:
@@ -682,6 +752,9 @@ def run_axon(args, wl):
         "gpu_launches": args.steps * (scan_launches + 1),
     }
 
+    if not args.no_workloads and world == 1:
+        line["workloads"] = {w.name: bench_prefill_workload(w, dev) for w in W.WORKLOADS
+                             if w.name not in ("tiny_f32", wl.name)}
     if not args.no_decode_bench:
         line["decode"] = bench_decode(dev)
         line["prefill_zoh"] = bench_zoh_prefill(wl, sets, params, (y, cc, ss), ws, dev)
@@ -691,10 +764,7 @@ def run_axon(args, wl):
         line["ssd"] = bench_ssd(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inp_cpu = {**params_cpu, **{k: v.cpu() for k, v in sets[0].items()}}
-        rate, units, secs, ch = time_oracle(wl, inp_cpu, args.cpu_budget)
-        line["cpu_baseline"] = {"value": rate / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                "sample": f"{ch} of {E} channels x {L} tokens (prefill), "
-                                          f"{secs:.1f} s, fp64 C oracle, single thread"}
+        line["cpu_baseline"] = cpu_baselines(wl, inp_cpu, args.cpu_budget)
     if rank == 0:
         print(json.dumps(line), flush=True)
     barrier(dev)
@@ -709,11 +779,13 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["axon", "reference"], default="axon")
-    ap.add_argument("--workload", default="bit_axon_layer", choices=[w.name for w in W.WORKLOADS])
+    ap.add_argument("--workload", default="long_seq", choices=[w.name for w in W.WORKLOADS])
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-bench", action="store_true",
                     help="skip the separate cached-decode measurement (decode workload shapes)")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the prefills of the other measured workloads")
     ap.add_argument("--no-block-bench", action="store_true",
                     help="skip the whole-layer measurement (input/output projections around the scan)")
     ap.add_argument("--decode-only", action="store_true",

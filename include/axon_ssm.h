@@ -322,8 +322,8 @@ AXON_API axon_status axon_ssm_carry_fold(int P, int r, int B, int E, int N, cons
  * The Mamba-2 (SSD) layer core: one scalar decay per head (wiki page
  * "Selective State Space Models (Mamba)", section "Mamba-2 block (SSD)":
  * d_state 128, headdim 64), computed as a chunked scan on the tensor cores
- * (the SSD article: masked matrix products inside 64-token chunks, a carried
- * state between them).  Per batch row b and head h, state S (P x N):
+ * (the SSD article: masked matrix products inside chunks of tokens, a carried
+ * state between them; this library's chunks are 128 tokens).  Per batch row b and head h, state S (P x N):
  *   dt = clip(softplus(dt_raw[b,t,h] + dt_bias[h]), 1e-4, 100),
  *   S  = exp(dt * A_h) S + dt * x[b,t,h,:] B[b,t,:]^T,  A_h = -exp(A_log[h]),
  *   y[b,t,h,:] = S C[b,t,:] + D[h] x[b,t,h,:].
@@ -345,7 +345,12 @@ AXON_API axon_status axon_ssm_carry_fold(int P, int r, int B, int E, int N, cons
  * an int), the per-chunk decays and weights, and the pieces' local states.
  * The flag is cleared by each call and set to 1 if a wait of the walk for its
  * tensor-core products gave up (the outputs are then undefined); it is
- * written on the stream, so read it after the call completes.  Other
+ * written on the stream, so read it after the call completes (the Python
+ * binding's ssd_scan reads it and raises).  A walk that gave up first waits,
+ * with the same bound, for every product it issued to finish, and only then
+ * frees its tensor memory; if that wait gives up as well, it leaves the
+ * tensor memory allocated rather than risk a late product writing into
+ * columns another block has since allocated.  Other
  * conventions as above.
  */
 AXON_API size_t axon_ssd_workspace_bytes(int B, int L, int H, int P, int N, int segments);

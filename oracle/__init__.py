@@ -5,7 +5,9 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 its Python binding) never does, and this package never imports the product.
 
 The arithmetic lives in ``axon_ssm_oracle.c`` (plain C, double precision, one
-thread).  This module compiles it with gcc on first use and exposes numpy
+thread; a second build of the same file with -fopenmp spreads independent
+channels over the host's cores for the full-size checks, with identical
+bits).  This module compiles it with gcc on first use and exposes numpy
 wrappers.  Every function cites the passage of the page "Axon-SSM: Selective
 State Space Model for Apple Silicon" (or the wiki page "Selective State Space
 Models (Mamba)") that it follows; see the C source for the step list.
@@ -30,33 +32,41 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "axon_ssm_oracle.c")
 _BUILD_DIR = os.path.join(_HERE, "_build")
 _LIB_PATH = os.path.join(_BUILD_DIR, "liboracle_axon_ssm.so")
+_LIB_OMP_PATH = os.path.join(_BUILD_DIR, "liboracle_axon_ssm_omp.so")
 _lock = threading.Lock()
-_lib = None
+_libs = {}
 
 _dp = ctypes.POINTER(ctypes.c_double)
 
 
-def build(force: bool = False) -> str:
-    """Compile the C oracle into a shared library with gcc (no -ffast-math)."""
+def build(force: bool = False, openmp: bool = False) -> str:
+    """Compile the C oracle into a shared library with gcc (no -ffast-math).
+
+    ``openmp=True`` builds the same source a second time with -fopenmp: its
+    channel loop then runs on all host cores (OMP_NUM_THREADS caps them), with
+    each channel's arithmetic unchanged, so both builds give identical bits.
+    """
     os.makedirs(_BUILD_DIR, exist_ok=True)
-    stale = (not os.path.exists(_LIB_PATH)
-             or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    path = _LIB_OMP_PATH if openmp else _LIB_PATH
+    stale = (not os.path.exists(path)
+             or os.path.getmtime(path) < os.path.getmtime(_SRC))
     if force or stale:
-        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        tmp = path + f".tmp{os.getpid()}"
         cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fno-fast-math",
-               "-ffp-contract=off", "-o", tmp, _SRC, "-lm"]
+               "-ffp-contract=off", *(["-fopenmp"] if openmp else []), "-o", tmp, _SRC, "-lm"]
         subprocess.run(cmd, check=True)
-        os.replace(tmp, _LIB_PATH)
-    return _LIB_PATH
+        os.replace(tmp, path)
+    return path
 
 
-def _load():
-    global _lib
+def _load(openmp: bool = False):
     with _lock:
-        if _lib is None:
+        lib = _libs.get(openmp)
+        if lib is None:
             # AXON_ORACLE_LIB points the pins at another build of this source
             # (the mutation tests plant mistakes in copies of it).
-            path = os.environ.get("AXON_ORACLE_LIB") or build()
+            env = os.environ.get("AXON_ORACLE_LIB_OMP" if openmp else "AXON_ORACLE_LIB")
+            path = env or build(openmp=openmp)
             lib = ctypes.CDLL(path)
             lib.oracle_silu.restype = ctypes.c_double
             lib.oracle_silu.argtypes = [ctypes.c_double]
@@ -74,8 +84,15 @@ def _load():
             lib.oracle_conv_silu.argtypes = [ctypes.c_int] * 4 + [_dp] * 5
             lib.oracle_ssd_scan.restype = ctypes.c_int
             lib.oracle_ssd_scan.argtypes = [ctypes.c_int] * 5 + [_dp] * 10
-            _lib = lib
-    return _lib
+            lib.oracle_threads.restype = ctypes.c_int
+            lib.oracle_threads.argtypes = []
+            _libs[openmp] = lib
+    return lib
+
+
+def threads(parallel: bool = False) -> int:
+    """Host threads the prefill's channel loop uses in the chosen build."""
+    return int(_load(parallel).oracle_threads())
 
 
 def _f64(a) -> np.ndarray:
@@ -120,12 +137,13 @@ def scan_core(u, dt, A, Bm, Cm, D=0.0, h0=None, zoh=False):
 
 
 def scan_fwd(x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
-             conv_cache=None, ssm_state=None, zoh=False):
+             conv_cache=None, ssm_state=None, zoh=False, parallel=False):
     """Layer core over a sequence (prefill), fp64.
 
     x, z, dt_raw: (B,L,E); Bm, Cm: (B,L,N); conv_w (E,K); conv_b, dt_bias, D (E,);
     A_log (E,N); conv_cache (B,K-1,E) or None; ssm_state (B,E,N) or None.
     Returns (y (B,L,E), conv_cache_out (B,K-1,E), ssm_state_out (B,E,N)).
+    ``parallel`` runs the OpenMP build of the same source (identical bits).
     """
     x, z, dt_raw, Bm, Cm = (_f64(v) for v in (x, z, dt_raw, Bm, Cm))
     conv_w, conv_b, dt_bias, A_log, D = (_f64(v) for v in (conv_w, conv_b, dt_bias, A_log, D))
@@ -138,7 +156,7 @@ def scan_fwd(x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
     y = np.zeros((Bsz, L, E))
     cc_out = np.zeros((Bsz, K - 1, E))
     ss_out = np.zeros((Bsz, E, N))
-    rc = _load().oracle_ssm_scan_fwd(Bsz, L, E, N, K, _ptr(x), _ptr(z), _ptr(dt_raw),
+    rc = _load(parallel).oracle_ssm_scan_fwd(Bsz, L, E, N, K, _ptr(x), _ptr(z), _ptr(dt_raw),
                                      _ptr(Bm), _ptr(Cm), _ptr(conv_w), _ptr(conv_b),
                                      _ptr(dt_bias), _ptr(A_log), _ptr(D), _ptr(cc), _ptr(ss),
                                      _ptr(y), _ptr(cc_out), _ptr(ss_out), int(bool(zoh)))

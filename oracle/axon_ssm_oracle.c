@@ -2,7 +2,8 @@
  * axon_ssm_oracle.c -- TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT PATH.
  *
  * A plain, slow, single-threaded fp64 CPU statement of the selective-scan (S6)
- * layer core described on the page "Axon-SSM: Selective State Space Model for
+ * layer core (a second build of this file with -fopenmp runs independent
+ * channels on several host cores, with each channel's arithmetic unchanged) described on the page "Axon-SSM: Selective State Space Model for
  * Apple Silicon" (bit-axon docs).  Only the test suite, the smoke check and the
  * CPU-baseline leg of the benchmark may load it.  It shares no code, header,
  * table or helper with the CUDA library; neither includes the other.
@@ -34,6 +35,9 @@
 #include <stddef.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORACLE_DT_MIN 1e-4   /* epsilon of the dt clip ("Selective mechanism") */
 #define ORACLE_DT_MAX 100.0  /* dt_max of the dt clip */
@@ -83,8 +87,62 @@ void oracle_scan_core(int L, int N, const double *u, const double *dt,
 }
 
 /*
+ * Steps 1-3 above for one (b, e) channel.  Scratch: xpad holds L + K - 1
+ * values, h and A hold N.  Channels share nothing, so the caller may run them
+ * in any order (or at the same time) on the same arrays.
+ */
+static void oracle_channel(int b, int e, int L, int E, int N, int K,
+                           const double *x, const double *z, const double *dt_raw,
+                           const double *Bm, const double *Cm,
+                           const double *conv_w, const double *conv_b,
+                           const double *dt_bias, const double *A_log, const double *D,
+                           const double *conv_cache_in, const double *ssm_state_in,
+                           double *y, double *conv_cache_out, double *ssm_state_out,
+                           int zoh, double *xpad, double *h, double *A)
+{
+    const int KM1 = K - 1;
+    /* 1. padded input stream for this channel */
+    for (int j = 0; j < KM1; ++j)
+        xpad[j] = conv_cache_in ? conv_cache_in[((size_t)b * KM1 + j) * E + e] : 0.0;
+    for (int t = 0; t < L; ++t)
+        xpad[KM1 + t] = x[((size_t)b * L + t) * E + e];
+    for (int n = 0; n < N; ++n) {
+        h[n] = ssm_state_in ? ssm_state_in[((size_t)b * E + e) * N + n] : 0.0;
+        A[n] = -exp(A_log[(size_t)e * N + n]);
+    }
+    /* 2. the per-step update */
+    for (int t = 0; t < L; ++t) {
+        size_t idx = ((size_t)b * L + t) * E + e;
+        double xc = conv_b[e];
+        for (int k = 0; k < K; ++k) xc += conv_w[(size_t)e * K + k] * xpad[t + k];
+        double u = oracle_silu(xc);
+        double dt = oracle_dt(dt_raw[idx] + dt_bias[e]);
+        double acc = 0.0;
+        for (int n = 0; n < N; ++n) {
+            size_t bn = ((size_t)b * L + t) * N + n;
+            double abar = exp(dt * A[n]);
+            double bbar = zoh ? expm1(dt * A[n]) / A[n] * Bm[bn] : dt * Bm[bn];
+            h[n] = abar * h[n] + bbar * u;
+            acc += Cm[bn] * h[n];
+        }
+        double y_ssm = acc + D[e] * u;
+        y[idx] = y_ssm * oracle_silu(z[idx]);
+    }
+    /* 3. final caches (written after all reads, so in == out is fine) */
+    for (int j = 0; j < KM1; ++j)
+        conv_cache_out[((size_t)b * KM1 + j) * E + e] = xpad[L + j];
+    for (int n = 0; n < N; ++n)
+        ssm_state_out[((size_t)b * E + e) * N + n] = h[n];
+}
+
+/*
  * The layer core over a whole sequence (prefill).  Returns 0 on success,
  * -1 on bad sizes or a failed temporary allocation.
+ *
+ * The default build is one plain loop over the channels.  A second build of
+ * this same file with -fopenmp hands the channels to the host's cores (the
+ * pragma below is ignored otherwise); each channel's arithmetic is the same
+ * either way, so both builds give identical bits.
  */
 int oracle_ssm_scan_fwd(int B, int L, int E, int N, int K,
                         const double *x, const double *z, const double *dt_raw,
@@ -96,50 +154,33 @@ int oracle_ssm_scan_fwd(int B, int L, int E, int N, int K,
                         int zoh)
 {
     if (B < 0 || L < 0 || E < 0 || N <= 0 || K <= 0) return -1;
-    const int KM1 = K - 1;
-    double *xpad = (double *)malloc(sizeof(double) * ((size_t)L + KM1));
-    double *h = (double *)malloc(sizeof(double) * (size_t)N);
-    double *A = (double *)malloc(sizeof(double) * (size_t)N);
-    if (!xpad || !h || !A) { free(xpad); free(h); free(A); return -1; }
-
+    int failed = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic, 4) reduction(| : failed)
     for (int b = 0; b < B; ++b) {
         for (int e = 0; e < E; ++e) {
-            /* 1. padded input stream for this channel */
-            for (int j = 0; j < KM1; ++j)
-                xpad[j] = conv_cache_in ? conv_cache_in[((size_t)b * KM1 + j) * E + e] : 0.0;
-            for (int t = 0; t < L; ++t)
-                xpad[KM1 + t] = x[((size_t)b * L + t) * E + e];
-            for (int n = 0; n < N; ++n) {
-                h[n] = ssm_state_in ? ssm_state_in[((size_t)b * E + e) * N + n] : 0.0;
-                A[n] = -exp(A_log[(size_t)e * N + n]);
-            }
-            /* 2. the per-step update */
-            for (int t = 0; t < L; ++t) {
-                size_t idx = ((size_t)b * L + t) * E + e;
-                double xc = conv_b[e];
-                for (int k = 0; k < K; ++k) xc += conv_w[(size_t)e * K + k] * xpad[t + k];
-                double u = oracle_silu(xc);
-                double dt = oracle_dt(dt_raw[idx] + dt_bias[e]);
-                double acc = 0.0;
-                for (int n = 0; n < N; ++n) {
-                    size_t bn = ((size_t)b * L + t) * N + n;
-                    double abar = exp(dt * A[n]);
-                    double bbar = zoh ? expm1(dt * A[n]) / A[n] * Bm[bn] : dt * Bm[bn];
-                    h[n] = abar * h[n] + bbar * u;
-                    acc += Cm[bn] * h[n];
-                }
-                double y_ssm = acc + D[e] * u;
-                y[idx] = y_ssm * oracle_silu(z[idx]);
-            }
-            /* 3. final caches (written after all reads, so in == out is fine) */
-            for (int j = 0; j < KM1; ++j)
-                conv_cache_out[((size_t)b * KM1 + j) * E + e] = xpad[L + j];
-            for (int n = 0; n < N; ++n)
-                ssm_state_out[((size_t)b * E + e) * N + n] = h[n];
+            double *xpad = (double *)malloc(sizeof(double) * ((size_t)L + K - 1));
+            double *h = (double *)malloc(sizeof(double) * (size_t)N);
+            double *A = (double *)malloc(sizeof(double) * (size_t)N);
+            if (xpad && h && A)
+                oracle_channel(b, e, L, E, N, K, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias,
+                               A_log, D, conv_cache_in, ssm_state_in, y, conv_cache_out,
+                               ssm_state_out, zoh, xpad, h, A);
+            else
+                failed = 1;
+            free(xpad); free(h); free(A);
         }
     }
-    free(xpad); free(h); free(A);
-    return 0;
+    return failed ? -1 : 0;
+}
+
+/* Host threads the channel loop uses: 1 in the default build. */
+int oracle_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }
 
 /*

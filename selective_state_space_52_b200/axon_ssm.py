@@ -383,10 +383,25 @@ def carry_fold(r, A_log, h_loc_all, dt_sum_all, *, stream=None):
     return out
 
 
-def ssd_scan(x, dt_raw, Bm, Cm, params: dict, h0=None, *, out=None, workspace=None, stream=None, segments=0):
+def ssd_error_flag(workspace) -> int:
+    """The SSD walk's error flag (the workspace's first int) after the call
+    that used ``workspace`` has completed: 1 if a wait for a tensor-core
+    product gave up.  Synchronises the device."""
+    torch.cuda.synchronize(workspace.device)
+    return int(workspace[:4].view(torch.int32).item())
+
+
+def ssd_scan(x, dt_raw, Bm, Cm, params: dict, h0=None, *, out=None, workspace=None, stream=None, segments=0,
+             check=True):
     """The Mamba-2 (SSD) layer core on x (B,L,H,P) bf16; ``params`` holds
     dt_bias, A_log, D (H,) float32; ``segments`` = 0 lets the library cut the
-    sequence for the current device.  Returns (y, h_out (B,H,P,N))."""
+    sequence for the current device.  Returns (y, h_out (B,H,P,N)).
+
+    With ``check`` (the default) the call waits for the device and reads the
+    walk's error flag from the workspace, raising ``AxonError``
+    (AXON_ERR_TIMEOUT) if a wait for a tensor-core product gave up, in which
+    case y and h_out are undefined.  ``check=False`` returns without waiting;
+    the caller then reads the flag with ``ssd_error_flag(workspace)``."""
     Bsz, L, H, P = x.shape
     N = Bm.shape[2]
     if out is None:
@@ -401,4 +416,6 @@ def ssd_scan(x, dt_raw, Bm, Cm, params: dict, h0=None, *, out=None, workspace=No
     axon_ssd_scan_fwd(Bsz, L, H, P, N, _dtype_code(x.dtype), x, dt_raw, params["dt_bias"], params["A_log"],
                       Bm, Cm, params["D"], h0, y, h_out, segments, workspace,
                       workspace.numel() * workspace.element_size(), stream=stream)
+    if check and L > 0 and Bsz * H > 0 and ssd_error_flag(workspace) != 0:
+        raise AxonError(6, "axon_ssd_scan_fwd (a wait for a tensor-core product gave up)")
     return y, h_out

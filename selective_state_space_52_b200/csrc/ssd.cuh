@@ -233,8 +233,8 @@ template <> struct SsdSmem<true> {
     static constexpr int SH = XW + 16384;        // S^T rows, hi part: 128 (n) x 64 (p) bf16
     static constexpr int SL = SH + 16384;        // lo part
     static constexpr int PR = SL + 16384;        // two buffers of (acum, e, w, v) x 128 floats
-    static constexpr int MB = PR + 2 * 4 * kSsdQ * 4;   // mbarriers: Gram, state, outputs
-    static constexpr int SLOT = MB + 24;         // tensor-memory address
+    static constexpr int MB = PR + 2 * 4 * kSsdQ * 4;   // mbarriers: Gram, state, outputs, drain
+    static constexpr int SLOT = MB + 32;         // tensor-memory address
     static constexpr int BYTES = SLOT + 8;
     static constexpr int TOTAL = BYTES + 1024;   // with the alignment pad
     // tensor memory: G (0..127); the state product (128..191); M as the A
@@ -252,7 +252,7 @@ template <> struct SsdSmem<false> {
     static constexpr int SH = -1, SL = -1;
     static constexpr int PR = XW + 16384;
     static constexpr int MB = PR + 2 * 4 * kSsdQ * 4;
-    static constexpr int SLOT = MB + 24;
+    static constexpr int SLOT = MB + 32;
     static constexpr int BYTES = SLOT + 8;
     static constexpr int TOTAL = BYTES + 1024;
     static constexpr int TMEM_COLS = 64;
@@ -295,6 +295,7 @@ __global__ void __launch_bounds__(kFull ? kSsdFullThreads : kSsdThreads, kFull ?
         c_end = min(min(nC, (k + 1) * p.cps), c_begin + p.cpp);
     }
     const uint32_t mbG = sb + Lay::MB, mbS = sb + Lay::MB + 8, mbY = sb + Lay::MB + 16;
+    const uint32_t mbF = sb + Lay::MB + 24;   // drain: every product thread 0 issued has completed
 
     // ---- copies of chunk c's rows: B/C rows rBC + (NT/16) k, piece tid%16; x rows
     // rX + (NT/8) k, piece tid%8; the prep values into buffer `slot`
@@ -331,6 +332,7 @@ __global__ void __launch_bounds__(kFull ? kSsdFullThreads : kSsdThreads, kFull ?
         mbar_init(mbG, 1);
         mbar_init(mbS, 1);
         mbar_init(mbY, 1);
+        mbar_init(mbF, 1);
     }
     if (w == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sb + Lay::SLOT),
@@ -578,7 +580,23 @@ __global__ void __launch_bounds__(kFull ? kSsdFullThreads : kSsdThreads, kFull ?
     }
 
     cp_async_wait_0();                         // this thread's copies in flight
-    if (!ok_all) atomicExch(p.err, 1);
+    // A wait that gave up (in the loop, or in the last chunk after its final
+    // barrier) leaves products thread 0 issued possibly still running: before
+    // the tensor memory is freed, one more commit from thread 0 on the drain
+    // barrier tracks the completion of all of them, waited for with the same
+    // bound.  If that wait gives up too, the tensor memory is not freed (a
+    // late product must not land in columns another CTA has allocated).
+    const bool failed = __syncthreads_or(!ok_all);
+    bool drained = true;
+    if (failed) {
+        if (tid == 0) {
+            tc_fence_after();
+            umma_commit(mbF);
+        }
+        drained = mbar_wait(mbF, 0u);
+        drained = !__syncthreads_or(!drained);
+        if (tid == 0) atomicExch(p.err, 1);
+    }
     if constexpr (kFull) {
         if (seg == p.segs - 1) {
 #pragma unroll
@@ -593,7 +611,8 @@ __global__ void __launch_bounds__(kFull ? kSsdFullThreads : kSsdThreads, kFull ?
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (w == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(Lay::TMEM_COLS));
+    if (w == 0 && drained)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(Lay::TMEM_COLS));
 }
 
 }  // namespace axon

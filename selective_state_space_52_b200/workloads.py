@@ -17,6 +17,13 @@ Distributions ("config-0 distributions"), for every workload below:
 The Mamba-block workload adds a bimodal dt: even channels u = 1e-4 (long
 memory), odd channels u = 1.0 (fast forgetting), same dt_raw noise.
 
+Test inputs (``params="random"``, the default of ``custom``) make every
+per-channel parameter differ from one channel to the next, as a trained layer's
+do (A_log is a learned per-state parameter that log(1..N) only initialises):
+  conv_b ~ N(0, 0.1^2) per channel;  D ~ N(0, 1) per channel;
+  A_log[e, n] = log(n + 1) + N(0, 0.1^2) per (channel, state).
+The five measured workloads keep the initialisation above.
+
 The Mamba-2 (SSD) workloads (``SSD_WORKLOADS``): x ~ N(0, 1) (B,L,H,64),
 dt_raw ~ N(0, 0.5), B, C ~ N(0, 1) (B,L,128) in bf16; per head dt_bias =
 log(expm1(u)), u ~ logUniform[1e-3, 1e-1], A_log = log(Uniform[1, 16]) and
@@ -50,6 +57,7 @@ class Workload:
     dt_mode: str = "logu"        # "logu" or "bimodal"
     decode_steps: int = 0        # cached single-token steps after the prefill
     note: str = ""
+    params: str = "init"         # "init": conv_b 0, D 1, A_log log(1..N); "random": per-channel draws
     N: int = N_STATE
     K: int = K_CONV
 
@@ -78,8 +86,8 @@ WORKLOADS = [
 WORKLOAD_BY_NAME = {w.name: w for w in WORKLOADS}
 
 
-def custom(B, L, E, io="f32", seed=0, dt_mode="logu", name="custom") -> Workload:
-    return Workload(name, B, L, E, io, seed, dt_mode=dt_mode)
+def custom(B, L, E, io="f32", seed=0, dt_mode="logu", name="custom", params="random") -> Workload:
+    return Workload(name, B, L, E, io, seed, dt_mode=dt_mode, params=params)
 
 
 def _gen(seed: int) -> torch.Generator:
@@ -102,9 +110,16 @@ def make_params(wl: Workload, g: torch.Generator | None = None) -> dict:
         lo, hi = math.log(1e-3), math.log(1e-1)
         u = torch.exp(lo + (hi - lo) * torch.rand(E, generator=g, dtype=torch.float64))
     dt_bias = torch.log(torch.expm1(u)).to(torch.float32)
-    A_log = torch.log(torch.arange(1, N + 1, dtype=torch.float64)).to(torch.float32)
+    A_log = torch.log(torch.arange(1, N + 1, dtype=torch.float64))
     A_log = A_log.unsqueeze(0).expand(E, N).contiguous()
     D = torch.ones(E, dtype=torch.float32)
+    if wl.params == "random":
+        conv_b = torch.randn(E, generator=g, dtype=torch.float32) * 0.1
+        D = torch.randn(E, generator=g, dtype=torch.float32)
+        A_log = A_log + torch.randn(E, N, generator=g, dtype=torch.float64) * 0.1
+    elif wl.params != "init":
+        raise ValueError(f"params must be 'init' or 'random', not {wl.params!r}")
+    A_log = A_log.to(torch.float32)
     return {"conv_w": conv_w, "conv_b": conv_b, "dt_bias": dt_bias, "A_log": A_log, "D": D}
 
 
@@ -172,16 +187,18 @@ class BlockWorkload:
     note: str = ""
     N: int = N_STATE
     K: int = K_CONV
+    params: str = "init"
 
     def core(self) -> Workload:
         """The layer-core workload with the same per-channel parameters."""
-        return Workload(self.name, self.B, self.L, self.E, "bf16", self.seed)
+        return Workload(self.name, self.B, self.L, self.E, "bf16", self.seed, params=self.params)
 
 
 BLOCK_WORKLOADS = [
     BlockWorkload("bit_axon_block", 1, 2048, 2560, 7680, 11,
                   note="the Bit-Axon layer: D=2560, expand 3 -> E=7680, bf16"),
-    BlockWorkload("small_block", 2, 100, 256, 768, 12, note="small layer for parity tests"),
+    BlockWorkload("small_block", 2, 100, 256, 768, 12, note="small layer for parity tests",
+                  params="random"),
 ]
 BLOCK_WORKLOAD_BY_NAME = {w.name: w for w in BLOCK_WORKLOADS}
 

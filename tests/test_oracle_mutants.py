@@ -75,3 +75,16 @@ def test_unmutated_oracle_passes_the_pins(tmp_path):
                         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
                        env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-2000:]
+
+
+def test_openmp_build_passes_the_pins(tmp_path):
+    """The OpenMP build of the same source (channels spread over host cores)
+    passes every pin, like the default single-threaded build."""
+    lib = tmp_path / "liboracle_omp.so"
+    subprocess.run(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-fno-fast-math",
+                    "-ffp-contract=off", "-fopenmp", "-o", str(lib), SRC, "-lm"], check=True)
+    env = dict(os.environ, AXON_ORACLE_LIB=str(lib), OMP_NUM_THREADS="4")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:]

@@ -582,3 +582,17 @@ def test_ssd_without_input_only_decays_the_state():
     y_ref = np.einsum("blh,bhpn,bln->blhp", dec, d["h0"], d["Cm"]) + d["D"][None, None, :, None] * d["x"]
     np.testing.assert_allclose(y, y_ref, rtol=1e-11, atol=1e-11)
     np.testing.assert_allclose(hL, dec[:, -1][:, :, None, None] * d["h0"], rtol=1e-11, atol=1e-11)
+
+
+@pytest.mark.skipif(bool(os.environ.get("AXON_ORACLE_LIB")),
+                    reason="compares the two builds of the real source only")
+def test_openmp_build_is_bit_identical():
+    """The OpenMP build runs each channel's arithmetic unchanged: its prefill
+    equals the single-threaded build's bit for bit, caches included."""
+    rng = np.random.default_rng(11)
+    d = rand_layer(rng, 3, 70, 37)
+    serial = run_layer(d)
+    par = run_layer(d, parallel=True)
+    for a, b in zip(serial, par):
+        np.testing.assert_array_equal(a, b)
+    assert oracle.threads(parallel=False) == 1

@@ -164,7 +164,7 @@ def test_dt_clip_edges(cuda_lib, io, shift):
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_bimodal_dt_long_and_fast_memory(cuda_lib, io):
-    wl = W.Workload("bimodal_small", 2, 777, 40, io, 9, dt_mode="bimodal")
+    wl = W.Workload("bimodal_small", 2, 777, 40, io, 9, dt_mode="bimodal", params="random")
     inp = W.make_inputs(wl, with_state=True)
     compare_scan(inp, io, what="bimodal")
 
