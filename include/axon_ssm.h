@@ -192,6 +192,27 @@ AXON_API axon_status axon_ssm_scan_fwd_segments(
     void *workspace, size_t workspace_bytes, int num_segments, axon_stream_t stream);
 
 /*
+ * The prefill with one kernel forced, for tests and tuning: the split-chunk
+ * quadrant scan (a block of `runs` warps per 8 channels; each chunk of the
+ * sequence is cut into `runs` runs of consecutive tokens, one per warp, whose
+ * aggregates (decay product, local end state) are folded into every run's
+ * entering state -- the chunked associative scan of the SSD article applied
+ * to the diagonal recurrence of the Axon-SSM page).  runs is 1, 2, 4 or 8
+ * (else AXON_ERR_INVALID_ARG); shapes whose staging does not fit return
+ * AXON_ERR_UNSUPPORTED.  `disc` as for axon_ssm_scan_fwd_ex.  No workspace.
+ * Other arguments, layouts and errors are those of axon_ssm_scan_fwd; results
+ * agree with the library's own plan to float32 rounding.
+ */
+AXON_API axon_status axon_ssm_scan_fwd_qsplit(
+    int B, int L, int E, int N, int K, axon_dtype io, axon_discretization disc, int runs,
+    const void *x, const void *z, const void *dt_raw,
+    const void *Bm, const void *Cm,
+    const float *conv_w, const float *conv_b,
+    const float *dt_bias, const float *A_log, const float *D,
+    const void *conv_cache_in, const float *ssm_state_in,
+    void *y, void *conv_cache_out, float *ssm_state_out, axon_stream_t stream);
+
+/*
  * The prefill (axon_ssm_scan_fwd_segments semantics) for callers that cannot
  * provide scratch memory.  The pages have no counterpart; this is a
  * convenience of the library.

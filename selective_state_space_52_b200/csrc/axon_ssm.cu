@@ -14,6 +14,7 @@
 #include "device_math.cuh"
 #include "scan_chunked.cuh"
 #include "scan_octo.cuh"
+#include "scan_qsplit.cuh"
 #include "scan_quad.cuh"
 #include "scan_seq.cuh"
 #include "step.cuh"
@@ -208,6 +209,39 @@ axon_status launch_quad(const ChunkParams& prm, cudaStream_t st) {
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
 
+// Split-chunk quadrant scan: W warps per 8 channels, each chunk cut into W
+// runs (R = 32 tokens per run for W = 1, else 16).
+template <class Io, int W, bool Z>
+axon_status launch_qsplit_t(const ChunkParams& prm, cudaStream_t st) {
+    constexpr int R = W == 1 ? 32 : 16;
+    auto kern = scan_qsplit_kernel<Io, W, R, Z>;
+    static std::atomic<unsigned long long> smem_set{0};
+    if (!allow_max_smem(kern, smem_set)) return AXON_ERR_CUDA;
+    const int smem = QsplitSmem(W, R, Io::kBytes).total;
+    const long long ctas = (long long)prm.B * ((prm.E + kQsCh - 1) / kQsCh);
+    if (ctas > 0x7fffffffLL) return AXON_ERR_UNSUPPORTED;
+    kern<<<(unsigned)ctas, 32 * W, smem, st>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+}
+
+template <class Io, bool Z>
+axon_status launch_qsplit(const ChunkParams& prm, int W, cudaStream_t st) {
+    switch (W) {
+        case 1: return launch_qsplit_t<Io, 1, Z>(prm, st);
+        case 2: return launch_qsplit_t<Io, 2, Z>(prm, st);
+        case 4: return launch_qsplit_t<Io, 4, Z>(prm, st);
+        case 8: return launch_qsplit_t<Io, 8, Z>(prm, st);
+    }
+    return AXON_ERR_UNSUPPORTED;
+}
+
+bool qsplit_fits(int B, int L, int E, int io_bytes, int W) {
+    (void)B; (void)L;
+    const int R = W == 1 ? 32 : 16;
+    return (long long)(W * R + kK) * E * io_bytes < (1LL << 31) &&
+           QsplitSmem(W, R, io_bytes).total <= device_max_smem_optin();
+}
+
 template <class Io, int W, int R, bool Z>
 axon_status launch_chunked_t(const ChunkParams& prm, int smem, cudaStream_t st) {
     auto kern = scan_chunked_kernel<Io, W, R, Z>;
@@ -256,7 +290,7 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
                       const void* conv_cache_in, const float* ssm_state_in,
                       void* y, void* conv_cache_out, float* ssm_state_out,
                       void* workspace, size_t workspace_bytes, int num_segments,
-                      cudaStream_t stream, bool zoh = false) {
+                      cudaStream_t stream, bool zoh = false, int qsplit_runs = 0) {
     axon_status st = check_shape(B, L, E, N, K, io);
     if (st != AXON_OK) return st;
     if (num_segments < 0) return AXON_ERR_INVALID_ARG;
@@ -293,8 +327,18 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
     int P = 1;
     int seg = L > 0 ? L : 1;
     bool chunked = false, quad = false, octo = false;
+    int qsplit = 0;                              // runs per chunk of the split-chunk quadrant scan
     ChunkPlan cplan{};
-    if (L > 0) {
+    if (qsplit_runs != 0) {
+        if (qsplit_runs != 1 && qsplit_runs != 2 && qsplit_runs != 4 && qsplit_runs != 8)
+            return AXON_ERR_INVALID_ARG;
+        if (num_segments != 1) return AXON_ERR_INVALID_ARG;
+        if (L > 0) {
+            if (device_max_smem_optin() <= 0) return AXON_ERR_CUDA;
+            if (!qsplit_fits(B, L, E, (int)io_bytes(io), qsplit_runs)) return AXON_ERR_UNSUPPORTED;
+            qsplit = qsplit_runs;
+        }
+    } else if (L > 0) {
         if (num_segments > kMaxSegments) return AXON_ERR_INVALID_ARG;
         if (num_segments > 1) {
             P = num_segments;                  // forced time split (segment carry)
@@ -329,7 +373,7 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
             return AXON_ERR_INVALID_ARG;
     }
 
-    if (chunked || quad || octo) {
+    if (chunked || quad || octo || qsplit) {
         ChunkParams cp;
         cp.B = B; cp.L = L; cp.E = E;
         cp.ET = quad ? kQuadCh : (octo ? kOctoCh : cplan.ET);
@@ -339,6 +383,11 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
         cp.conv_w = conv_w; cp.conv_b = conv_b; cp.dt_bias = dt_bias; cp.A_log = A_log; cp.D = D;
         cp.conv_cache_in = conv_cache_in; cp.ssm_state_in = ssm_state_in;
         cp.y = y; cp.conv_cache_out = conv_cache_out; cp.ssm_state_out = ssm_state_out;
+        if (qsplit) {
+            if (io == AXON_BF16)
+                return zoh ? launch_qsplit<IoBF16, true>(cp, qsplit, stream) : launch_qsplit<IoBF16, false>(cp, qsplit, stream);
+            return zoh ? launch_qsplit<IoF32, true>(cp, qsplit, stream) : launch_qsplit<IoF32, false>(cp, qsplit, stream);
+        }
         if (octo) {
             if (io == AXON_BF16) return zoh ? launch_octo<IoBF16, true>(cp, stream) : launch_octo<IoBF16, false>(cp, stream);
             return zoh ? launch_octo<IoF32, true>(cp, stream) : launch_octo<IoF32, false>(cp, stream);
@@ -554,6 +603,22 @@ axon_status axon_ssm_scan_fwd_ex(int B, int L, int E, int N, int K, axon_dtype i
                      conv_cache_in, ssm_state_in, y, conv_cache_out, ssm_state_out,
                      workspace, workspace_bytes, num_segments,
                      reinterpret_cast<cudaStream_t>(stream), disc == AXON_DISC_ZOH);
+}
+
+axon_status axon_ssm_scan_fwd_qsplit(int B, int L, int E, int N, int K, axon_dtype io,
+                                     axon_discretization disc, int runs,
+                                     const void* x, const void* z, const void* dt_raw,
+                                     const void* Bm, const void* Cm,
+                                     const float* conv_w, const float* conv_b,
+                                     const float* dt_bias, const float* A_log, const float* D,
+                                     const void* conv_cache_in, const float* ssm_state_in,
+                                     void* y, void* conv_cache_out, float* ssm_state_out,
+                                     axon_stream_t stream) {
+    if (disc != AXON_DISC_FIRST_ORDER && disc != AXON_DISC_ZOH) return AXON_ERR_UNSUPPORTED;
+    if (runs == 0) return AXON_ERR_INVALID_ARG;
+    return scan_impl(B, L, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, conv_b, dt_bias, A_log, D,
+                     conv_cache_in, ssm_state_in, y, conv_cache_out, ssm_state_out,
+                     nullptr, 0, 1, reinterpret_cast<cudaStream_t>(stream), disc == AXON_DISC_ZOH, runs);
 }
 
 axon_status axon_ssm_scan_fwd_noalloc(int B, int L, int E, int N, int K, axon_dtype io,

@@ -1,0 +1,478 @@
+// scan_qsplit.cuh -- quadrant scan with each chunk split in time over W warps.
+//
+// A CTA of W warps owns 8 consecutive channels of one batch row for the whole
+// sequence.  In every warp lane = 8 g + c handles channel c and the state
+// quadrant g (states 4g .. 4g+3), so the B and C values a lane needs are the
+// same for the 8 lanes of its quarter warp.  The sequence is walked in chunks
+// of W * R tokens; warp w takes the run of R tokens w*R .. w*R + R - 1 of each
+// chunk.  Per chunk and warp:
+//
+//   1. copies (cp.async, one chunk ahead, double buffered) of its run's x
+//      rows with a 3-token halo, the z and dt_raw rows of the 8 channels and
+//      the B, C rows into the warp's own shared memory; bf16 B and C rows are
+//      widened to float32 once per warp (not once per lane);
+//   2. the per-(token, channel) prologue, once: lane (g, c) takes tokens
+//      g*R/4 .. g*R/4 + R/4 - 1 of channel c (conv window in registers), writes
+//      (dt, dt, f, f) -- f = dt*u first order, u for ZOH -- and keeps D*u and
+//      SiLU(z) of its tokens in registers;
+//   3. W > 1: a first pass from a zero state over the run keeps the R decays
+//      a = 2^(dt * A log2 e) of its 4 states in registers and yields the run's
+//      aggregate (prod a = 2^(A log2 e * sum dt), local end state H); after one
+//      CTA barrier each warp folds the aggregates of the runs before it into
+//      the chunk's entering state, h = A_j h + H_j (the intra-block pass and
+//      inter-block carry of the SSD article's chunked scan, applied to the
+//      diagonal recurrence), and the second pass walks the run again from that
+//      state with the stored decays: no second exponential;
+//      W == 1: one pass with the carried state, decays computed on the way;
+//   4. the partial C . h of each token (sum over the lane's quadrant) goes
+//      through shared memory to the lane that owns the token's prologue, which
+//      adds the four quadrants and stores y = (C . h + D u) SiLU(z).
+// The last warp's end state is the next chunk's entering state (shared
+// memory, double buffered by chunk parity, so one barrier per chunk suffices).
+//
+// Recurrence and gating: Axon-SSM page, recurrence equation, "Selective
+// mechanism", "Diagonal state matrix", "Gating"; with kZoh the exact
+// zero-order-hold Bbar of section "ZOH discretisation".
+#pragma once
+
+#include "device_math.cuh"
+#include "scan_chunked.cuh"   // ChunkParams, cp.async helpers, SmemIo, f2
+
+namespace axon {
+
+constexpr int kQsCh = 8;   // channels per CTA
+
+// Byte layout of the shared memory: W per-warp areas, then the CTA's
+// aggregate and entering-state slots.  Identical on host and device.
+struct QsplitSmem {
+    int xs, zs, ds, bs, cs, stage;   // one staging buffer (io dtype); two per warp
+    int bf, cf;                      // float32 B, C rows of the run (bf16 io)
+    int pf;                          // (dt, dt, f, f) per (token, channel)
+    int red;                         // partial sums, one row of R + 4 floats per lane
+    int warp_bytes;
+    int agg, entry, total;
+    __host__ __device__ static int pad(int r, int RQ) { return r + r / RQ; }
+    __host__ __device__ QsplitSmem(int W, int R, int io_bytes) {
+        const int RQ = R / 4;
+        const int XB = kQsCh * io_bytes;
+        const int RB = kN * io_bytes;
+        int off = 0;
+        xs = off; off += (pad(R + kK - 2, RQ) + 1) * XB;
+        zs = off; off += (pad(R - 1, RQ) + 1) * XB;
+        ds = off; off += (pad(R - 1, RQ) + 1) * XB;
+        bs = off; off += R * RB;
+        cs = off; off += R * RB;
+        stage = (off + 15) & ~15;
+        off = 2 * stage;
+        bf = off; off += io_bytes == 2 ? R * kN * 4 : 0;
+        cf = off; off += io_bytes == 2 ? R * kN * 4 : 0;
+        pf = off; off += R * kQsCh * 16;
+        red = off; off += 32 * (R + 4) * 4;
+        warp_bytes = (off + 127) & ~127;
+        off = W * warp_bytes;
+        agg = off; off += W > 1 ? 2 * W * 32 * 32 : 0;       // [parity][warp][lane] (A0..3, H0..3)
+        entry = off; off += W > 1 ? 2 * 32 * 16 : 0;         // [parity][lane] h0..3
+        total = off;
+    }
+};
+
+template <class Io, int W, int R, bool kZoh>
+__global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(ChunkParams p) {
+    static_assert(R % 16 == 0 && R <= 32, "R: 16 or 32 tokens per run");
+    static_assert(W == 1 || W == 2 || W == 4 || W == 8, "W: 1, 2, 4 or 8 runs per chunk");
+    using TT = typename Io::T;
+    using SI = SmemIo<Io>;
+    constexpr int S = Io::kBytes;
+    constexpr int XB = kQsCh * S;            // bytes of one staged x/z/dt row (8 channels)
+    constexpr int RB = kN * S;               // bytes of one staged B/C row
+    constexpr int RQ = R / 4;                // tokens per lane in the prologue
+    constexpr int T = W * R;                 // tokens per chunk
+    constexpr int P = XB / 16;               // 16-byte pieces per staged x/z/dt row
+    constexpr int PB = RB / 16;              // 16-byte pieces per B/C row
+    constexpr int NXP = (R + kK - 1) * P, NX = (NXP + 31) / 32;
+    constexpr int NZP = R * P, NZ = (NZP + 31) / 32;
+    constexpr int NBP = R * PB, NB = (NBP + 31) / 32;
+    constexpr bool kWiden = S == 2;          // bf16 B/C rows are widened to float32
+    extern __shared__ __align__(16) unsigned char smem[];
+
+    const int lane = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5;          // run of the chunk
+    const int tiles = (p.E + kQsCh - 1) / kQsCh;
+    const int b = blockIdx.x / tiles;
+    const int e0 = (blockIdx.x - b * tiles) * kQsCh;
+    const int ne = min(kQsCh, p.E - e0);     // 8, or 4 for an fp32 tail
+    const int g = lane >> 3;                 // state quadrant
+    const int c = lane & 7;                  // channel in the tile
+    const bool active = c < ne;
+    const int e = e0 + (active ? c : 0);
+    const QsplitSmem lay(W, R, S);
+    unsigned char* ws = smem + w * lay.warp_bytes;
+
+    const unsigned char* xg = static_cast<const unsigned char*>(p.x);
+    const unsigned char* zg = static_cast<const unsigned char*>(p.z);
+    const unsigned char* dg = static_cast<const unsigned char*>(p.dt_raw);
+    const unsigned char* bg = static_cast<const unsigned char*>(p.Bm);
+    const unsigned char* cg = static_cast<const unsigned char*>(p.Cm);
+    const unsigned char* ccg = static_cast<const unsigned char*>(p.conv_cache_in);
+    const int row_bytes = p.E * S;           // the host keeps (T + K) * E * S below 2^31
+    const int npc = (ne * S + 15) / 16;      // pieces of a row inside the tile
+    const size_t tile_off = (size_t)b * p.L * row_bytes + (size_t)e0 * S;
+
+    // ---- this lane's share of a run's copies: shared-memory destinations and
+    // byte offsets from the run's first row, fixed for all chunks
+    int xsd[NX], xgo[NX], zsd[NZ], zgo[NZ], bso[NB];
+    bool xok[NX], zok[NZ], bok[NB];
+#pragma unroll
+    for (int i = 0; i < NX; ++i) {
+        const int q = lane + 32 * i, r = q / P, pc = q % P;
+        xok[i] = q < NXP && pc < npc;
+        xsd[i] = lay.xs + QsplitSmem::pad(r, RQ) * XB + pc * 16;
+        xgo[i] = (r - (kK - 1)) * row_bytes + pc * 16;
+    }
+#pragma unroll
+    for (int i = 0; i < NZ; ++i) {
+        const int q = lane + 32 * i, r = q / P, pc = q % P;
+        zok[i] = q < NZP && pc < npc;
+        zsd[i] = QsplitSmem::pad(r, RQ) * XB + pc * 16;
+        zgo[i] = r * row_bytes + pc * 16;
+    }
+#pragma unroll
+    for (int i = 0; i < NB; ++i) {
+        const int q = lane + 32 * i;
+        bok[i] = q < NBP;
+        bso[i] = (q / PB) * RB + (q % PB) * 16;
+    }
+
+    // copies of chunk k's run of this warp into stage st
+    auto prefetch = [&](int k, int st) {
+        unsigned char* sb = ws + st * lay.stage;
+        const int t0 = k * T + w * R;
+        if (t0 >= kK - 1 && t0 + R <= p.L) {
+            // every row of the run and its halo lies inside the sequence
+            const unsigned char* xr = xg + tile_off + (size_t)t0 * row_bytes;
+            const unsigned char* zr = zg + tile_off + (size_t)t0 * row_bytes;
+            const unsigned char* dr = dg + tile_off + (size_t)t0 * row_bytes;
+            const size_t bc0 = ((size_t)b * p.L + t0) * RB;
+#pragma unroll
+            for (int i = 0; i < NX; ++i)
+                if (xok[i]) cp_async16(sb + xsd[i], xr + xgo[i], true);
+#pragma unroll
+            for (int i = 0; i < NZ; ++i)
+                if (zok[i]) {
+                    cp_async16(sb + lay.zs + zsd[i], zr + zgo[i], true);
+                    cp_async16(sb + lay.ds + zsd[i], dr + zgo[i], true);
+                }
+#pragma unroll
+            for (int i = 0; i < NB; ++i)
+                if (bok[i]) {
+                    cp_async16(sb + lay.bs + bso[i], bg + bc0 + bso[i], true);
+                    cp_async16(sb + lay.cs + bso[i], cg + bc0 + bso[i], true);
+                }
+            return;
+        }
+        // the sequence's first rows (halo from the conv cache or zeros) or a
+        // ragged end (rows past L zero-filled)
+        for (int q = lane; q < NXP; q += 32) {
+            const int r = q / P, pc = q % P;
+            const int t = t0 - (kK - 1) + r;
+            const void* src = xg;
+            bool ok = false;
+            if (pc < npc) {
+                if (t >= 0 && t < p.L) {
+                    src = xg + tile_off + (size_t)t * row_bytes + pc * 16;
+                    ok = true;
+                } else if (t < 0 && ccg != nullptr) {
+                    src = ccg + ((size_t)b * (kK - 1) + (kK - 1 + t)) * row_bytes + (size_t)e0 * S + pc * 16;
+                    ok = true;
+                }
+            }
+            cp_async16(sb + lay.xs + QsplitSmem::pad(r, RQ) * XB + pc * 16, src, ok);
+        }
+        for (int q = lane; q < NZP; q += 32) {
+            const int r = q / P, pc = q % P;
+            const int t = t0 + r;
+            const bool ok = t < p.L && pc < npc;
+            const size_t go = ok ? tile_off + (size_t)t * row_bytes + pc * 16 : 0;
+            const int so = QsplitSmem::pad(r, RQ) * XB + pc * 16;
+            cp_async16(sb + lay.zs + so, zg + go, ok);
+            cp_async16(sb + lay.ds + so, dg + go, ok);
+        }
+        for (int q = lane; q < NBP; q += 32) {
+            const int r = q / PB, pc = q % PB;
+            const int t = t0 + r;
+            const bool ok = t < p.L;
+            const size_t go = ok ? ((size_t)b * p.L + t) * RB + pc * 16 : 0;
+            cp_async16(sb + lay.bs + r * RB + pc * 16, bg + go, ok);
+            cp_async16(sb + lay.cs + r * RB + pc * 16, cg + go, ok);
+        }
+    };
+
+    // ---- per-lane constants: the channel's conv / dt / D parameters, the
+    // quadrant's A log2 e (and 1/A for ZOH) and the initial state
+    const float w0 = __ldg(p.conv_w + (size_t)e * kK + 0);
+    const float w1 = __ldg(p.conv_w + (size_t)e * kK + 1);
+    const float w2 = __ldg(p.conv_w + (size_t)e * kK + 2);
+    const float w3 = __ldg(p.conv_w + (size_t)e * kK + 3);
+    const float cb = __ldg(p.conv_b + e);
+    const float db = __ldg(p.dt_bias + e);
+    const float Dv = __ldg(p.D + e);
+    float2 s01, s23, iA01 = f2(0.f, 0.f), iA23 = f2(0.f, 0.f), h01, h23;
+    {
+        const float4 al = __ldg(reinterpret_cast<const float4*>(p.A_log + (size_t)e * kN) + g);
+        s01 = f2(-expf(al.x) * kLog2e, -expf(al.y) * kLog2e);
+        s23 = f2(-expf(al.z) * kLog2e, -expf(al.w) * kLog2e);
+        if constexpr (kZoh) {
+            iA01 = f2(kLog2e / s01.x, kLog2e / s01.y);
+            iA23 = f2(kLog2e / s23.x, kLog2e / s23.y);
+        }
+        float4 h0 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (p.ssm_state_in && active)
+            h0 = reinterpret_cast<const float4*>(p.ssm_state_in + ((size_t)b * p.E + e) * kN)[g];
+        h01 = f2(h0.x, h0.y);
+        h23 = f2(h0.z, h0.w);
+    }
+
+    // y of token (chunk start) + w*R + g*RQ + j, channel e: ybase + (t0 + j) * row_bytes
+    unsigned char* ybase = static_cast<unsigned char*>(p.y) + tile_off + (size_t)(w * R + g * RQ) * row_bytes + c * S;
+    const int nck = (p.L + T - 1) / T;
+    float4* pf = reinterpret_cast<float4*>(ws + lay.pf);          // [token][channel] (dt, dt, f, f)
+    float* red = reinterpret_cast<float*>(ws + lay.red);          // [lane][token] partial C . h
+    const float* bfs = reinterpret_cast<const float*>(ws + lay.bf);
+    const float* cfs = reinterpret_cast<const float*>(ws + lay.cf);
+
+    // B / C values of token t for this lane's quadrant (float32 rows)
+    auto bq = [&](const unsigned char* sb, int t) -> float4 {
+        if constexpr (kWiden) return *reinterpret_cast<const float4*>(bfs + t * kN + 4 * g);
+        else return *reinterpret_cast<const float4*>(sb + lay.bs + t * RB + 16 * g);
+    };
+    auto cq = [&](const unsigned char* sb, int t) -> float4 {
+        if constexpr (kWiden) return *reinterpret_cast<const float4*>(cfs + t * kN + 4 * g);
+        else return *reinterpret_cast<const float4*>(sb + lay.cs + t * RB + 16 * g);
+    };
+    // the ZOH input factor of token t's 4 states from dt and the decays
+    auto zoh4 = [&](float dt, float2 a01, float2 a23, float2& z01, float2& z23) {
+        const float2 x01 = __fmul2_rn(f2(dt, dt), s01), x23 = __fmul2_rn(f2(dt, dt), s23);
+        z01 = f2(zoh_bbar(dt, x01.x * kLn2, a01.x, iA01.x), zoh_bbar(dt, x01.y * kLn2, a01.y, iA01.y));
+        z23 = f2(zoh_bbar(dt, x23.x * kLn2, a23.x, iA23.x), zoh_bbar(dt, x23.y * kLn2, a23.y, iA23.y));
+    };
+
+    float2* agg = reinterpret_cast<float2*>(smem + lay.agg);       // W > 1
+    float4* entry = reinterpret_cast<float4*>(smem + lay.entry);   // W > 1
+
+    prefetch(0, 0);
+    cp_async_commit();
+    for (int k = 0; k < nck; ++k) {
+        const int st = k & 1;
+        const int t0 = k * T;                // chunk start
+        const int tr = t0 + w * R;           // this warp's run start
+        const bool full = tr + R <= p.L;
+        __syncwarp();                        // every lane is done with the stage refilled below
+        if (k + 1 < nck) prefetch(k + 1, st ^ 1);
+        cp_async_commit();
+        cp_async_wait_1();                   // this lane's copies of chunk k have landed
+        __syncwarp();                        // ... and every lane's
+        const unsigned char* sb = ws + st * lay.stage;
+
+        // ---- widen the run's B and C rows to float32 (bf16 io)
+        if constexpr (kWiden) {
+#pragma unroll
+            for (int q = lane; q < 2 * R; q += 32) {
+                const int t = q >> 1;
+                const unsigned char* src = sb + ((q & 1) ? lay.cs : lay.bs) + t * RB;
+                float* dst = const_cast<float*>((q & 1) ? cfs : bfs) + t * kN;
+                float v[8];
+                SI::ld8(src, v);
+                *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<float4*>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
+                SI::ld8(src + 16, v);
+                *reinterpret_cast<float4*>(dst + 8) = make_float4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<float4*>(dst + 12) = make_float4(v[4], v[5], v[6], v[7]);
+            }
+        }
+
+        // ---- prologue: lane (g, c) takes tokens g*RQ .. g*RQ + RQ - 1 of channel c
+        float Du[RQ], gz[RQ];
+        {
+            const unsigned char* xc = sb + lay.xs + c * S;
+            const int tb = g * RQ;
+            float xm3 = SI::ld(xc + QsplitSmem::pad(tb + 0, RQ) * XB);
+            float xm2 = SI::ld(xc + QsplitSmem::pad(tb + 1, RQ) * XB);
+            float xm1 = SI::ld(xc + QsplitSmem::pad(tb + 2, RQ) * XB);
+#pragma unroll
+            for (int i = 0; i < RQ; ++i) {
+                const int t = tb + i;
+                const float xt = SI::ld(xc + QsplitSmem::pad(t + 3, RQ) * XB);
+                float xv = fmaf(w0, xm3, cb);
+                xv = fmaf(w1, xm2, xv);
+                xv = fmaf(w2, xm1, xv);
+                xv = fmaf(w3, xt, xv);
+                xm3 = xm2; xm2 = xm1; xm1 = xt;
+                const float u = silu(xv);
+                const int tp = t + g;            // padded row of token t (t / RQ == g)
+                const float dt = dt_from_raw(SI::ld(sb + lay.ds + tp * XB + c * S) + db);
+                const bool live = full || tr + t < p.L;
+                const float dtl = live ? dt : 0.0f;        // dt = 0: decay 1, no input
+                const float f = live ? (kZoh ? u : dt * u) : 0.0f;
+                pf[t * kQsCh + c] = make_float4(dtl, dtl, f, f);
+                Du[i] = Dv * u;
+                gz[i] = silu(SI::ld(sb + lay.zs + tp * XB + c * S));
+            }
+        }
+        __syncwarp();
+
+        float part[R];
+        if constexpr (W == 1) {
+            // ---- one pass from the carried state, in blocks of 4 tokens: the
+            // block's decays and inputs first, then its state updates
+#pragma unroll
+            for (int tb = 0; tb < R; tb += 4) {
+                float2 a01[4], a23[4], u01[4], u23[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int t = tb + i;
+                    const float4 v = pf[t * kQsCh + c];
+                    const float4 Bq = bq(sb, t);
+                    const float2 arg01 = __fmul2_rn(f2(v.x, v.y), s01);
+                    const float2 arg23 = __fmul2_rn(f2(v.x, v.y), s23);
+                    a01[i] = f2(ex2_approx(arg01.x), ex2_approx(arg01.y));
+                    a23[i] = f2(ex2_approx(arg23.x), ex2_approx(arg23.y));
+                    u01[i] = __fmul2_rn(f2(v.z, v.w), f2(Bq.x, Bq.y));
+                    u23[i] = __fmul2_rn(f2(v.z, v.w), f2(Bq.z, Bq.w));
+                    if constexpr (kZoh) {
+                        float2 z01, z23;
+                        zoh4(v.x, a01[i], a23[i], z01, z23);
+                        u01[i] = __fmul2_rn(u01[i], z01);
+                        u23[i] = __fmul2_rn(u23[i], z23);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int t = tb + i;
+                    const float4 Cq = cq(sb, t);
+                    h01 = __ffma2_rn(a01[i], h01, u01[i]);
+                    h23 = __ffma2_rn(a23[i], h23, u23[i]);
+                    const float2 pq = __ffma2_rn(f2(Cq.z, Cq.w), h23, __fmul2_rn(f2(Cq.x, Cq.y), h01));
+                    part[t] = pq.x + pq.y;
+                }
+            }
+        } else {
+            // ---- first pass: the run from a zero state; keep the decays
+            float2 a01[R], a23[R];
+            float2 H01 = f2(0.f, 0.f), H23 = f2(0.f, 0.f);
+            float dsum = 0.f;
+#pragma unroll
+            for (int t = 0; t < R; ++t) {
+                const float4 v = pf[t * kQsCh + c];
+                const float4 Bq = bq(sb, t);
+                const float2 arg01 = __fmul2_rn(f2(v.x, v.y), s01);
+                const float2 arg23 = __fmul2_rn(f2(v.x, v.y), s23);
+                a01[t] = f2(ex2_approx(arg01.x), ex2_approx(arg01.y));
+                a23[t] = f2(ex2_approx(arg23.x), ex2_approx(arg23.y));
+                float2 u01 = __fmul2_rn(f2(v.z, v.w), f2(Bq.x, Bq.y));
+                float2 u23 = __fmul2_rn(f2(v.z, v.w), f2(Bq.z, Bq.w));
+                if constexpr (kZoh) {
+                    float2 z01, z23;
+                    zoh4(v.x, a01[t], a23[t], z01, z23);
+                    u01 = __fmul2_rn(u01, z01);
+                    u23 = __fmul2_rn(u23, z23);
+                }
+                H01 = __ffma2_rn(a01[t], H01, u01);
+                H23 = __ffma2_rn(a23[t], H23, u23);
+                dsum += v.x;
+            }
+            // the run's aggregate: prod_t a_t = 2^(A log2 e * sum_t dt_t)
+            {
+                const float2 q01 = __fmul2_rn(f2(dsum, dsum), s01);
+                const float2 q23 = __fmul2_rn(f2(dsum, dsum), s23);
+                float2* slot = agg + ((k & 1) * W + w) * 32 * 4 + lane * 4;
+                reinterpret_cast<float4*>(slot)[0] =
+                    make_float4(ex2_approx(q01.x), ex2_approx(q01.y), ex2_approx(q23.x), ex2_approx(q23.y));
+                reinterpret_cast<float4*>(slot)[1] = make_float4(H01.x, H01.y, H23.x, H23.y);
+            }
+            __syncthreads();                 // every run's aggregate of chunk k is written
+            // ---- the state entering this run: the chunk's entering state (the
+            // last run's end state of chunk k-1) folded through runs 0 .. w-1
+            if (k > 0) {
+                const float4 he = entry[(k & 1) * 32 + lane];
+                h01 = f2(he.x, he.y);
+                h23 = f2(he.z, he.w);
+            }
+            for (int j = 0; j < w; ++j) {
+                const float4* slot = reinterpret_cast<const float4*>(agg + ((k & 1) * W + j) * 32 * 4 + lane * 4);
+                const float4 A = slot[0], H = slot[1];
+                h01 = __ffma2_rn(f2(A.x, A.y), h01, f2(H.x, H.y));
+                h23 = __ffma2_rn(f2(A.z, A.w), h23, f2(H.z, H.w));
+            }
+            // ---- second pass: the run again from its true entering state
+#pragma unroll
+            for (int t = 0; t < R; ++t) {
+                const float4 v = pf[t * kQsCh + c];
+                const float4 Bq = bq(sb, t);
+                float2 u01 = __fmul2_rn(f2(v.z, v.w), f2(Bq.x, Bq.y));
+                float2 u23 = __fmul2_rn(f2(v.z, v.w), f2(Bq.z, Bq.w));
+                if constexpr (kZoh) {
+                    float2 z01, z23;
+                    zoh4(v.x, a01[t], a23[t], z01, z23);
+                    u01 = __fmul2_rn(u01, z01);
+                    u23 = __fmul2_rn(u23, z23);
+                }
+                const float4 Cq = cq(sb, t);
+                h01 = __ffma2_rn(a01[t], h01, u01);
+                h23 = __ffma2_rn(a23[t], h23, u23);
+                const float2 pq = __ffma2_rn(f2(Cq.z, Cq.w), h23, __fmul2_rn(f2(Cq.x, Cq.y), h01));
+                part[t] = pq.x + pq.y;
+            }
+            if (w == W - 1) entry[((k + 1) & 1) * 32 + lane] = make_float4(h01.x, h01.y, h23.x, h23.y);
+        }
+
+        // ---- sum the four quadrants' partials of each token: lane (g, c)
+        // gets those of tokens g*RQ .. g*RQ + RQ - 1 of channel c
+        {
+            float* mine = red + lane * (R + 4);
+#pragma unroll
+            for (int t = 0; t < R; t += 4)
+                *reinterpret_cast<float4*>(mine + t) = make_float4(part[t], part[t + 1], part[t + 2], part[t + 3]);
+            __syncwarp();
+            float tot[RQ];
+#pragma unroll
+            for (int j = 0; j < RQ; ++j) tot[j] = 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float* src = red + (8 * q + c) * (R + 4) + g * RQ;
+#pragma unroll
+                for (int j = 0; j < RQ; j += 4) {
+                    const float4 v = *reinterpret_cast<const float4*>(src + j);
+                    tot[j] += v.x; tot[j + 1] += v.y; tot[j + 2] += v.z; tot[j + 3] += v.w;
+                }
+            }
+            unsigned char* yrow = ybase + (size_t)t0 * row_bytes;
+#pragma unroll
+            for (int j = 0; j < RQ; ++j)
+                if (active && (full || tr + g * RQ + j < p.L))
+                    Io::store(reinterpret_cast<TT*>(yrow + j * row_bytes), (tot[j] + Du[j]) * gz[j]);
+        }
+    }
+
+    // ---- final caches: the last run holds the sequence's end state
+    if (active && w == W - 1)
+        reinterpret_cast<float4*>(p.ssm_state_out + ((size_t)b * p.E + e) * kN)[g] =
+            make_float4(h01.x, h01.y, h23.x, h23.y);
+    if (active && w == 0 && g == 0) {
+        // the last K-1 raw inputs of conv_cache_in ++ x (all read before any write: may alias)
+        const TT* xs = static_cast<const TT*>(p.x);
+        const TT* cc = static_cast<const TT*>(p.conv_cache_in);
+        TT v[kK - 1];
+#pragma unroll
+        for (int j = 0; j < kK - 1; ++j) {
+            const int t = p.L - (kK - 1) + j;
+            if (t >= 0) v[j] = xs[((size_t)b * p.L + t) * p.E + e];
+            else if (cc) v[j] = cc[((size_t)b * (kK - 1) + (kK - 1 + t)) * p.E + e];
+            else v[j] = TT(0.0f);
+        }
+        TT* co = static_cast<TT*>(p.conv_cache_out);
+#pragma unroll
+        for (int j = 0; j < kK - 1; ++j) co[((size_t)b * (kK - 1) + j) * p.E + e] = v[j];
+    }
+}
+
+}  // namespace axon
