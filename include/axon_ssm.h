@@ -404,13 +404,17 @@ AXON_API axon_status axon_ssd_scan_fwd(
  *   y               = layer core          axon_ssm_scan_fwd on (x, z, dt_raw, B, C)
  *   out             = y W_out             W_out (E, Dm); out (B,L,Dm)
  *
- * Weights are row-major bf16 ("activations times weights").  The four matrix
- * products are plain bf16 GEMMs with float32 accumulation run by cuBLASLt
- * (one handle per device, created on first use); the conv stage and the layer
- * core run in this library's kernels.  The intermediates x, z, u, dt_raw, B,
- * C and y are stored in bf16 inside `workspace`, which must hold at least
+ * Weights are row-major bf16 ("activations times weights").  The three
+ * projections run on this library's tcgen05 GEMM (axon_gemm_bf16; float32
+ * accumulation): one launch writes x and z, one writes dt_raw, B and C, one
+ * the output.  The conv stage and the layer core run in this library's
+ * kernels too.  The intermediates x, z, u, dt_raw, B, C and y are stored in
+ * bf16 inside `workspace`, which must hold at least
  * axon_ssm_block_workspace_bytes(...) bytes (16-byte aligned; it also serves
- * as the GEMMs' and the scan's scratch).  Caches and parameters as for
+ * as the scan's scratch).  Its first 4 bytes (an int) are an error flag,
+ * cleared by each call and set to 1 if a wait of a GEMM for its copies or
+ * tensor-core products gave up (the outputs are then undefined); read it
+ * after the call completes.  Caches and parameters as for
  * axon_ssm_scan_fwd (in == out allowed); conv_cache_out receives the last K-1
  * rows of x.  Dm and E must be multiples of 8 (AXON_ERR_ALIGNMENT); io other
  * than AXON_BF16, N != 16 or K != 4 return AXON_ERR_UNSUPPORTED; out and the
@@ -427,6 +431,20 @@ AXON_API axon_status axon_ssm_block_fwd(
     const void *conv_cache_in, const float *ssm_state_in,
     void *out, void *conv_cache_out, float *ssm_state_out,
     void *workspace, size_t workspace_bytes, axon_stream_t stream);
+
+/*
+ * The projection GEMM the whole layer uses, on its own (tests and timing):
+ * C (M x N) = A (M x K) W (K x N), all row-major bf16 with row strides lda,
+ * ldw, ldc (elements), float32 accumulation, written as bf16.  Runs on the
+ * tcgen05 tensor cores (tiles of 128 x 256, TMA-fed, accumulators in tensor
+ * memory).  N, lda, ldw and ldc must be multiples of 8 and A, W, C 16-byte
+ * aligned (AXON_ERR_ALIGNMENT); C must not overlap A or W; K == 0 with M, N
+ * > 0 is AXON_ERR_INVALID_ARG.  `err` (a device int, or NULL) is set to 1 if
+ * a wait of the kernel for its copies or products gave up (C is then
+ * undefined); it is not cleared by the call.  Enqueued on `stream`.
+ */
+AXON_API axon_status axon_gemm_bf16(int M, int N, int K, const void *A, int lda, const void *W, int ldw,
+                                    void *C, int ldc, int *err, axon_stream_t stream);
 
 #ifdef __cplusplus
 }

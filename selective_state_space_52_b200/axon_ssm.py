@@ -53,6 +53,8 @@ _lib.axon_ssm_scan_fwd_segments.argtypes = _SCAN_ARGS + [_i, _vp]
 _lib.axon_ssm_scan_fwd_noalloc.restype = _i
 _lib.axon_ssm_scan_fwd_noalloc.argtypes = [_i] * 6 + [_vp] * 15 + [_i, _vp]
 NOALLOC_SCRATCH_BYTES = 16 << 20
+_lib.axon_ssm_scan_fwd_qsplit.restype = _i
+_lib.axon_ssm_scan_fwd_qsplit.argtypes = [_i] * 8 + [_vp] * 15 + [_vp]
 _lib.axon_ssm_scan_fwd_ex.restype = _i
 _lib.axon_ssm_scan_fwd_ex.argtypes = [_i] * 7 + [_vp] * 15 + [_vp, _sz, _i, _vp]
 _lib.axon_ssm_step_ex.restype = _i
@@ -72,6 +74,8 @@ _lib.axon_ssd_workspace_bytes.restype = _sz
 _lib.axon_ssd_workspace_bytes.argtypes = [_i] * 6
 _lib.axon_ssd_scan_fwd.restype = _i
 _lib.axon_ssd_scan_fwd.argtypes = [_i] * 6 + [_vp] * 10 + [_i, _vp, _sz, _vp]
+_lib.axon_gemm_bf16.restype = _i
+_lib.axon_gemm_bf16.argtypes = [_i] * 3 + [_vp, _i, _vp, _i, _vp, _i, _vp, _vp]
 _lib.axon_ssm_block_workspace_bytes.restype = _sz
 _lib.axon_ssm_block_workspace_bytes.argtypes = [_i] * 7
 _lib.axon_ssm_block_fwd.restype = _i
@@ -184,6 +188,21 @@ def axon_ssm_scan_fwd_noalloc(B, L, E, N, K, io, x, z, dt_raw, Bm, Cm, conv_w, c
     return rc
 
 
+def axon_ssm_scan_fwd_qsplit(B, L, E, N, K, io, disc, runs, x, z, dt_raw, Bm, Cm, conv_w, conv_b,
+                             dt_bias, A_log, D, conv_cache_in, ssm_state_in, y, conv_cache_out,
+                             ssm_state_out, stream=None, *, raise_on_error=True) -> int:
+    """The prefill on the split-chunk quadrant scan with `runs` warps per 8
+    channels (1, 2, 4 or 8), for tests and tuning."""
+    rc = _lib.axon_ssm_scan_fwd_qsplit(B, L, E, N, K, io, int(disc), int(runs), _p(x), _p(z),
+                                       _p(dt_raw), _p(Bm), _p(Cm), _p(conv_w), _p(conv_b),
+                                       _p(dt_bias), _p(A_log), _p(D), _p(conv_cache_in),
+                                       _p(ssm_state_in), _p(y), _p(conv_cache_out),
+                                       _p(ssm_state_out), _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_ssm_scan_fwd_qsplit")
+    return rc
+
+
 def axon_ssm_scan_fwd_ex(B, L, E, N, K, io, disc, x, z, dt_raw, Bm, Cm, conv_w, conv_b,
                          dt_bias, A_log, D, conv_cache_in, ssm_state_in, y, conv_cache_out,
                          ssm_state_out, workspace, workspace_bytes, num_segments=0, stream=None, *,
@@ -272,19 +291,43 @@ def axon_ssm_block_fwd(B, L, Dm, E, N, K, io, X, W_in, W_x, W_out, conv_w, conv_
     return rc
 
 
+def axon_gemm_bf16(M, N, K, A, lda, W, ldw, C, ldc, err=None, stream=None, *, raise_on_error=True) -> int:
+    rc = _lib.axon_gemm_bf16(M, N, K, _p(A), int(lda), _p(W), int(ldw), _p(C), int(ldc), _p(err),
+                             _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_gemm_bf16")
+    return rc
+
+
+def gemm_bf16(A, W, *, out=None, stream=None, check=True):
+    """C = A @ W for row-major bf16 A (M x K) and W (K x N) on the library's
+    tcgen05 GEMM (float32 accumulation).  With ``check`` the call waits for the
+    device and raises AxonError (AXON_ERR_TIMEOUT) if a wait of the kernel gave up."""
+    M, K = A.shape
+    N = W.shape[1]
+    C = torch.empty(M, N, dtype=torch.bfloat16, device=A.device) if out is None else out
+    err = torch.zeros(1, dtype=torch.int32, device=A.device)
+    axon_gemm_bf16(M, N, K, A, A.stride(0), W, W.stride(0), C, C.stride(0), err, stream=stream)
+    if check and int(err.item()) != 0:
+        raise AxonError(6, "axon_gemm_bf16 (a wait for a copy or a tensor-core product gave up)")
+    return C
+
+
 # ------------------------------------------------------------ conveniences
 PARAM_KEYS = ("conv_w", "conv_b", "dt_bias", "A_log", "D")
 WEIGHT_KEYS = ("W_in", "W_x", "W_out")
 
 
 def scan_fwd(x, z, dt_raw, Bm, Cm, params: dict, cache=None, *, num_segments=None,
-             out=None, workspace=None, stream=None, discretization="first_order"):
+             out=None, workspace=None, stream=None, discretization="first_order", runs=None):
     """Prefill over (B, L, E) inputs on the GPU.
 
     ``params`` holds conv_w, conv_b, dt_bias, A_log, D (float32, on the device);
     ``cache`` is None or (conv_cache, ssm_state).  Returns
     ``(y, (conv_cache, ssm_state))`` -- the cache pair of the Axon-SSM page's
     "Autoregressive decoding" section, ready for the next call or for ``step``.
+    ``runs`` (tests and tuning) forces the split-chunk quadrant scan with that
+    many warps per 8 channels.
     """
     Bsz, L, E = x.shape
     K = params["conv_w"].shape[1]
@@ -308,7 +351,10 @@ def scan_fwd(x, z, dt_raw, Bm, Cm, params: dict, cache=None, *, num_segments=Non
     wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
     args = (Bsz, L, E, N, K, io, x, z, dt_raw, Bm, Cm, *(params[k] for k in PARAM_KEYS),
             cc_in, ss_in, y, cc_out, ss_out, workspace, wsz)
-    if discretization != "first_order":
+    if runs is not None:
+        axon_ssm_scan_fwd_qsplit(Bsz, L, E, N, K, io, _DISC[discretization], runs, *args[6:-2],
+                                 stream=stream)
+    elif discretization != "first_order":
         axon_ssm_scan_fwd_ex(Bsz, L, E, N, K, io, _DISC[discretization], *args[6:],
                              num_segments or 0, stream=stream)
     elif num_segments is None:
@@ -336,12 +382,23 @@ def step(x, z, dt_raw, Bm, Cm, params: dict, cache, *, y=None, stream=None,
     return y
 
 
-def block_fwd(X, weights: dict, params: dict, cache=None, *, out=None, workspace=None, stream=None):
+def block_error_flag(workspace) -> int:
+    """The whole layer's GEMM error flag (the workspace's first int) after the
+    call that used ``workspace`` has completed.  Synchronises the device."""
+    torch.cuda.synchronize(workspace.device)
+    return int(workspace[:4].view(torch.int32).item())
+
+
+def block_fwd(X, weights: dict, params: dict, cache=None, *, out=None, workspace=None, stream=None,
+              check=True):
     """The whole Axon-SSM layer on (B, L, Dm) bf16 input ``X``.
 
     ``weights`` holds W_in (Dm, 2E), W_x (E, E+2N), W_out (E, Dm) in bf16;
     ``params`` and ``cache`` as for ``scan_fwd``.  Returns
-    ``(out, (conv_cache, ssm_state))``.
+    ``(out, (conv_cache, ssm_state))``.  With ``check`` (the default) the call
+    waits for the device and raises AxonError (AXON_ERR_TIMEOUT) if a wait of
+    a projection GEMM gave up; ``check=False`` returns at once (read the flag
+    with ``block_error_flag(workspace)``).
     """
     Bsz, L, Dm = X.shape
     E = weights["W_in"].shape[1] // 2
@@ -363,6 +420,8 @@ def block_fwd(X, weights: dict, params: dict, cache=None, *, out=None, workspace
     axon_ssm_block_fwd(Bsz, L, Dm, E, N, K, io, X, weights["W_in"], weights["W_x"], weights["W_out"],
                        *(params[k] for k in PARAM_KEYS), cc_in, ss_in, y, cc_out, ss_out,
                        workspace, wsz, stream=stream)
+    if check and Bsz * E > 0 and block_error_flag(workspace) != 0:
+        raise AxonError(6, "axon_ssm_block_fwd (a wait of a projection GEMM gave up)")
     return y, (cc_out, ss_out)
 
 

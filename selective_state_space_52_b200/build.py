@@ -3,8 +3,9 @@
     python -m selective_state_space_52_b200.build [--force] [--verbose]
 
 The shared library is written next to this file, so it ships with the source
-tree; nothing is installed into site-packages.  cudart is linked statically,
-cuBLASLt (the whole-layer entry point's GEMMs) dynamically from the toolkit.
+tree; nothing is installed into site-packages.  cudart is linked statically;
+no other library is linked (the tensor-map encoder is looked up in the driver
+at run time).
 """
 from __future__ import annotations
 
@@ -24,7 +25,7 @@ LIB = os.path.join(PKG, "libaxon_ssm.so")
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--use_fast_math", "-Xcompiler", "-fPIC",
               "-Xcompiler", "-fvisibility=hidden", "-shared", "-cudart", "static"]
-LINK_LIBS = ["-lcublasLt"]    # the block's plain GEMMs
+LINK_LIBS = []
 
 
 def _nvcc() -> str:

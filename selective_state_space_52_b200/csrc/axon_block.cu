@@ -4,23 +4,26 @@
 //
 // Axon-SSM page, "Gating": (x, z) = split(W_in X) and y_out = W_out (y_ssm *
 // SiLU(z)); "Selective mechanism": (dt, B, C) = f_proj(conv output), read as
-// one linear map E -> E + 2N.  The four projections are plain bf16 GEMMs with
-// float32 accumulation, run by cuBLASLt; the conv stage and the scan are this
-// library's kernels.
-#include <cublasLt.h>
+// one linear map E -> E + 2N.  The three projections are this library's
+// tcgen05 GEMM (gemm_tc.cuh): one launch writes x and z, one writes dt_raw, B
+// and C, one the output; the conv stage and the scan are this library's
+// kernels too.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 
 #include "axon_ssm.h"
 #include "conv_silu.cuh"
 #include "device_math.cuh"
+#include "gemm_tc.cuh"
 
 namespace axon {
 namespace {
 
-constexpr size_t kGemmWorkspace = size_t(32) << 20;   // cuBLASLt scratch inside the caller's workspace
 constexpr size_t kAlign = 256;
 constexpr int kMaxBlockDevices = 64;
 
@@ -32,15 +35,17 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
     return a0 < b0 + nb && b0 < a0 + na;
 }
 
-// Byte offsets of the intermediates inside the caller's workspace.
+// Byte offsets of the intermediates inside the caller's workspace; the first
+// 256 bytes hold the GEMMs' error flag.
 struct BlockPlan {
-    size_t x, z, u, dt, bm, cm, y, scan_ws, scan_ws_bytes, gemm_ws, total;
+    size_t flag, x, z, u, dt, bm, cm, y, scan_ws, scan_ws_bytes, total;
 };
 
 bool plan_block(int B, int L, int E, int N, int K, BlockPlan* p) {
     const size_t M = (size_t)B * L;
     const size_t act = round_up(M * E * 2), bc = round_up(M * N * 2);
     size_t off = 0;
+    p->flag = off; off += kAlign;
     p->x = off; off += act;
     p->z = off; off += act;
     p->u = off; off += act;
@@ -50,64 +55,80 @@ bool plan_block(int B, int L, int E, int N, int K, BlockPlan* p) {
     p->y = off; off += act;
     p->scan_ws_bytes = axon_ssm_scan_workspace_bytes(B, L, E, N, K, AXON_BF16);
     p->scan_ws = off; off += round_up(p->scan_ws_bytes);
-    p->gemm_ws = off; off += kGemmWorkspace;
     p->total = off;
     return true;
 }
 
-// One cuBLASLt handle per device, created on first use with that device current.
-std::mutex g_lt_mu;
-cublasLtHandle_t g_lt[kMaxBlockDevices] = {};
-
-axon_status lt_handle(cublasLtHandle_t* out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return AXON_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxBlockDevices) return AXON_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_lt_mu);
-    if (!g_lt[dev] && cublasLtCreate(&g_lt[dev]) != CUBLAS_STATUS_SUCCESS) {
-        g_lt[dev] = nullptr;
-        return AXON_ERR_CUDA;
-    }
-    *out = g_lt[dev];
-    return AXON_OK;
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
 }
 
-// Row-major C (M x Nc, ldc) = A (M x Kd, lda) * W (Kd x Nc, ldw), bf16 in and
-// out, float32 accumulation.  In cuBLASLt's column-major terms this is
-// C^T (Nc x M) = W^T (Nc x Kd) * A^T (Kd x M), no transposes.
-axon_status gemm_rm(cublasLtHandle_t lt, int M, int Nc, int Kd, const void* A, int lda,
-                    const void* W, int ldw, void* C, int ldc, void* ws, size_t ws_bytes,
-                    cudaStream_t st) {
-    if (M == 0 || Nc == 0) return AXON_OK;
-    cublasLtMatmulDesc_t op = nullptr;
-    cublasLtMatrixLayout_t dw = nullptr, da = nullptr, dc = nullptr;
-    cublasLtMatmulPreference_t pref = nullptr;
-    axon_status rc = AXON_ERR_CUDA;
-    const float alpha = 1.0f, beta = 0.0f;
-    cublasLtMatmulHeuristicResult_t heur{};
-    int found = 0;
-    if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS) goto done;
-    if (cublasLtMatrixLayoutCreate(&dw, CUDA_R_16BF, Nc, Kd, ldw) != CUBLAS_STATUS_SUCCESS) goto done;
-    if (cublasLtMatrixLayoutCreate(&da, CUDA_R_16BF, Kd, M, lda) != CUBLAS_STATUS_SUCCESS) goto done;
-    if (cublasLtMatrixLayoutCreate(&dc, CUDA_R_16BF, Nc, M, ldc) != CUBLAS_STATUS_SUCCESS) goto done;
-    if (cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS) goto done;
-    if (cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws_bytes,
-                                             sizeof(ws_bytes)) != CUBLAS_STATUS_SUCCESS) goto done;
-    if (cublasLtMatmulAlgoGetHeuristic(lt, op, dw, da, dc, dc, pref, 1, &heur, &found) != CUBLAS_STATUS_SUCCESS ||
-        found == 0) {
-        rc = AXON_ERR_UNSUPPORTED;
-        goto done;
+// A 2-D bf16 tensor map over a row-major (rows x cols, row stride ld
+// elements) array, boxes of box_cols x box_rows, 128-byte swizzle,
+// out-of-bounds elements read as zero.
+bool tensor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_cols,
+                uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {ld * 2};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+std::atomic<int> g_gemm_sms[kMaxBlockDevices];
+std::atomic<unsigned long long> g_gemm_smem_set{0};
+
+// Row-major outputs (M x N) = A (M x K, row stride lda) * W (K x N, row
+// stride ldw), bf16 in and out, float32 accumulation, on the tcgen05 GEMM.
+// Strides, base addresses and column splits must be 16-byte multiples.
+axon_status gemm_tc(int M, int N, int K, const void* A, int lda, const void* W, int ldw, const GemmOut* outs,
+                    int nout, int* err, cudaStream_t st) {
+    if (M == 0 || N == 0) return AXON_OK;
+    if (K == 0 || nout < 1 || nout > 3) return AXON_ERR_UNSUPPORTED;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxBlockDevices) return AXON_ERR_CUDA;
+    int sms = g_gemm_sms[dev].load(std::memory_order_relaxed);
+    if (sms <= 0) {
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            return AXON_ERR_CUDA;
+        g_gemm_sms[dev].store(sms, std::memory_order_relaxed);
     }
-    if (cublasLtMatmul(lt, op, &alpha, W, dw, A, da, &beta, C, dc, C, dc, &heur.algo, ws, ws_bytes, st) ==
-        CUBLAS_STATUS_SUCCESS)
-        rc = AXON_OK;
-done:
-    if (pref) cublasLtMatmulPreferenceDestroy(pref);
-    if (dc) cublasLtMatrixLayoutDestroy(dc);
-    if (da) cublasLtMatrixLayoutDestroy(da);
-    if (dw) cublasLtMatrixLayoutDestroy(dw);
-    if (op) cublasLtMatmulDescDestroy(op);
-    return rc;
+    const unsigned long long bit = 1ull << dev;
+    if (!(g_gemm_smem_set.load(std::memory_order_acquire) & bit)) {
+        if (cudaFuncSetAttribute(gemm_bf16_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGmSmem) !=
+            cudaSuccess)
+            return AXON_ERR_CUDA;
+        g_gemm_smem_set.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    CUtensorMap ta, tw;
+    if (!tensor_map(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)lda, kGmBK, kGmBM) ||
+        !tensor_map(&tw, W, (uint64_t)K, (uint64_t)N, (uint64_t)ldw, 64, kGmBK))
+        return AXON_ERR_CUDA;
+    GemmParams p{};
+    p.M = M; p.N = N; p.K = K;
+    p.tiles_m = (M + kGmBM - 1) / kGmBM;
+    p.tiles_n = (N + kGmBN - 1) / kGmBN;
+    p.nout = nout;
+    for (int i = 0; i < nout; ++i) p.out[i] = outs[i];
+    p.err = err;
+    const long long tiles = (long long)p.tiles_m * p.tiles_n;
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    gemm_bf16_tc_kernel<<<grid, kGmThreads, kGmSmem, st>>>(ta, tw, p);
+    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
 
 }  // namespace
@@ -166,25 +187,21 @@ axon_status axon_ssm_block_fwd(int B, int L, int Dm, int E, int N, int K, axon_d
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     unsigned char* ws = static_cast<unsigned char*>(workspace);
-    void* x = ws + plan.x;
-    void* z = ws + plan.z;
-    void* u = ws + plan.u;
-    void* dt = ws + plan.dt;
-    void* bm = ws + plan.bm;
-    void* cm = ws + plan.cm;
-    void* y = ws + plan.y;
-    void* gws = ws + plan.gemm_ws;
+    int* err = reinterpret_cast<int*>(ws + plan.flag);
+    __nv_bfloat16* x = reinterpret_cast<__nv_bfloat16*>(ws + plan.x);
+    __nv_bfloat16* z = reinterpret_cast<__nv_bfloat16*>(ws + plan.z);
+    __nv_bfloat16* u = reinterpret_cast<__nv_bfloat16*>(ws + plan.u);
+    __nv_bfloat16* dt = reinterpret_cast<__nv_bfloat16*>(ws + plan.dt);
+    __nv_bfloat16* bm = reinterpret_cast<__nv_bfloat16*>(ws + plan.bm);
+    __nv_bfloat16* cm = reinterpret_cast<__nv_bfloat16*>(ws + plan.cm);
+    __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(ws + plan.y);
     const int Mi = (int)M;
-    const unsigned char* wx = static_cast<const unsigned char*>(W_x);
-    const unsigned char* win = static_cast<const unsigned char*>(W_in);
     axon_status rc = AXON_OK;
+    if (cudaMemsetAsync(err, 0, sizeof(int), st) != cudaSuccess) return AXON_ERR_CUDA;
     if (L > 0) {
-        cublasLtHandle_t lt = nullptr;
-        if ((rc = lt_handle(&lt)) != AXON_OK) return rc;
-        // (x, z) = split(X W_in): the two column halves of W_in
-        if ((rc = gemm_rm(lt, Mi, E, Dm, X, Dm, win, 2 * E, x, E, gws, kGemmWorkspace, st)) != AXON_OK) return rc;
-        if ((rc = gemm_rm(lt, Mi, E, Dm, X, Dm, win + (size_t)E * 2, 2 * E, z, E, gws, kGemmWorkspace, st)) != AXON_OK)
-            return rc;
+        // (x, z) = split(X W_in): one GEMM over the 2E columns of W_in
+        const GemmOut xz[2] = {{x, E, 0}, {z, E, E}};
+        if ((rc = gemm_tc(Mi, 2 * E, Dm, X, Dm, W_in, 2 * E, xz, 2, err, st)) != AXON_OK) return rc;
         // u = SiLU(conv(x))
         ConvParams cp{B, L, E, x, conv_w, conv_b, conv_cache_in, u};
         const dim3 grid((unsigned)((E / 8 + kConvThreads - 1) / kConvThreads),
@@ -192,14 +209,9 @@ axon_status axon_ssm_block_fwd(int B, int L, int Dm, int E, int N, int K, axon_d
         if (grid.y > 65535u || grid.z > 65535u) return AXON_ERR_UNSUPPORTED;
         conv_silu_kernel<IoBF16><<<grid, kConvThreads, 0, st>>>(cp);
         if (cudaGetLastError() != cudaSuccess) return AXON_ERR_CUDA;
-        // (dt_raw, B, C) = split(u W_x): columns [0, E), [E, E+N), [E+N, E+2N)
-        const int ldx = E + 2 * N;
-        if ((rc = gemm_rm(lt, Mi, E, E, u, E, wx, ldx, dt, E, gws, kGemmWorkspace, st)) != AXON_OK) return rc;
-        if ((rc = gemm_rm(lt, Mi, N, E, u, E, wx + (size_t)E * 2, ldx, bm, N, gws, kGemmWorkspace, st)) != AXON_OK)
-            return rc;
-        if ((rc = gemm_rm(lt, Mi, N, E, u, E, wx + (size_t)(E + N) * 2, ldx, cm, N, gws, kGemmWorkspace, st)) !=
-            AXON_OK)
-            return rc;
+        // (dt_raw, B, C) = split(u W_x): columns [0, E), [E, E+N), [E+N, E+2N), one GEMM
+        const GemmOut dbc[3] = {{dt, E, 0}, {bm, N, E}, {cm, N, E + N}};
+        if ((rc = gemm_tc(Mi, E + 2 * N, E, u, E, W_x, E + 2 * N, dbc, 3, err, st)) != AXON_OK) return rc;
     }
     // the fused layer core: conv, SiLU, dt, recurrence, D skip, SiLU(z) gate, caches
     rc = axon_ssm_scan_fwd_segments(B, L, E, N, K, AXON_BF16, x, z, dt, bm, cm, conv_w, conv_b, dt_bias,
@@ -208,9 +220,22 @@ axon_status axon_ssm_block_fwd(int B, int L, int Dm, int E, int N, int K, axon_d
                                     stream);
     if (rc != AXON_OK || L == 0) return rc;
     // out = y W_out
-    cublasLtHandle_t lt = nullptr;
-    if ((rc = lt_handle(&lt)) != AXON_OK) return rc;
-    return gemm_rm(lt, Mi, Dm, E, y, E, W_out, Dm, out, Dm, gws, kGemmWorkspace, st);
+    const GemmOut o[1] = {{static_cast<__nv_bfloat16*>(out), Dm, 0}};
+    return gemm_tc(Mi, Dm, E, y, E, W_out, Dm, o, 1, err, st);
+}
+
+axon_status axon_gemm_bf16(int M, int N, int K, const void* A, int lda, const void* W, int ldw, void* C, int ldc,
+                           int* err, axon_stream_t stream) {
+    if (M < 0 || N < 0 || K < 0 || lda < K || ldw < N || ldc < N) return AXON_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return AXON_OK;
+    if (K == 0 || !A || !W || !C) return AXON_ERR_INVALID_ARG;
+    if (N % 8 || lda % 8 || ldw % 8 || ldc % 8 || !aligned16(A) || !aligned16(W) || !aligned16(C) ||
+        (err && (reinterpret_cast<uintptr_t>(err) & 3u)))
+        return AXON_ERR_ALIGNMENT;
+    if (overlaps(C, (size_t)M * ldc * 2, A, (size_t)M * lda * 2) || overlaps(C, (size_t)M * ldc * 2, W, (size_t)K * ldw * 2))
+        return AXON_ERR_INVALID_ARG;
+    const GemmOut o[1] = {{static_cast<__nv_bfloat16*>(C), ldc, 0}};
+    return gemm_tc(M, N, K, A, lda, W, ldw, o, 1, err, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

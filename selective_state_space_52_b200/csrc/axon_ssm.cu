@@ -210,10 +210,10 @@ axon_status launch_quad(const ChunkParams& prm, cudaStream_t st) {
 }
 
 // Split-chunk quadrant scan: W warps per 8 channels, each chunk cut into W
-// runs (R = 32 tokens per run for W = 1, else 16).
+// runs (R = 32 tokens per run for W = 1, else 8).
 template <class Io, int W, bool Z>
 axon_status launch_qsplit_t(const ChunkParams& prm, cudaStream_t st) {
-    constexpr int R = W == 1 ? 32 : 16;
+    constexpr int R = W == 1 ? 32 : 8;
     auto kern = scan_qsplit_kernel<Io, W, R, Z>;
     static std::atomic<unsigned long long> smem_set{0};
     if (!allow_max_smem(kern, smem_set)) return AXON_ERR_CUDA;
@@ -237,7 +237,7 @@ axon_status launch_qsplit(const ChunkParams& prm, int W, cudaStream_t st) {
 
 bool qsplit_fits(int B, int L, int E, int io_bytes, int W) {
     (void)B; (void)L;
-    const int R = W == 1 ? 32 : 16;
+    const int R = W == 1 ? 32 : 8;
     return (long long)(W * R + kK) * E * io_bytes < (1LL << 31) &&
            QsplitSmem(W, R, io_bytes).total <= device_max_smem_optin();
 }

@@ -16,17 +16,18 @@
 //      (dt, dt, f, f) -- f = dt*u first order, u for ZOH -- and keeps D*u and
 //      SiLU(z) of its tokens in registers;
 //   3. W > 1: a first pass from a zero state over the run keeps the R decays
-//      a = 2^(dt * A log2 e) of its 4 states in registers and yields the run's
-//      aggregate (prod a = 2^(A log2 e * sum dt), local end state H); after one
-//      CTA barrier each warp folds the aggregates of the runs before it into
-//      the chunk's entering state, h = A_j h + H_j (the intra-block pass and
+//      a = 2^(dt * A log2 e) and inputs dt*u*B of its 4 states in registers and
+//      yields the run's aggregate (prod a, local end state H); after one CTA
+//      barrier each warp folds the aggregates of the runs before it into the
+//      chunk's entering state, h = A_j h + H_j (the intra-block pass and
 //      inter-block carry of the SSD article's chunked scan, applied to the
-//      diagonal recurrence), and the second pass walks the run again from that
-//      state with the stored decays: no second exponential;
+//      diagonal recurrence), and the second pass walks the run again from
+//      that state with the stored decays and inputs: no second exponential;
 //      W == 1: one pass with the carried state, decays computed on the way;
-//   4. the partial C . h of each token (sum over the lane's quadrant) goes
-//      through shared memory to the lane that owns the token's prologue, which
-//      adds the four quadrants and stores y = (C . h + D u) SiLU(z).
+//   4. the partial C . h of each token (sum over the lane's quadrant) is summed
+//      over the four quadrants by a shuffle reduce-scatter that leaves each
+//      lane with the tokens whose prologue it ran, and the lane stores
+//      y = (C . h + D u) SiLU(z).
 // The last warp's end state is the next chunk's entering state (shared
 // memory, double buffered by chunk parity, so one barrier per chunk suffices).
 //
@@ -47,8 +48,7 @@ constexpr int kQsCh = 8;   // channels per CTA
 struct QsplitSmem {
     int xs, zs, ds, bs, cs, stage;   // one staging buffer (io dtype); two per warp
     int bf, cf;                      // float32 B, C rows of the run (bf16 io)
-    int pf;                          // (dt, dt, f, f) per (token, channel)
-    int red;                         // partial sums, one row of R + 4 floats per lane
+    int pf;                          // (dt, f) per (token, channel)
     int warp_bytes;
     int agg, entry, total;
     __host__ __device__ static int pad(int r, int RQ) { return r + r / RQ; }
@@ -66,8 +66,7 @@ struct QsplitSmem {
         off = 2 * stage;
         bf = off; off += io_bytes == 2 ? R * kN * 4 : 0;
         cf = off; off += io_bytes == 2 ? R * kN * 4 : 0;
-        pf = off; off += R * kQsCh * 16;
-        red = off; off += 32 * (R + 4) * 4;
+        pf = off; off += R * kQsCh * 8;
         warp_bytes = (off + 127) & ~127;
         off = W * warp_bytes;
         agg = off; off += W > 1 ? 2 * W * 32 * 32 : 0;       // [parity][warp][lane] (A0..3, H0..3)
@@ -78,7 +77,7 @@ struct QsplitSmem {
 
 template <class Io, int W, int R, bool kZoh>
 __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(ChunkParams p) {
-    static_assert(R % 16 == 0 && R <= 32, "R: 16 or 32 tokens per run");
+    static_assert(R == 8 || R == 16 || R == 32, "R: 8, 16 or 32 tokens per run");
     static_assert(W == 1 || W == 2 || W == 4 || W == 8, "W: 1, 2, 4 or 8 runs per chunk");
     using TT = typename Io::T;
     using SI = SmemIo<Io>;
@@ -235,8 +234,7 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
     // y of token (chunk start) + w*R + g*RQ + j, channel e: ybase + (t0 + j) * row_bytes
     unsigned char* ybase = static_cast<unsigned char*>(p.y) + tile_off + (size_t)(w * R + g * RQ) * row_bytes + c * S;
     const int nck = (p.L + T - 1) / T;
-    float4* pf = reinterpret_cast<float4*>(ws + lay.pf);          // [token][channel] (dt, dt, f, f)
-    float* red = reinterpret_cast<float*>(ws + lay.red);          // [lane][token] partial C . h
+    float2* pf = reinterpret_cast<float2*>(ws + lay.pf);          // [token][channel] (dt, f)
     const float* bfs = reinterpret_cast<const float*>(ws + lay.bf);
     const float* cfs = reinterpret_cast<const float*>(ws + lay.cf);
 
@@ -313,7 +311,7 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
                 const bool live = full || tr + t < p.L;
                 const float dtl = live ? dt : 0.0f;        // dt = 0: decay 1, no input
                 const float f = live ? (kZoh ? u : dt * u) : 0.0f;
-                pf[t * kQsCh + c] = make_float4(dtl, dtl, f, f);
+                pf[t * kQsCh + c] = make_float2(dtl, f);
                 Du[i] = Dv * u;
                 gz[i] = silu(SI::ld(sb + lay.zs + tp * XB + c * S));
             }
@@ -330,14 +328,15 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int t = tb + i;
-                    const float4 v = pf[t * kQsCh + c];
+                    const float2 v = pf[t * kQsCh + c];
                     const float4 Bq = bq(sb, t);
-                    const float2 arg01 = __fmul2_rn(f2(v.x, v.y), s01);
-                    const float2 arg23 = __fmul2_rn(f2(v.x, v.y), s23);
+                    const float2 dd = f2(v.x, v.x), ff = f2(v.y, v.y);
+                    const float2 arg01 = __fmul2_rn(dd, s01);
+                    const float2 arg23 = __fmul2_rn(dd, s23);
                     a01[i] = f2(ex2_approx(arg01.x), ex2_approx(arg01.y));
                     a23[i] = f2(ex2_approx(arg23.x), ex2_approx(arg23.y));
-                    u01[i] = __fmul2_rn(f2(v.z, v.w), f2(Bq.x, Bq.y));
-                    u23[i] = __fmul2_rn(f2(v.z, v.w), f2(Bq.z, Bq.w));
+                    u01[i] = __fmul2_rn(ff, f2(Bq.x, Bq.y));
+                    u23[i] = __fmul2_rn(ff, f2(Bq.z, Bq.w));
                     if constexpr (kZoh) {
                         float2 z01, z23;
                         zoh4(v.x, a01[i], a23[i], z01, z23);
@@ -356,38 +355,37 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
                 }
             }
         } else {
-            // ---- first pass: the run from a zero state; keep the decays
-            float2 a01[R], a23[R];
+            // ---- first pass: the run from a zero state; keep decays and inputs
+            float2 a01[R], a23[R], u01[R], u23[R];
             float2 H01 = f2(0.f, 0.f), H23 = f2(0.f, 0.f);
-            float dsum = 0.f;
+            float2 P01 = f2(1.f, 1.f), P23 = f2(1.f, 1.f);
 #pragma unroll
             for (int t = 0; t < R; ++t) {
-                const float4 v = pf[t * kQsCh + c];
+                const float2 v = pf[t * kQsCh + c];
                 const float4 Bq = bq(sb, t);
-                const float2 arg01 = __fmul2_rn(f2(v.x, v.y), s01);
-                const float2 arg23 = __fmul2_rn(f2(v.x, v.y), s23);
+                const float2 dd = f2(v.x, v.x), ff = f2(v.y, v.y);
+                const float2 arg01 = __fmul2_rn(dd, s01);
+                const float2 arg23 = __fmul2_rn(dd, s23);
                 a01[t] = f2(ex2_approx(arg01.x), ex2_approx(arg01.y));
                 a23[t] = f2(ex2_approx(arg23.x), ex2_approx(arg23.y));
-                float2 u01 = __fmul2_rn(f2(v.z, v.w), f2(Bq.x, Bq.y));
-                float2 u23 = __fmul2_rn(f2(v.z, v.w), f2(Bq.z, Bq.w));
+                u01[t] = __fmul2_rn(ff, f2(Bq.x, Bq.y));
+                u23[t] = __fmul2_rn(ff, f2(Bq.z, Bq.w));
                 if constexpr (kZoh) {
                     float2 z01, z23;
                     zoh4(v.x, a01[t], a23[t], z01, z23);
-                    u01 = __fmul2_rn(u01, z01);
-                    u23 = __fmul2_rn(u23, z23);
+                    u01[t] = __fmul2_rn(u01[t], z01);
+                    u23[t] = __fmul2_rn(u23[t], z23);
                 }
-                H01 = __ffma2_rn(a01[t], H01, u01);
-                H23 = __ffma2_rn(a23[t], H23, u23);
-                dsum += v.x;
+                H01 = __ffma2_rn(a01[t], H01, u01[t]);
+                H23 = __ffma2_rn(a23[t], H23, u23[t]);
+                P01 = __fmul2_rn(P01, a01[t]);
+                P23 = __fmul2_rn(P23, a23[t]);
             }
-            // the run's aggregate: prod_t a_t = 2^(A log2 e * sum_t dt_t)
+            // the run's aggregate (prod a, H) for the other warps
             {
-                const float2 q01 = __fmul2_rn(f2(dsum, dsum), s01);
-                const float2 q23 = __fmul2_rn(f2(dsum, dsum), s23);
-                float2* slot = agg + ((k & 1) * W + w) * 32 * 4 + lane * 4;
-                reinterpret_cast<float4*>(slot)[0] =
-                    make_float4(ex2_approx(q01.x), ex2_approx(q01.y), ex2_approx(q23.x), ex2_approx(q23.y));
-                reinterpret_cast<float4*>(slot)[1] = make_float4(H01.x, H01.y, H23.x, H23.y);
+                float4* slot = reinterpret_cast<float4*>(agg + ((k & 1) * W + w) * 32 * 4 + lane * 4);
+                slot[0] = make_float4(P01.x, P01.y, P23.x, P23.y);
+                slot[1] = make_float4(H01.x, H01.y, H23.x, H23.y);
             }
             __syncthreads();                 // every run's aggregate of chunk k is written
             // ---- the state entering this run: the chunk's entering state (the
@@ -406,44 +404,34 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
             // ---- second pass: the run again from its true entering state
 #pragma unroll
             for (int t = 0; t < R; ++t) {
-                const float4 v = pf[t * kQsCh + c];
-                const float4 Bq = bq(sb, t);
-                float2 u01 = __fmul2_rn(f2(v.z, v.w), f2(Bq.x, Bq.y));
-                float2 u23 = __fmul2_rn(f2(v.z, v.w), f2(Bq.z, Bq.w));
-                if constexpr (kZoh) {
-                    float2 z01, z23;
-                    zoh4(v.x, a01[t], a23[t], z01, z23);
-                    u01 = __fmul2_rn(u01, z01);
-                    u23 = __fmul2_rn(u23, z23);
-                }
                 const float4 Cq = cq(sb, t);
-                h01 = __ffma2_rn(a01[t], h01, u01);
-                h23 = __ffma2_rn(a23[t], h23, u23);
+                h01 = __ffma2_rn(a01[t], h01, u01[t]);
+                h23 = __ffma2_rn(a23[t], h23, u23[t]);
                 const float2 pq = __ffma2_rn(f2(Cq.z, Cq.w), h23, __fmul2_rn(f2(Cq.x, Cq.y), h01));
                 part[t] = pq.x + pq.y;
             }
             if (w == W - 1) entry[((k + 1) & 1) * 32 + lane] = make_float4(h01.x, h01.y, h23.x, h23.y);
         }
 
-        // ---- sum the four quadrants' partials of each token: lane (g, c)
-        // gets those of tokens g*RQ .. g*RQ + RQ - 1 of channel c
+        // ---- reduce-scatter of the quadrant partials over lanes 16 and 8
+        // apart: quadrants {0, 1} keep the first half of the run's tokens and
+        // {2, 3} the second, then each quadrant keeps its own R/4 tokens, so
+        // lane (g, c) ends with the totals of tokens g*RQ .. g*RQ + RQ - 1
         {
-            float* mine = red + lane * (R + 4);
+            const bool hi = (g & 2) != 0, lo = (g & 1) != 0;
+            float half[R / 2];
 #pragma unroll
-            for (int t = 0; t < R; t += 4)
-                *reinterpret_cast<float4*>(mine + t) = make_float4(part[t], part[t + 1], part[t + 2], part[t + 3]);
-            __syncwarp();
+            for (int i = 0; i < R / 2; ++i) {
+                const float keep = hi ? part[R / 2 + i] : part[i];
+                const float send = hi ? part[i] : part[R / 2 + i];
+                half[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+            }
             float tot[RQ];
 #pragma unroll
-            for (int j = 0; j < RQ; ++j) tot[j] = 0.f;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float* src = red + (8 * q + c) * (R + 4) + g * RQ;
-#pragma unroll
-                for (int j = 0; j < RQ; j += 4) {
-                    const float4 v = *reinterpret_cast<const float4*>(src + j);
-                    tot[j] += v.x; tot[j + 1] += v.y; tot[j + 2] += v.z; tot[j + 3] += v.w;
-                }
+            for (int j = 0; j < RQ; ++j) {
+                const float keep = lo ? half[RQ + j] : half[j];
+                const float send = lo ? half[j] : half[RQ + j];
+                tot[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
             }
             unsigned char* yrow = ybase + (size_t)t0 * row_bytes;
 #pragma unroll

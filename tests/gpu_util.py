@@ -71,7 +71,8 @@ def to_dev(inp: dict, device="cuda") -> dict:
     return {k: (v.to(device).contiguous() if v is not None else None) for k, v in inp.items()}
 
 
-def run_gpu_scan(inp_cpu: dict, num_segments=None, with_state=True, guarded=True):
+def run_gpu_scan(inp_cpu: dict, num_segments=None, with_state=True, guarded=True, runs=None,
+                 discretization="first_order"):
     """Run the CUDA prefill on `inp_cpu` (a workloads dict); returns numpy outputs."""
     d = to_dev(inp_cpu)
     x = d["x"]
@@ -84,7 +85,8 @@ def run_gpu_scan(inp_cpu: dict, num_segments=None, with_state=True, guarded=True
     gcc = Guarded((Bsz, K - 1, E), x.dtype)
     gss = Guarded((Bsz, E, N), torch.float32)
     y, (cc, ss) = axon_ssm.scan_fwd(d["x"], d["z"], d["dt_raw"], d["B"], d["C"], params, cache,
-                                    num_segments=num_segments, out=(gy.t, gcc.t, gss.t))
+                                    num_segments=num_segments, out=(gy.t, gcc.t, gss.t), runs=runs,
+                                    discretization=discretization)
     torch.cuda.synchronize()
     if guarded:
         for g, name in ((gy, "y"), (gcc, "conv_cache"), (gss, "ssm_state")):
@@ -92,17 +94,19 @@ def run_gpu_scan(inp_cpu: dict, num_segments=None, with_state=True, guarded=True
     return (y.float().cpu().numpy(), cc.cpu(), ss.cpu().numpy())
 
 
-def oracle_scan(inp_cpu: dict, with_state=True):
+def oracle_scan(inp_cpu: dict, with_state=True, zoh=False):
     cc = inp_cpu.get("conv_cache") if with_state else None
     ss = inp_cpu.get("ssm_state") if with_state else None
     return oracle.scan_fwd(inp_cpu["x"], inp_cpu["z"], inp_cpu["dt_raw"], inp_cpu["B"],
                            inp_cpu["C"], inp_cpu["conv_w"], inp_cpu["conv_b"],
-                           inp_cpu["dt_bias"], inp_cpu["A_log"], inp_cpu["D"], cc, ss)
+                           inp_cpu["dt_bias"], inp_cpu["A_log"], inp_cpu["D"], cc, ss, zoh=zoh)
 
 
-def compare_scan(inp_cpu: dict, io: str, num_segments=None, with_state=True, what=""):
-    y, cc, ss = run_gpu_scan(inp_cpu, num_segments=num_segments, with_state=with_state)
-    y_ref, cc_ref, ss_ref = oracle_scan(inp_cpu, with_state=with_state)
+def compare_scan(inp_cpu: dict, io: str, num_segments=None, with_state=True, what="", runs=None,
+                 zoh=False):
+    y, cc, ss = run_gpu_scan(inp_cpu, num_segments=num_segments, with_state=with_state, runs=runs,
+                             discretization="zoh" if zoh else "first_order")
+    y_ref, cc_ref, ss_ref = oracle_scan(inp_cpu, with_state=with_state, zoh=zoh)
     stats = check_close(y, y_ref, tol_for(io, y_ref), what + " y")
     check_close(ss, ss_ref, state_tol(ss_ref), what + " ssm_state")
     # conv cache: bit-exact copy of raw inputs

@@ -235,7 +235,7 @@ def test_block_workspace_query(lib):
     q.restype = ctypes.c_size_t
     q.argtypes = [ctypes.c_int] * 7
     need = q(1, 2048, 2560, 7680, 16, 4, 1)
-    assert need >= 5 * 2048 * 7680 * 2 + (32 << 20)      # five (M, E) bf16 intermediates + GEMM scratch
+    assert need >= 5 * 2048 * 7680 * 2 + 2 * 2048 * 16 * 2   # x, z, u, dt_raw, y (M, E) and B, C (M, N) in bf16
     assert q(1, 2048, 2560, 7680, 16, 4, 0) == 0          # fp32 io: not supported
     assert _block(lib, ws_bytes=need - 1, L=2048, Dm=2560, E=7680) == WORKSPACE
 

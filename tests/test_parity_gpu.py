@@ -281,3 +281,44 @@ def test_step_matches_oracle_step(cuda_lib, io):
     check_close(y.float().cpu().numpy(), y_ref, tol_for(io, y_ref), "step y")
     check_close(ss.cpu().numpy(), ss_ref, state_tol(ss_ref), "step state")
     assert torch.equal(cc.cpu(), torch.from_numpy(cc_ref).to(cc.dtype))
+
+
+# The split-chunk quadrant scan with each number of runs per chunk (W warps per
+# 8 channels; W = 1: runs of 32 tokens, else 16): single tokens, ragged runs
+# and chunks, chunks whose last runs lie wholly past L, several batch rows, an
+# fp32 tail tile (E % 8 == 4), both discretisations.
+QSPLIT_SHAPES = [(1, 64, 1), (1, 64, 17), (2, 40, 100), (1, 2048, 300), (3, 24, 515), (1, 16, 2049)]
+
+
+@pytest.mark.parametrize("zoh", [False, True])
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("runs", [1, 2, 4, 8])
+@pytest.mark.parametrize("B,E,L", QSPLIT_SHAPES)
+def test_split_chunk_scan_shapes(cuda_lib, runs, io, zoh, B, E, L):
+    wl = W.custom(B, L, E, io=io, seed=5100 + 3 * E + L + runs)
+    inp = W.make_inputs(wl, with_state=True)
+    compare_scan(inp, io, with_state=(L % 2 == 1), runs=runs, zoh=zoh,
+                 what=f"qsplit W{runs} B{B} E{E} L{L} {io} zoh={zoh}")
+
+
+@pytest.mark.parametrize("runs", [1, 2, 8])
+def test_split_chunk_scan_fp32_tail_tile(cuda_lib, runs):
+    inp = W.make_inputs(W.custom(2, 77, 36, io="f32", seed=5200 + runs), with_state=True)
+    compare_scan(inp, "f32", runs=runs, what=f"qsplit tail W{runs}")
+
+
+@pytest.mark.parametrize("runs", [1, 4])
+def test_split_chunk_scan_in_place_caches(cuda_lib, runs):
+    from selective_state_space_52_b200 import axon_ssm
+    inp = W.make_inputs(W.custom(1, 333, 64, io="bf16", seed=5300 + runs), with_state=True)
+    d = to_dev(inp)
+    params = {k: d[k] for k in axon_ssm.PARAM_KEYS}
+    cc, ss = d["conv_cache"].clone(), d["ssm_state"].clone()
+    y = torch.empty_like(d["x"])
+    axon_ssm.scan_fwd(d["x"], d["z"], d["dt_raw"], d["B"], d["C"], params, (cc, ss), out=(y, cc, ss),
+                      runs=runs)
+    torch.cuda.synchronize()
+    y_ref, cc_ref, ss_ref = oracle_scan(inp)
+    check_close(y.float().cpu().numpy(), y_ref, tol_for("bf16", y_ref), "qsplit in-place y")
+    check_close(ss.cpu().numpy(), ss_ref, state_tol(ss_ref), "qsplit in-place state")
+    assert torch.equal(cc.cpu(), torch.from_numpy(cc_ref).to(cc.dtype))
