@@ -136,10 +136,11 @@ def step_model(wl) -> dict:
 # translation unit that plans and launches it.  A committed ncu figure counts
 # only while these files are unchanged.
 KERNEL_SOURCES = {
-    "scan": ("axon_ssm.cu", "device_math.cuh", "scan_chunked.cuh", "scan_octo.cuh", "scan_quad.cuh",
-             "scan_seq.cuh"),
+    "scan": ("axon_ssm.cu", "device_math.cuh", "scan_chunked.cuh", "scan_octo.cuh", "scan_qsplit.cuh",
+             "scan_quad.cuh", "scan_seq.cuh"),
     "step": ("axon_ssm.cu", "device_math.cuh", "step.cuh"),
-    "ssd": ("axon_ssd.cu", "device_math.cuh", "scan_chunked.cuh", "ssd.cuh"),
+    "ssd": ("axon_ssd.cu", "device_math.cuh", "scan_chunked.cuh", "ssd.cuh", "tc_ops.cuh"),
+    "gemm": ("axon_block.cu", "gemm_tc.cuh", "tc_ops.cuh"),
 }
 
 

@@ -90,11 +90,36 @@ bool tensor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, 
 }
 
 std::atomic<int> g_gemm_sms[kMaxBlockDevices];
-std::atomic<unsigned long long> g_gemm_smem_set{0};
+std::atomic<unsigned long long> g_gemm_smem_set[2];
+
+template <int BN>
+axon_status launch_gemm(int M, int N, int K, const CUtensorMap& ta, const void* W, int ldw, GemmParams p, int sms,
+                        cudaStream_t st) {
+    using Cfg = GemmCfg<BN>;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxBlockDevices) return AXON_ERR_CUDA;
+    const unsigned long long bit = 1ull << dev;
+    std::atomic<unsigned long long>& set = g_gemm_smem_set[BN == 256 ? 0 : 1];
+    if (!(set.load(std::memory_order_acquire) & bit)) {
+        if (cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
+            cudaSuccess)
+            return AXON_ERR_CUDA;
+        set.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    CUtensorMap tw;
+    if (!tensor_map(&tw, W, (uint64_t)K, (uint64_t)N, (uint64_t)ldw, 64, kGmBK)) return AXON_ERR_CUDA;
+    p.tiles_m = (M + kGmBM - 1) / kGmBM;
+    p.tiles_n = (N + BN - 1) / BN;
+    const long long tiles = (long long)p.tiles_m * p.tiles_n;
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    gemm_bf16_tc_kernel<BN><<<grid, kGmThreads, Cfg::kSmem, st>>>(ta, tw, p);
+    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+}
 
 // Row-major outputs (M x N) = A (M x K, row stride lda) * W (K x N, row
-// stride ldw), bf16 in and out, float32 accumulation, on the tcgen05 GEMM.
-// Strides, base addresses and column splits must be 16-byte multiples.
+// stride ldw), bf16 in and out, float32 accumulation, on the tcgen05 GEMM
+// (128 x 256 tiles).  Strides, base addresses and column splits must be
+// 16-byte multiples.
 axon_status gemm_tc(int M, int N, int K, const void* A, int lda, const void* W, int ldw, const GemmOut* outs,
                     int nout, int* err, cudaStream_t st) {
     if (M == 0 || N == 0) return AXON_OK;
@@ -107,28 +132,14 @@ axon_status gemm_tc(int M, int N, int K, const void* A, int lda, const void* W, 
             return AXON_ERR_CUDA;
         g_gemm_sms[dev].store(sms, std::memory_order_relaxed);
     }
-    const unsigned long long bit = 1ull << dev;
-    if (!(g_gemm_smem_set.load(std::memory_order_acquire) & bit)) {
-        if (cudaFuncSetAttribute(gemm_bf16_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGmSmem) !=
-            cudaSuccess)
-            return AXON_ERR_CUDA;
-        g_gemm_smem_set.fetch_or(bit, std::memory_order_acq_rel);
-    }
-    CUtensorMap ta, tw;
-    if (!tensor_map(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)lda, kGmBK, kGmBM) ||
-        !tensor_map(&tw, W, (uint64_t)K, (uint64_t)N, (uint64_t)ldw, 64, kGmBK))
-        return AXON_ERR_CUDA;
+    CUtensorMap ta;
+    if (!tensor_map(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)lda, kGmBK, kGmBM)) return AXON_ERR_CUDA;
     GemmParams p{};
     p.M = M; p.N = N; p.K = K;
-    p.tiles_m = (M + kGmBM - 1) / kGmBM;
-    p.tiles_n = (N + kGmBN - 1) / kGmBN;
     p.nout = nout;
     for (int i = 0; i < nout; ++i) p.out[i] = outs[i];
     p.err = err;
-    const long long tiles = (long long)p.tiles_m * p.tiles_n;
-    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    gemm_bf16_tc_kernel<<<grid, kGmThreads, kGmSmem, st>>>(ta, tw, p);
-    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+    return launch_gemm<256>(M, N, K, ta, W, ldw, p, sms, st);
 }
 
 }  // namespace

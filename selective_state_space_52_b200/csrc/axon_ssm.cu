@@ -242,6 +242,22 @@ bool qsplit_fits(int B, int L, int E, int io_bytes, int W) {
            QsplitSmem(W, R, io_bytes).total <= device_max_smem_optin();
 }
 
+// Runs per chunk of the split-chunk quadrant scan for an unsplit first-order
+// prefill, or 0 where another kernel is faster.  Measured on B200 (prefill
+// time against the eighths / quadrant scans and the run-split chunked
+// kernel): eight runs per chunk win below about 20 channels per SM (where
+// the CTAs of 8 channels alone leave the SMs nearly idle), one run per chunk
+// from 48 to 511 channels per SM; the eighths scan keeps 20 to 47, and the
+// one-thread-per-channel walk 512 and up.
+int plan_qsplit(int B, int L, int E, int io_bytes, int sms) {
+    const long long channels = (long long)B * E;
+    int W = 0;
+    if (channels < (long long)sms * 20) W = 8;
+    else if (channels >= (long long)sms * 48 && channels < (long long)sms * 512) W = 1;
+    if (W == 0 || device_max_smem_optin() <= 0 || !qsplit_fits(B, L, E, io_bytes, W)) return 0;
+    return W;
+}
+
 template <class Io, int W, int R, bool Z>
 axon_status launch_chunked_t(const ChunkParams& prm, int smem, cudaStream_t st) {
     auto kern = scan_chunked_kernel<Io, W, R, Z>;
@@ -347,6 +363,8 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
             if (sms <= 0) return AXON_ERR_CUDA;
             if (num_segments == 0 && use_time_split(B, L, E, sms)) {
                 P = plan_segments(B, L, E, sms);
+            } else if (!zoh && (qsplit = plan_qsplit(B, L, E, (int)io_bytes(io), sms)) > 0) {
+                // the split-chunk quadrant scan (first order)
             } else if (use_quad(B, E, (int)io_bytes(io), sms, zoh)) {
                 quad = true;                   // unsplit: the quadrant scan
             } else if (use_octo(B, E, (int)io_bytes(io), sms, zoh)) {

@@ -4,19 +4,20 @@
 // output projections; "Selective mechanism": f_proj, one linear map of the
 // conv output).
 //
-// Persistent, warp-specialised, one CTA per SM (192 threads):
+// Persistent, warp-specialised, one CTA per SM (192 threads), output tiles of
+// 128 x BN (the layer uses BN = 256; 128-column tiles measured slower):
 //   warp 0 (one thread)  TMA producer: per 64-deep K block, the A tile
-//                        (128 rows x 64, K-major) and the W tile (64 x 256,
-//                        N-major, four 64-column boxes), 128-byte swizzle,
-//                        into a ring of kGmStages shared-memory stages;
-//   warp 1 (one thread)  MMA issuer: four tcgen05.mma (M 128, N 256, K 16)
-//                        per stage into one of two float32 accumulators in
-//                        tensor memory (2 x 256 columns); each stage is handed
-//                        back to the producer by a tcgen05.commit;
+//                        (128 rows x 64, K-major) and the W tile (64 x BN,
+//                        N-major, 64-column boxes), 128-byte swizzle, into a
+//                        ring of shared-memory stages (4 for BN 256, 6 for 128);
+//   warp 1 (one thread)  MMA issuer: four tcgen05.mma (M 128, N BN, K 16)
+//                        per stage into one of 512 / BN float32 accumulators
+//                        in tensor memory; each stage is handed back to the
+//                        producer by a tcgen05.commit;
 //   warps 2-5            epilogue: tensor memory -> registers (thread = row)
 //                        -> bf16, stored straight to global memory, while the
 //                        MMA issuer fills the other accumulator.
-// Output tiles (128 x 256) go round-robin over the CTAs, M fastest, so the
+// Output tiles go round-robin over the CTAs, M fastest, so the
 // CTAs running at once share W tiles in L2.  The output columns may be split
 // over up to three row-major destinations (columns [c_k, c_{k+1}) go to
 // destination k at column - c_k), so one GEMM writes x and z, or dt_raw, B
@@ -33,15 +34,21 @@
 namespace axon {
 
 constexpr int kGmBM = 128;          // rows of an output tile (the MMA's M)
-constexpr int kGmBN = 256;          // columns of an output tile (the MMA's N)
 constexpr int kGmBK = 64;           // K per stage: one 128-byte swizzle row of bf16
-constexpr int kGmStages = 4;
 constexpr int kGmThreads = 192;
 constexpr int kGmABytes = kGmBM * kGmBK * 2;          // 16 KB
-constexpr int kGmBBytes = kGmBK * kGmBN * 2;          // 32 KB
-constexpr int kGmStageBytes = kGmABytes + kGmBBytes;
-constexpr int kGmBarOff = kGmStages * kGmStageBytes;  // mbarriers after the stages
-constexpr int kGmSmem = kGmBarOff + 256 + 1024;       // + barriers, slot, flag + alignment pad
+
+// Shared-memory plan for output tiles of BN columns (the MMA's N): as many
+// stages of (A 16 KB + W BN x 128 bytes) as fit, then the mbarriers.
+template <int BN>
+struct GemmCfg {
+    static constexpr int kBBytes = kGmBK * BN * 2;
+    static constexpr int kStageBytes = kGmABytes + kBBytes;
+    static constexpr int kStages = BN == 256 ? 4 : 6;
+    static constexpr int kAccs = 512 / BN;            // tensor-memory accumulators (512 columns)
+    static constexpr int kBarOff = kStages * kStageBytes;
+    static constexpr int kSmem = kBarOff + 256 + 1024;  // + barriers, slot, flags + alignment pad
+};
 
 struct GemmOut {
     __nv_bfloat16* ptr;   // row-major destination
@@ -57,9 +64,13 @@ struct GemmParams {
     int* err;             // set to 1 when a wait gave up (may be null)
 };
 
+template <int kGmBN>
 __global__ void __launch_bounds__(kGmThreads, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                         GemmParams p) {
+    using Cfg = GemmCfg<kGmBN>;
+    constexpr int kGmStages = Cfg::kStages, kGmStageBytes = Cfg::kStageBytes, kGmBarOff = Cfg::kBarOff;
+    constexpr int kAccs = Cfg::kAccs;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;   // swizzled tiles want 1024-byte alignment
@@ -70,10 +81,10 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     auto full = [&](int s) { return bar + 8u * s; };                       // stage loaded
     auto empty = [&](int s) { return bar + 8u * (kGmStages + s); };        // stage consumed
     auto tfull = [&](int a) { return bar + 8u * (2 * kGmStages + a); };    // accumulator ready
-    auto tempty = [&](int a) { return bar + 8u * (2 * kGmStages + 2 + a); };  // accumulator drained
-    const uint32_t drain = bar + 8u * (2 * kGmStages + 4);
-    const uint32_t slot = bar + 8u * (2 * kGmStages + 5);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kGmBarOff + 8 * (2 * kGmStages + 6));
+    auto tempty = [&](int a) { return bar + 8u * (2 * kGmStages + kAccs + a); };  // accumulator drained
+    const uint32_t drain = bar + 8u * (2 * kGmStages + 2 * kAccs);
+    const uint32_t slot = bar + 8u * (2 * kGmStages + 2 * kAccs + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kGmBarOff + 8 * (2 * kGmStages + 2 * kAccs + 2));
     volatile int* drained = abort_flag + 1;     // set once every issued product has finished
 
     if (threadIdx.x == 0) {
@@ -81,7 +92,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             mbar_init(full(s), 1);
             mbar_init(empty(s), 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < kAccs; ++a) {
             mbar_init(tfull(a), 1);
             mbar_init(tempty(a), 4);             // one arrival per epilogue warp
         }
@@ -94,7 +105,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(sm + kGmBarOff + 8 * (2 * kGmStages + 5));
+    const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(sm + kGmBarOff + 8 * (2 * kGmStages + 2 * kAccs + 1));
 
     const int ntiles = p.tiles_m * p.tiles_n;
     const int kblocks = (p.K + kGmBK - 1) / kGmBK;
@@ -157,7 +168,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                 }
                 if (!ok) { fail(); break; }
                 umma_commit(tfull(a));               // the accumulator is complete
-                if (++a == 2) { a = 0; aph ^= 1u; }
+                if (++a == kAccs) { a = 0; aph ^= 1u; }
             }
             // every product issued has finished before the tensor memory is freed
             umma_commit(drain);
@@ -201,7 +212,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty(a));   // the MMA issuer may refill this accumulator
-            if (++a == 2) { a = 0; aph ^= 1u; }
+            if (++a == kAccs) { a = 0; aph ^= 1u; }
         }
     }
 

@@ -39,7 +39,7 @@ __device__ __forceinline__ void step_cp_async16(void* smem_dst, const void* gmem
 
 constexpr int kStepThreads = 128;  // 32 channels x 4 lanes
 constexpr int kStepChan = kStepThreads / 4;
-constexpr int kStepStages = 8;     // state rows in flight per lane (shared-memory ring)
+constexpr int kStepStages = 4;     // state rows in flight per lane (shared-memory ring)
 constexpr int kStepMaxRows = 32;   // batch rows per block
 
 // grid = (ceil(E / 32), ceil(B / rows)) blocks of 128 threads, rows <= 32.

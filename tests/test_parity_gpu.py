@@ -42,22 +42,22 @@ def test_chunked_kernel_small_shapes(cuda_lib, io, B, E, L):
     compare_scan(inp, io, num_segments=1, with_state=(L % 2 == 1), what=f"chunked B{B} L{L} E{E} {io}")
 
 
-# Shapes that steer the planner to each unsplit kernel on a 148-SM B200: the
-# run-split chunked kernel below 8 channels per SM (channels per tile ET =
-# ceil(E / (148 / B)), W the largest of 32/16/8 with ET*W <= 512 whose shared
-# memory fits, partial last tiles when E % ET != 0), the eighths scan from 8
-# to 47 channels per SM (to 127 with exact ZOH), the quadrant scan from 48 to
-# 511 (first order; from 128 with ZOH), the direct walk above.
+# Shapes that steer the first-order planner to each unsplit kernel on a
+# 148-SM B200: the split-chunk quadrant scan with 8 runs per chunk below 20
+# channels per SM, the eighths scan from 20 to 47, the split-chunk scan with
+# one run per chunk from 48 to 511, the direct walk (one thread per channel)
+# above.  (The exact-ZOH planner keeps the eighths / quadrant / run-split
+# chunked kernels; tests/test_zoh_gpu.py covers it.)
 PLANNER_SHAPES = [
-    (1, 1000, 300),     # ET 7, partial last tile, W 16
-    (1, 7680, 200),     # 52 channels per SM: quadrant scan
+    (1, 1000, 300),     # 6.8 channels per SM, fp32 tail tile: split-chunk, 8 runs
+    (1, 7680, 200),     # 52 channels per SM: split-chunk, 1 run
     (2, 2048, 300),     # 28 channels per SM: eighths scan
-    (1, 1096, 200),     # ET 8, W 32
-    (1, 1600, 200),     # 10.8 channels per SM: eighths scan
-    (1, 14800, 100),    # 100 channels per SM: quadrant scan
-    (1, 29600, 40),     # 200 channels per SM: quadrant scan
-    (8, 4800, 40),      # 259 channels per SM: quadrant scan
-    (16, 4800, 24),     # 519 channels per SM: direct walk, W 1
+    (1, 1096, 200),     # 7.4 channels per SM: split-chunk, 8 runs
+    (1, 1600, 200),     # 10.8 channels per SM: split-chunk, 8 runs
+    (1, 14800, 100),    # 100 channels per SM: split-chunk, 1 run
+    (1, 29600, 40),     # 200 channels per SM: split-chunk, 1 run
+    (8, 4800, 40),      # 259 channels per SM: split-chunk, 1 run
+    (16, 4800, 24),     # 519 channels per SM: direct walk
 ]
 
 
