@@ -578,6 +578,49 @@ def bench_prefill_workload(wl, dev, launches: int = 20) -> dict:
                     "over the MUFU peak"}
 
 
+def run_single_kernel(args, wl, dev) -> dict:
+    """The prefill of `wl` (library plan) or one projection GEMM, 3 warm-up
+    calls and one timed call: a short program for profiling one kernel."""
+    from selective_state_space_52_b200 import axon_ssm
+    stream = torch.cuda.current_stream(dev)
+    if args.gemm_only:
+        M, N, K = (int(v) for v in args.gemm_only.split(","))
+        g = torch.Generator().manual_seed(M + N + K)
+        A = torch.randn(M, K, generator=g).to(torch.bfloat16).to(dev)
+        Wt = (torch.randn(K, N, generator=g) / K ** 0.5).to(torch.bfloat16).to(dev)
+        C = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+
+        def call():
+            axon_ssm.gemm_bf16(A, Wt, out=C, check=False)
+        what = {"kernel": "axon_gemm_bf16", "M": M, "N": N, "K": K}
+        flops = 2 * M * N * K
+    else:
+        inp = {k: v.to(dev) for k, v in W.make_inputs(wl).items()}
+        params = {k: inp[k] for k in axon_ssm.PARAM_KEYS}
+        out = (torch.empty_like(inp["x"]), torch.empty(wl.B, wl.K - 1, wl.E, dtype=wl.torch_io, device=dev),
+               torch.empty(wl.B, wl.E, wl.N, dtype=torch.float32, device=dev))
+        io_code = axon_ssm.AXON_BF16 if wl.io == "bf16" else axon_ssm.AXON_F32
+        ws = torch.empty(max(axon_ssm.axon_ssm_scan_workspace_bytes(wl.B, wl.L, wl.E, wl.N, wl.K, io_code), 16),
+                         dtype=torch.uint8, device=dev)
+
+        def call():
+            axon_ssm.scan_fwd(inp["x"], inp["z"], inp["dt_raw"], inp["B"], inp["C"], params, None, out=out,
+                              workspace=ws)
+        what = {"kernel": "prefill", "workload": workload_desc(wl)}
+        flops = None
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream); call(); b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b)
+    what["us"] = ms * 1e3
+    if flops:
+        what["tflops"] = flops / (ms / 1e3) / 1e12
+    return what
+
+
 def workload_desc(wl) -> str:
     return (f"{wl.name}: B{wl.B} L{wl.L} E{wl.E} N{wl.N} K{wl.K}, {wl.io} io, fp32 state; "
             "step = prefill + 1 cached decode token")
@@ -794,6 +837,12 @@ def main(argv=None):
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the cached-decode measurement and print it as one JSON line "
                          "(for profiling the step kernel alone)")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="run only the workload's prefill (library plan): 3 warm-up calls and one timed call, "
+                         "printed as one JSON line (for profiling the prefill kernel alone)")
+    ap.add_argument("--gemm-only", default=None, metavar="M,N,K",
+                    help="run only the projection GEMM (axon_gemm_bf16) on random bf16 operands of this shape: "
+                         "3 warm-up calls and one timed call (for profiling it alone)")
     ap.add_argument("--ssd-only", action="store_true",
                     help="run only the Mamba-2 (SSD) layer-core measurement and print it as one JSON line "
                          "(for profiling its kernels alone)")
@@ -808,6 +857,13 @@ def main(argv=None):
         dev = torch.device("cuda", 0)
         torch.cuda.set_device(dev)
         print(json.dumps({"decode": bench_decode(dev)}), flush=True)
+        return 0
+    if args.prefill_only or args.gemm_only:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA GPU for --prefill-only / --gemm-only")
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps(run_single_kernel(args, wl, dev)), flush=True)
         return 0
     if args.ssd_only:
         if not torch.cuda.is_available():

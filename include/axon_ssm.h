@@ -198,7 +198,8 @@ AXON_API axon_status axon_ssm_scan_fwd_segments(
  * aggregates (decay product, local end state) are folded into every run's
  * entering state -- the chunked associative scan of the SSD article applied
  * to the diagonal recurrence of the Axon-SSM page).  runs is 1, 2, 4 or 8
- * (else AXON_ERR_INVALID_ARG); shapes whose staging does not fit return
+ * (one run per chunk: 32-token runs; several: 16-token runs; else
+ * AXON_ERR_INVALID_ARG); shapes whose staging does not fit return
  * AXON_ERR_UNSUPPORTED.  `disc` as for axon_ssm_scan_fwd_ex.  No workspace.
  * Other arguments, layouts and errors are those of axon_ssm_scan_fwd; results
  * agree with the library's own plan to float32 rounding.

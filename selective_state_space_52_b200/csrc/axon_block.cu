@@ -90,7 +90,7 @@ bool tensor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, 
 }
 
 std::atomic<int> g_gemm_sms[kMaxBlockDevices];
-std::atomic<unsigned long long> g_gemm_smem_set[2];
+std::atomic<unsigned long long> g_gemm_smem_set[2];   // per tile width: 256, 192
 
 template <int BN>
 axon_status launch_gemm(int M, int N, int K, const CUtensorMap& ta, const void* W, int ldw, GemmParams p, int sms,
@@ -100,6 +100,7 @@ axon_status launch_gemm(int M, int N, int K, const CUtensorMap& ta, const void* 
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxBlockDevices) return AXON_ERR_CUDA;
     const unsigned long long bit = 1ull << dev;
     std::atomic<unsigned long long>& set = g_gemm_smem_set[BN == 256 ? 0 : 1];
+    static_assert(BN == 256 || BN == 192, "tile widths of the layer's GEMM");
     if (!(set.load(std::memory_order_acquire) & bit)) {
         if (cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
             cudaSuccess)
@@ -117,9 +118,13 @@ axon_status launch_gemm(int M, int N, int K, const CUtensorMap& ta, const void* 
 }
 
 // Row-major outputs (M x N) = A (M x K, row stride lda) * W (K x N, row
-// stride ldw), bf16 in and out, float32 accumulation, on the tcgen05 GEMM
-// (128 x 256 tiles).  Strides, base addresses and column splits must be
-// 16-byte multiples.
+// stride ldw), bf16 in and out, float32 accumulation, on the tcgen05 GEMM.
+// Strides, base addresses and column splits must be 16-byte multiples.  Tiles
+// are 256 columns wide unless 192-column tiles cut waves x width by a quarter
+// or more: a tile's time is about proportional to its width and the last wave
+// runs as long as a full one, but 192-column tiles run a little less
+// efficiently (measured on the layer: the 2048 x 2560 output projection gains,
+// 160 tiles of 256 taking two waves on 148 SMs; the wider ones lose).
 axon_status gemm_tc(int M, int N, int K, const void* A, int lda, const void* W, int ldw, const GemmOut* outs,
                     int nout, int* err, cudaStream_t st) {
     if (M == 0 || N == 0) return AXON_OK;
@@ -139,6 +144,10 @@ axon_status gemm_tc(int M, int N, int K, const void* A, int lda, const void* W, 
     p.nout = nout;
     for (int i = 0; i < nout; ++i) p.out[i] = outs[i];
     p.err = err;
+    const long long tm = (M + kGmBM - 1) / kGmBM;
+    const long long w256 = (tm * ((N + 255) / 256) + sms - 1) / sms;
+    const long long w192 = (tm * ((N + 191) / 192) + sms - 1) / sms;
+    if (4 * w192 * 192 <= 3 * w256 * 256) return launch_gemm<192>(M, N, K, ta, W, ldw, p, sms, st);
     return launch_gemm<256>(M, N, K, ta, W, ldw, p, sms, st);
 }
 

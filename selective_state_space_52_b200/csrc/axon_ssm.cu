@@ -211,9 +211,8 @@ axon_status launch_quad(const ChunkParams& prm, cudaStream_t st) {
 
 // Split-chunk quadrant scan: W warps per 8 channels, each chunk cut into W
 // runs (R = 32 tokens per run for W = 1, else 8).
-template <class Io, int W, bool Z>
+template <class Io, int W, int R, bool Z>
 axon_status launch_qsplit_t(const ChunkParams& prm, cudaStream_t st) {
-    constexpr int R = W == 1 ? 32 : 8;
     auto kern = scan_qsplit_kernel<Io, W, R, Z>;
     static std::atomic<unsigned long long> smem_set{0};
     if (!allow_max_smem(kern, smem_set)) return AXON_ERR_CUDA;
@@ -224,31 +223,35 @@ axon_status launch_qsplit_t(const ChunkParams& prm, cudaStream_t st) {
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
 
+// W runs per chunk: one run of 32 tokens, or W runs of 16
 template <class Io, bool Z>
 axon_status launch_qsplit(const ChunkParams& prm, int W, cudaStream_t st) {
     switch (W) {
-        case 1: return launch_qsplit_t<Io, 1, Z>(prm, st);
-        case 2: return launch_qsplit_t<Io, 2, Z>(prm, st);
-        case 4: return launch_qsplit_t<Io, 4, Z>(prm, st);
-        case 8: return launch_qsplit_t<Io, 8, Z>(prm, st);
+        case 1: return launch_qsplit_t<Io, 1, 32, Z>(prm, st);
+        case 2: return launch_qsplit_t<Io, 2, 16, Z>(prm, st);
+        case 4: return launch_qsplit_t<Io, 4, 16, Z>(prm, st);
+        case 8: return launch_qsplit_t<Io, 8, 16, Z>(prm, st);
     }
     return AXON_ERR_UNSUPPORTED;
 }
 
+// Tokens per run of the split-chunk scan with W runs per chunk.
+int qsplit_run_len(int W) { return W == 1 ? 32 : 16; }
+
 bool qsplit_fits(int B, int L, int E, int io_bytes, int W) {
     (void)B; (void)L;
-    const int R = W == 1 ? 32 : 8;
+    const int R = qsplit_run_len(W);
     return (long long)(W * R + kK) * E * io_bytes < (1LL << 31) &&
            QsplitSmem(W, R, io_bytes).total <= device_max_smem_optin();
 }
 
-// Runs per chunk of the split-chunk quadrant scan for an unsplit first-order
+// Shape code of the split-chunk quadrant scan for an unsplit first-order
 // prefill, or 0 where another kernel is faster.  Measured on B200 (prefill
 // time against the eighths / quadrant scans and the run-split chunked
-// kernel): eight runs per chunk win below about 20 channels per SM (where
-// the CTAs of 8 channels alone leave the SMs nearly idle), one run per chunk
-// from 48 to 511 channels per SM; the eighths scan keeps 20 to 47, and the
-// one-thread-per-channel walk 512 and up.
+// kernel): eight runs of 16 tokens per chunk win below about 20 channels per
+// SM (where the CTAs of 8 channels alone leave the SMs nearly idle), one run of 32 tokens per
+// chunk from 48 to 511 channels per SM; the eighths scan keeps 20 to 47, and
+// the one-thread-per-channel walk 512 and up.
 int plan_qsplit(int B, int L, int E, int io_bytes, int sms) {
     const long long channels = (long long)B * E;
     int W = 0;
@@ -306,7 +309,7 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
                       const void* conv_cache_in, const float* ssm_state_in,
                       void* y, void* conv_cache_out, float* ssm_state_out,
                       void* workspace, size_t workspace_bytes, int num_segments,
-                      cudaStream_t stream, bool zoh = false, int qsplit_runs = 0) {
+                      cudaStream_t stream, bool zoh = false, int forced_qsplit = 0) {
     axon_status st = check_shape(B, L, E, N, K, io);
     if (st != AXON_OK) return st;
     if (num_segments < 0) return AXON_ERR_INVALID_ARG;
@@ -345,14 +348,14 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
     bool chunked = false, quad = false, octo = false;
     int qsplit = 0;                              // runs per chunk of the split-chunk quadrant scan
     ChunkPlan cplan{};
-    if (qsplit_runs != 0) {
-        if (qsplit_runs != 1 && qsplit_runs != 2 && qsplit_runs != 4 && qsplit_runs != 8)
+    if (forced_qsplit != 0) {
+        if (forced_qsplit != 1 && forced_qsplit != 2 && forced_qsplit != 4 && forced_qsplit != 8)
             return AXON_ERR_INVALID_ARG;
         if (num_segments != 1) return AXON_ERR_INVALID_ARG;
         if (L > 0) {
             if (device_max_smem_optin() <= 0) return AXON_ERR_CUDA;
-            if (!qsplit_fits(B, L, E, (int)io_bytes(io), qsplit_runs)) return AXON_ERR_UNSUPPORTED;
-            qsplit = qsplit_runs;
+            if (!qsplit_fits(B, L, E, (int)io_bytes(io), forced_qsplit)) return AXON_ERR_UNSUPPORTED;
+            qsplit = forced_qsplit;
         }
     } else if (L > 0) {
         if (num_segments > kMaxSegments) return AXON_ERR_INVALID_ARG;

@@ -5,11 +5,12 @@
 // conv output).
 //
 // Persistent, warp-specialised, one CTA per SM (192 threads), output tiles of
-// 128 x BN (the layer uses BN = 256; 128-column tiles measured slower):
+// 128 x BN, BN = 256 or 192 (whichever fills the SMs in less time; 128-column
+// tiles measured slower):
 //   warp 0 (one thread)  TMA producer: per 64-deep K block, the A tile
 //                        (128 rows x 64, K-major) and the W tile (64 x BN,
 //                        N-major, 64-column boxes), 128-byte swizzle, into a
-//                        ring of shared-memory stages (4 for BN 256, 6 for 128);
+//                        ring of shared-memory stages (4 for BN 256, 5 for 192);
 //   warp 1 (one thread)  MMA issuer: four tcgen05.mma (M 128, N BN, K 16)
 //                        per stage into one of 512 / BN float32 accumulators
 //                        in tensor memory; each stage is handed back to the
@@ -44,8 +45,9 @@ template <int BN>
 struct GemmCfg {
     static constexpr int kBBytes = kGmBK * BN * 2;
     static constexpr int kStageBytes = kGmABytes + kBBytes;
-    static constexpr int kStages = BN == 256 ? 4 : 6;
-    static constexpr int kAccs = 512 / BN;            // tensor-memory accumulators (512 columns)
+    static constexpr int kStages = BN == 256 ? 4 : (BN == 192 ? 5 : 6);
+    static constexpr int kAccs = 512 / BN;            // tensor-memory accumulators (of 512 columns)
+    static constexpr int kAccStride = BN > 128 ? 256 : 128;   // their first columns: 0, 256 (or 128 apart)
     static constexpr int kBarOff = kStages * kStageBytes;
     static constexpr int kSmem = kBarOff + 256 + 1024;  // + barriers, slot, flags + alignment pad
 };
@@ -153,7 +155,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
                 if (!mbar_wait(tempty(a), aph ^ 1u)) { fail(); break; }
                 tc_fence_after();
-                const uint32_t d = tbase + (uint32_t)(a * kGmBN);
+                const uint32_t d = tbase + (uint32_t)(a * Cfg::kAccStride);
                 bool ok = true;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(full(s), ph) || *abort_flag) { ok = false; break; }
@@ -186,7 +188,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             tc_fence_after();
             const int m = (tile % p.tiles_m) * kGmBM + row;
             const int n0 = (tile / p.tiles_m) * kGmBN;
-            const uint32_t tl = tbase + (uint32_t)(a * kGmBN) + ((uint32_t)(32 * q) << 16);
+            const uint32_t tl = tbase + (uint32_t)(a * Cfg::kAccStride) + ((uint32_t)(32 * q) << 16);
 #pragma unroll 1
             for (int c0 = 0; c0 < kGmBN; c0 += 16) {
                 float v[16];

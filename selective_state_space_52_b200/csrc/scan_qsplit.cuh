@@ -9,20 +9,20 @@
 //
 //   1. copies (cp.async, one chunk ahead, double buffered) of its run's x
 //      rows with a 3-token halo, the z and dt_raw rows of the 8 channels and
-//      the B, C rows into the warp's own shared memory; bf16 B and C rows are
-//      widened to float32 once per warp (not once per lane);
+//      the B, C rows into the warp's own shared memory;
 //   2. the per-(token, channel) prologue, once: lane (g, c) takes tokens
 //      g*R/4 .. g*R/4 + R/4 - 1 of channel c (conv window in registers), writes
 //      (dt, dt, f, f) -- f = dt*u first order, u for ZOH -- and keeps D*u and
 //      SiLU(z) of its tokens in registers;
-//   3. W > 1: a first pass from a zero state over the run keeps the R decays
-//      a = 2^(dt * A log2 e) and inputs dt*u*B of its 4 states in registers and
-//      yields the run's aggregate (prod a, local end state H); after one CTA
-//      barrier each warp folds the aggregates of the runs before it into the
-//      chunk's entering state, h = A_j h + H_j (the intra-block pass and
-//      inter-block carry of the SSD article's chunked scan, applied to the
-//      diagonal recurrence), and the second pass walks the run again from
-//      that state with the stored decays and inputs: no second exponential;
+//   3. W > 1: a first pass from a zero state over the run computes the
+//      decays a = 2^(dt * A log2 e), the local states H_t, the decay products
+//      P_t, and keeps per token C_t . H_t and C_t P_t; its end (P, H) is the
+//      run's aggregate.  After one CTA barrier each warp folds the
+//      aggregates of the runs before it into the chunk's entering state,
+//      h = P_j h + H_j (the intra-block pass and inter-block carry of the SSD
+//      article's chunked scan, applied to the diagonal recurrence), and the
+//      second pass needs no recurrence and no exponential:
+//      C_t . h_t = C_t . H_t + (C_t P_t) . h_in;
 //      W == 1: one pass with the carried state, decays computed on the way;
 //   4. the partial C . h of each token (sum over the lane's quadrant) is summed
 //      over the four quadrants by a shuffle reduce-scatter that leaves each
@@ -47,8 +47,8 @@ constexpr int kQsCh = 8;   // channels per CTA
 // aggregate and entering-state slots.  Identical on host and device.
 struct QsplitSmem {
     int xs, zs, ds, bs, cs, stage;   // one staging buffer (io dtype); two per warp
-    int bf, cf;                      // float32 B, C rows of the run (bf16 io)
     int pf;                          // (dt, f) per (token, channel)
+    int dz;                          // (D u, SiLU(z)) per (token, channel), W > 1
     int warp_bytes;
     int agg, entry, total;
     __host__ __device__ static int pad(int r, int RQ) { return r + r / RQ; }
@@ -64,12 +64,11 @@ struct QsplitSmem {
         cs = off; off += R * RB;
         stage = (off + 15) & ~15;
         off = 2 * stage;
-        bf = off; off += io_bytes == 2 ? R * kN * 4 : 0;
-        cf = off; off += io_bytes == 2 ? R * kN * 4 : 0;
         pf = off; off += R * kQsCh * 8;
+        dz = off; off += W > 1 ? R * kQsCh * 8 : 0;
         warp_bytes = (off + 127) & ~127;
         off = W * warp_bytes;
-        agg = off; off += W > 1 ? 2 * W * 32 * 32 : 0;       // [parity][warp][lane] (A0..3, H0..3)
+        agg = off; off += W > 1 ? 2 * W * 2 * 32 * 16 : 0;   // [parity][warp][A | H][lane] float4
         entry = off; off += W > 1 ? 2 * 32 * 16 : 0;         // [parity][lane] h0..3
         total = off;
     }
@@ -77,7 +76,7 @@ struct QsplitSmem {
 
 template <class Io, int W, int R, bool kZoh>
 __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(ChunkParams p) {
-    static_assert(R == 8 || R == 16 || R == 32, "R: 8, 16 or 32 tokens per run");
+    static_assert(R == 16 || R == 32, "R: 16 or 32 tokens per run");
     static_assert(W == 1 || W == 2 || W == 4 || W == 8, "W: 1, 2, 4 or 8 runs per chunk");
     using TT = typename Io::T;
     using SI = SmemIo<Io>;
@@ -91,7 +90,6 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
     constexpr int NXP = (R + kK - 1) * P, NX = (NXP + 31) / 32;
     constexpr int NZP = R * P, NZ = (NZP + 31) / 32;
     constexpr int NBP = R * PB, NB = (NBP + 31) / 32;
-    constexpr bool kWiden = S == 2;          // bf16 B/C rows are widened to float32
     extern __shared__ __align__(16) unsigned char smem[];
 
     const int lane = threadIdx.x & 31;
@@ -117,56 +115,42 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
     const int npc = (ne * S + 15) / 16;      // pieces of a row inside the tile
     const size_t tile_off = (size_t)b * p.L * row_bytes + (size_t)e0 * S;
 
-    // ---- this lane's share of a run's copies: shared-memory destinations and
-    // byte offsets from the run's first row, fixed for all chunks
-    int xsd[NX], xgo[NX], zsd[NZ], zgo[NZ], bso[NB];
-    bool xok[NX], zok[NZ], bok[NB];
-#pragma unroll
-    for (int i = 0; i < NX; ++i) {
-        const int q = lane + 32 * i, r = q / P, pc = q % P;
-        xok[i] = q < NXP && pc < npc;
-        xsd[i] = lay.xs + QsplitSmem::pad(r, RQ) * XB + pc * 16;
-        xgo[i] = (r - (kK - 1)) * row_bytes + pc * 16;
-    }
-#pragma unroll
-    for (int i = 0; i < NZ; ++i) {
-        const int q = lane + 32 * i, r = q / P, pc = q % P;
-        zok[i] = q < NZP && pc < npc;
-        zsd[i] = QsplitSmem::pad(r, RQ) * XB + pc * 16;
-        zgo[i] = r * row_bytes + pc * 16;
-    }
-#pragma unroll
-    for (int i = 0; i < NB; ++i) {
-        const int q = lane + 32 * i;
-        bok[i] = q < NBP;
-        bso[i] = (q / PB) * RB + (q % PB) * 16;
-    }
-
     // copies of chunk k's run of this warp into stage st
     auto prefetch = [&](int k, int st) {
         unsigned char* sb = ws + st * lay.stage;
         const int t0 = k * T + w * R;
         if (t0 >= kK - 1 && t0 + R <= p.L) {
-            // every row of the run and its halo lies inside the sequence
+            // every row of the run and its halo lies inside the sequence;
+            // this lane's pieces: x (with halo), z and dt rows, B and C rows
             const unsigned char* xr = xg + tile_off + (size_t)t0 * row_bytes;
             const unsigned char* zr = zg + tile_off + (size_t)t0 * row_bytes;
             const unsigned char* dr = dg + tile_off + (size_t)t0 * row_bytes;
             const size_t bc0 = ((size_t)b * p.L + t0) * RB;
 #pragma unroll
-            for (int i = 0; i < NX; ++i)
-                if (xok[i]) cp_async16(sb + xsd[i], xr + xgo[i], true);
+            for (int i = 0; i < NX; ++i) {
+                const int q = lane + 32 * i, r = q / P, pc = q % P;
+                if (q < NXP && pc < npc)
+                    cp_async16(sb + lay.xs + QsplitSmem::pad(r, RQ) * XB + pc * 16,
+                               xr + (r - (kK - 1)) * row_bytes + pc * 16, true);
+            }
 #pragma unroll
-            for (int i = 0; i < NZ; ++i)
-                if (zok[i]) {
-                    cp_async16(sb + lay.zs + zsd[i], zr + zgo[i], true);
-                    cp_async16(sb + lay.ds + zsd[i], dr + zgo[i], true);
+            for (int i = 0; i < NZ; ++i) {
+                const int q = lane + 32 * i, r = q / P, pc = q % P;
+                if (q < NZP && pc < npc) {
+                    const int so = QsplitSmem::pad(r, RQ) * XB + pc * 16, go = r * row_bytes + pc * 16;
+                    cp_async16(sb + lay.zs + so, zr + go, true);
+                    cp_async16(sb + lay.ds + so, dr + go, true);
                 }
+            }
 #pragma unroll
-            for (int i = 0; i < NB; ++i)
-                if (bok[i]) {
-                    cp_async16(sb + lay.bs + bso[i], bg + bc0 + bso[i], true);
-                    cp_async16(sb + lay.cs + bso[i], cg + bc0 + bso[i], true);
+            for (int i = 0; i < NB; ++i) {
+                const int q = lane + 32 * i;
+                if (q < NBP) {
+                    const int o = (q / PB) * RB + (q % PB) * 16;
+                    cp_async16(sb + lay.bs + o, bg + bc0 + o, true);
+                    cp_async16(sb + lay.cs + o, cg + bc0 + o, true);
                 }
+            }
             return;
         }
         // the sequence's first rows (halo from the conv cache or zeros) or a
@@ -235,18 +219,21 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
     unsigned char* ybase = static_cast<unsigned char*>(p.y) + tile_off + (size_t)(w * R + g * RQ) * row_bytes + c * S;
     const int nck = (p.L + T - 1) / T;
     float2* pf = reinterpret_cast<float2*>(ws + lay.pf);          // [token][channel] (dt, f)
-    const float* bfs = reinterpret_cast<const float*>(ws + lay.bf);
-    const float* cfs = reinterpret_cast<const float*>(ws + lay.cf);
 
-    // B / C values of token t for this lane's quadrant (float32 rows)
-    auto bq = [&](const unsigned char* sb, int t) -> float4 {
-        if constexpr (kWiden) return *reinterpret_cast<const float4*>(bfs + t * kN + 4 * g);
-        else return *reinterpret_cast<const float4*>(sb + lay.bs + t * RB + 16 * g);
+    // B / C values of token t for this lane's quadrant, from the staged rows
+    // (a float4, or four bf16 values widened in registers: the 8 lanes of a
+    // quarter warp read the same 8 bytes, one shared-memory wavefront)
+    auto quad_of = [&](const unsigned char* row) -> float4 {
+        if constexpr (S == 4) {
+            return *reinterpret_cast<const float4*>(row + 16 * g);
+        } else {
+            const uint2 q = *reinterpret_cast<const uint2*>(row + 8 * g);
+            return make_float4(__uint_as_float(q.x << 16), __uint_as_float(q.x & 0xffff0000u),
+                               __uint_as_float(q.y << 16), __uint_as_float(q.y & 0xffff0000u));
+        }
     };
-    auto cq = [&](const unsigned char* sb, int t) -> float4 {
-        if constexpr (kWiden) return *reinterpret_cast<const float4*>(cfs + t * kN + 4 * g);
-        else return *reinterpret_cast<const float4*>(sb + lay.cs + t * RB + 16 * g);
-    };
+    auto bq = [&](const unsigned char* sb, int t) -> float4 { return quad_of(sb + lay.bs + t * RB); };
+    auto cq = [&](const unsigned char* sb, int t) -> float4 { return quad_of(sb + lay.cs + t * RB); };
     // the ZOH input factor of token t's 4 states from dt and the decays
     auto zoh4 = [&](float dt, float2 a01, float2 a23, float2& z01, float2& z23) {
         const float2 x01 = __fmul2_rn(f2(dt, dt), s01), x23 = __fmul2_rn(f2(dt, dt), s23);
@@ -254,7 +241,7 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
         z23 = f2(zoh_bbar(dt, x23.x * kLn2, a23.x, iA23.x), zoh_bbar(dt, x23.y * kLn2, a23.y, iA23.y));
     };
 
-    float2* agg = reinterpret_cast<float2*>(smem + lay.agg);       // W > 1
+    float4* agg = reinterpret_cast<float4*>(smem + lay.agg);       // W > 1: [parity][warp][A | H][lane]
     float4* entry = reinterpret_cast<float4*>(smem + lay.entry);   // W > 1
 
     prefetch(0, 0);
@@ -271,25 +258,12 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
         __syncwarp();                        // ... and every lane's
         const unsigned char* sb = ws + st * lay.stage;
 
-        // ---- widen the run's B and C rows to float32 (bf16 io)
-        if constexpr (kWiden) {
-#pragma unroll
-            for (int q = lane; q < 2 * R; q += 32) {
-                const int t = q >> 1;
-                const unsigned char* src = sb + ((q & 1) ? lay.cs : lay.bs) + t * RB;
-                float* dst = const_cast<float*>((q & 1) ? cfs : bfs) + t * kN;
-                float v[8];
-                SI::ld8(src, v);
-                *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
-                *reinterpret_cast<float4*>(dst + 4) = make_float4(v[4], v[5], v[6], v[7]);
-                SI::ld8(src + 16, v);
-                *reinterpret_cast<float4*>(dst + 8) = make_float4(v[0], v[1], v[2], v[3]);
-                *reinterpret_cast<float4*>(dst + 12) = make_float4(v[4], v[5], v[6], v[7]);
-            }
-        }
-
         // ---- prologue: lane (g, c) takes tokens g*RQ .. g*RQ + RQ - 1 of channel c
-        float Du[RQ], gz[RQ];
+        // D u and SiLU(z) of the lane's prologue tokens: registers for one run
+        // per chunk, shared memory for several (their walk keeps more live)
+        constexpr int RQr = W == 1 ? RQ : 1;
+        float Du[RQr], gz[RQr];
+        float2* dzs = reinterpret_cast<float2*>(ws + lay.dz);
         {
             const unsigned char* xc = sb + lay.xs + c * S;
             const int tb = g * RQ;
@@ -312,21 +286,23 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
                 const float dtl = live ? dt : 0.0f;        // dt = 0: decay 1, no input
                 const float f = live ? (kZoh ? u : dt * u) : 0.0f;
                 pf[t * kQsCh + c] = make_float2(dtl, f);
-                Du[i] = Dv * u;
-                gz[i] = silu(SI::ld(sb + lay.zs + tp * XB + c * S));
+                const float du = Dv * u, gzv = silu(SI::ld(sb + lay.zs + tp * XB + c * S));
+                if constexpr (W == 1) { Du[i] = du; gz[i] = gzv; }
+                else dzs[t * kQsCh + c] = make_float2(du, gzv);
             }
         }
         __syncwarp();
 
         float part[R];
         if constexpr (W == 1) {
-            // ---- one pass from the carried state, in blocks of 4 tokens: the
-            // block's decays and inputs first, then its state updates
+            // ---- one pass from the carried state, in blocks of kBlk tokens:
+            // the block's decays and inputs first, then its state updates
+            constexpr int kBlk = 4;
 #pragma unroll
-            for (int tb = 0; tb < R; tb += 4) {
-                float2 a01[4], a23[4], u01[4], u23[4];
+            for (int tb = 0; tb < R; tb += kBlk) {
+                float2 a01[kBlk], a23[kBlk], u01[kBlk], u23[kBlk];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < kBlk; ++i) {
                     const int t = tb + i;
                     const float2 v = pf[t * kQsCh + c];
                     const float4 Bq = bq(sb, t);
@@ -345,7 +321,7 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < kBlk; ++i) {
                     const int t = tb + i;
                     const float4 Cq = cq(sb, t);
                     h01 = __ffma2_rn(a01[i], h01, u01[i]);
@@ -355,8 +331,13 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
                 }
             }
         } else {
-            // ---- first pass: the run from a zero state; keep decays and inputs
-            float2 a01[R], a23[R], u01[R], u23[R];
+            // ---- first pass: the run from a zero state.  With h_in the state
+            // entering the run, P_t the product of its decays up to t and
+            // H_t the state reached from zero, h_t = P_t h_in + H_t, so
+            // C_t . h_t = C_t . H_t + (C_t P_t) . h_in: keep the local partial
+            // C_t . H_t and Q_t = C_t P_t of every token, and (P, H) at the end.
+            float2 q01[R], q23[R];
+            float pl[R];
             float2 H01 = f2(0.f, 0.f), H23 = f2(0.f, 0.f);
             float2 P01 = f2(1.f, 1.f), P23 = f2(1.f, 1.f);
 #pragma unroll
@@ -366,26 +347,32 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
                 const float2 dd = f2(v.x, v.x), ff = f2(v.y, v.y);
                 const float2 arg01 = __fmul2_rn(dd, s01);
                 const float2 arg23 = __fmul2_rn(dd, s23);
-                a01[t] = f2(ex2_approx(arg01.x), ex2_approx(arg01.y));
-                a23[t] = f2(ex2_approx(arg23.x), ex2_approx(arg23.y));
-                u01[t] = __fmul2_rn(ff, f2(Bq.x, Bq.y));
-                u23[t] = __fmul2_rn(ff, f2(Bq.z, Bq.w));
+                const float2 a01 = f2(ex2_approx(arg01.x), ex2_approx(arg01.y));
+                const float2 a23 = f2(ex2_approx(arg23.x), ex2_approx(arg23.y));
+                float2 i01 = __fmul2_rn(ff, f2(Bq.x, Bq.y));
+                float2 i23 = __fmul2_rn(ff, f2(Bq.z, Bq.w));
                 if constexpr (kZoh) {
                     float2 z01, z23;
-                    zoh4(v.x, a01[t], a23[t], z01, z23);
-                    u01[t] = __fmul2_rn(u01[t], z01);
-                    u23[t] = __fmul2_rn(u23[t], z23);
+                    zoh4(v.x, a01, a23, z01, z23);
+                    i01 = __fmul2_rn(i01, z01);
+                    i23 = __fmul2_rn(i23, z23);
                 }
-                H01 = __ffma2_rn(a01[t], H01, u01[t]);
-                H23 = __ffma2_rn(a23[t], H23, u23[t]);
-                P01 = __fmul2_rn(P01, a01[t]);
-                P23 = __fmul2_rn(P23, a23[t]);
+                H01 = __ffma2_rn(a01, H01, i01);
+                H23 = __ffma2_rn(a23, H23, i23);
+                P01 = __fmul2_rn(P01, a01);
+                P23 = __fmul2_rn(P23, a23);
+                const float4 Cq = cq(sb, t);
+                const float2 c01 = f2(Cq.x, Cq.y), c23 = f2(Cq.z, Cq.w);
+                const float2 pq = __ffma2_rn(c23, H23, __fmul2_rn(c01, H01));
+                pl[t] = pq.x + pq.y;
+                q01[t] = __fmul2_rn(c01, P01);
+                q23[t] = __fmul2_rn(c23, P23);
             }
             // the run's aggregate (prod a, H) for the other warps
             {
-                float4* slot = reinterpret_cast<float4*>(agg + ((k & 1) * W + w) * 32 * 4 + lane * 4);
+                float4* slot = agg + ((k & 1) * W + w) * 64 + lane;
                 slot[0] = make_float4(P01.x, P01.y, P23.x, P23.y);
-                slot[1] = make_float4(H01.x, H01.y, H23.x, H23.y);
+                slot[32] = make_float4(H01.x, H01.y, H23.x, H23.y);
             }
             __syncthreads();                 // every run's aggregate of chunk k is written
             // ---- the state entering this run: the chunk's entering state (the
@@ -396,20 +383,20 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
                 h23 = f2(he.z, he.w);
             }
             for (int j = 0; j < w; ++j) {
-                const float4* slot = reinterpret_cast<const float4*>(agg + ((k & 1) * W + j) * 32 * 4 + lane * 4);
-                const float4 A = slot[0], H = slot[1];
+                const float4* slot = agg + ((k & 1) * W + j) * 64 + lane;
+                const float4 A = slot[0], H = slot[32];
                 h01 = __ffma2_rn(f2(A.x, A.y), h01, f2(H.x, H.y));
                 h23 = __ffma2_rn(f2(A.z, A.w), h23, f2(H.z, H.w));
             }
-            // ---- second pass: the run again from its true entering state
+            // ---- second pass: every token's C . h from the entering state,
+            // no chain; then the run's end state
 #pragma unroll
             for (int t = 0; t < R; ++t) {
-                const float4 Cq = cq(sb, t);
-                h01 = __ffma2_rn(a01[t], h01, u01[t]);
-                h23 = __ffma2_rn(a23[t], h23, u23[t]);
-                const float2 pq = __ffma2_rn(f2(Cq.z, Cq.w), h23, __fmul2_rn(f2(Cq.x, Cq.y), h01));
-                part[t] = pq.x + pq.y;
+                const float2 pq = __ffma2_rn(q23[t], h23, __fmul2_rn(q01[t], h01));
+                part[t] = pl[t] + (pq.x + pq.y);
             }
+            h01 = __ffma2_rn(P01, h01, H01);
+            h23 = __ffma2_rn(P23, h23, H23);
             if (w == W - 1) entry[((k + 1) & 1) * 32 + lane] = make_float4(h01.x, h01.y, h23.x, h23.y);
         }
 
@@ -435,9 +422,13 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
             }
             unsigned char* yrow = ybase + (size_t)t0 * row_bytes;
 #pragma unroll
-            for (int j = 0; j < RQ; ++j)
-                if (active && (full || tr + g * RQ + j < p.L))
-                    Io::store(reinterpret_cast<TT*>(yrow + j * row_bytes), (tot[j] + Du[j]) * gz[j]);
+            for (int j = 0; j < RQ; ++j) {
+                if (!active || (!full && tr + g * RQ + j >= p.L)) continue;
+                float du, gzv;
+                if constexpr (W == 1) { du = Du[j]; gzv = gz[j]; }
+                else { const float2 v = dzs[(g * RQ + j) * kQsCh + c]; du = v.x; gzv = v.y; }
+                Io::store(reinterpret_cast<TT*>(yrow + j * row_bytes), (tot[j] + du) * gzv);
+            }
         }
     }
 
