@@ -28,15 +28,16 @@ from gpu_util import to_dev
 pytestmark = pytest.mark.gpu
 
 
-def block_close(got, ref_rounded, ref_plain, what):
+def block_close(got, ref_rounded, ref_plain, what, elem_tol=1e-2):
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref_rounded, dtype=np.float64)
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
     assert np.all(np.isfinite(got)), what + ": non-finite"
     scale = max(float(np.sqrt(np.mean(ref ** 2))), 1e-30)
     err = np.abs(got - ref) / np.maximum(scale, np.abs(ref))
-    assert err.max() <= 1e-2, (f"{what}: {int((err > 1e-2).sum())} of {err.size} elements beyond 1% "
-                                f"of scale against the bf16-rounding oracle; worst {float(err.max()):.3g}")
+    assert err.max() <= elem_tol, (f"{what}: {int((err > elem_tol).sum())} of {err.size} elements beyond "
+                                   f"{elem_tol:.0%} of scale against the bf16-rounding oracle; "
+                                   f"worst {float(err.max()):.3g}")
     plain = np.asarray(ref_plain, dtype=np.float64)
     rel = np.linalg.norm(got - plain) / max(np.linalg.norm(plain), 1e-30)
     assert rel <= 1e-2, f"{what}: normwise error {rel:.3g} against the plain fp64 oracle"
@@ -62,13 +63,13 @@ def ref_block(inp, with_state, bf16_intermediates):
                             bf16_intermediates=bf16_intermediates)
 
 
-def check_block(inp, with_state, what):
+def check_block(inp, with_state, what, elem_tol=1e-2):
     got = run_block(inp, with_state)
     rounded = ref_block(inp, with_state, True)
     plain = ref_block(inp, with_state, False)
     for name, g, r, p in zip(("out", "ssm_state", "conv_cache"), (got[0], got[2], got[1]),
                              (rounded[0], rounded[2], rounded[1]), (plain[0], plain[2], plain[1])):
-        block_close(g, r, p, f"{what} {name}")
+        block_close(g, r, p, f"{what} {name}", elem_tol)
 
 
 @pytest.mark.parametrize("with_state", [False, True])
@@ -83,6 +84,22 @@ def test_bit_axon_block_full_width(cuda_lib):
     bw = W.BLOCK_WORKLOAD_BY_NAME["bit_axon_block"]
     inp = W.make_block_inputs(bw, with_state=True, L=48)
     check_block(inp, True, "bit-axon block")
+
+
+def test_bit_axon_block_full_size(cuda_lib):
+    """The Bit-Axon layer at the measured size (B1 L2048 D2560 E7680): every
+    projection runs several waves of persistent tiles, with a partial last
+    wave.  Elementwise bound 2% of scale against the bf16-rounding oracle:
+    over 2048 x 7680 stored intermediates a few land, in float32, on the other
+    side of a bf16 rounding boundary than in fp64 (one bf16 ulp each), and one
+    such flip in a long-memory channel moves that token's y, which the output
+    projection spreads over the whole output row -- measured: 11 of 5.2 M
+    outputs above 1%, worst 1.37%, all in one token row, the same whether or
+    not the projections' last wave was split over the SMs.  The normwise bound
+    against the plain fp64 oracle stays 1%."""
+    bw = W.BLOCK_WORKLOAD_BY_NAME["bit_axon_block"]
+    inp = W.make_block_inputs(bw, with_state=True)
+    check_block(inp, True, "bit-axon block, full size", elem_tol=2e-2)
 
 
 def test_block_empty_sequence_copies_caches(cuda_lib):
