@@ -53,7 +53,8 @@ constexpr int kStepMaxRows = 32;   // batch rows per block
 //    shared-memory ring with cp.async (a lane reads back only its own copies);
 //  - A = -exp(A_log) is formed once per lane.
 // The conv/SiLU/dt prologue of four consecutive rows is spread over the four
-// lanes of a channel; C . h is finished with two shuffles.
+// lanes of a channel; C . h is finished with two shuffles.  y and the shifted
+// conv caches of all the block's rows leave at the end as 16-byte pieces.
 template <class Io, bool kZoh>
 __global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int rows) {
     using T = typename Io::T;
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int ro
 
     __shared__ __align__(16) unsigned char small[kStepMaxRows][kSmall][kWin];
     __shared__ __align__(16) unsigned char bcs[kStepMaxRows][2][kN * S];
+    __shared__ __align__(16) unsigned char yst[kStepMaxRows][kWin];   // y of the block's rows
     __shared__ float4 ring[kStepStages][kStepThreads];
 
     {   // (1) every row's small inputs and B/C rows, 16-byte pieces
@@ -98,10 +100,10 @@ __global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int ro
         }
         asm volatile("cp.async.commit_group;\n" ::: "memory");
     }
-    auto issue = [&](int j) {   // (2) row j's state piece -> this lane's ring slot
-        step_cp_async16(&ring[j % kStepStages][tid],
-                        reinterpret_cast<const float4*>(p.ssm_state + ((size_t)(b0 + j) * p.E + ec) * kN) + q, true);
-    };
+    // (2) row j's state piece -> this lane's ring slot; rows are E*N floats apart
+    const size_t srow = (size_t)p.E * kN;
+    const float* sbase = p.ssm_state + ((size_t)b0 * p.E + ec) * kN + 4 * q;
+    auto issue = [&](int j) { step_cp_async16(&ring[j % kStepStages][tid], sbase + (size_t)j * srow, true); };
 #pragma unroll
     for (int j = 0; j < kStepStages - 1; ++j) {
         if (j < nb) issue(j);
@@ -126,8 +128,8 @@ __global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int ro
     const int co = (ec - e0) * S;                     // this channel's byte offset in a window
     // Rows go in rounds of four: lane q computes the conv / SiLU / dt prologue
     // and SiLU(z) of row j0+q only; each row's dt and dt*u reach the other
-    // three lanes of the channel by shuffles, and the row's owner lane writes
-    // y and the shifted cache.
+    // three lanes of the channel by shuffles, and the row's owner lane puts
+    // its y in shared memory.
 #pragma unroll 1
     for (int j0 = 0; j0 < nb; j0 += 4) {
         const int jq = min(j0 + q, nb - 1);
@@ -169,18 +171,33 @@ __global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int ro
             }
             acc += __shfl_xor_sync(0xffffffffu, acc, 1);
             acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            if (live) {
-                const size_t ch = (size_t)b * p.E + e;
-                reinterpret_cast<float4*>(p.ssm_state + ch * kN)[q] = make_float4(h[0], h[1], h[2], h[3]);
-                if (q == k) {
-                    Io::store(static_cast<T*>(p.y) + ch, fmaf(Dv, uq, acc) * gzq);
-                    // shift the cache: drop the oldest input, append x_t (exact copies of the raw bits)
-                    T* cc = static_cast<T*>(p.conv_cache) + (size_t)b * (kK - 1) * p.E + e;
-                    cc[0] = *reinterpret_cast<const T*>(&small[j][4][co]);
-                    cc[p.E] = *reinterpret_cast<const T*>(&small[j][5][co]);
-                    cc[2 * (size_t)p.E] = *reinterpret_cast<const T*>(&small[j][0][co]);
-                }
+            if (live) *reinterpret_cast<float4*>(const_cast<float*>(sbase) + (size_t)j * srow) =
+                          make_float4(h[0], h[1], h[2], h[3]);
+            if (live && q == k) Io::store(reinterpret_cast<T*>(&yst[j][co]), fmaf(Dv, uq, acc) * gzq);
+        }
+    }
+    // (3) y and the shifted conv caches of all rows, 16-byte pieces: cache row
+    // i <- cache row i+1, the last <- x_t (exact copies of the raw bits; every
+    // read of the old cache happened in (1), so in-place updates are safe)
+    __syncthreads();
+    {
+        constexpr int kPw = kWin / 16;
+        const size_t row_bytes = (size_t)p.E * S;
+        for (int i = tid; i < nb * kK * kPw; i += kStepThreads) {
+            const int j = i / (kK * kPw), t = i - j * (kK * kPw), k = t / kPw, pc = t - k * kPw;
+            const size_t col = (size_t)e0 * S + (size_t)pc * 16;
+            if (col + 16 > row_bytes) continue;          // E*S is a multiple of 16
+            const int b = b0 + j;
+            unsigned char* dst;
+            const unsigned char* src;
+            if (k == 0) {                                // y
+                dst = static_cast<unsigned char*>(p.y) + (size_t)b * row_bytes + col;
+                src = &yst[j][pc * 16];
+            } else {                                     // cache row k-1
+                dst = static_cast<unsigned char*>(p.conv_cache) + ((size_t)b * (kK - 1) + (k - 1)) * row_bytes + col;
+                src = k < kK - 1 ? &small[j][3 + k][pc * 16] : &small[j][0][pc * 16];
             }
+            *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
         }
     }
 }
