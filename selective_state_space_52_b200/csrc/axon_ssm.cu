@@ -532,6 +532,15 @@ axon_status axon_ssm_scan_fwd_segments(int B, int L, int E, int N, int K, axon_d
 }
 
 namespace {
+// Batch rows per decode block: the fewest, in rounds of four, whose grid of
+// ceil(E / 32) x ceil(B / rows) blocks fits the resident slots in one wave.
+int step_rows(int B, int E, long long slots) {
+    const long long bx = (E + kStepChan - 1) / kStepChan;
+    int rows = B < 4 ? B : 4;
+    while (rows < kStepMaxRows && rows < B && bx * ((B + rows - 1) / rows) > slots) rows += 4;
+    return rows;
+}
+
 axon_status step_impl(int B, int E, int N, int K, axon_dtype io,
                       const void* x, const void* z, const void* dt_raw,
                       const void* Bm, const void* Cm,
@@ -567,23 +576,24 @@ axon_status step_impl(int B, int E, int N, int K, axon_dtype io,
     prm.x = x; prm.z = z; prm.dt_raw = dt_raw; prm.Bm = Bm; prm.Cm = Cm;
     prm.conv_w = conv_w; prm.conv_b = conv_b; prm.dt_bias = dt_bias; prm.A_log = A_log; prm.D = D;
     prm.conv_cache = conv_cache; prm.ssm_state = ssm_state; prm.y = y;
-    // batch rows per block: the fewest that keep the grid within ~8 resident
-    // blocks of 128 threads per SM (one wave), so each block's copy ring runs
-    // over several rows
     const int sms = device_sm_count();
     if (sms <= 0) return AXON_ERR_CUDA;
-    const long long bx = (E + kStepChan - 1) / kStepChan;
-    int rows = 1;
-    while (rows < kStepMaxRows && rows < B && bx * ((B + rows - 1) / rows) > 8LL * sms) rows *= 2;
-    const dim3 grid((unsigned)bx, (unsigned)((B + rows - 1) / rows));
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (io == AXON_BF16) {
-        if (zoh) step_kernel<IoBF16, true><<<grid, kStepThreads, 0, s>>>(prm, rows);
-        else step_kernel<IoBF16, false><<<grid, kStepThreads, 0, s>>>(prm, rows);
-    } else {
-        if (zoh) step_kernel<IoF32, true><<<grid, kStepThreads, 0, s>>>(prm, rows);
-        else step_kernel<IoF32, false><<<grid, kStepThreads, 0, s>>>(prm, rows);
+    void (*kern)(StepParams, int);
+    if (io == AXON_BF16) kern = zoh ? step_kernel<IoBF16, true> : step_kernel<IoBF16, false>;
+    else kern = zoh ? step_kernel<IoF32, true> : step_kernel<IoF32, false>;
+    // resident blocks per SM of this instance (a property of the compiled
+    // kernel, queried once)
+    static std::atomic<int> occupancy[4];
+    const int ki = (io == AXON_BF16 ? 2 : 0) + (zoh ? 1 : 0);
+    int per_sm = occupancy[ki].load(std::memory_order_relaxed);
+    if (per_sm <= 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kStepThreads, 0) != cudaSuccess || per_sm <= 0)
+            return AXON_ERR_CUDA;
+        occupancy[ki].store(per_sm, std::memory_order_relaxed);
     }
+    const int rows = step_rows(B, E, (long long)per_sm * sms);
+    const dim3 grid((unsigned)((E + kStepChan - 1) / kStepChan), (unsigned)((B + rows - 1) / rows));
+    kern<<<grid, kStepThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(prm, rows);
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
 }  // namespace

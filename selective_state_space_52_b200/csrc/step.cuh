@@ -3,11 +3,12 @@
 // float32 states, run one token of conv + SiLU + dt + recurrence + gate, write
 // y, the shifted conv cache and the updated state in place.
 //
-// The step is bound by HBM traffic on the state read-modify-write (2 x 64 bytes
-// of the 148 bytes per channel it moves at bf16).  The state moves as 16-byte
-// pieces, four lanes per channel, through per-lane asynchronous-copy rings, and
-// every other input arrives through shared memory in one copy per block, so the
-// HBM traffic of later rows overlaps the arithmetic of the current one.
+// The step moves 148 bytes per channel at bf16, 128 of them the float32 state
+// read and written back, and does 22 transcendentals per channel.  With the
+// work spread thinly (one token), what limits it is the instructions issued
+// per channel and the bytes each SM keeps in flight, so the kernel loads
+// straight from global memory into registers, a round of four batch rows at a
+// time, and keeps the per-row bookkeeping small.
 #pragma once
 
 #include "device_math.cuh"
@@ -31,84 +32,68 @@ struct StepParams {
     void* y;
 };
 
-__device__ __forceinline__ void step_cp_async16(void* smem_dst, const void* gmem_src, bool valid) {
-    const unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
-    const int n = valid ? 16 : 0;   // 0 source bytes: zero-fill
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem_src), "r"(n) : "memory");
-}
-
 constexpr int kStepThreads = 128;  // 32 channels x 4 lanes
 constexpr int kStepChan = kStepThreads / 4;
-constexpr int kStepStages = 4;     // state rows in flight per lane (shared-memory ring)
 constexpr int kStepMaxRows = 32;   // batch rows per block
 
+// a raw io value as float (exact)
+__device__ __forceinline__ float step_f(float v) { return v; }
+__device__ __forceinline__ float step_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Four consecutive values of a B or C row (8 bytes at bf16, 16 at fp32), read
+// through the non-coherent path: B and C are never written by the step.
+template <class Io> struct StepQuad;
+template <> struct StepQuad<IoBF16> {
+    uint2 v;
+    __device__ __forceinline__ void load(const void* row, int q) {
+        v = __ldg(reinterpret_cast<const uint2*>(row) + q);
+    }
+    __device__ __forceinline__ void unpack(float (&r)[4]) const {
+        r[0] = __uint_as_float(v.x << 16); r[1] = __uint_as_float(v.x & 0xffff0000u);
+        r[2] = __uint_as_float(v.y << 16); r[3] = __uint_as_float(v.y & 0xffff0000u);
+    }
+};
+template <> struct StepQuad<IoF32> {
+    float4 v;
+    __device__ __forceinline__ void load(const void* row, int q) {
+        v = __ldg(reinterpret_cast<const float4*>(row) + q);
+    }
+    __device__ __forceinline__ void unpack(float (&r)[4]) const {
+        r[0] = v.x; r[1] = v.y; r[2] = v.z; r[3] = v.w;
+    }
+};
+
 // grid = (ceil(E / 32), ceil(B / rows)) blocks of 128 threads, rows <= 32.
-// Four lanes share a channel, each owning four consecutive states (one 16-byte
-// vector), so a warp's state traffic is one contiguous 512-byte run.  A block
-// owns 32 channels and walks `rows` batch rows:
-//  - at the start it copies, for all its rows, the channels' x, z, dt_raw and
-//    K-1 cache entries and the B_t, C_t rows into shared memory (one
-//    cooperative cp.async group, one barrier);
-//  - every lane streams its state pieces through a private kStepStages-deep
-//    shared-memory ring with cp.async (a lane reads back only its own copies);
-//  - A = -exp(A_log) is formed once per lane.
-// The conv/SiLU/dt prologue of four consecutive rows is spread over the four
-// lanes of a channel; C . h is finished with two shuffles.  y and the shifted
-// conv caches of all the block's rows leave at the end as 16-byte pieces.
+// Lane (c, q) = thread 4c + q owns channel e0 + c and the state quadrant
+// 4q .. 4q+3 (one 16-byte vector), so a warp's state traffic is one
+// contiguous 512-byte run.  The block walks its rows in rounds of four:
+//  - every lane loads the four rows' state vectors and B, C quadrants, and
+//    the raw inputs (x, z, dt_raw, K-1 cached values) of round row q, all
+//    issued before the first use, so they are in flight together;
+//  - lane q runs the conv / SiLU / dt prologue and SiLU(z) of round row q; a
+//    row's dt and input factor reach the other three lanes of the channel by
+//    shuffles;
+//  - each lane updates its quadrant of the four rows and stores the states;
+//    the four per-quadrant partial C . h are summed by a two-step shuffle
+//    reduce-scatter that leaves round row q's total on lane q, which writes
+//    that row's y and shifted conv cache.
+// State, cache and y are read and written by the same thread (plain loads:
+// the state and cache are updated in place); lanes past E compute channel
+// E-1 and store nothing.
 template <class Io, bool kZoh>
 __global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int rows) {
     using T = typename Io::T;
     constexpr int S = Io::kBytes;
-    constexpr int kSmall = 3 + (kK - 1);              // x, z, dt_raw, cache rows 0..K-2
-    constexpr int kWin = kStepChan * S;               // bytes of a 32-channel window
     const int tid = threadIdx.x;
-    const int q = tid & 3;                            // states 4q .. 4q+3
-    const int c = tid >> 2;
-    const int e0 = blockIdx.x * kStepChan;
-    const int e = e0 + c;
+    const int q = tid & 3;
+    const int e = blockIdx.x * kStepChan + (tid >> 2);
     const int b0 = blockIdx.y * rows;
     const int nb = min(rows, p.B - b0);
-    // Every lane stays to the end (the shuffles below need full warps); lanes
-    // past E compute channel E-1 and store nothing.
     const bool live = e < p.E;
     const int ec = live ? e : p.E - 1;
+    const size_t E = (size_t)p.E;
+    const size_t srow = E * kN;                       // floats between consecutive rows' states
 
-    __shared__ __align__(16) unsigned char small[kStepMaxRows][kSmall][kWin];
-    __shared__ __align__(16) unsigned char bcs[kStepMaxRows][2][kN * S];
-    __shared__ __align__(16) unsigned char yst[kStepMaxRows][kWin];   // y of the block's rows
-    __shared__ float4 ring[kStepStages][kStepThreads];
-
-    {   // (1) every row's small inputs and B/C rows, 16-byte pieces
-        constexpr int kPw = kWin / 16, kPb = kN * S / 16;
-        constexpr int kPer = kSmall * kPw + 2 * kPb;   // pieces per row
-        const size_t row_bytes = (size_t)p.E * S;
-        for (int i = tid; i < nb * kPer; i += kStepThreads) {
-            const int j = i / kPer, t = i - j * kPer, b = b0 + j;
-            if (t < kSmall * kPw) {
-                const int k = t / kPw, pc = t - k * kPw;
-                const size_t col = (size_t)e0 * S + (size_t)pc * 16;
-                const bool ok = col + 16 <= row_bytes;           // E*S is a multiple of 16
-                const unsigned char* base;
-                if (k < 3) base = static_cast<const unsigned char*>(k == 0 ? p.x : (k == 1 ? p.z : p.dt_raw)) + (size_t)b * row_bytes;
-                else base = static_cast<const unsigned char*>(p.conv_cache) + ((size_t)b * (kK - 1) + (k - 3)) * row_bytes;
-                step_cp_async16(&small[j][k][pc * 16], ok ? base + col : static_cast<const void*>(p.x), ok);
-            } else {
-                const int u = t - kSmall * kPw, w2 = u / kPb, pc = u - w2 * kPb;
-                const unsigned char* base = static_cast<const unsigned char*>(w2 ? p.Cm : p.Bm) + (size_t)b * kN * S;
-                step_cp_async16(&bcs[j][w2][pc * 16], base + pc * 16, true);
-            }
-        }
-        asm volatile("cp.async.commit_group;\n" ::: "memory");
-    }
-    // (2) row j's state piece -> this lane's ring slot; rows are E*N floats apart
-    const size_t srow = (size_t)p.E * kN;
-    const float* sbase = p.ssm_state + ((size_t)b0 * p.E + ec) * kN + 4 * q;
-    auto issue = [&](int j) { step_cp_async16(&ring[j % kStepStages][tid], sbase + (size_t)j * srow, true); };
-#pragma unroll
-    for (int j = 0; j < kStepStages - 1; ++j) {
-        if (j < nb) issue(j);
-        asm volatile("cp.async.commit_group;\n" ::: "memory");
-    }
     const float4 w = __ldg(reinterpret_cast<const float4*>(p.conv_w) + ec);
     const float cb = __ldg(p.conv_b + ec);
     const float db = __ldg(p.dt_bias + ec);
@@ -122,82 +107,79 @@ __global__ void __launch_bounds__(kStepThreads) step_kernel(StepParams p, int ro
         A2[2] = -ex2_approx(a4.z * kLog2e) * kLog2e;
         A2[3] = -ex2_approx(a4.w * kLog2e) * kLog2e;
     }
-    asm volatile("cp.async.wait_group %0;\n" ::"n"(kStepStages - 1) : "memory");   // (1) landed
-    __syncthreads();
+    const T* xg = static_cast<const T*>(p.x);
+    const T* zg = static_cast<const T*>(p.z);
+    const T* dg = static_cast<const T*>(p.dt_raw);
+    T* cc = static_cast<T*>(p.conv_cache);
+    T* yg = static_cast<T*>(p.y);
+    const unsigned char* Bg = static_cast<const unsigned char*>(p.Bm);
+    const unsigned char* Cg = static_cast<const unsigned char*>(p.Cm);
 
-    const int co = (ec - e0) * S;                     // this channel's byte offset in a window
-    // Rows go in rounds of four: lane q computes the conv / SiLU / dt prologue
-    // and SiLU(z) of row j0+q only; each row's dt and dt*u reach the other
-    // three lanes of the channel by shuffles, and the row's owner lane puts
-    // its y in shared memory.
 #pragma unroll 1
     for (int j0 = 0; j0 < nb; j0 += 4) {
-        const int jq = min(j0 + q, nb - 1);
-        float uq, dtq, dtuq, gzq;
-        {
-            const float x_t = Io::sload(&small[jq][0][co]);
-            float xc = fmaf(w.x, Io::sload(&small[jq][3][co]), cb);
-            xc = fmaf(w.y, Io::sload(&small[jq][4][co]), xc);
-            xc = fmaf(w.z, Io::sload(&small[jq][5][co]), xc);
-            xc = fmaf(w.w, x_t, xc);
-            uq = silu(xc);
-            dtq = dt_from_raw(Io::sload(&small[jq][2][co]) + db);
-            dtuq = kZoh ? uq : dtq * uq;                  // input factor of Bbar u
-            gzq = silu(Io::sload(&small[jq][1][co]));
-        }
+        const int nr = min(4, nb - j0);               // rows of this round (block-uniform)
+        // ---- loads of the round, all before the first use
+        const size_t rq = (size_t)(b0 + j0 + min(q, nr - 1));   // this lane's prologue row
+        const T xr = xg[rq * E + ec];                  // raw bits: also the cache's new last row
+        const float z_t = Io::load(zg + rq * E + ec);
+        const float d_t = Io::load(dg + rq * E + ec);
+        T* ccq = cc + rq * (kK - 1) * E + ec;          // cache rows 0 .. K-2 of row rq
+        const T c0 = ccq[0], c1 = ccq[E], c2 = ccq[2 * E];
+        float* st = p.ssm_state + ((size_t)(b0 + j0) * E + ec) * kN + 4 * q;   // row j0's state vector
+        const size_t bco = (size_t)(b0 + j0) * kN * S;                          // row j0's B / C row
+        float4 hs[4];
+        StepQuad<Io> Bq[4], Cq[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const int j = j0 + k;
-            if (j >= nb) break;                           // block-uniform
-            const int b = b0 + j;
-            if (j + kStepStages - 1 < nb) issue(j + kStepStages - 1);
-            asm volatile("cp.async.commit_group;\n" ::: "memory");
-            asm volatile("cp.async.wait_group %0;\n" ::"n"(kStepStages - 1) : "memory");   // row j landed
+            if (k < nr) {
+                hs[k] = *reinterpret_cast<const float4*>(st + k * srow);
+                Bq[k].load(Bg + bco + k * kN * S, q);
+                Cq[k].load(Cg + bco + k * kN * S, q);
+            }
+        }
+        // ---- prologue of row rq: conv over (cache 0, 1, 2, x_t), SiLU, dt, gate
+        float xc = fmaf(w.x, step_f(c0), cb);
+        xc = fmaf(w.y, step_f(c1), xc);
+        xc = fmaf(w.z, step_f(c2), xc);
+        xc = fmaf(w.w, step_f(xr), xc);
+        const float uq = silu(xc);
+        const float dtq = dt_from_raw(d_t + db);
+        const float fq = kZoh ? uq : dtq * uq;        // input factor of Bbar u
+        const float gzq = silu(z_t);
+        // ---- the round's rows: quadrant update, state store, partial C . h
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (k >= nr) break;                       // block-uniform
             const float dt = __shfl_sync(0xffffffffu, dtq, k, 4);
-            const float dtu = __shfl_sync(0xffffffffu, dtuq, k, 4);
-            float Bq[4], Cq[4];
-            Io::sload4(&bcs[j][0][4 * q * S], Bq);
-            Io::sload4(&bcs[j][1][4 * q * S], Cq);
-            const float4 hq = ring[j % kStepStages][tid];
-            float h[4] = {hq.x, hq.y, hq.z, hq.w};
-            float acc = 0.0f;
+            const float f = __shfl_sync(0xffffffffu, fq, k, 4);
+            float Bv[4], Cv[4];
+            Bq[k].unpack(Bv);
+            Cq[k].unpack(Cv);
+            float h[4] = {hs[k].x, hs[k].y, hs[k].z, hs[k].w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const float a = ex2_approx(dt * A2[i]);
                 // first-order: (dt u) B;  ZOH: u ((exp(dt A) - 1) / A) B
-                const float uin = kZoh ? dtu * zoh_bbar(dt, dt * A2[i] * kLn2, a, kLog2e / A2[i]) : dtu;
-                h[i] = fmaf(a, h[i], uin * Bq[i]);
-                acc = fmaf(Cq[i], h[i], acc);
+                const float uin = kZoh ? f * zoh_bbar(dt, dt * A2[i] * kLn2, a, kLog2e / A2[i]) : f;
+                h[i] = fmaf(a, h[i], uin * Bv[i]);
+                acc[k] = fmaf(Cv[i], h[i], acc[k]);
             }
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            if (live) *reinterpret_cast<float4*>(const_cast<float*>(sbase) + (size_t)j * srow) =
-                          make_float4(h[0], h[1], h[2], h[3]);
-            if (live && q == k) Io::store(reinterpret_cast<T*>(&yst[j][co]), fmaf(Dv, uq, acc) * gzq);
+            if (live) *reinterpret_cast<float4*>(st + k * srow) = make_float4(h[0], h[1], h[2], h[3]);
         }
-    }
-    // (3) y and the shifted conv caches of all rows, 16-byte pieces: cache row
-    // i <- cache row i+1, the last <- x_t (exact copies of the raw bits; every
-    // read of the old cache happened in (1), so in-place updates are safe)
-    __syncthreads();
-    {
-        constexpr int kPw = kWin / 16;
-        const size_t row_bytes = (size_t)p.E * S;
-        for (int i = tid; i < nb * kK * kPw; i += kStepThreads) {
-            const int j = i / (kK * kPw), t = i - j * (kK * kPw), k = t / kPw, pc = t - k * kPw;
-            const size_t col = (size_t)e0 * S + (size_t)pc * 16;
-            if (col + 16 > row_bytes) continue;          // E*S is a multiple of 16
-            const int b = b0 + j;
-            unsigned char* dst;
-            const unsigned char* src;
-            if (k == 0) {                                // y
-                dst = static_cast<unsigned char*>(p.y) + (size_t)b * row_bytes + col;
-                src = &yst[j][pc * 16];
-            } else {                                     // cache row k-1
-                dst = static_cast<unsigned char*>(p.conv_cache) + ((size_t)b * (kK - 1) + (k - 1)) * row_bytes + col;
-                src = k < kK - 1 ? &small[j][3 + k][pc * 16] : &small[j][0][pc * 16];
-            }
-            *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+        // ---- reduce-scatter over the channel's four lanes: lanes with q & 2
+        // keep rows 2, 3 (then q & 1 picks the odd row), so lane q ends with
+        // the total of round row q
+        const bool hi = (q & 2) != 0, lo = (q & 1) != 0;
+        const float r0 = (hi ? acc[2] : acc[0]) + __shfl_xor_sync(0xffffffffu, hi ? acc[0] : acc[2], 2);
+        const float r1 = (hi ? acc[3] : acc[1]) + __shfl_xor_sync(0xffffffffu, hi ? acc[1] : acc[3], 2);
+        const float tot = (lo ? r1 : r0) + __shfl_xor_sync(0xffffffffu, lo ? r0 : r1, 1);
+        if (live && q < nr) {
+            Io::store(yg + rq * E + ec, fmaf(Dv, uq, tot) * gzq);
+            // shifted cache: row i <- row i+1, the last <- x_t (raw bits)
+            ccq[0] = c1;
+            ccq[E] = c2;
+            ccq[2 * E] = xr;
         }
     }
 }
