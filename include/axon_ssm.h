@@ -354,9 +354,9 @@ AXON_API axon_status axon_ssm_carry_fold(int P, int r, int B, int E, int N, cons
  * NULL (zeros); h_out (B,H,P,N) float32, may be h0 itself.  P == 64, N == 128
  * and io == AXON_BF16 only (else AXON_ERR_UNSUPPORTED).  The products run on
  * the tcgen05 tensor cores with bf16 operands (the decayed chunk Gram matrix
- * with D on its diagonal, the dt-weighted x, and the carried state split in
- * two bf16 parts) and float32 accumulators; the carried state itself is
- * float32.  To fill the GPU when B * H is small the sequence is cut into
+ * with D on its diagonal and the carried state, each split in two bf16 parts,
+ * hi and the rounding residual lo; the dt-weighted x) and float32
+ * accumulators; the carried state itself is float32.  To fill the GPU when B * H is small the sequence is cut into
  * `segments` runs of whole 128-token chunks (0: chosen for the current
  * device, about one walk per SM; capped at one per chunk and 64): a first
  * walk over pieces of every segment but the last gives their local end

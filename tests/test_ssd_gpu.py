@@ -4,15 +4,15 @@ the products on tcgen05 tensor-core MMAs into tensor memory) against the fp64
 oracle's ``ssd_scan`` on the same bf16 inputs, for one segment, forced
 segment counts and the automatic plan.
 
-Tolerance.  The tensor-core products take bf16 operands: the decayed chunk
-Gram matrix G_ij exp(acum_i - acum_j) dt_j (plus D on its diagonal) and the
-weighted x rows w_j x_j (relative rounding 2^-9 each); the carried state
-enters the inter-chunk term as two bf16 parts (about 2^-17); accumulation and
-the carried state are float32.  The errors of the
-many products summed into each output are independent, so the error is a
-fraction of a percent of the output's rms scale: elementwise |got - ref| <=
-3e-2 * max(rms(ref), |ref|) and normwise ||got - ref|| / ||ref|| <= 1e-2, for
-y and for the final state.
+Tolerance: the bf16 output bound, elementwise |got - ref| <= 2e-2 *
+max(1, |ref|) per head, and normwise ||got - ref|| / ||ref|| <= 1e-2, for y
+and for the final state.  The tensor-core products take bf16 operands: the
+decayed chunk Gram matrix M = G_ij exp(acum_i - acum_j) dt_j (plus D on its
+diagonal) and the carried state each enter as a hi + lo pair of bf16 parts
+(about 16 significant bits), the weighted x rows w_j x_j as one bf16 value,
+x itself is exact; accumulation and the carried state are float32.  The
+float64 model of these roundings (tests/test_ssd_rounding_model.py) stays
+within 0.6 of the bound on the Mamba-2 workload's most cancelling heads.
 """
 import math
 
@@ -31,10 +31,9 @@ def close(got, ref, what):
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (what, got.shape, ref.shape)
     assert np.all(np.isfinite(got)), what + ": non-finite"
-    scale = max(float(np.sqrt(np.mean(ref ** 2))), 1e-30)
-    err = np.abs(got - ref) / np.maximum(scale, np.abs(ref))
+    err = np.abs(got - ref) / np.maximum(1.0, np.abs(ref))
     rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
-    assert err.max() <= 3e-2, f"{what}: worst {err.max():.3g} of scale, {int((err > 3e-2).sum())} elements; normwise {rel:.3g}"
+    assert err.max() <= 2e-2, f"{what}: worst {err.max():.3g} of max(1, |ref|), {int((err > 2e-2).sum())} elements; normwise {rel:.3g}"
     assert rel <= 1e-2, f"{what}: normwise {rel:.3g}"
 
 

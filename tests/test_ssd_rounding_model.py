@@ -1,17 +1,21 @@
 """The error budget behind the SSD GPU tests' tolerance, made checkable on CPU.
 
 A float32 / bf16 model of the arithmetic the SSD walk performs (not its code):
-128-token chunks; the decayed Gram matrix M rounded to bf16, with D on its
-diagonal and, below the diagonal 32-token blocks, the decay factorised as
-2^(acum_i - acum_r) * dt_j 2^(acum_r - acum_j) (r the block's last token);
-the state weights w_j x_j rounded to bf16; the carried state float32, entering
+128-token chunks; the decayed Gram matrix M, with D on its diagonal and, below
+the diagonal 32-token blocks, the decay factorised as
+2^(acum_i - acum_r) * dt_j 2^(acum_r - acum_j) (r the block's last token),
+entering M x as a bf16 pair (hi = M rounded, lo = the residual rounded); the
+state weights w_j x_j rounded to bf16; the carried state float32, entering
 C S^T as a bf16 pair (hi = its top 16 bits, lo = the rest rounded); products
 accumulated exactly (float64 here, float32 on the GPU); y rounded to bf16.
 Against the fp64 oracle on the GPU tests' inputs this model stays within
-2% of max(rms, |ref|) elementwise and 0.5% normwise per head, so the GPU
-tests' 3% / 1% bounds leave room for float32 accumulation order.  With a
-single bf16 copy of the state instead of the pair, one case exceeds 3%:
-that is why the kernel splits it.
+half of the bf16 output bound |got - ref| <= 2e-2 max(1, |ref|) elementwise
+(0.6 of it on the Mamba-2 workload's most cancelling heads) and 0.5%
+normwise per head, so the GPU tests' bound leaves room for float32
+accumulation order.  With a single bf16 copy of M, heads of the Mamba-2
+workload exceed that bound; with a single bf16 copy of the state instead of
+the pair, one small case exceeds 3% of max(rms, |ref|): that is why the
+kernel splits both.
 """
 import math
 
@@ -45,7 +49,7 @@ def dt_of(v):
     return np.clip(sp, 1e-4, 100.0)
 
 
-def model(inp, with_state, split_state=True):
+def model(inp, with_state, split_state=True, split_m=True, heads=None):
     x = inp["x"].float().numpy().astype(np.float64)
     dtr = inp["dt_raw"].float().numpy().astype(np.float64)
     Bm = inp["B"].float().numpy().astype(np.float64)
@@ -58,7 +62,7 @@ def model(inp, with_state, split_state=True):
     y = np.zeros_like(x)
     hout = np.zeros((Bs, H, P, N))
     for b in range(Bs):
-        for h in range(H):
+        for h in (range(H) if heads is None else heads):
             A2 = f32(-math.exp(Alog[h]) * LOG2E)
             S = f32(inp["h0"][b, h].numpy()) if with_state else np.zeros((P, N))
             for t0 in range(0, L, Q):
@@ -87,7 +91,11 @@ def model(inp, with_state, split_state=True):
                             blk = G[rows, cols] * d * dt[j][None, :]
                             blk[np.arange(BLK), np.arange(BLK)] += D[h]
                             M[rows, cols] = blk
-                M = bf(M)
+                if split_m:
+                    Mh = bf(M)
+                    M = Mh + bf(M - Mh)
+                else:
+                    M = bf(M)
                 if split_state:
                     Sh = hi_part(S)
                     Sb = Sh + bf(S - Sh)
@@ -102,10 +110,16 @@ def model(inp, with_state, split_state=True):
 
 
 def errors(got, ref):
-    scale = max(float(np.sqrt(np.mean(ref ** 2))), 1e-30)
-    err = np.abs(got - ref) / np.maximum(scale, np.abs(ref))
+    """(worst |got - ref| / max(1, |ref|), normwise relative error)"""
+    err = np.abs(got - ref) / np.maximum(1.0, np.abs(ref))
     rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-30)
     return float(err.max()), float(rel)
+
+
+def errors_of_scale(got, ref):
+    """worst |got - ref| / max(rms(ref), |ref|)"""
+    scale = max(float(np.sqrt(np.mean(ref ** 2))), 1e-30)
+    return float((np.abs(got - ref) / np.maximum(scale, np.abs(ref))).max())
 
 
 def oracle_ref(inp, with_state):
@@ -124,8 +138,8 @@ def test_rounding_model_within_budget(L, with_state):
     for hd in range(y.shape[2]):
         ey, ry = errors(y[:, :, hd], y_ref[:, :, hd])
         eh, rh = errors(h[:, hd], h_ref[:, hd])
-        assert ey <= 2e-2 and ry <= 5e-3, (L, with_state, hd, ey, ry)
-        assert eh <= 2e-2 and rh <= 5e-3, (L, with_state, hd, eh, rh)
+        assert ey <= 1e-2 and ry <= 5e-3, (L, with_state, hd, ey, ry)
+        assert eh <= 1e-2 and rh <= 5e-3, (L, with_state, hd, eh, rh)
 
 
 def test_rounding_model_at_the_clip_bounds():
@@ -140,8 +154,8 @@ def test_rounding_model_at_the_clip_bounds():
     for hd in range(3):
         ey, ry = errors(y[:, :, hd], y_ref[:, :, hd])
         eh, rh = errors(h[:, hd], h_ref[:, hd])
-        assert ey <= 2e-2 and ry <= 5e-3, (hd, ey, ry)
-        assert eh <= 2e-2 and rh <= 5e-3, (hd, eh, rh)
+        assert ey <= 1e-2 and ry <= 5e-3, (hd, ey, ry)
+        assert eh <= 1e-2 and rh <= 5e-3, (hd, eh, rh)
 
 
 def test_single_bf16_state_copy_would_break_the_bound():
@@ -151,5 +165,31 @@ def test_single_bf16_state_copy_would_break_the_bound():
     inp = W.make_ssd_inputs(W.SSD_WORKLOAD_BY_NAME["small_ssd"], with_state=True, L=1000)
     y, _ = model(inp, True, split_state=False)
     y_ref, _ = oracle_ref(inp, True)
-    worst = max(errors(y[:, :, hd], y_ref[:, :, hd])[0] for hd in range(y.shape[2]))
+    worst = max(errors_of_scale(y[:, :, hd], y_ref[:, :, hd]) for hd in range(y.shape[2]))
     assert worst > 3e-2, worst
+
+
+# heads of the Mamba-2 workload (B1 L4096, 64 heads) whose outputs cancel most
+MAMBA2_HEADS = (22, 31, 41)
+
+
+def test_m_split_keeps_the_mamba2_heads_within_the_bound():
+    """Why the walk splits M: on the Mamba-2 workload's most cancelling heads,
+    a single bf16 copy of M puts elements beyond 2e-2 max(1, |ref|); the
+    hi + lo pair keeps them within 0.6 of it (what remains is the rounding of
+    w x to bf16 and of y itself)."""
+    sw = W.SSD_WORKLOAD_BY_NAME["mamba2_ssd"]
+    inp = W.make_ssd_inputs(sw, with_state=True)
+    heads = list(MAMBA2_HEADS)
+    sub = {k: v for k, v in inp.items()}
+    sub["x"], sub["dt_raw"] = inp["x"][:, :, heads], inp["dt_raw"][:, :, heads]
+    for k in ("dt_bias", "A_log", "D"):
+        sub[k] = inp[k][heads]
+    sub["h0"] = inp["h0"][:, heads]
+    y_ref, _ = oracle_ref(sub, True)
+    y1, _ = model(sub, True, split_m=False)
+    y2, _ = model(sub, True, split_m=True)
+    single = max(errors(y1[:, :, hd], y_ref[:, :, hd])[0] for hd in range(len(heads)))
+    pair = max(errors(y2[:, :, hd], y_ref[:, :, hd])[0] for hd in range(len(heads)))
+    assert single > 2e-2, single
+    assert pair <= 1.2e-2, pair
