@@ -447,6 +447,21 @@ AXON_API axon_status axon_ssm_block_fwd(
 AXON_API axon_status axon_gemm_bf16(int M, int N, int K, const void *A, int lda, const void *W, int ldw,
                                     void *C, int ldc, int *err, axon_stream_t stream);
 
+/*
+ * The FMA-pipe exp2 on its own (tests): y[i] = 2^x[i] for x[i] <= 0, computed
+ * with float32 fused multiply-adds instead of the MUFU unit -- Cody and
+ * Waite's reduction 2^x = 2^n 2^f, n = round(x), f in [-1/2, 1/2], 2^f by a
+ * degree-6 minimax polynomial with constant term 1 (relative error within
+ * 1.3 * 2^-24; 2^0 is exactly 1), 2^n added to the exponent field; x below
+ * -126 gives 2^-126.  Kernels whose MUFU pipe is their busiest can take part
+ * of their decays exp(dt A) = 2^(dt A log2 e) this way (page "Axon-SSM:
+ * Selective State Space Model for Apple Silicon", "ZOH discretisation").
+ * x and y are n float32 device values, 16-byte aligned; y may be x itself,
+ * not otherwise overlap it.  n < 0 or a NULL pointer with n > 0 is
+ * AXON_ERR_INVALID_ARG.  Enqueued on `stream`.
+ */
+AXON_API axon_status axon_exp2_fma(const float *x, float *y, long long n, axon_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -75,6 +75,8 @@ _lib.axon_ssd_workspace_bytes.argtypes = [_i] * 6
 _lib.axon_ssd_scan_fwd.restype = _i
 _lib.axon_ssd_scan_fwd.argtypes = [_i] * 6 + [_vp] * 10 + [_i, _vp, _sz, _vp]
 _lib.axon_gemm_bf16.restype = _i
+_lib.axon_exp2_fma.restype = _i
+_lib.axon_exp2_fma.argtypes = [_vp, _vp, ctypes.c_longlong, _vp]
 _lib.axon_gemm_bf16.argtypes = [_i] * 3 + [_vp, _i, _vp, _i, _vp, _i, _vp, _vp]
 _lib.axon_ssm_block_workspace_bytes.restype = _sz
 _lib.axon_ssm_block_workspace_bytes.argtypes = [_i] * 7
@@ -297,6 +299,23 @@ def axon_gemm_bf16(M, N, K, A, lda, W, ldw, C, ldc, err=None, stream=None, *, ra
     if raise_on_error:
         _check(rc, "axon_gemm_bf16")
     return rc
+
+
+def axon_exp2_fma(x, y, n, stream=None, *, raise_on_error=True) -> int:
+    rc = _lib.axon_exp2_fma(_p(x), _p(y), int(n), _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_exp2_fma")
+    return rc
+
+
+def exp2_fma(x, *, out=None, stream=None):
+    """2^x of a contiguous float32 CUDA tensor through the FMA-pipe exp2."""
+    import torch
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("exp2_fma: x must be a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x) if out is None else out
+    axon_exp2_fma(x.data_ptr(), y.data_ptr(), x.numel(), stream=stream)
+    return y
 
 
 def gemm_bf16(A, W, *, out=None, stream=None, check=True):

@@ -471,6 +471,18 @@ axon_status static_scratch_address(void** out) {
 
 using namespace axon;
 
+namespace axon {
+// y = 2^x through exp2_fma2 (the FMA-pipe exp2), two values per thread.
+__global__ void exp2_fma_kernel(const float* x, float* y, long long n) {
+    const long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const bool pair = i + 1 < n;
+    const float2 v = exp2_fma2(make_float2(x[i], pair ? x[i + 1] : x[i]));
+    y[i] = v.x;
+    if (pair) y[i + 1] = v.y;
+}
+}  // namespace axon
+
 extern "C" {
 
 int axon_ssm_abi_version(void) { return kAbiVersion; }
@@ -719,6 +731,18 @@ axon_status axon_ssm_carry_fold(int P, int r, int B, int E, int N, const float* 
     const size_t total = (size_t)B * E * kN;
     carry_fold_kernel<<<(unsigned)((total + 127) / 128), 128, 0, static_cast<cudaStream_t>(stream)>>>(
         r, B, E, A_log, h_loc, dt_sum, h_in);
+    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+}
+
+axon_status axon_exp2_fma(const float* x, float* y, long long n, axon_stream_t stream) {
+    if (n < 0) return AXON_ERR_INVALID_ARG;
+    if (n == 0) return AXON_OK;
+    if (!x || !y) return AXON_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y)) return AXON_ERR_ALIGNMENT;
+    if (overlaps(x, (size_t)n * 4, y, (size_t)n * 4) && x != y) return AXON_ERR_INVALID_ARG;
+    const long long threads = (n + 1) / 2;
+    if ((threads + 255) / 256 > 0x7fffffffLL) return AXON_ERR_UNSUPPORTED;
+    exp2_fma_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
 

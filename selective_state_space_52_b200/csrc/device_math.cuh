@@ -37,6 +37,35 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return y;
 }
 
+// 2^x for a pair of x <= 0 on the FMA pipe (packed float32 pairs), for
+// kernels whose MUFU pipe is the busiest: Cody and Waite's reduction
+// 2^x = 2^n 2^f, n = round(x), f = x - n in [-1/2, 1/2] (exact: adding
+// 1.5 * 2^23 rounds to an integer, subtracting it back and then n from x are
+// exact), 2^f by the degree-6 polynomial with constant term 1 (2^0 is exactly
+// 1, a masked token's decay) minimising the largest relative error on
+// [-1/2, 1/2] (Remez exchange; coefficients from
+// selective_state_space_52_b200/exp2_poly_fit.py, rounded to float32; the
+// float32 evaluation stays within 1.3 * 2^-24 relative), and 2^n added to the
+// exponent field (n << 23: the low 9 bits of 1.5 * 2^23 are zero, so the
+// sum's bit pattern shifted left by 23 is n << 23).  x is clamped at -126, so
+// the result stays a normal float (2^-126 where MUFU's ftz form gives 0).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    constexpr float kRound = 12582912.0f;            // 1.5 * 2^23
+    const float2 xc = make_float2(fmaxf(x.x, -126.0f), fmaxf(x.y, -126.0f));
+    const float2 j = __fadd2_rn(xc, make_float2(kRound, kRound));
+    const float2 n = __fadd2_rn(j, make_float2(-kRound, -kRound));
+    const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), xc);
+    float2 p = make_float2(0x1.446c7ep-13f, 0x1.446c7ep-13f);
+    p = __ffma2_rn(p, f, make_float2(0x1.5f88fep-10f, 0x1.5f88fep-10f));
+    p = __ffma2_rn(p, f, make_float2(0x1.3b29e4p-7f, 0x1.3b29e4p-7f));
+    p = __ffma2_rn(p, f, make_float2(0x1.c6ae2cp-5f, 0x1.c6ae2cp-5f));
+    p = __ffma2_rn(p, f, make_float2(0x1.ebfbe0p-3f, 0x1.ebfbe0p-3f));
+    p = __ffma2_rn(p, f, make_float2(0x1.62e432p-1f, 0x1.62e432p-1f));
+    p = __ffma2_rn(p, f, make_float2(1.0f, 1.0f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
+}
+
 // SiLU(v) = v * sigmoid(v) = v / (1 + 2^(-v log2 e)).  For v -> -inf the
 // exponential overflows to +inf and the reciprocal to 0, giving -0.
 __device__ __forceinline__ float silu(float v) {

@@ -147,6 +147,13 @@ template <> struct SmemIo<IoBF16> {
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
+// State pairs (of 8) whose decays the direct walk computes on the FMA pipe
+// (exp2_fma2) instead of MUFU: the walk issues 16 MUFU decays and 6 prologue
+// transcendentals per token and channel against about 70 other instructions,
+// so MUFU is its busiest pipe; each pair moved costs about 12 issue slots and
+// frees 16 cycles of the MUFU pipe.
+constexpr int kDirectFmaPairs = 0;
+
 // Walks the flat indices w = tid, tid + NT, ... of a (rows x per_row) grid of
 // copy pieces as (row, piece) pairs without a division per step: the stride NT
 // is split once into whole rows (drow) and a remainder (dpc).
@@ -354,7 +361,8 @@ __global__ void __launch_bounds__(512, kMinBlocks) scan_chunked_kernel(ChunkPara
                     for (int hh = 0; hh < 2; ++hh) {
                         const int pq = 2 * q + hh;
                         const float2 arg = __fmul2_rn(dt2, s2[pq]);
-                        const float2 a = f2(ex2_approx(arg.x), ex2_approx(arg.y));
+                        // the first kDirectFmaPairs state pairs on the FMA pipe, the rest on MUFU
+                        const float2 a = pq < kDirectFmaPairs ? exp2_fma2(arg) : f2(ex2_approx(arg.x), ex2_approx(arg.y));
                         const float2 bb = hh ? f2(bv.z, bv.w) : f2(bv.x, bv.y);
                         const float2 cc = hh ? f2(cv.z, cv.w) : f2(cv.x, cv.y);
                         float2 uin2 = dtu2;

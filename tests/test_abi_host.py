@@ -362,3 +362,16 @@ def test_ssd_wait_probe_rejects_bad_arguments(lib):
     assert f(FAKE + 2, 64, None) == INVALID                     # not 4-byte aligned
     assert f(FAKE, 0, None) == INVALID
     assert f(FAKE, (1 << 16) + 1, None) == INVALID
+
+
+def test_exp2_fma_argument_checks(lib):
+    """The FMA-pipe exp2's host checks (nothing is launched on an error)."""
+    f = lib.axon_exp2_fma
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p]
+    assert f(None, None, 0, None) == 0                          # nothing to do
+    assert f(FAKE, FAKE + 4096, -1, None) == INVALID
+    assert f(None, FAKE, 8, None) == INVALID
+    assert f(FAKE, None, 8, None) == INVALID
+    assert f(FAKE + 4, FAKE + 4096, 8, None) == ALIGNMENT
+    assert f(FAKE, FAKE + 16, 8, None) == INVALID               # partial overlap
