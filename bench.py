@@ -846,6 +846,9 @@ def main(argv=None):
     ap.add_argument("--ssd-only", action="store_true",
                     help="run only the Mamba-2 (SSD) layer-core measurement and print it as one JSON line "
                          "(for profiling its kernels alone)")
+    ap.add_argument("--block-only", action="store_true",
+                    help="run only the whole-layer measurement (key block) and print it as one JSON line "
+                         "(for profiling the layer's kernels alone)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)     # at least 3 untimed warm-up steps
     wl = W.WORKLOAD_BY_NAME[args.workload]
@@ -871,6 +874,13 @@ def main(argv=None):
         dev = torch.device("cuda", 0)
         torch.cuda.set_device(dev)
         print(json.dumps({"ssd": bench_ssd(dev)}), flush=True)
+        return 0
+    if args.block_only:
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA GPU for --block-only")
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps({"block": bench_block(dev)}), flush=True)
         return 0
     return run_axon(args, wl)
 

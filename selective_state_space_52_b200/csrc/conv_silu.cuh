@@ -21,10 +21,39 @@ struct ConvParams {
 constexpr int kConvRun = 32;     // tokens per thread
 constexpr int kConvThreads = 128;
 
+// 8 consecutive io values <-> float32: one 16-byte vector at bf16, two at fp32
+__device__ __forceinline__ void conv_ld8(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 q = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void conv_ld8(const float* p, float (&v)[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void conv_st8(__nv_bfloat16* p, const float (&v)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+__device__ __forceinline__ void conv_st8(float* p, const float (&v)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
 // One thread: 8 consecutive channels (one 16-byte bf16 vector, two fp32
-// vectors) of one batch row over kConvRun consecutive tokens; the K-1 previous
-// inputs of each channel slide in registers.  grid = (ceil(E/8 / 128),
-// ceil(L / kConvRun), B).  E is a multiple of 8.
+// vectors) of one batch row over kConvRun consecutive tokens, loaded and
+// stored as whole vectors; the K-1 previous inputs of each channel slide in
+// registers.  grid = (ceil(E/8 / 128), ceil(L / kConvRun), B).  E is a
+// multiple of 8 and the rows 16-byte aligned.
 template <class Io>
 __global__ void __launch_bounds__(kConvThreads) conv_silu_kernel(ConvParams p) {
     using T = typename Io::T;
@@ -38,7 +67,7 @@ __global__ void __launch_bounds__(kConvThreads) conv_silu_kernel(ConvParams p) {
     const T* cc = static_cast<const T*>(p.conv_cache_in);
     T* u = static_cast<T*>(p.u);
 
-    float w[8][kK], cbias[8], win[8][kK - 1];
+    float w[8][kK], cbias[8], win[kK - 1][8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         const float4 wv = __ldg(reinterpret_cast<const float4*>(p.conv_w) + e0 + c);
@@ -49,25 +78,29 @@ __global__ void __launch_bounds__(kConvThreads) conv_silu_kernel(ConvParams p) {
 #pragma unroll
     for (int j = 0; j < kK - 1; ++j) {
         const int t = t0 - (kK - 1) + j;
-        const T* row = nullptr;
-        if (t >= 0) row = x + ((size_t)b * p.L + t) * p.E + e0;
-        else if (cc) row = cc + ((size_t)b * (kK - 1) + (kK - 1 + t)) * p.E + e0;
+        if (t >= 0) conv_ld8(x + ((size_t)b * p.L + t) * p.E + e0, win[j]);
+        else if (cc) conv_ld8(cc + ((size_t)b * (kK - 1) + (kK - 1 + t)) * p.E + e0, win[j]);
+        else {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) win[c][j] = row ? Io::load(row + c) : 0.0f;
+            for (int c = 0; c < 8; ++c) win[j][c] = 0.0f;
+        }
     }
-    for (int t = t0; t < t1; ++t) {
-        const T* row = x + ((size_t)b * p.L + t) * p.E + e0;
-        T* out = u + ((size_t)b * p.L + t) * p.E + e0;
+    const T* row = x + ((size_t)b * p.L + t0) * p.E + e0;
+    T* out = u + ((size_t)b * p.L + t0) * p.E + e0;
+#pragma unroll 4
+    for (int t = t0; t < t1; ++t, row += p.E, out += p.E) {
+        float xt[8], o[8];
+        conv_ld8(row, xt);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            const float xt = Io::load(row + c);
-            float xc = fmaf(w[c][0], win[c][0], cbias[c]);
-            xc = fmaf(w[c][1], win[c][1], xc);
-            xc = fmaf(w[c][2], win[c][2], xc);
-            xc = fmaf(w[c][3], xt, xc);
-            win[c][0] = win[c][1]; win[c][1] = win[c][2]; win[c][2] = xt;
-            Io::store(out + c, silu(xc));
+            float xc = fmaf(w[c][0], win[0][c], cbias[c]);
+            xc = fmaf(w[c][1], win[1][c], xc);
+            xc = fmaf(w[c][2], win[2][c], xc);
+            xc = fmaf(w[c][3], xt[c], xc);
+            win[0][c] = win[1][c]; win[1][c] = win[2][c]; win[2][c] = xt[c];
+            o[c] = silu(xc);
         }
+        conv_st8(out, o);
     }
 }
 

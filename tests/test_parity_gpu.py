@@ -283,6 +283,29 @@ def test_step_matches_oracle_step(cuda_lib, io):
     assert torch.equal(cc.cpu(), torch.from_numpy(cc_ref).to(cc.dtype))
 
 
+# Decode blocks that walk several rounds of four rows and end on a partial one
+# (B = 30: blocks of 12 rows, the last with 6; B = 50 with E % 32 == 8: a
+# channel tail in every round), through the occupancy-sized row plan.
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("B,E", [(30, 4096), (50, 2056)])
+def test_step_multi_round_blocks(cuda_lib, io, B, E):
+    from selective_state_space_52_b200 import axon_ssm
+    wl = W.custom(B, 1, E, io=io, seed=91 + B)
+    inp = W.make_inputs(wl, with_state=True)
+    d = to_dev(inp)
+    params = {k: d[k] for k in axon_ssm.PARAM_KEYS}
+    cc, ss = d["conv_cache"].clone(), d["ssm_state"].clone()
+    y = axon_ssm.step(*(d[k][:, 0].contiguous() for k in ("x", "z", "dt_raw", "B", "C")), params, (cc, ss))
+    torch.cuda.synchronize()
+    y_ref, cc_ref, ss_ref = oracle.step(inp["x"][:, 0], inp["z"][:, 0], inp["dt_raw"][:, 0],
+                                        inp["B"][:, 0], inp["C"][:, 0], inp["conv_w"],
+                                        inp["conv_b"], inp["dt_bias"], inp["A_log"], inp["D"],
+                                        inp["conv_cache"], inp["ssm_state"])
+    check_close(y.float().cpu().numpy(), y_ref, tol_for(io, y_ref), "step y")
+    check_close(ss.cpu().numpy(), ss_ref, state_tol(ss_ref), "step state")
+    assert torch.equal(cc.cpu(), torch.from_numpy(cc_ref).to(cc.dtype))
+
+
 # The split-chunk quadrant scan with each number of runs per chunk (W warps per
 # 8 channels; W = 1: runs of 32 tokens, else 16): single tokens, ragged runs
 # and chunks, chunks whose last runs lie wholly past L, several batch rows, an
