@@ -314,10 +314,11 @@ AXON_API axon_status axon_ssm_step_ex(
  * with one exchange of per-slice summaries (the chunked associative scan of
  * the SSD article, devices as blocks; the recurrence's decay over a run of
  * tokens is exp(A * sum dt), Axon-SSM page, recurrence equation):
- *   1. every slice r >= 1 runs axon_ssm_scan_fwd from a ZERO state (its conv
- *      cache = the last K-1 inputs of slice r-1) for its end state h_loc_r,
- *      and axon_ssm_dt_sum for dt_sum_r; slice 0 runs from the true initial
- *      state, its end state is h_loc_0 and its output is final;
+ *   1. every slice r >= 1 runs axon_ssm_scan_state from a ZERO state (its
+ *      conv cache = the last K-1 inputs of slice r-1) for its end state
+ *      h_loc_r and dt_sum_r in one pass (or axon_ssm_scan_fwd and
+ *      axon_ssm_dt_sum); slice 0 runs axon_ssm_scan_fwd from the true
+ *      initial state, its end state is h_loc_0 and its output is final;
  *   2. the P (h_loc, dt_sum) pairs are exchanged (one all-gather);
  *   3. axon_ssm_carry_fold gives slice r its entering state
  *      h = h_loc_0; h = exp(A * dt_sum_j) * h + h_loc_j for j = 1 .. r-1;
@@ -338,6 +339,28 @@ AXON_API axon_status axon_ssm_dt_sum(int B, int L, int E, axon_dtype io, const v
 
 AXON_API axon_status axon_ssm_carry_fold(int P, int r, int B, int E, int N, const float *A_log,
                                          const float *h_loc, const float *dt_sum, float *h_in,
+                                         axon_stream_t stream);
+
+/*
+ * The state-only prefill of step 1 above: the conv + SiLU, dt and recurrence
+ * of axon_ssm_scan_fwd (first order) without the output side -- no z, C, D
+ * or y -- writing only the final caches (conv_cache_out: the last K-1 raw
+ * inputs; ssm_state_out: h_L) and dt_sum (B,E) float32 = the sum over t of the
+ * same step sizes the recurrence used, added in a fixed order (the same bits
+ * on every run).  Layouts, ownership and the NULL conventions of
+ * conv_cache_in / ssm_state_in as in axon_ssm_scan_fwd; L == 0 copies the
+ * caches and zeroes dt_sum.  Each cache may be updated in place
+ * (conv_cache_out == conv_cache_in, ssm_state_out == ssm_state_in); the
+ * outputs must not otherwise overlap each other or the inputs
+ * (AXON_ERR_INVALID_ARG); every pointer 16-byte aligned (AXON_ERR_ALIGNMENT).
+ * Enqueued on `stream`; needs no workspace.
+ */
+AXON_API axon_status axon_ssm_scan_state(int B, int L, int E, int N, int K, axon_dtype io,
+                                         const void *x, const void *dt_raw, const void *Bm,
+                                         const float *conv_w, const float *conv_b,
+                                         const float *dt_bias, const float *A_log,
+                                         const void *conv_cache_in, const float *ssm_state_in,
+                                         void *conv_cache_out, float *ssm_state_out, float *dt_sum,
                                          axon_stream_t stream);
 
 /*

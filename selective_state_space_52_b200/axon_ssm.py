@@ -68,6 +68,8 @@ _lib.axon_ssm_dt_sum.restype = _i
 _lib.axon_ssm_dt_sum.argtypes = [_i] * 4 + [_vp] * 3 + [_vp]
 _lib.axon_ssm_carry_fold.restype = _i
 _lib.axon_ssm_carry_fold.argtypes = [_i] * 5 + [_vp] * 4 + [_vp]
+_lib.axon_ssm_scan_state.restype = _i
+_lib.axon_ssm_scan_state.argtypes = [_i] * 6 + [_vp] * 12 + [_vp]
 _lib.axon_ssd_wait_probe.restype = _i
 _lib.axon_ssd_wait_probe.argtypes = [_vp, _i, _vp]
 _lib.axon_ssd_workspace_bytes.restype = _sz
@@ -252,6 +254,17 @@ def axon_ssm_carry_fold(P, r, B, E, N, A_log, h_loc, dt_sum, h_in, stream=None, 
                                   _stream(stream))
     if raise_on_error:
         _check(rc, "axon_ssm_carry_fold")
+    return rc
+
+
+def axon_ssm_scan_state(B, L, E, N, K, io, x, dt_raw, Bm, conv_w, conv_b, dt_bias, A_log,
+                        conv_cache_in, ssm_state_in, conv_cache_out, ssm_state_out, dt_sum, stream=None, *,
+                        raise_on_error=True) -> int:
+    rc = _lib.axon_ssm_scan_state(B, L, E, N, K, io, _p(x), _p(dt_raw), _p(Bm), _p(conv_w), _p(conv_b),
+                                  _p(dt_bias), _p(A_log), _p(conv_cache_in), _p(ssm_state_in),
+                                  _p(conv_cache_out), _p(ssm_state_out), _p(dt_sum), _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_ssm_scan_state")
     return rc
 
 
@@ -450,6 +463,23 @@ def dt_sum(dt_raw, dt_bias, *, stream=None):
     out = torch.empty(Bsz, E, dtype=torch.float32, device=dt_raw.device)
     axon_ssm_dt_sum(Bsz, L, E, _dtype_code(dt_raw.dtype), dt_raw, dt_bias, out, stream=stream)
     return out
+
+
+def scan_state(x, dt_raw, Bm, params: dict, cache=None, *, stream=None):
+    """The state-only prefill (first order): returns ((conv_cache, ssm_state),
+    dt_sum) -- the final caches and the (B, E) float32 sum of the step sizes --
+    without z, C, D or y."""
+    Bsz, L, E = x.shape
+    K = params["conv_w"].shape[1]
+    N = params["A_log"].shape[1]
+    cc_in, ss_in = (None, None) if cache is None else cache
+    dev = x.device
+    cc_out = torch.empty(Bsz, K - 1, E, dtype=x.dtype, device=dev)
+    ss_out = torch.empty(Bsz, E, N, dtype=torch.float32, device=dev)
+    dts = torch.empty(Bsz, E, dtype=torch.float32, device=dev)
+    axon_ssm_scan_state(Bsz, L, E, N, K, _dtype_code(x.dtype), x, dt_raw, Bm, params["conv_w"], params["conv_b"],
+                        params["dt_bias"], params["A_log"], cc_in, ss_in, cc_out, ss_out, dts, stream=stream)
+    return (cc_out, ss_out), dts
 
 
 def carry_fold(r, A_log, h_loc_all, dt_sum_all, *, stream=None):

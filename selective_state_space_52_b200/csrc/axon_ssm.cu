@@ -211,9 +211,9 @@ axon_status launch_quad(const ChunkParams& prm, cudaStream_t st) {
 
 // Split-chunk quadrant scan: W warps per 8 channels, each chunk cut into W
 // runs (R = 32 tokens per run for W = 1, else 8).
-template <class Io, int W, int R, bool Z>
+template <class Io, int W, int R, bool Z, bool S = false>
 axon_status launch_qsplit_t(const ChunkParams& prm, cudaStream_t st) {
-    auto kern = scan_qsplit_kernel<Io, W, R, Z>;
+    auto kern = scan_qsplit_kernel<Io, W, R, Z, S>;
     static std::atomic<unsigned long long> smem_set{0};
     if (!allow_max_smem(kern, smem_set)) return AXON_ERR_CUDA;
     const int smem = QsplitSmem(W, R, Io::kBytes).total;
@@ -223,14 +223,14 @@ axon_status launch_qsplit_t(const ChunkParams& prm, cudaStream_t st) {
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
 
-// W runs per chunk: one run of 32 tokens, or W runs of 16
-template <class Io, bool Z>
+// W runs per chunk: one run of 32 tokens, or W runs of 16 (S: the state-only form)
+template <class Io, bool Z, bool S = false>
 axon_status launch_qsplit(const ChunkParams& prm, int W, cudaStream_t st) {
     switch (W) {
-        case 1: return launch_qsplit_t<Io, 1, 32, Z>(prm, st);
-        case 2: return launch_qsplit_t<Io, 2, 16, Z>(prm, st);
-        case 4: return launch_qsplit_t<Io, 4, 16, Z>(prm, st);
-        case 8: return launch_qsplit_t<Io, 8, 16, Z>(prm, st);
+        case 1: return launch_qsplit_t<Io, 1, 32, Z, S>(prm, st);
+        case 2: return launch_qsplit_t<Io, 2, 16, Z, S>(prm, st);
+        case 4: return launch_qsplit_t<Io, 4, 16, Z, S>(prm, st);
+        case 8: return launch_qsplit_t<Io, 8, 16, Z, S>(prm, st);
     }
     return AXON_ERR_UNSUPPORTED;
 }
@@ -395,7 +395,7 @@ axon_status scan_impl(int B, int L, int E, int N, int K, axon_dtype io,
     }
 
     if (chunked || quad || octo || qsplit) {
-        ChunkParams cp;
+        ChunkParams cp{};
         cp.B = B; cp.L = L; cp.E = E;
         cp.ET = quad ? kQuadCh : (octo ? kOctoCh : cplan.ET);
         cp.tiles_per_b = quad ? (E + kQuadCh - 1) / kQuadCh : (octo ? E / kOctoCh : cplan.tiles_per_b);
@@ -744,6 +744,63 @@ axon_status axon_exp2_fma(const float* x, float* y, long long n, axon_stream_t s
     if ((threads + 255) / 256 > 0x7fffffffLL) return AXON_ERR_UNSUPPORTED;
     exp2_fma_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
+}
+
+axon_status axon_ssm_scan_state(int B, int L, int E, int N, int K, axon_dtype io,
+                                const void* x, const void* dt_raw, const void* Bm,
+                                const float* conv_w, const float* conv_b,
+                                const float* dt_bias, const float* A_log,
+                                const void* conv_cache_in, const float* ssm_state_in,
+                                void* conv_cache_out, float* ssm_state_out, float* dt_sum,
+                                axon_stream_t stream) {
+    axon_status st = check_shape(B, L, E, N, K, io);
+    if (st != AXON_OK) return st;
+    if (B == 0 || E == 0) return AXON_OK;
+    if (!conv_w || !conv_b || !dt_bias || !A_log || !conv_cache_out || !ssm_state_out || !dt_sum)
+        return AXON_ERR_INVALID_ARG;
+    if (L > 0 && (!x || !dt_raw || !Bm)) return AXON_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, dt_raw, Bm, conv_w, conv_b, dt_bias, A_log, conv_cache_in, ssm_state_in,
+                          conv_cache_out, ssm_state_out, dt_sum};
+    for (const void* q : ptrs)
+        if (q && !aligned16(q)) return AXON_ERR_ALIGNMENT;
+    const size_t sio = io_bytes(io);
+    const size_t n_in = (size_t)B * L * E * sio, n_b = (size_t)B * L * kN * sio;
+    const size_t n_cc = (size_t)B * (kK - 1) * E * sio, n_ss = (size_t)B * E * kN * sizeof(float);
+    const size_t n_dt = (size_t)B * E * sizeof(float);
+    // outputs: disjoint from each other and from every input, except each cache
+    // may be updated in place (conv_cache_out == conv_cache_in, state likewise)
+    const void* outs[] = {conv_cache_out, ssm_state_out, dt_sum};
+    const size_t nouts[] = {n_cc, n_ss, n_dt};
+    for (int i = 0; i < 3; ++i) {
+        for (int j = i + 1; j < 3; ++j)
+            if (overlaps(outs[i], nouts[i], outs[j], nouts[j])) return AXON_ERR_INVALID_ARG;
+        if (overlaps(outs[i], nouts[i], x, n_in) || overlaps(outs[i], nouts[i], dt_raw, n_in) ||
+            overlaps(outs[i], nouts[i], Bm, n_b))
+            return AXON_ERR_INVALID_ARG;
+    }
+    if (conv_cache_in != conv_cache_out && overlaps(conv_cache_in, n_cc, conv_cache_out, n_cc))
+        return AXON_ERR_INVALID_ARG;
+    if (ssm_state_in != ssm_state_out && overlaps(ssm_state_in, n_ss, ssm_state_out, n_ss))
+        return AXON_ERR_INVALID_ARG;
+    if (overlaps(conv_cache_in, n_cc, ssm_state_out, n_ss) || overlaps(conv_cache_in, n_cc, dt_sum, n_dt) ||
+        overlaps(ssm_state_in, n_ss, conv_cache_out, n_cc) || overlaps(ssm_state_in, n_ss, dt_sum, n_dt))
+        return AXON_ERR_INVALID_ARG;
+    const int sms = device_sm_count();
+    if (sms <= 0) return AXON_ERR_CUDA;
+    // the prefill's split-chunk plan, or (where the prefill prefers another
+    // kernel) eight runs per chunk for few channels and one run for many
+    int W = plan_qsplit(B, L, E, (int)sio, sms);
+    if (W == 0) W = (long long)B * E < (long long)sms * 48 ? 8 : 1;
+    if (!qsplit_fits(B, L, E, (int)sio, W)) return AXON_ERR_UNSUPPORTED;
+    ChunkParams cp{};
+    cp.B = B; cp.L = L; cp.E = E;
+    cp.x = x; cp.z = nullptr; cp.dt_raw = dt_raw; cp.Bm = Bm; cp.Cm = nullptr;
+    cp.conv_w = conv_w; cp.conv_b = conv_b; cp.dt_bias = dt_bias; cp.A_log = A_log; cp.D = nullptr;
+    cp.conv_cache_in = conv_cache_in; cp.ssm_state_in = ssm_state_in;
+    cp.y = nullptr; cp.conv_cache_out = conv_cache_out; cp.ssm_state_out = ssm_state_out;
+    cp.dt_sum = dt_sum;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return io == AXON_BF16 ? launch_qsplit<IoBF16, false, true>(cp, W, s) : launch_qsplit<IoF32, false, true>(cp, W, s);
 }
 
 }  // extern "C"

@@ -65,6 +65,7 @@ struct ChunkParams {
     void* y;
     void* conv_cache_out;
     float* ssm_state_out;
+    float* dt_sum;               // state-only split-chunk scan: (B, E) sum of the step sizes, else unused
 };
 
 constexpr int kSkew = 16;   // bytes added per run of rows (breaks bank aliasing between runs)

@@ -50,7 +50,7 @@ struct QsplitSmem {
     int pf;                          // (dt, f) per (token, channel)
     int dz;                          // (D u, SiLU(z)) per (token, channel), W > 1
     int warp_bytes;
-    int agg, entry, total;
+    int agg, entry, dts, total;
     __host__ __device__ static int pad(int r, int RQ) { return r + r / RQ; }
     __host__ __device__ QsplitSmem(int W, int R, int io_bytes) {
         const int RQ = R / 4;
@@ -70,12 +70,17 @@ struct QsplitSmem {
         off = W * warp_bytes;
         agg = off; off += W > 1 ? 2 * W * 2 * 32 * 16 : 0;   // [parity][warp][A | H][lane] float4
         entry = off; off += W > 1 ? 2 * 32 * 16 : 0;         // [parity][lane] h0..3
+        dts = off; off += W * kQsCh * 4;                     // state-only: [warp][channel] dt sums
         total = off;
     }
 };
 
-template <class Io, int W, int R, bool kZoh>
+// kState (first order only): the state-only form for a time split's first
+// pass -- no z, C, D, y: it walks the states to the end and writes the final
+// caches and, per channel, the sum of the step sizes (p.dt_sum).
+template <class Io, int W, int R, bool kZoh, bool kState = false>
 __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(ChunkParams p) {
+    static_assert(!(kZoh && kState), "the state-only form is first order");
     static_assert(R == 16 || R == 32, "R: 16 or 32 tokens per run");
     static_assert(W == 1 || W == 2 || W == 4 || W == 8, "W: 1, 2, 4 or 8 runs per chunk");
     using TT = typename Io::T;
@@ -138,7 +143,7 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
                 const int q = lane + 32 * i, r = q / P, pc = q % P;
                 if (q < NZP && pc < npc) {
                     const int so = QsplitSmem::pad(r, RQ) * XB + pc * 16, go = r * row_bytes + pc * 16;
-                    cp_async16(sb + lay.zs + so, zr + go, true);
+                    if constexpr (!kState) cp_async16(sb + lay.zs + so, zr + go, true);
                     cp_async16(sb + lay.ds + so, dr + go, true);
                 }
             }
@@ -148,7 +153,7 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
                 if (q < NBP) {
                     const int o = (q / PB) * RB + (q % PB) * 16;
                     cp_async16(sb + lay.bs + o, bg + bc0 + o, true);
-                    cp_async16(sb + lay.cs + o, cg + bc0 + o, true);
+                    if constexpr (!kState) cp_async16(sb + lay.cs + o, cg + bc0 + o, true);
                 }
             }
             return;
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
             const bool ok = t < p.L && pc < npc;
             const size_t go = ok ? tile_off + (size_t)t * row_bytes + pc * 16 : 0;
             const int so = QsplitSmem::pad(r, RQ) * XB + pc * 16;
-            cp_async16(sb + lay.zs + so, zg + go, ok);
+            if constexpr (!kState) cp_async16(sb + lay.zs + so, zg + go, ok);
             cp_async16(sb + lay.ds + so, dg + go, ok);
         }
         for (int q = lane; q < NBP; q += 32) {
@@ -186,7 +191,7 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
             const bool ok = t < p.L;
             const size_t go = ok ? ((size_t)b * p.L + t) * RB + pc * 16 : 0;
             cp_async16(sb + lay.bs + r * RB + pc * 16, bg + go, ok);
-            cp_async16(sb + lay.cs + r * RB + pc * 16, cg + go, ok);
+            if constexpr (!kState) cp_async16(sb + lay.cs + r * RB + pc * 16, cg + go, ok);
         }
     };
 
@@ -198,7 +203,7 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
     const float w3 = __ldg(p.conv_w + (size_t)e * kK + 3);
     const float cb = __ldg(p.conv_b + e);
     const float db = __ldg(p.dt_bias + e);
-    const float Dv = __ldg(p.D + e);
+    const float Dv = kState ? 0.0f : __ldg(p.D + e);     // D may be null for the state-only form
     float2 s01, s23, iA01 = f2(0.f, 0.f), iA23 = f2(0.f, 0.f), h01, h23;
     {
         const float4 al = __ldg(reinterpret_cast<const float4*>(p.A_log + (size_t)e * kN) + g);
@@ -244,6 +249,7 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
     float4* agg = reinterpret_cast<float4*>(smem + lay.agg);       // W > 1: [parity][warp][A | H][lane]
     float4* entry = reinterpret_cast<float4*>(smem + lay.entry);   // W > 1
 
+    float dt_acc = 0.0f;                     // state-only: sum of this lane's step sizes
     prefetch(0, 0);
     cp_async_commit();
     for (int k = 0; k < nck; ++k) {
@@ -286,9 +292,13 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
                 const float dtl = live ? dt : 0.0f;        // dt = 0: decay 1, no input
                 const float f = live ? (kZoh ? u : dt * u) : 0.0f;
                 pf[t * kQsCh + c] = make_float2(dtl, f);
-                const float du = Dv * u, gzv = silu(SI::ld(sb + lay.zs + tp * XB + c * S));
-                if constexpr (W == 1) { Du[i] = du; gz[i] = gzv; }
-                else dzs[t * kQsCh + c] = make_float2(du, gzv);
+                if constexpr (kState) {
+                    dt_acc += dtl;                 // the step sizes of the lane's tokens
+                } else {
+                    const float du = Dv * u, gzv = silu(SI::ld(sb + lay.zs + tp * XB + c * S));
+                    if constexpr (W == 1) { Du[i] = du; gz[i] = gzv; }
+                    else dzs[t * kQsCh + c] = make_float2(du, gzv);
+                }
             }
         }
         __syncwarp();
@@ -323,11 +333,13 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
 #pragma unroll
                 for (int i = 0; i < kBlk; ++i) {
                     const int t = tb + i;
-                    const float4 Cq = cq(sb, t);
                     h01 = __ffma2_rn(a01[i], h01, u01[i]);
                     h23 = __ffma2_rn(a23[i], h23, u23[i]);
-                    const float2 pq = __ffma2_rn(f2(Cq.z, Cq.w), h23, __fmul2_rn(f2(Cq.x, Cq.y), h01));
-                    part[t] = pq.x + pq.y;
+                    if constexpr (!kState) {
+                        const float4 Cq = cq(sb, t);
+                        const float2 pq = __ffma2_rn(f2(Cq.z, Cq.w), h23, __fmul2_rn(f2(Cq.x, Cq.y), h01));
+                        part[t] = pq.x + pq.y;
+                    }
                 }
             }
         } else {
@@ -361,12 +373,14 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
                 H23 = __ffma2_rn(a23, H23, i23);
                 P01 = __fmul2_rn(P01, a01);
                 P23 = __fmul2_rn(P23, a23);
-                const float4 Cq = cq(sb, t);
-                const float2 c01 = f2(Cq.x, Cq.y), c23 = f2(Cq.z, Cq.w);
-                const float2 pq = __ffma2_rn(c23, H23, __fmul2_rn(c01, H01));
-                pl[t] = pq.x + pq.y;
-                q01[t] = __fmul2_rn(c01, P01);
-                q23[t] = __fmul2_rn(c23, P23);
+                if constexpr (!kState) {
+                    const float4 Cq = cq(sb, t);
+                    const float2 c01 = f2(Cq.x, Cq.y), c23 = f2(Cq.z, Cq.w);
+                    const float2 pq = __ffma2_rn(c23, H23, __fmul2_rn(c01, H01));
+                    pl[t] = pq.x + pq.y;
+                    q01[t] = __fmul2_rn(c01, P01);
+                    q23[t] = __fmul2_rn(c23, P23);
+                }
             }
             // the run's aggregate (prod a, H) for the other warps
             {
@@ -390,10 +404,12 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
             }
             // ---- second pass: every token's C . h from the entering state,
             // no chain; then the run's end state
+            if constexpr (!kState) {
 #pragma unroll
-            for (int t = 0; t < R; ++t) {
-                const float2 pq = __ffma2_rn(q23[t], h23, __fmul2_rn(q01[t], h01));
-                part[t] = pl[t] + (pq.x + pq.y);
+                for (int t = 0; t < R; ++t) {
+                    const float2 pq = __ffma2_rn(q23[t], h23, __fmul2_rn(q01[t], h01));
+                    part[t] = pl[t] + (pq.x + pq.y);
+                }
             }
             h01 = __ffma2_rn(P01, h01, H01);
             h23 = __ffma2_rn(P23, h23, H23);
@@ -404,7 +420,7 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
         // apart: quadrants {0, 1} keep the first half of the run's tokens and
         // {2, 3} the second, then each quadrant keeps its own R/4 tokens, so
         // lane (g, c) ends with the totals of tokens g*RQ .. g*RQ + RQ - 1
-        {
+        if constexpr (!kState) {
             const bool hi = (g & 2) != 0, lo = (g & 1) != 0;
             float half[R / 2];
 #pragma unroll
@@ -451,6 +467,21 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
         TT* co = static_cast<TT*>(p.conv_cache_out);
 #pragma unroll
         for (int j = 0; j < kK - 1; ++j) co[((size_t)b * (kK - 1) + j) * p.E + e] = v[j];
+    }
+    if constexpr (kState) {
+        // the channel's sum of step sizes: its four quadrant lanes in every warp
+        // hold the sums of disjoint tokens; added in a fixed order
+        float v = dt_acc;
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        float* dts = reinterpret_cast<float*>(smem + lay.dts);
+        if (g == 0) dts[w * kQsCh + c] = v;
+        __syncthreads();
+        if (active && w == 0 && g == 0) {
+            float tot = 0.0f;
+            for (int j = 0; j < W; ++j) tot += dts[j * kQsCh + c];
+            p.dt_sum[(size_t)b * p.E + e] = tot;
+        }
     }
 }
 

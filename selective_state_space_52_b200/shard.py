@@ -33,15 +33,19 @@ import torch
 class SliceOps:
     """The per-slice operations: scan(x, z, dt_raw, B, C, params, cache) ->
     (y, (conv_cache, ssm_state)); dt_sum(dt_raw, dt_bias) -> (B,E); fold(r,
-    A_log, h_loc_all (P,B,E,N), dt_sum_all (P,B,E)) -> (B,E,N)."""
+    A_log, h_loc_all (P,B,E,N), dt_sum_all (P,B,E)) -> (B,E,N); optionally
+    scan_state(x, dt_raw, B, params, cache) -> ((conv_cache, ssm_state),
+    dt_sum), the first pass of a slice r >= 1 in one state-only scan."""
     scan: Callable
     dt_sum: Callable
     fold: Callable
+    scan_state: Callable | None = None
 
 
 def cuda_ops() -> SliceOps:
     from . import axon_ssm
-    return SliceOps(scan=axon_ssm.scan_fwd, dt_sum=axon_ssm.dt_sum, fold=axon_ssm.carry_fold)
+    return SliceOps(scan=axon_ssm.scan_fwd, dt_sum=axon_ssm.dt_sum, fold=axon_ssm.carry_fold,
+                    scan_state=axon_ssm.scan_state)
 
 
 def slice_tail(x: torch.Tensor, K: int) -> torch.Tensor:
@@ -53,12 +57,16 @@ def slice_tail(x: torch.Tensor, K: int) -> torch.Tensor:
 
 
 def first_pass(r: int, sl: dict, params: dict, halo, cache0, ops: SliceOps):
-    """Phase 2 for slice r: returns (y, caches, h_loc, dt_sum)."""
+    """Phase 2 for slice r: returns (y, caches, h_loc, dt_sum); y is None for
+    r >= 1 with a state-only scan (only slice 0's first-pass y is final)."""
     if r == 0:
         y, caches = ops.scan(sl["x"], sl["z"], sl["dt_raw"], sl["B"], sl["C"], params, cache0)
         # the same dtype as every other slice's sum: the exchange gathers equal buffers
         dts = torch.zeros(caches[1].shape[:2], dtype=caches[1].dtype, device=caches[1].device)
         return y, caches, caches[1], dts
+    if ops.scan_state is not None:
+        caches, dts = ops.scan_state(sl["x"], sl["dt_raw"], sl["B"], params, (halo, None))
+        return None, caches, caches[1], dts
     y, caches = ops.scan(sl["x"], sl["z"], sl["dt_raw"], sl["B"], sl["C"], params, (halo, None))
     return y, caches, caches[1], ops.dt_sum(sl["dt_raw"], params["dt_bias"])
 

@@ -66,3 +66,54 @@ def test_time_split_over_slices(cuda_lib, io, B, E, L, P, with_state):
     check_close(y, y_ref, tol_for(io, y_ref), f"slices y B{B} E{E} L{L} P{P} {io}")
     check_close(ss.cpu().numpy(), ss_ref, state_tol(ss_ref), "slices state")
     assert torch.equal(cc.cpu(), torch.from_numpy(cc_ref).to(cc.dtype))
+
+
+# The state-only first pass (axon_ssm_scan_state): the oracle's final caches
+# and the sum of the step sizes, on shapes that take each run count of the
+# split-chunk scan (few channels: 8 runs per chunk, many: 1), ragged lengths,
+# with and without initial caches, in place, and an empty sequence.
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("B,E,L", [(1, 64, 1), (2, 40, 301), (1, 2048, 1000), (3, 264, 77), (2, 7680, 129),
+                                   (64, 7680, 33)])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_scan_state_matches_oracle(cuda_lib, io, B, E, L, with_state):
+    from selective_state_space_52_b200 import axon_ssm
+    inp = W.make_inputs(W.custom(B, L, E, io=io, seed=9400 + E + L), with_state=True)
+    d = to_dev(inp)
+    params = {k: d[k] for k in ("conv_w", "conv_b", "dt_bias", "A_log", "D")}
+    cache = (d["conv_cache"], d["ssm_state"]) if with_state else None
+    (cc, ss), dts = axon_ssm.scan_state(d["x"], d["dt_raw"], d["B"], params, cache)
+    torch.cuda.synchronize()
+    _, cc_ref, ss_ref = oracle.scan_fwd(inp["x"], inp["z"], inp["dt_raw"], inp["B"], inp["C"], inp["conv_w"],
+                                        inp["conv_b"], inp["dt_bias"], inp["A_log"], inp["D"],
+                                        inp["conv_cache"] if with_state else None,
+                                        inp["ssm_state"] if with_state else None, parallel=True)
+    check_close(ss.cpu().numpy(), ss_ref, state_tol(ss_ref), "scan_state state")
+    assert torch.equal(cc.cpu(), torch.from_numpy(cc_ref).to(cc.dtype))
+    v = inp["dt_raw"].double().numpy() + inp["dt_bias"].double().numpy()
+    ref = np.clip(np.logaddexp(0.0, v), 1e-4, 100.0).sum(axis=1)
+    np.testing.assert_allclose(dts.cpu().double().numpy(), ref, rtol=2e-5)
+    # the same bits on a second run (a fixed summation order), and in place
+    (cc2, ss2), dts2 = axon_ssm.scan_state(d["x"], d["dt_raw"], d["B"], params, cache)
+    assert torch.equal(dts, dts2) and torch.equal(ss, ss2)
+    if with_state:
+        cci, ssi = d["conv_cache"].clone(), d["ssm_state"].clone()
+        Bsz, K, N = B, inp["conv_w"].shape[1], inp["A_log"].shape[1]
+        dt3 = torch.empty(B, E, dtype=torch.float32, device="cuda")
+        axon_ssm.axon_ssm_scan_state(B, L, E, N, K, 1 if io == "bf16" else 0, d["x"], d["dt_raw"], d["B"],
+                                     params["conv_w"], params["conv_b"], params["dt_bias"], params["A_log"],
+                                     cci, ssi, cci, ssi, dt3)
+        torch.cuda.synchronize()
+        assert torch.equal(cci, cc) and torch.equal(ssi, ss) and torch.equal(dt3, dts)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_scan_state_empty_sequence(cuda_lib, io):
+    from selective_state_space_52_b200 import axon_ssm
+    inp = W.make_inputs(W.custom(2, 0, 40, io=io, seed=9500), with_state=True)
+    d = to_dev(inp)
+    params = {k: d[k] for k in ("conv_w", "conv_b", "dt_bias", "A_log", "D")}
+    (cc, ss), dts = axon_ssm.scan_state(d["x"], d["dt_raw"], d["B"], params, (d["conv_cache"], d["ssm_state"]))
+    torch.cuda.synchronize()
+    assert torch.equal(cc, d["conv_cache"]) and torch.equal(ss, d["ssm_state"])
+    assert torch.count_nonzero(dts).item() == 0
