@@ -9,8 +9,9 @@ the same steps at the C level):
   1. all-gather every slice's last K-1 inputs: slice r's conv cache is slice
      r-1's tail (slice 0 uses the sequence's own conv cache);
   2. first pass: slice 0 scans from the sequence's initial state -- its y and
-     end state are final; slice r >= 1 scans from a zero state for its end
-     state h_loc_r and sums its dt (axon_ssm_dt_sum);
+     end state are final; slice r >= 1 runs a state-only scan from a zero
+     state for its end state h_loc_r and the sum of its dt
+     (axon_ssm_scan_state; or a full scan and axon_ssm_dt_sum);
   3. all-gather the (h_loc, dt_sum) pairs;
   4. slice r >= 1 folds them into its entering state (axon_ssm_carry_fold) and
      scans again from it: its y and end caches are final.
