@@ -375,3 +375,40 @@ def test_exp2_fma_argument_checks(lib):
     assert f(FAKE, None, 8, None) == INVALID
     assert f(FAKE + 4, FAKE + 4096, 8, None) == ALIGNMENT
     assert f(FAKE, FAKE + 16, 8, None) == INVALID               # partial overlap
+
+
+def _scan_state(lib, **over):
+    a = dict(B=1, L=64, E=32, N=16, K=4, io=0)
+    names = ["x", "dt_raw", "Bm", "conv_w", "conv_b", "dt_bias", "A_log", "cc_in", "ss_in", "cc_out", "ss_out", "dts"]
+    for i, n in enumerate(names):
+        a[n] = FAKE + (i << 32)
+    a["cc_in"] = a["ss_in"] = None
+    a.update(over)
+    f = lib.axon_ssm_scan_state
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 12 + [ctypes.c_void_p]
+    return f(a["B"], a["L"], a["E"], a["N"], a["K"], a["io"], *(a[n] for n in names), None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(N=8), UNSUPPORTED),
+    (dict(K=3), UNSUPPORTED),
+    (dict(io=7), UNSUPPORTED),
+    (dict(E=30), ALIGNMENT),                       # fp32 needs E % 4 == 0
+    (dict(B=-1), INVALID),
+    (dict(dts=None), INVALID),
+    (dict(x=None), INVALID),
+    (dict(Bm=None), INVALID),
+    (dict(conv_w=FAKE + 8), ALIGNMENT),
+    (dict(ss_out=FAKE + (9 << 32) + 16), INVALID),    # overlaps the conv cache output
+    (dict(dts=FAKE), INVALID),                        # overlaps x
+    (dict(cc_in=FAKE + (9 << 32) + 16), INVALID),     # partly overlaps the conv cache output
+])
+def test_scan_state_argument_checks(lib, over, status):
+    """The state-only scan's host checks: nothing is launched on an error."""
+    assert _scan_state(lib, **over) == status
+
+
+def test_scan_state_empty_is_ok(lib):
+    assert _scan_state(lib, B=0) == OK
+    assert _scan_state(lib, E=0) == OK
