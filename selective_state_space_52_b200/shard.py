@@ -66,8 +66,12 @@ def first_pass(r: int, sl: dict, params: dict, halo, cache0, ops: SliceOps):
         dts = torch.zeros(caches[1].shape[:2], dtype=caches[1].dtype, device=caches[1].device)
         return y, caches, caches[1], dts
     if ops.scan_state is not None:
-        caches, dts = ops.scan_state(sl["x"], sl["dt_raw"], sl["B"], params, (halo, None))
-        return None, caches, caches[1], dts
+        try:
+            caches, dts = ops.scan_state(sl["x"], sl["dt_raw"], sl["B"], params, (halo, None))
+            return None, caches, caches[1], dts
+        except Exception as ex:                      # a shape the state-only scan does not take
+            if getattr(ex, "status", None) != 2:     # AXON_ERR_UNSUPPORTED
+                raise
     y, caches = ops.scan(sl["x"], sl["z"], sl["dt_raw"], sl["B"], sl["C"], params, (halo, None))
     return y, caches, caches[1], ops.dt_sum(sl["dt_raw"], params["dt_bias"])
 
