@@ -111,6 +111,46 @@ def measured_peaks():
                 "source": "fallback"}
 
 
+# float32 operations per token x channel of the layer core (conv 4 FMA, dt*u
+# and 16 (dt A) products, 16 (dt u) B products, 16 state FMAs, 16 C.h FMAs,
+# D u and the gate product): the FMA side of the combined roofline
+FP32_OPS_PER_TOKEN_CH = 70
+
+
+def measure_peaks_in_run(dev) -> dict:
+    """The roofline's denominators measured in this run: the HBM copy rate
+    (1 GiB copied, read + write bytes, best of 5), and the MUFU exp2 and float32
+    FMA rates of this library's throughput probes (axon_peak_probe: 8 blocks of
+    256 threads per SM, 8 independent chains per thread, best of 5)."""
+    from selective_state_space_52_b200 import axon_ssm
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    blocks = sms * 8
+    out = torch.empty(blocks * 256, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def best(fn, reps=5):
+        fn()
+        torch.cuda.synchronize(dev)
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream); fn(); b.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(b) / 1e3)
+        return min(ts)
+
+    res = {"source": "measured in this run (bench.py measure_peaks_in_run)"}
+    for kind, name, iters in ((0, "mufu_gops", 4096), (1, "ffma_gops", 16384)):
+        secs = best(lambda: axon_ssm.axon_peak_probe(kind, out, blocks, iters))
+        res[name] = blocks * 256 * 8 * iters / secs / 1e9
+    src = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+    dst = torch.empty_like(src)
+    secs = best(lambda: dst.copy_(src))
+    res["hbm_copy_gbs"] = 2 * src.numel() / secs / 1e9
+    del src, dst
+    return res
+
+
 def scan_model(wl) -> dict:
     """Algorithmic bytes and MUFU operations of one prefill launch."""
     s = 2 if wl.io == "bf16" else 4
@@ -771,6 +811,13 @@ def run_axon(args, wl):
     hbm_ach = sm["bytes"] / (scan_ms / 1e3) / 1e9
     traffic = ncu_traffic("scan", wl.name, sm["token_ch"])
     stm = step_model(wl)
+    pin = measure_peaks_in_run(dev)
+    # the combined roofline with this run's peaks: the slowest of the bytes,
+    # the MUFU ops and the float32 ops at their measured rates
+    t_roof = {"hbm": sm["bytes"] / (pin["hbm_copy_gbs"] * 1e9),
+              "mufu": sm["mufu"] / (pin["mufu_gops"] * 1e9),
+              "fp32": FP32_OPS_PER_TOKEN_CH * sm["token_ch"] / (pin["ffma_gops"] * 1e9)}
+    bound_in_run = max(t_roof, key=t_roof.get)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
@@ -787,7 +834,13 @@ def run_axon(args, wl):
                      "kernel_ms": scan_ms, "algorithmic_bytes": sm["bytes"],
                      "hbm": {"achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": hbm_ach / peaks["hbm_gbs"],
-                             "peak_source": peaks["source"]}},
+                             "peak_source": peaks["source"]},
+                     "in_run": {"bound": bound_in_run, "frac": t_roof[bound_in_run] / (scan_ms / 1e3),
+                                "roofline_us": {k: v * 1e6 for k, v in t_roof.items()},
+                                "note": "max(algorithmic bytes / HBM copy, 22 MUFU ops / MUFU rate, "
+                                        f"{FP32_OPS_PER_TOKEN_CH} FP32 ops / FFMA rate) per token x channel, "
+                                        "each rate measured in this run (peaks_in_run)"}},
+        "peaks_in_run": pin,
         "decode_step": {"us": step_ms * 1e3, "algorithmic_bytes": stm["bytes"],
                         "hbm_gbs": stm["bytes"] / (step_ms / 1e3) / 1e9},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -803,6 +856,9 @@ def run_axon(args, wl):
                              if w.name not in ("tiny_f32", wl.name)}
     if not args.no_decode_bench:
         line["decode"] = bench_decode(dev)
+        line["decode"]["cold_frac_hbm_copy_in_run"] = (line["decode"]["algorithmic_bytes"] /
+                                                       (line["decode"]["cold_us"] / 1e6) / 1e9 /
+                                                       pin["hbm_copy_gbs"])
         line["prefill_zoh"] = bench_zoh_prefill(wl, sets, params, (y, cc, ss), ws, dev)
     if not args.no_block_bench and world == 1:
         line["block"] = bench_block(dev)

@@ -485,6 +485,19 @@ AXON_API axon_status axon_gemm_bf16(int M, int N, int K, const void *A, int lda,
  */
 AXON_API axon_status axon_exp2_fma(const float *x, float *y, long long n, axon_stream_t stream);
 
+/*
+ * Throughput probes for the roofline's compute denominators, measured in the
+ * same run as the kernels they rate (bench.py): `blocks` blocks of 256
+ * threads, each thread running 8 independent chains for `iters` steps --
+ * kind 0: y = 2^(y * c) on the MUFU unit (one exp2 per step), kind 1: y =
+ * y * a + b (one float32 FMA per step).  Ops executed = blocks * 256 * 8 *
+ * iters.  `out` (blocks * 256 float32 device values, 16-byte aligned)
+ * receives one sum per thread so the work is kept.  Other kinds are
+ * AXON_ERR_UNSUPPORTED, blocks <= 0, iters < 0 or out == NULL
+ * AXON_ERR_INVALID_ARG.  Enqueued on `stream`.
+ */
+AXON_API axon_status axon_peak_probe(int kind, float *out, int blocks, long long iters, axon_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -78,6 +78,8 @@ _lib.axon_ssd_scan_fwd.restype = _i
 _lib.axon_ssd_scan_fwd.argtypes = [_i] * 6 + [_vp] * 10 + [_i, _vp, _sz, _vp]
 _lib.axon_gemm_bf16.restype = _i
 _lib.axon_exp2_fma.restype = _i
+_lib.axon_peak_probe.restype = _i
+_lib.axon_peak_probe.argtypes = [_i, _vp, _i, ctypes.c_longlong, _vp]
 _lib.axon_exp2_fma.argtypes = [_vp, _vp, ctypes.c_longlong, _vp]
 _lib.axon_gemm_bf16.argtypes = [_i] * 3 + [_vp, _i, _vp, _i, _vp, _i, _vp, _vp]
 _lib.axon_ssm_block_workspace_bytes.restype = _sz
@@ -318,6 +320,13 @@ def axon_exp2_fma(x, y, n, stream=None, *, raise_on_error=True) -> int:
     rc = _lib.axon_exp2_fma(_p(x), _p(y), int(n), _stream(stream))
     if raise_on_error:
         _check(rc, "axon_exp2_fma")
+    return rc
+
+
+def axon_peak_probe(kind, out, blocks, iters, stream=None, *, raise_on_error=True) -> int:
+    rc = _lib.axon_peak_probe(int(kind), _p(out), int(blocks), int(iters), _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_peak_probe")
     return rc
 
 

@@ -11,6 +11,7 @@
 
 #include "axon_ssm.h"
 #include "carry.cuh"
+#include "probe.cuh"
 #include "device_math.cuh"
 #include "scan_chunked.cuh"
 #include "scan_octo.cuh"
@@ -801,6 +802,16 @@ axon_status axon_ssm_scan_state(int B, int L, int E, int N, int K, axon_dtype io
     cp.dt_sum = dt_sum;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return io == AXON_BF16 ? launch_qsplit<IoBF16, false, true>(cp, W, s) : launch_qsplit<IoF32, false, true>(cp, W, s);
+}
+
+axon_status axon_peak_probe(int kind, float* out, int blocks, long long iters, axon_stream_t stream) {
+    if (kind != 0 && kind != 1) return AXON_ERR_UNSUPPORTED;
+    if (blocks <= 0 || iters < 0 || !out) return AXON_ERR_INVALID_ARG;
+    if (!aligned16(out)) return AXON_ERR_ALIGNMENT;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (kind == 0) peak_probe_kernel<0><<<(unsigned)blocks, 256, 0, st>>>(out, iters);
+    else peak_probe_kernel<1><<<(unsigned)blocks, 256, 0, st>>>(out, iters);
+    return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
 
 }  // extern "C"

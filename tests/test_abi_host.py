@@ -412,3 +412,14 @@ def test_scan_state_argument_checks(lib, over, status):
 def test_scan_state_empty_is_ok(lib):
     assert _scan_state(lib, B=0) == OK
     assert _scan_state(lib, E=0) == OK
+
+
+def test_peak_probe_argument_checks(lib):
+    f = lib.axon_peak_probe
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_void_p]
+    assert f(2, FAKE, 1, 1, None) == UNSUPPORTED
+    assert f(0, None, 1, 1, None) == INVALID
+    assert f(0, FAKE, 0, 1, None) == INVALID
+    assert f(1, FAKE, 1, -1, None) == INVALID
+    assert f(0, FAKE + 4, 1, 1, None) == ALIGNMENT
