@@ -148,6 +148,14 @@ def measure_peaks_in_run(dev) -> dict:
     secs = best(lambda: dst.copy_(src))
     res["hbm_copy_gbs"] = 2 * src.numel() / secs / 1e9
     del src, dst
+    # the dense bf16 tensor rate as the library GEMM reaches it (a denominator only)
+    n = 8192
+    a = torch.randn(n, n, device=dev).to(torch.bfloat16)
+    b = torch.randn(n, n, device=dev).to(torch.bfloat16)
+    c = torch.empty(n, n, dtype=torch.bfloat16, device=dev)
+    secs = best(lambda: torch.matmul(a, b, out=c))
+    res["bf16_gemm_tflops"] = 2 * n ** 3 / secs / 1e12
+    del a, b, c
     return res
 
 
@@ -862,8 +870,12 @@ def run_axon(args, wl):
         line["prefill_zoh"] = bench_zoh_prefill(wl, sets, params, (y, cc, ss), ws, dev)
     if not args.no_block_bench and world == 1:
         line["block"] = bench_block(dev)
+        line["block"]["gemm_frac_of_bf16_gemm_in_run"] = (line["block"]["gemm_tflops_over_layer_time"] /
+                                                          pin["bf16_gemm_tflops"])
         line["time_split"] = bench_time_split(wl, sets[0], params, dev)
         line["ssd"] = bench_ssd(dev)
+        line["ssd"]["tensor"]["frac_of_bf16_gemm_in_run"] = (line["ssd"]["tensor"]["achieved"] /
+                                                             pin["bf16_gemm_tflops"])
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         inp_cpu = {**params_cpu, **{k: v.cpu() for k, v in sets[0].items()}}
         line["cpu_baseline"] = cpu_baselines(wl, inp_cpu, args.cpu_budget)
