@@ -93,6 +93,29 @@ __device__ __forceinline__ float dt_from_raw(float v) {
     return fminf(fmaxf(softplus(v), kDtMin), kDtMax);
 }
 
+// silu and dt_from_raw on a pair of values (two tokens), with the products,
+// sums and polynomial on the paired float32 pipe (FMUL2 / FADD2 / FFMA2) and
+// the roundings the scalar forms above compile to (the series as three FMAs),
+// so a pair gives what two scalar calls give.
+__device__ __forceinline__ float2 silu2(float2 v) {
+    const float2 a = __fmul2_rn(v, make_float2(-kLog2e, -kLog2e));
+    const float2 d = __fadd2_rn(make_float2(ex2_approx(a.x), ex2_approx(a.y)), make_float2(1.0f, 1.0f));
+    return __fmul2_rn(v, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+}
+__device__ __forceinline__ float2 dt_from_raw2(float2 v) {
+    const float2 a = __fmul2_rn(make_float2(fabsf(v.x), fabsf(v.y)), make_float2(-kLog2e, -kLog2e));
+    const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+    float2 r = __ffma2_rn(e, make_float2(-0.25f, -0.25f), make_float2(0.33333334f, 0.33333334f));
+    r = __ffma2_rn(e, r, make_float2(-0.5f, -0.5f));
+    r = __ffma2_rn(e, r, make_float2(1.0f, 1.0f));
+    const float2 series = __fmul2_rn(e, r);
+    const float2 onep = __fadd2_rn(e, make_float2(1.0f, 1.0f));
+    const float2 via = __fmul2_rn(make_float2(lg2_approx(onep.x), lg2_approx(onep.y)), make_float2(kLn2, kLn2));
+    const float2 l = make_float2(e.x < 0.015625f ? series.x : via.x, e.y < 0.015625f ? series.y : via.y);
+    const float2 sp = __fadd2_rn(make_float2(fmaxf(v.x, 0.0f), fmaxf(v.y, 0.0f)), l);
+    return make_float2(fminf(fmaxf(sp.x, kDtMin), kDtMax), fminf(fmaxf(sp.y, kDtMin), kDtMax));
+}
+
 // Exact zero-order-hold input factor (Axon-SSM page, "ZOH discretisation"):
 // Bbar = (exp(dt A) - 1) / A * B.  With x = dt*A <= 0 and a = exp(x) already
 // evaluated, this returns Bbar / B = dt * phi(x), phi(x) = expm1(x) / x:

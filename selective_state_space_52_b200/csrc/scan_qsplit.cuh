@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
     constexpr int XB = kQsCh * S;            // bytes of one staged x/z/dt row (8 channels)
     constexpr int RB = kN * S;               // bytes of one staged B/C row
     constexpr int RQ = R / 4;                // tokens per lane in the prologue
+    static_assert(RQ % 2 == 0, "the prologue runs tokens in pairs");
     constexpr int T = W * R;                 // tokens per chunk
     constexpr int P = XB / 16;               // 16-byte pieces per staged x/z/dt row
     constexpr int PB = RB / 16;              // 16-byte pieces per B/C row
@@ -277,27 +278,41 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
             float xm2 = SI::ld(xc + QsplitSmem::pad(tb + 1, RQ) * XB);
             float xm1 = SI::ld(xc + QsplitSmem::pad(tb + 2, RQ) * XB);
 #pragma unroll
-            for (int i = 0; i < RQ; ++i) {
+            for (int i = 0; i < RQ; i += 2) {   // tokens t and t + 1 as one float32 pair
                 const int t = tb + i;
-                const float xt = SI::ld(xc + QsplitSmem::pad(t + 3, RQ) * XB);
-                float xv = fmaf(w0, xm3, cb);
-                xv = fmaf(w1, xm2, xv);
-                xv = fmaf(w2, xm1, xv);
-                xv = fmaf(w3, xt, xv);
-                xm3 = xm2; xm2 = xm1; xm1 = xt;
-                const float u = silu(xv);
+                const float xt0 = SI::ld(xc + QsplitSmem::pad(t + 3, RQ) * XB);
+                const float xt1 = SI::ld(xc + QsplitSmem::pad(t + 4, RQ) * XB);
+                float xv0 = fmaf(w0, xm3, cb);
+                xv0 = fmaf(w1, xm2, xv0);
+                xv0 = fmaf(w2, xm1, xv0);
+                xv0 = fmaf(w3, xt0, xv0);
+                float xv1 = fmaf(w0, xm2, cb);
+                xv1 = fmaf(w1, xm1, xv1);
+                xv1 = fmaf(w2, xt0, xv1);
+                xv1 = fmaf(w3, xt1, xv1);
+                xm3 = xm1; xm2 = xt0; xm1 = xt1;
+                const float2 u = silu2(make_float2(xv0, xv1));
                 const int tp = t + g;            // padded row of token t (t / RQ == g)
-                const float dt = dt_from_raw(SI::ld(sb + lay.ds + tp * XB + c * S) + db);
-                const bool live = full || tr + t < p.L;
-                const float dtl = live ? dt : 0.0f;        // dt = 0: decay 1, no input
-                const float f = live ? (kZoh ? u : dt * u) : 0.0f;
-                pf[t * kQsCh + c] = make_float2(dtl, f);
-                if constexpr (kState) {
-                    dt_acc += dtl;                 // the step sizes of the lane's tokens
+                const float2 dt = dt_from_raw2(__fadd2_rn(make_float2(SI::ld(sb + lay.ds + tp * XB + c * S),
+                                                                      SI::ld(sb + lay.ds + (tp + 1) * XB + c * S)),
+                                                          make_float2(db, db)));
+                // dt = 0 past the sequence end: decay 1, no input
+                const bool live0 = full || tr + t < p.L, live1 = full || tr + t + 1 < p.L;
+                const float2 fu = kZoh ? u : __fmul2_rn(dt, u);
+                pf[t * kQsCh + c] = make_float2(live0 ? dt.x : 0.0f, live0 ? fu.x : 0.0f);
+                pf[(t + 1) * kQsCh + c] = make_float2(live1 ? dt.y : 0.0f, live1 ? fu.y : 0.0f);
+                if constexpr (kState) {            // the step sizes of the lane's tokens
+                    dt_acc += (live0 ? dt.x : 0.0f);
+                    dt_acc += (live1 ? dt.y : 0.0f);
                 } else {
-                    const float du = Dv * u, gzv = silu(SI::ld(sb + lay.zs + tp * XB + c * S));
-                    if constexpr (W == 1) { Du[i] = du; gz[i] = gzv; }
-                    else dzs[t * kQsCh + c] = make_float2(du, gzv);
+                    const float2 du = __fmul2_rn(make_float2(Dv, Dv), u);
+                    const float2 gzv = silu2(make_float2(SI::ld(sb + lay.zs + tp * XB + c * S),
+                                                         SI::ld(sb + lay.zs + (tp + 1) * XB + c * S)));
+                    if constexpr (W == 1) { Du[i] = du.x; gz[i] = gzv.x; Du[i + 1] = du.y; gz[i + 1] = gzv.y; }
+                    else {
+                        dzs[t * kQsCh + c] = make_float2(du.x, gzv.x);
+                        dzs[(t + 1) * kQsCh + c] = make_float2(du.y, gzv.y);
+                    }
                 }
             }
         }
