@@ -429,13 +429,14 @@ AXON_API axon_status axon_ssd_scan_fwd(
  *   out             = y W_out             W_out (E, Dm); out (B,L,Dm)
  *
  * Weights are row-major bf16 ("activations times weights").  The three
- * projections run on this library's tcgen05 GEMM (axon_gemm_bf16; float32
+ * projections run on this library's tcgen05 GEMM (axon_gemm_bf16_plan's
+ * automatic tiling with the workspace's stream-K scratch; float32
  * accumulation): one launch writes x and z, one writes dt_raw, B and C, one
  * the output.  The conv stage and the layer core run in this library's
  * kernels too.  The intermediates x, z, u, dt_raw, B, C and y are stored in
  * bf16 inside `workspace`, which must hold at least
  * axon_ssm_block_workspace_bytes(...) bytes (16-byte aligned; it also serves
- * as the scan's scratch).  Its first 4 bytes (an int) are an error flag,
+ * as the scan's scratch and the GEMMs' stream-K scratch).  Its first 4 bytes (an int) are an error flag,
  * cleared by each call and set to 1 if a wait of a GEMM for its copies or
  * tensor-core products gave up (the outputs are then undefined); read it
  * after the call completes.  Caches and parameters as for
@@ -460,8 +461,9 @@ AXON_API axon_status axon_ssm_block_fwd(
  * The projection GEMM the whole layer uses, on its own (tests and timing):
  * C (M x N) = A (M x K) W (K x N), all row-major bf16 with row strides lda,
  * ldw, ldc (elements), float32 accumulation, written as bf16.  Runs on the
- * tcgen05 tensor cores (tiles of 128 x 256, TMA-fed, accumulators in tensor
- * memory).  N, lda, ldw and ldc must be multiples of 8 and A, W, C 16-byte
+ * tcgen05 tensor cores (TMA-fed, accumulators in tensor memory): from 256
+ * rows on CTA pairs, 256 x 256 tiles, whole tiles; below on single CTAs,
+ * 128 x 256 or 128 x 192 tiles.  N, lda, ldw and ldc must be multiples of 8 and A, W, C 16-byte
  * aligned (AXON_ERR_ALIGNMENT); C must not overlap A or W; K == 0 with M, N
  * > 0 is AXON_ERR_INVALID_ARG.  `err` (a device int, or NULL) is set to 1 if
  * a wait of the kernel for its copies or products gave up (C is then
@@ -469,6 +471,42 @@ AXON_API axon_status axon_ssm_block_fwd(
  */
 AXON_API axon_status axon_gemm_bf16(int M, int N, int K, const void *A, int lda, const void *W, int ldw,
                                     void *C, int ldc, int *err, axon_stream_t stream);
+
+/*
+ * axon_gemm_bf16 with its tiling chosen by the caller (tests and timing):
+ *   AXON_GEMM_AUTO          what axon_gemm_bf16 picks (given the workspace);
+ *   AXON_GEMM_SINGLE_256    one CTA per 128 x 256 output tile;
+ *   AXON_GEMM_SINGLE_192    one CTA per 128 x 192 output tile;
+ *   AXON_GEMM_PAIR          a cluster of two CTAs (two SMs) per 256 x 256
+ *                           output tile, the tensor cores of both running one
+ *                           product of 256 rows (each CTA stages half of the
+ *                           W tile), whole tiles round-robin over the pairs;
+ *   AXON_GEMM_PAIR_STREAMK  the same tiles with the tiles x K-blocks
+ *                           iterations split evenly over the pairs
+ *                           (stream-K): a tile split between pairs is
+ *                           finished by the pair holding its first K blocks,
+ *                           which adds the others' float32 partial sums
+ *                           (kept in `workspace`) in a fixed order, so the
+ *                           result does not depend on timing.
+ * The pair plans return AXON_ERR_UNSUPPORTED if no two-CTA cluster fits on
+ * the device.  `workspace` (device, 16-byte aligned, not overlapping A, W or
+ * C) may be NULL except for AXON_GEMM_PAIR_STREAMK, which needs
+ * axon_gemm_workspace_bytes() bytes (AXON_ERR_WORKSPACE otherwise); the
+ * call clears its first bytes (flags) on `stream` before the product.  Any
+ * other plan is AXON_ERR_INVALID_ARG; the other arguments and errors are those
+ * of axon_gemm_bf16.
+ */
+enum {
+    AXON_GEMM_AUTO = 0,
+    AXON_GEMM_SINGLE_256 = 1,
+    AXON_GEMM_SINGLE_192 = 2,
+    AXON_GEMM_PAIR = 3,
+    AXON_GEMM_PAIR_STREAMK = 4
+};
+AXON_API size_t axon_gemm_workspace_bytes(void);
+AXON_API axon_status axon_gemm_bf16_plan(int M, int N, int K, const void *A, int lda, const void *W, int ldw,
+                                         void *C, int ldc, int *err, int plan, void *workspace,
+                                         size_t workspace_bytes, axon_stream_t stream);
 
 /*
  * The FMA-pipe exp2 on its own (tests): y[i] = 2^x[i] for x[i] <= 0, computed

@@ -82,6 +82,10 @@ _lib.axon_peak_probe.restype = _i
 _lib.axon_peak_probe.argtypes = [_i, _vp, _i, ctypes.c_longlong, _vp]
 _lib.axon_exp2_fma.argtypes = [_vp, _vp, ctypes.c_longlong, _vp]
 _lib.axon_gemm_bf16.argtypes = [_i] * 3 + [_vp, _i, _vp, _i, _vp, _i, _vp, _vp]
+_lib.axon_gemm_bf16_plan.restype = _i
+_lib.axon_gemm_bf16_plan.argtypes = [_i] * 3 + [_vp, _i, _vp, _i, _vp, _i, _vp, _i, _vp, _sz, _vp]
+_lib.axon_gemm_workspace_bytes.restype = _sz
+_lib.axon_gemm_workspace_bytes.argtypes = []
 _lib.axon_ssm_block_workspace_bytes.restype = _sz
 _lib.axon_ssm_block_workspace_bytes.argtypes = [_i] * 7
 _lib.axon_ssm_block_fwd.restype = _i
@@ -316,6 +320,23 @@ def axon_gemm_bf16(M, N, K, A, lda, W, ldw, C, ldc, err=None, stream=None, *, ra
     return rc
 
 
+# tilings of axon_gemm_bf16_plan (include/axon_ssm.h)
+GEMM_AUTO, GEMM_SINGLE_256, GEMM_SINGLE_192, GEMM_PAIR, GEMM_PAIR_STREAMK = 0, 1, 2, 3, 4
+
+
+def axon_gemm_workspace_bytes() -> int:
+    return int(_lib.axon_gemm_workspace_bytes())
+
+
+def axon_gemm_bf16_plan(M, N, K, A, lda, W, ldw, C, ldc, err=None, plan=GEMM_AUTO, workspace=None,
+                        workspace_bytes=0, stream=None, *, raise_on_error=True) -> int:
+    rc = _lib.axon_gemm_bf16_plan(M, N, K, _p(A), int(lda), _p(W), int(ldw), _p(C), int(ldc), _p(err),
+                                  int(plan), _p(workspace), int(workspace_bytes), _stream(stream))
+    if raise_on_error:
+        _check(rc, "axon_gemm_bf16_plan")
+    return rc
+
+
 def axon_exp2_fma(x, y, n, stream=None, *, raise_on_error=True) -> int:
     rc = _lib.axon_exp2_fma(_p(x), _p(y), int(n), _stream(stream))
     if raise_on_error:
@@ -340,15 +361,20 @@ def exp2_fma(x, *, out=None, stream=None):
     return y
 
 
-def gemm_bf16(A, W, *, out=None, stream=None, check=True):
+def gemm_bf16(A, W, *, out=None, stream=None, check=True, plan=GEMM_AUTO, workspace=None):
     """C = A @ W for row-major bf16 A (M x K) and W (K x N) on the library's
-    tcgen05 GEMM (float32 accumulation).  With ``check`` the call waits for the
-    device and raises AxonError (AXON_ERR_TIMEOUT) if a wait of the kernel gave up."""
+    tcgen05 GEMM (float32 accumulation; ``plan``: one of the GEMM_* tilings,
+    ``workspace``: a uint8 CUDA tensor of axon_gemm_workspace_bytes() bytes,
+    needed by GEMM_PAIR_STREAMK).  With ``check`` the call waits for the
+    device and raises AxonError (AXON_ERR_TIMEOUT) if a wait of the kernel
+    gave up."""
     M, K = A.shape
     N = W.shape[1]
     C = torch.empty(M, N, dtype=torch.bfloat16, device=A.device) if out is None else out
     err = torch.zeros(1, dtype=torch.int32, device=A.device)
-    axon_gemm_bf16(M, N, K, A, A.stride(0), W, W.stride(0), C, C.stride(0), err, stream=stream)
+    nws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    axon_gemm_bf16_plan(M, N, K, A, A.stride(0), W, W.stride(0), C, C.stride(0), err, plan, workspace, nws,
+                        stream=stream)
     if check and int(err.item()) != 0:
         raise AxonError(6, "axon_gemm_bf16 (a wait for a copy or a tensor-core product gave up)")
     return C

@@ -64,7 +64,31 @@ struct GemmParams {
     int nout;             // destinations (1..3), sorted by col0, out[0].col0 == 0
     GemmOut out[3];
     int* err;             // set to 1 when a wait gave up (may be null)
+    // CTA-pair kernel, stream-K split (null: whole tiles round-robin):
+    float* sk_partial;    // [pair][CTA][16 column chunks][4 quads][128 rows] float4 partial sums
+    int* sk_flag;         // [pair][CTA][4 epilogue warps], zero at launch; 1 once published
+    int sk_dp_tiles;      // the first tiles (a multiple of the pairs) go whole, round-robin
 };
+
+// Output row m, columns n .. n + 15 (bf16), as two 8-column (16-byte)
+// pieces, each into the destination that owns its columns; columns past N
+// are dropped.
+__device__ __forceinline__ void gemm_store16(const GemmParams& p, int m, int n, const float (&v)[16]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int col = n + 8 * h;
+        if (col < p.N) {
+            const int k = (p.nout > 2 && col >= p.out[2].col0) ? 2 : ((p.nout > 1 && col >= p.out[1].col0) ? 1 : 0);
+            const GemmOut o = k == 2 ? p.out[2] : (k == 1 ? p.out[1] : p.out[0]);
+            uint4 pk;
+            pk.x = pack_bf16(v[8 * h + 0], v[8 * h + 1]);
+            pk.y = pack_bf16(v[8 * h + 2], v[8 * h + 3]);
+            pk.z = pack_bf16(v[8 * h + 4], v[8 * h + 5]);
+            pk.w = pack_bf16(v[8 * h + 6], v[8 * h + 7]);
+            *reinterpret_cast<uint4*>(o.ptr + (size_t)m * o.ld + (col - o.col0)) = pk;
+        }
+    }
+}
 
 template <int kGmBN>
 __global__ void __launch_bounds__(kGmThreads, 1)
@@ -184,7 +208,9 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         int a = 0;
         uint32_t aph = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            if (!mbar_wait(tfull(a), aph) || *abort_flag) { fail(); break; }
+            // the warp decides together: the tensor-memory loads below are warp-wide
+            const bool ready = mbar_wait(tfull(a), aph) && !*abort_flag;
+            if (!__all_sync(0xffffffffu, ready)) { fail(); break; }
             tc_fence_after();
             const int m = (tile % p.tiles_m) * kGmBM + row;
             const int n0 = (tile / p.tiles_m) * kGmBN;
@@ -193,23 +219,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             for (int c0 = 0; c0 < kGmBN; c0 += 16) {
                 float v[16];
                 tmem_ld16(tl + c0, v);               // warp-wide: rows past M take part too
-                if (m < p.M) {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {    // two 8-column (16-byte) pieces
-                        const int col = n0 + c0 + 8 * h;
-                        if (col < p.N) {
-                            const int k = (p.nout > 2 && col >= p.out[2].col0) ? 2
-                                          : ((p.nout > 1 && col >= p.out[1].col0) ? 1 : 0);
-                            const GemmOut o = k == 2 ? p.out[2] : (k == 1 ? p.out[1] : p.out[0]);
-                            uint4 pk;
-                            pk.x = pack_bf16(v[8 * h + 0], v[8 * h + 1]);
-                            pk.y = pack_bf16(v[8 * h + 2], v[8 * h + 3]);
-                            pk.z = pack_bf16(v[8 * h + 4], v[8 * h + 5]);
-                            pk.w = pack_bf16(v[8 * h + 6], v[8 * h + 7]);
-                            *reinterpret_cast<uint4*>(o.ptr + (size_t)m * o.ld + (col - o.col0)) = pk;
-                        }
-                    }
-                }
+                if (m < p.M) gemm_store16(p, m, n0 + c0, v);
             }
             tc_fence_before();
             __syncwarp();

@@ -423,3 +423,36 @@ def test_peak_probe_argument_checks(lib):
     assert f(0, FAKE, 0, 1, None) == INVALID
     assert f(1, FAKE, 1, -1, None) == INVALID
     assert f(0, FAKE + 4, 1, 1, None) == ALIGNMENT
+
+
+def test_gemm_plan_argument_checks(lib):
+    """The tiling-choosing GEMM entry: plan range, the stream-K workspace
+    (missing, too small, misaligned, overlapping an operand) -- all refused
+    before anything is enqueued."""
+    q = lib.axon_gemm_workspace_bytes
+    q.restype = ctypes.c_size_t
+    q.argtypes = []
+    need = q()
+    assert need == 128 * 2 * 128 * 256 * 4 + 128 * 2 * 4 * 4   # 128 pairs: two 128 x 256 float32 partials, 8 flags
+    f = lib.axon_gemm_bf16_plan
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p, ctypes.c_int] * 3 + [ctypes.c_void_p, ctypes.c_int,
+                                                                          ctypes.c_void_p, ctypes.c_size_t,
+                                                                          ctypes.c_void_p]
+    A, W, C, ws = FAKE, FAKE + (1 << 32), FAKE + (2 << 32), FAKE + (3 << 32)
+
+    def call(plan, workspace=ws, nbytes=need, **kw):
+        a = dict(M=256, N=256, K=64)
+        a.update(kw)
+        return f(a["M"], a["N"], a["K"], A, a["K"], W, a["N"], C, a["N"], None, plan, workspace, nbytes, None)
+
+    assert call(5) == INVALID
+    assert call(-1) == INVALID
+    assert call(4, workspace=None, nbytes=0) == WORKSPACE          # stream-K needs the workspace
+    assert call(4, nbytes=need - 1) == WORKSPACE
+    assert call(4, workspace=ws + 4) == ALIGNMENT
+    assert call(3, workspace=ws + 4) == ALIGNMENT                  # a given workspace is checked for every plan
+    assert call(4, workspace=A + 64) == INVALID                     # overlaps A
+    assert call(4, workspace=C - 1024) == INVALID                   # overlaps C
+    assert call(4, M=0) == OK                                       # empty product
+    assert call(4, N=12) == ALIGNMENT                               # N % 8
