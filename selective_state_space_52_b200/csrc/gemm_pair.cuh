@@ -24,7 +24,9 @@
 //                        each finished accumulator to both "ready" barriers;
 //   warps 2-5            epilogue: this CTA's 128 accumulator rows (tensor
 //                        memory -> registers, 64 columns a round -> bf16 ->
-//                        global), then one arrival per warp on CTA 0's
+//                        a swizzled per-warp shared buffer -> global, 128
+//                        contiguous bytes of four rows per store
+//                        instruction), then one arrival per warp on CTA 0's
 //                        "drained" barrier (8 in all), so the issuer may
 //                        refill that accumulator.
 // Work: whole tiles round-robin over the pairs, M fastest (pairs running at
@@ -62,7 +64,9 @@ struct GemmPairCfg {
     static constexpr int kStages = 6;
     static constexpr int kAccs = 2;                                    // 256-column accumulators
     static constexpr int kBarOff = kStages * kStageBytes;
-    static constexpr int kSmem = kBarOff + 256 + 1024;                 // + barriers, slot, flags + alignment pad
+    static constexpr int kEpiOff = kBarOff + 256;                      // after the barriers, slot, flags
+    static constexpr int kEpiBytes = 4 * 32 * 128;                     // per epilogue warp: 32 rows x 64 bf16
+    static constexpr int kSmem = kEpiOff + kEpiBytes + 1024;           // + alignment pad
 };
 
 __global__ void __launch_bounds__(kGmThreads, 1)
@@ -223,7 +227,6 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             const bool ready = mbar_wait(tfull(a), aph) && !*abort_flag;
             if (!__all_sync(0xffffffffu, ready)) { fail(); return false; }
             tc_fence_after();
-            const int m = (tile % p.tiles_m) * kGpTileM + kGmBM * (int)rank + row;
             const int n0 = (tile / p.tiles_m) * kGpTileN;
             const uint32_t tl = tbase + (uint32_t)(a * kGpTileN) + ((uint32_t)(32 * q) << 16);
             // 64 accumulator columns per round: two 32-column loads in flight
@@ -238,6 +241,33 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                     v[j] = __uint_as_float(r0[j]);
                     v[32 + j] = __uint_as_float(r1[j]);
                 }
+            };
+            // 64 columns of the warp's 32 rows as bf16, through the warp's
+            // shared-memory buffer (16-byte chunks XOR-swizzled by row: both
+            // the row-wise writes and the reads below are conflict-free), so
+            // that each store instruction writes 128 contiguous bytes of four
+            // rows instead of 16 bytes of 32
+            unsigned char* ebuf = sm + Cfg::kEpiOff + q * (32 * 128);
+            const int mrow0 = (tile % p.tiles_m) * kGpTileM + kGmBM * (int)rank + 32 * q;
+            auto store64 = [&](int c0, const float (&v)[64]) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint4 pk;
+                    pk.x = pack_bf16(v[8 * j + 0], v[8 * j + 1]);
+                    pk.y = pack_bf16(v[8 * j + 2], v[8 * j + 3]);
+                    pk.z = pack_bf16(v[8 * j + 4], v[8 * j + 5]);
+                    pk.w = pack_bf16(v[8 * j + 6], v[8 * j + 7]);
+                    *reinterpret_cast<uint4*>(ebuf + lane * 128 + ((j ^ (lane & 7)) * 16)) = pk;
+                }
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = (lane >> 3) + 4 * i, ch = lane & 7;
+                    const uint4 pk = *reinterpret_cast<const uint4*>(ebuf + r * 128 + ((ch ^ (r & 7)) * 16));
+                    const int mm = mrow0 + r, col = n0 + c0 + 8 * ch;
+                    if (mm < p.M && col < p.N) gemm_store8(p, mm, col, pk);
+                }
+                __syncwarp();
             };
             if (kb0 > 0) {
                 // a later part of the tile: publish the float32 partial for the
@@ -315,11 +345,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                             }
                         }
                     }
-                    if (m < p.M) {
-#pragma unroll
-                        for (int h = 0; h < 4; ++h)
-                            gemm_store16(p, m, n0 + c0 + 16 * h, *reinterpret_cast<const float(*)[16]>(v + 16 * h));
-                    }
+                    store64(c0, v);
                 }
             }
             tc_fence_before();

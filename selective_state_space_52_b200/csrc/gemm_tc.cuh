@@ -70,6 +70,14 @@ struct GemmParams {
     int sk_dp_tiles;      // the first tiles (a multiple of the pairs) go whole, round-robin
 };
 
+// Output row m, columns col .. col + 7: one 16-byte piece of bf16 into the
+// destination that owns those columns (col < N).
+__device__ __forceinline__ void gemm_store8(const GemmParams& p, int m, int col, uint4 pk) {
+    const int k = (p.nout > 2 && col >= p.out[2].col0) ? 2 : ((p.nout > 1 && col >= p.out[1].col0) ? 1 : 0);
+    const GemmOut o = k == 2 ? p.out[2] : (k == 1 ? p.out[1] : p.out[0]);
+    *reinterpret_cast<uint4*>(o.ptr + (size_t)m * o.ld + (col - o.col0)) = pk;
+}
+
 // Output row m, columns n .. n + 15 (bf16), as two 8-column (16-byte)
 // pieces, each into the destination that owns its columns; columns past N
 // are dropped.
