@@ -22,8 +22,9 @@ constexpr int kConvRun = 32;     // tokens per thread
 constexpr int kConvThreads = 128;
 
 // 8 consecutive io values <-> float32: one 16-byte vector at bf16, two at fp32
+// (loads through the read-only path: x is never written by the kernel)
 __device__ __forceinline__ void conv_ld8(const __nv_bfloat16* p, float (&v)[8]) {
-    const uint4 q = *reinterpret_cast<const uint4*>(p);
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -32,7 +33,7 @@ __device__ __forceinline__ void conv_ld8(const __nv_bfloat16* p, float (&v)[8]) 
     }
 }
 __device__ __forceinline__ void conv_ld8(const float* p, float (&v)[8]) {
-    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 __device__ __forceinline__ void conv_st8(__nv_bfloat16* p, const float (&v)[8]) {
@@ -53,7 +54,10 @@ __device__ __forceinline__ void conv_st8(float* p, const float (&v)[8]) {
 // vectors) of one batch row over kConvRun consecutive tokens, loaded and
 // stored as whole vectors; the K-1 previous inputs of each channel slide in
 // registers.  grid = (ceil(E/8 / 128), ceil(L / kConvRun), B).  E is a
-// multiple of 8 and the rows 16-byte aligned.
+// multiple of 8 and the rows 16-byte aligned.  x and u never overlap (the
+// layer's workspace holds them apart), so the loads of later tokens may run
+// ahead of the stores of earlier ones: without that promise each token's
+// load waited for the previous token's store, one memory latency per token.
 template <class Io>
 __global__ void __launch_bounds__(kConvThreads) conv_silu_kernel(ConvParams p) {
     using T = typename Io::T;
@@ -63,9 +67,9 @@ __global__ void __launch_bounds__(kConvThreads) conv_silu_kernel(ConvParams p) {
     const int b = blockIdx.z;
     const int t0 = blockIdx.y * kConvRun;
     const int t1 = min(p.L, t0 + kConvRun);
-    const T* x = static_cast<const T*>(p.x);
+    const T* __restrict__ x = static_cast<const T*>(p.x);
     const T* cc = static_cast<const T*>(p.conv_cache_in);
-    T* u = static_cast<T*>(p.u);
+    T* __restrict__ u = static_cast<T*>(p.u);
 
     float w[8][kK], cbias[8], win[kK - 1][8];
 #pragma unroll
@@ -85,9 +89,9 @@ __global__ void __launch_bounds__(kConvThreads) conv_silu_kernel(ConvParams p) {
             for (int c = 0; c < 8; ++c) win[j][c] = 0.0f;
         }
     }
-    const T* row = x + ((size_t)b * p.L + t0) * p.E + e0;
-    T* out = u + ((size_t)b * p.L + t0) * p.E + e0;
-#pragma unroll 4
+    const T* __restrict__ row = x + ((size_t)b * p.L + t0) * p.E + e0;
+    T* __restrict__ out = u + ((size_t)b * p.L + t0) * p.E + e0;
+#pragma unroll 8
     for (int t = t0; t < t1; ++t, row += p.E, out += p.E) {
         float xt[8], o[8];
         conv_ld8(row, xt);
