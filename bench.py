@@ -188,7 +188,7 @@ KERNEL_SOURCES = {
              "scan_quad.cuh", "scan_seq.cuh"),
     "step": ("axon_ssm.cu", "device_math.cuh", "step.cuh"),
     "ssd": ("axon_ssd.cu", "device_math.cuh", "scan_chunked.cuh", "ssd.cuh", "tc_ops.cuh"),
-    "gemm": ("axon_block.cu", "gemm_tc.cuh", "tc_ops.cuh"),
+    "gemm": ("axon_block.cu", "gemm_pair.cuh", "gemm_tc.cuh", "tc_ops.cuh"),
 }
 
 
@@ -640,10 +640,12 @@ def run_single_kernel(args, wl, dev) -> dict:
         A = torch.randn(M, K, generator=g).to(torch.bfloat16).to(dev)
         Wt = (torch.randn(K, N, generator=g) / K ** 0.5).to(torch.bfloat16).to(dev)
         C = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        gws = torch.empty(axon_ssm.axon_gemm_workspace_bytes(), dtype=torch.uint8, device=dev)
 
         def call():
-            axon_ssm.gemm_bf16(A, Wt, out=C, check=False)
-        what = {"kernel": "axon_gemm_bf16", "M": M, "N": N, "K": K}
+            # the automatic tiling with the stream-K scratch, as the layer runs it
+            axon_ssm.gemm_bf16(A, Wt, out=C, check=False, workspace=gws)
+        what = {"kernel": "axon_gemm_bf16_plan (automatic, with stream-K scratch)", "M": M, "N": N, "K": K}
         flops = 2 * M * N * K
     else:
         inp = {k: v.to(dev) for k, v in W.make_inputs(wl).items()}
