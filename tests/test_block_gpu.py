@@ -79,6 +79,16 @@ def test_small_block(cuda_lib, with_state):
     check_block(inp, with_state, "small block")
 
 
+def test_block_on_cta_pairs_ragged_rows(cuda_lib):
+    """A layer tall enough for the CTA-pair GEMM (M = B*L = 600: two full
+    256-row tiles and a ragged one), with fewer tiles than pairs in every
+    projection, so all three run the stream-K split (tiles shared by several
+    pairs, partials added by their owners); small widths keep the oracle quick."""
+    bw = W.BLOCK_WORKLOAD_BY_NAME["small_block"]
+    inp = W.make_block_inputs(bw, with_state=True, L=300)
+    check_block(inp, True, "small block, 600 rows")
+
+
 def test_bit_axon_block_full_width(cuda_lib):
     """The Bit-Axon layer's widths (D 2560, E 7680) on a short sequence."""
     bw = W.BLOCK_WORKLOAD_BY_NAME["bit_axon_block"]
