@@ -346,7 +346,7 @@ axon_status axon_ssm_block_fwd(int B, int L, int Dm, int E, int N, int K, axon_d
             return rc;
         // u = SiLU(conv(x))
         ConvParams cp{B, L, E, x, conv_w, conv_b, conv_cache_in, u};
-        const dim3 grid((unsigned)((E / 8 + kConvThreads - 1) / kConvThreads),
+        const dim3 grid((unsigned)((E / kConvCh + kConvThreads - 1) / kConvThreads),
                         (unsigned)((L + kConvRun - 1) / kConvRun), (unsigned)B);
         if (grid.y > 65535u || grid.z > 65535u) return AXON_ERR_UNSUPPORTED;
         conv_silu_kernel<IoBF16><<<grid, kConvThreads, 0, st>>>(cp);
