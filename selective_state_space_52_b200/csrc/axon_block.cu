@@ -128,7 +128,17 @@ axon_status launch_gemm(int M, int N, int K, const CUtensorMap& ta, const void* 
     p.tiles_n = (N + BN - 1) / BN;
     const long long tiles = (long long)p.tiles_m * p.tiles_n;
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    gemm_bf16_tc_kernel<BN><<<grid, kGmThreads, Cfg::kSmem, st>>>(ta, tw, p);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kGmThreads, 1, 1);
+    cfg.dynamicSmemBytes = Cfg::kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gemm_bf16_tc_kernel<BN>, ta, tw, p) != cudaSuccess) return AXON_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
 
@@ -145,8 +155,10 @@ cudaLaunchConfig_t pair_config(unsigned pairs, cudaStream_t st, cudaLaunchAttrib
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cfg;
 }
 
@@ -165,7 +177,7 @@ int gemm_pair_slots(int dev) {
         }
         g_pair_smem_set.fetch_or(bit, std::memory_order_acq_rel);
     }
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     const cudaLaunchConfig_t cfg = pair_config(1, nullptr, attr);
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, gemm_bf16_pair_kernel, &cfg) != cudaSuccess || clusters <= 0) {
@@ -203,11 +215,17 @@ axon_status launch_gemm_pair(int M, int N, int K, const CUtensorMap& ta, const v
         p.sk_flag = sk->flag;
         p.sk_dp_tiles = (int)dp;
     }
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     const cudaLaunchConfig_t cfg = pair_config((unsigned)np, st, attr);
     if (cudaLaunchKernelEx(&cfg, gemm_bf16_pair_kernel, ta, tw, p) != cudaSuccess) return AXON_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
+
+// Launches after the layer's first kernel carry the programmatic-serialization
+// attribute: each kernel signals griddepcontrol.launch_dependents early and
+// waits (griddepcontrol.wait) for its predecessor before touching global
+// memory, so a kernel's launch and its local set-up (barriers, tensor memory)
+// overlap the previous kernel's tail.
 
 // Row-major outputs (M x N) = A (M x K, row stride lda) * W (K x N, row
 // stride ldw), bf16 in and out, float32 accumulation, on the tcgen05 GEMM.
@@ -349,7 +367,16 @@ axon_status axon_ssm_block_fwd(int B, int L, int Dm, int E, int N, int K, axon_d
         const dim3 grid((unsigned)((E / kConvCh + kConvThreads - 1) / kConvThreads),
                         (unsigned)((L + kConvRun - 1) / kConvRun), (unsigned)B);
         if (grid.y > 65535u || grid.z > 65535u) return AXON_ERR_UNSUPPORTED;
-        conv_silu_kernel<IoBF16><<<grid, kConvThreads, 0, st>>>(cp);
+        cudaLaunchConfig_t ccfg{};
+        ccfg.gridDim = grid;
+        ccfg.blockDim = dim3(kConvThreads, 1, 1);
+        ccfg.stream = st;
+        cudaLaunchAttribute cat[1];
+        cat[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        cat[0].val.programmaticStreamSerializationAllowed = 1;
+        ccfg.attrs = cat;
+        ccfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&ccfg, conv_silu_kernel<IoBF16>, cp) != cudaSuccess) return AXON_ERR_CUDA;
         if (cudaGetLastError() != cudaSuccess) return AXON_ERR_CUDA;
         // (dt_raw, B, C) = split(u W_x): columns [0, E), [E, E+N), [E+N, E+2N), one GEMM
         const GemmOut dbc[3] = {{dt, E, 0}, {bm, N, E}, {cm, N, E + N}};

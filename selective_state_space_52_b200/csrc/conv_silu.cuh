@@ -6,6 +6,7 @@
 #pragma once
 
 #include "device_math.cuh"
+#include "tc_ops.cuh"
 
 namespace axon {
 
@@ -58,6 +59,8 @@ __device__ __forceinline__ void conv_st4(float* p, const float (&v)[4]) {
 template <class Io>
 __global__ void __launch_bounds__(kConvThreads) conv_silu_kernel(ConvParams p) {
     using T = typename Io::T;
+    grid_dep_launch();
+    grid_dep_wait();
     const int g = blockIdx.x * kConvThreads + threadIdx.x;   // channel group
     if (g * kConvCh >= p.E) return;
     const int e0 = g * kConvCh;

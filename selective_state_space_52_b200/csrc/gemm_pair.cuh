@@ -114,6 +114,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     tc_fence_before();
     cluster_sync_all();                          // both CTAs' barriers and tensor memory exist
     tc_fence_after();
+    grid_dep_launch();
+    grid_dep_wait();                             // the operands' producers have finished
     const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(sm + Cfg::kBarOff + 8 * (2 * kStages + 2 * kAccs + 1));
 
     const int kblocks = (p.K + kGmBK - 1) / kGmBK;

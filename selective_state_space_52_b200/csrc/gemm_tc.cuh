@@ -139,6 +139,8 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    grid_dep_launch();
+    grid_dep_wait();                             // the operands' producers have finished
     const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(sm + kGmBarOff + 8 * (2 * kGmStages + 2 * kAccs + 1));
 
     const int ntiles = p.tiles_m * p.tiles_n;

@@ -97,6 +97,10 @@ __global__ void __launch_bounds__(32 * W, kZoh ? 1 : 16 / W) scan_qsplit_kernel(
     constexpr int NZP = R * P, NZ = (NZP + 31) / 32;
     constexpr int NBP = R * PB, NB = (NBP + 31) / 32;
     extern __shared__ __align__(16) unsigned char smem[];
+    // a kernel launched after this one with programmatic serialization (the
+    // whole layer's output projection) may be scheduled now: it waits for
+    // this grid's completion before it reads y
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const int lane = threadIdx.x & 31;
     const int w = threadIdx.x >> 5;          // run of the chunk

@@ -124,6 +124,13 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols));
 }
 
+// Programmatic dependent launch: let the next kernel of the stream (launched
+// with the programmatic-serialization attribute) be scheduled now, and wait
+// until the kernels this one depends on have finished and their writes are
+// visible.  Both are no-ops when there is no such kernel.
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---- CTA pairs (cta_group::2): a cluster of two CTAs whose tensor cores
 // run one product of M = 256 rows, each CTA holding half of A (its 128 rows)
 // and half of B (N / 2 columns) at the same shared-memory offsets; the
