@@ -180,13 +180,27 @@ axon_status axon_ssd_scan_fwd(int B, int L, int H, int P, int N, axon_dtype io,
         if (cudaGetLastError() != cudaSuccess) return AXON_ERR_CUDA;
     }
     if (!allow_smem<true>() || !allow_smem<false>()) return AXON_ERR_CUDA;
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    auto config = [&](dim3 grid, unsigned threads, size_t smem) {
+        cudaLaunchConfig_t c{};
+        c.gridDim = grid;
+        c.blockDim = dim3(threads, 1, 1);
+        c.dynamicSmemBytes = smem;
+        c.stream = st;
+        c.attrs = pdl;
+        c.numAttrs = 1;
+        return c;
+    };
     if (segs > 1) {
-        ssd_chunk_scan_kernel<false><<<dim3((unsigned)H, (unsigned)((segs - 1) * pcs), (unsigned)B), kSsdThreads,
-                                       SsdSmem<false>::TOTAL, st>>>(p);
-        if (cudaGetLastError() != cudaSuccess) return AXON_ERR_CUDA;
+        const cudaLaunchConfig_t c = config(dim3((unsigned)H, (unsigned)((segs - 1) * pcs), (unsigned)B), kSsdThreads,
+                                            SsdSmem<false>::TOTAL);
+        if (cudaLaunchKernelEx(&c, ssd_chunk_scan_kernel<false>, p) != cudaSuccess) return AXON_ERR_CUDA;
     }
-    ssd_chunk_scan_kernel<true><<<dim3((unsigned)H, (unsigned)segs, (unsigned)B), kSsdFullThreads,
-                                  SsdSmem<true>::TOTAL, st>>>(p);
+    const cudaLaunchConfig_t c = config(dim3((unsigned)H, (unsigned)segs, (unsigned)B), kSsdFullThreads,
+                                        SsdSmem<true>::TOTAL);
+    if (cudaLaunchKernelEx(&c, ssd_chunk_scan_kernel<true>, p) != cudaSuccess) return AXON_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? AXON_OK : AXON_ERR_CUDA;
 }
 

@@ -111,6 +111,8 @@ __device__ __forceinline__ int tile_off(int r, int pc) {
 // below 2^-126 of G_ij dt_j.  Tokens past L get dt = 0, e = -inf, v = 0.
 // grid = (nC, ceil(H / 4), B), 128 threads: warp -> head, lane -> 4 tokens.
 __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_prep_kernel(SsdParams p) {
+    grid_dep_launch();
+    grid_dep_wait();
     const int c = blockIdx.x, b = blockIdx.z;
     const int lane = threadIdx.x & 31;
     const int h = blockIdx.y * 4 + (threadIdx.x >> 5);
@@ -204,6 +206,7 @@ template <> struct SsdSmem<false> {
 template <bool kFull>
 __global__ void __launch_bounds__(kFull ? kSsdFullThreads : kSsdThreads, kFull ? 1 : 3)
     ssd_chunk_scan_kernel(SsdParams p) {
+    grid_dep_launch();
     using Lay = SsdSmem<kFull>;
     constexpr int Q = kSsdQ, P = kSsdP, N = kSsdN;
     constexpr int NT = kFull ? kSsdFullThreads : kSsdThreads;
@@ -272,6 +275,7 @@ __global__ void __launch_bounds__(kFull ? kSsdFullThreads : kSsdThreads, kFull ?
                      "r"(Lay::TMEM_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
+    grid_dep_wait();                    // the prep values and the first walk's states are written
     if (c_begin < c_end) issue_chunk(c_begin, 0);
 
     // ---- the carried state, transposed: thread (n, hf) holds S[p][n] for its PH head columns
