@@ -492,7 +492,10 @@ AXON_API axon_status axon_gemm_bf16(int M, int N, int K, const void *A, int lda,
  * the device.  `workspace` (device, 16-byte aligned, not overlapping A, W or
  * C) may be NULL except for AXON_GEMM_PAIR_STREAMK, which needs
  * axon_gemm_workspace_bytes() bytes (AXON_ERR_WORKSPACE otherwise); the
- * call clears its first bytes (flags) on `stream` before the product.  Any
+ * call clears its first bytes (flags) on `stream` before the product.  The
+ * stream-K pairs wait (bounded) on one another's flags: the grid holds as
+ * many pairs as fit on the device, so when other work occupies SMs at the
+ * same time a wait may give up, and `err` is then set (C undefined).  Any
  * other plan is AXON_ERR_INVALID_ARG; the other arguments and errors are those
  * of axon_gemm_bf16.
  */
