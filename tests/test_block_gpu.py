@@ -16,6 +16,8 @@ changes a long-memory state's whole history).  So the GPU is checked two ways:
 Applied to the output, the final state and the final conv cache (the last rows
 of x, stored in bf16).
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -119,3 +121,37 @@ def test_block_empty_sequence_copies_caches(cuda_lib):
     assert out.shape == (bw.B, 0, bw.Dm)
     np.testing.assert_array_equal(cc, inp["conv_cache"].float().numpy())
     np.testing.assert_array_equal(ss, inp["ssm_state"].numpy())
+
+
+def test_back_to_back_layer_calls_share_a_workspace(cuda_lib):
+    """Three layer calls enqueued back to back on one stream with one shared
+    workspace and no synchronisation between them (inputs A, B, then A again;
+    CTA-pair projections with the stream-K split, kernels chained by
+    programmatic dependent launch): the two A outputs agree bit for bit and
+    B's matches B run on its own, so no kernel reads its inputs early or sees
+    flags or partial sums left by the call before."""
+    from selective_state_space_52_b200 import axon_ssm
+    bw = W.BLOCK_WORKLOAD_BY_NAME["small_block"]
+    ia = to_dev(W.make_block_inputs(bw, with_state=True, L=300))
+    ib = to_dev(W.make_block_inputs(dataclasses.replace(bw, seed=bw.seed + 101), with_state=True, L=300))
+
+    def call(d, ws):
+        weights = {k: d[k] for k in axon_ssm.WEIGHT_KEYS}
+        params = {k: d[k] for k in axon_ssm.PARAM_KEYS}
+        return axon_ssm.block_fwd(d["X"], weights, params, (d["conv_cache"], d["ssm_state"]), workspace=ws,
+                                  check=False)
+
+    E, N, K, Dm = bw.E, bw.N, bw.K, bw.Dm
+    ws = torch.empty(axon_ssm.axon_ssm_block_workspace_bytes(bw.B, 300, Dm, E, N, K), dtype=torch.uint8,
+                     device="cuda")
+    outs = [call(d, ws) for d in (ia, ib, ia)]
+    torch.cuda.synchronize()
+    assert axon_ssm.block_error_flag(ws) == 0
+    (a1, (ca1, sa1)), (b1, (cb1, sb1)), (a2, (ca2, sa2)) = outs
+    assert torch.equal(a1.view(torch.int16), a2.view(torch.int16))
+    assert torch.equal(sa1, sa2) and torch.equal(ca1.view(torch.int16), ca2.view(torch.int16))
+    ws2 = torch.empty_like(ws)
+    b2, (cb2, sb2) = call(ib, ws2)
+    torch.cuda.synchronize()
+    assert torch.equal(b1.view(torch.int16), b2.view(torch.int16))
+    assert torch.equal(sb1, sb2) and torch.equal(cb1.view(torch.int16), cb2.view(torch.int16))
