@@ -142,3 +142,21 @@ def test_gemm_plan_errors(cuda_lib, gemm_ws):
     ws_over_c = c.view(torch.uint8)
     assert call(256, 256, 256, a, 256, a, 256, c, 256, None, 4, ws_over_c, gemm_ws.numel(),
                 raise_on_error=False) == 1
+
+
+def test_gemm_stream_k_back_to_back_calls_share_a_workspace(cuda_lib, gemm_ws):
+    """Stream-K products enqueued back to back with one workspace and no
+    synchronisation (operands A, B, then A again): each call clears its flags
+    on the stream before it runs, so the two A results agree bit for bit and
+    B's matches B run on its own (no owner sees a flag or partial left by the
+    call before)."""
+    M, N, K = 2048, 2560, 7680
+    g = torch.Generator().manual_seed(21)
+    ops = [((torch.randn(M, K, generator=g) / K ** 0.25).to(torch.bfloat16).cuda(),
+            (torch.randn(K, N, generator=g) / K ** 0.25).to(torch.bfloat16).cuda()) for _ in range(2)]
+    outs = [cuda_lib.gemm_bf16(A, W, plan=4, workspace=gemm_ws, check=False) for A, W in (ops[0], ops[1], ops[0])]
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0].view(torch.int16), outs[2].view(torch.int16))
+    alone = cuda_lib.gemm_bf16(*ops[1], plan=4, workspace=torch.empty_like(gemm_ws))
+    torch.cuda.synchronize()
+    assert torch.equal(outs[1].view(torch.int16), alone.view(torch.int16))

@@ -163,3 +163,32 @@ def test_ssd_wait_gives_up_and_reports(cuda_lib):
     assert int(status.item()) == 1
     # the device still runs the SSD core afterwards
     test_ssd_small(cuda_lib, 130, True)
+
+
+def test_ssd_back_to_back_calls_share_a_workspace(cuda_lib):
+    """Three SSD calls enqueued back to back on one stream with one shared
+    workspace and no synchronisation between them (inputs A, B, then A again;
+    three segments, so the state-only walk and the carries run; the kernels
+    chained by programmatic dependent launch): the two A results agree bit
+    for bit and B's matches B run on its own."""
+    import dataclasses
+    from selective_state_space_52_b200 import axon_ssm
+    sw = W.SSD_WORKLOAD_BY_NAME["small_ssd"]
+    da = {k: v.cuda() for k, v in W.make_ssd_inputs(sw, with_state=True, L=1000).items()}
+    db = {k: v.cuda() for k, v in W.make_ssd_inputs(dataclasses.replace(sw, seed=sw.seed + 77), with_state=True,
+                                                   L=1000).items()}
+    nbytes = axon_ssm.axon_ssd_workspace_bytes(sw.B, 1000, sw.H, sw.P, sw.N, 3)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+
+    def call(d, w):
+        params = {k: d[k] for k in ("dt_bias", "A_log", "D")}
+        return axon_ssm.ssd_scan(d["x"], d["dt_raw"], d["B"], d["C"], params, d["h0"], workspace=w, segments=3,
+                                 check=False)
+
+    (ya1, ha1), (yb1, hb1), (ya2, ha2) = [call(d, ws) for d in (da, db, da)]
+    torch.cuda.synchronize()
+    assert axon_ssm.ssd_error_flag(ws) == 0
+    assert torch.equal(ya1.view(torch.int16), ya2.view(torch.int16)) and torch.equal(ha1, ha2)
+    yb2, hb2 = call(db, torch.empty_like(ws))
+    torch.cuda.synchronize()
+    assert torch.equal(yb1.view(torch.int16), yb2.view(torch.int16)) and torch.equal(hb1, hb2)
