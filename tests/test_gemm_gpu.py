@@ -73,8 +73,10 @@ def test_gemm_rejects_bad_arguments(cuda_lib):
     assert cuda_lib.axon_gemm_bf16(0, 16, 16, None, 16, None, 16, None, 16, raise_on_error=False) == 0  # empty
 
 
+# (9472, 512, 256): 74 pair tiles, as many as a B200 runs at once, so the
+# stream-K plan leaves no split tail (every tile whole through the split path)
 PLAN_SHAPES = [(1, 8, 8), (256, 256, 64), (256, 256, 7680), (300, 520, 104), (129, 264, 200), (1000, 4096, 1024),
-               (4096, 15360, 64), (2048, 2560, 7680), (2048, 7712, 7680), (2048, 15360, 2560)]
+               (4096, 15360, 64), (2048, 2560, 7680), (2048, 7712, 7680), (2048, 15360, 2560), (9472, 512, 256)]
 
 
 @pytest.fixture(scope="module")
